@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the PaTH attention hot path on B200.
+
+One step = the whole training hot path on one batch: path_attn_fwd then
+path_attn_bwd (UT prep, transport chain, attention forward, attention
+backward, UT adjoint, gate gradient) at B=8 H=24 L=4096 d=64 bf16, inputs
+resident in HBM. The decode step (B=32 H=32 d=128, cache 16384 -> 16448,
+64 steps) is timed after it and reported under "decode".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs the same workload on its own GPU (weak
+scaling: heads are independent, no collective on the data path); the step
+time is the max over ranks.
+
+Metric: algorithmic TFLOP/s = 11 * L^2 * d * B * H FLOP per step (forward
+3 L^2 d: QK^T, PV and the d x d block transport at 64-position blocks;
+backward 8 L^2 d) divided by the device time of a step. Also reported:
+tokens/s = B * L / step time, and the FlashAttention-equivalent 7 L^2 d count.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic_inputs as si  # noqa: E402
+
+WORKLOAD = "fwdbwd_bf16_l4096"
+DECODE = "decode_bf16_c16k"
+METRIC = "PaTH fwd+bwd TFLOP/s at L=4096 d=64 (algorithmic 11*L^2*d per head)"
+UNIT = "TFLOP/s"
+
+
+def algorithmic_flops(B, H, L, d):
+    return 11.0 * L * L * d * B * H
+
+
+def fa_equiv_flops(B, H, L, d):
+    return 7.0 * L * L * d * B * H
+
+
+def stage_flops(name, B, H, L, d, BT=128):
+    """Algorithmic FLOP of one launch of a stage (causal, leading order)."""
+    nh = B * H
+    per = {
+        "attn_fwd": 2.0 * L * L * d,                      # QK^T + PV
+        "attn_bwd_q": 3.0 * L * L * d,                    # S, dP, dQ
+        "attn_bwd_k": 4.0 * L * L * d + 2.0 * L * L * d * d / BT,  # S, dP, dV, dK + chain adjoint
+        "chain": 1.0 * L * L * d * d / BT,                # key-side block transport
+    }
+    return per.get(name, 0.0) * nh
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples of one GPU while the timed region runs."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "utilization.gpu")
+
+    def __init__(self, device):
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            pass
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 11:
+                    continue
+                if self.uuid and self.uuid.replace("GPU-", "") not in parts[1]:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        busy = [r for r in rows if (num(r[10]) or 0) > 50] or rows
+        sm = [num(r[2]) for r in busy if num(r[2]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in busy:
+            for n, v in zip(names, r[6:10]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(rows[0][3]), "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(busy)}
+
+
+def lib_call(name, *args):
+    import softmax_attention_block_b200 as P
+    return getattr(P.lib(), name)(*args)
+
+
+class StageTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("total_ms", ctypes.c_double),
+                ("count", ctypes.c_int)]
+
+
+def read_profile():
+    import softmax_attention_block_b200 as P
+    L = P.lib()
+    L.path_profile_read.argtypes = [ctypes.POINTER(StageTime), ctypes.c_int]
+    buf = (StageTime * 64)()
+    n = L.path_profile_read(buf, 64)
+    return {buf[i].name.decode(): (buf[i].total_ms, buf[i].count) for i in range(n)}
+
+
+# ---------------------------------------------------------------- reference arm
+def cpu_baseline_sample(w, heads=(0,)):
+    """Time the fp64 oracle (as it stands) on a bounded sample: the listed heads
+    of the workload, forward + backward. Returns (TFLOP/s, seconds, cores)."""
+    import oracle
+
+    x = si.workload_inputs(w.name, heads=list(heads))
+    orc = oracle.default()
+    t0 = time.perf_counter()
+    orc.fwd(x["q"], x["k"], x["v"], x["w"], x["beta"], x["log_f"])
+    orc.bwd(x["q"], x["k"], x["v"], x["w"], x["beta"], x["dout"], x["log_f"])
+    dt = time.perf_counter() - t0
+    flops = algorithmic_flops(1, len(heads), w.L, w.d)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return flops / dt / 1e12, dt, cores
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = si.WORKLOADS[WORKLOAD]
+    for _ in range(args.warmup):
+        cpu_baseline_sample(w)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        v, s, cores = cpu_baseline_sample(w)
+        vals.append(v)
+        secs.append(s)
+    value = statistics.mean(vals)
+    sample = (f"1 of {w.B * w.H} heads (b=0,h=0) of {WORKLOAD}, fwd+bwd, fp64 oracle; "
+              f"TFLOP/s on that head's 11*L^2*d FLOP")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * statistics.mean(secs), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+                       "sample": "1 head per step"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch.distributed as dist
+    import softmax_attention_block_b200 as P
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    P.lib()
+    peaks = load_peaks()
+
+    w = si.WORKLOADS[WORKLOAD]
+    xc = si.workload_inputs(WORKLOAD, seed=0)
+    x = {k: (v.to(dev) if v is not None else None) for k, v in xc.items()}
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    grads = {n: torch.empty_like(x["q"]) for n in ("dq", "dk", "dv", "dw")}
+    grads["dbeta"] = torch.empty_like(x["beta"])
+    ws_bytes = max(P.path_attn_workspace_bytes(w.B, w.H, w.L, w.d, w.dtype, True),
+                   P.path_attn_workspace_bytes(w.B, w.H, w.L, w.d, w.dtype, False))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def step(inp):
+        P.path_attn_fwd(inp["q"], inp["k"], inp["v"], inp["w"], inp["beta"], inp["log_f"],
+                        out=out, lse=lse, workspace=ws)
+        P.path_attn_bwd(inp["q"], inp["k"], inp["v"], inp["w"], inp["beta"], out, lse,
+                        inp["dout"], inp["log_f"], grads=grads, workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step(x)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    launches0 = P.lib().path_kernel_launch_count()
+    P.lib().path_profile_enable(1)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(x)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    P.lib().path_profile_enable(0)
+    launches = P.lib().path_kernel_launch_count() - launches0
+    clk = clocks.stop()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    stages = read_profile()
+    ms_step = ms_total / args.steps
+    flops = algorithmic_flops(w.B, w.H, w.L, w.d)
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    tokens = world * w.B * w.L / (ms_step * 1e-3)
+
+    # dominant stage -> roofline against the measured bf16 dense peak
+    stage_rows = {n: {"ms_per_launch": t / c, "launches": c, "share": 0.0}
+                  for n, (t, c) in stages.items()}
+    tot = sum(t for t, _ in stages.values()) or 1.0
+    for n, (t, _) in stages.items():
+        stage_rows[n]["share"] = t / tot
+    dom = max(stages, key=lambda n: stages[n][0]) if stages else None
+    roofline = None
+    if dom:
+        per_launch_ms = stages[dom][0] / stages[dom][1]
+        f = stage_flops(dom, w.B, w.H, w.L, w.d)
+        ach = f / (per_launch_ms * 1e-3) / 1e12 if f else None
+        peak = peaks["bf16_tflops_sustained"]
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak,
+                    "unit": "TFLOP/s", "frac": (ach / peak) if ach else None, "traffic": None,
+                    "peak_source": f"{peaks['source']} bf16 dense (sustained)"}
+
+    # end to end through the API with host buffers (pinned), copies in the timed region
+    e2e = None
+    if not args.no_e2e:
+        host = {k: (v.pin_memory() if v is not None else None) for k, v in xc.items()}
+        hout = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                for n, t in list(grads.items()) + [("out", out), ("lse", lse)]}
+        dev_in = {k: (torch.empty_like(v) if v is not None else None) for k, v in x.items()}
+        h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+        d2h = sum(v.numel() * v.element_size() for v in hout.values())
+
+        def e2e_step():
+            for k, v in host.items():
+                if v is not None:
+                    dev_in[k].copy_(v, non_blocking=True)
+            step(dev_in)
+            for n, t in list(grads.items()) + [("out", out), ("lse", lse)]:
+                hout[n].copy_(t, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+        e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del host, hout, dev_in
+
+    del x, out, lse, grads, ws
+    torch.cuda.empty_cache()
+    decode = None if args.no_decode else bench_decode(P, dev, peaks, world, max_over_ranks,
+                                                       barrier)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, s, cores = cpu_baseline_sample(w)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"1 of {w.B * w.H} heads of {WORKLOAD} fwd+bwd in fp64 ({s:.1f} s)"}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+                       "log_f": False, "l2": "inputs larger than L2 (each [B,H,L,d] bf16 "
+                       "tensor is 100.7 MB; 126 MB L2)",
+                       "parallelism": f"{world} rank(s), full workload per rank"},
+            "tokens_per_s": tokens,
+            "tflops_fa_equiv": world * fa_equiv_flops(w.B, w.H, w.L, w.d) / (ms_step * 1e-3) / 1e12,
+            "pct_bf16_peak": value / world / peaks["bf16_tflops_sustained"],
+            "stages": stage_rows, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clk, "decode": decode}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_decode(P, dev, peaks, world, max_over_ranks, barrier):
+    w = si.WORKLOADS[DECODE]
+    cap = w.n0 + w.steps
+    kc, vc, seq = si.make_decode_inputs(w.B, w.H, w.d, w.n0, cap, w.steps, w.dtype, seed=0)
+    kd, vd = kc.to(dev), vc.to(dev)
+    del kc, vc
+    sd = [{k: v.to(dev) for k, v in s.items()} for s in seq]
+    out = torch.empty((w.B, w.H, w.d), dtype=w.dtype, device=dev)
+    ws = torch.empty(P.path_decode_workspace_bytes(w.B, w.H, cap, w.d, w.dtype), dtype=torch.uint8,
+                     device=dev)
+    # warm-up on a copy of the first steps' state would change the cache; warm up on the
+    # first 3 steps then rewind n (the cache rows past n0 are overwritten by the timed run)
+    for t in range(3):
+        s = sd[t]
+        P.path_decode_step(s["q"], s["k_new"], s["v_new"], s["w"], s["beta"], kd, vd, w.n0 + t,
+                           out=out, workspace=ws)
+    torch.cuda.synchronize()
+    barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    P.lib().path_profile_enable(1)
+    e0.record(stream)
+    for t, s in enumerate(sd):
+        P.path_decode_step(s["q"], s["k_new"], s["v_new"], s["w"], s["beta"], kd, vd, w.n0 + t,
+                           out=out, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    P.lib().path_profile_enable(0)
+    stages = read_profile()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / w.steps
+    nh = w.B * w.H
+    n_avg = w.n0 + (w.steps - 1) / 2.0
+    bytes_step = 3.0 * nh * n_avg * w.d * 2  # read K, write K, read V (bf16)
+    gbs = world * bytes_step / (ms * 1e-3) / 1e9
+    chunk_ms = stages.get("decode_chunks", (0.0, 1))
+    per_launch = chunk_ms[0] / max(chunk_ms[1], 1)
+    ach = bytes_step / (per_launch * 1e-3) / 1e9 if per_launch else None
+    return {"workload": DECODE, "value": gbs, "unit": "GB/s", "us_per_step": ms * 1e3,
+            "bytes_per_step": bytes_step,
+            "roofline": {"kernel": "decode_chunks", "bound": "hbm", "achieved": ach,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"] if ach else None, "traffic": None,
+                         "peak_source": f"{peaks['source']} HBM copy"}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,159 @@
+/*
+ * path_attn.h — C ABI of the B200 (sm_100a) PaTH attention library
+ * (libpath_attn.so).
+ *
+ * PaTH attention ("PaTH Attention: Position Encoding via Accumulating
+ * Householder Transformations"). Per head, with 0-based positions and
+ *   H_s  = I - beta_s w_s w_s^T
+ *        (gist.science summary, section 2 "Kernmechanisme", transition
+ *         matrix; Paper-Notes page, "关键设计"),
+ * the logit of query i against key j <= i is
+ *   z_ij = scale * q_i^T H_i H_{i-1} ... H_{j+1} k_j + (c_i - c_j)
+ *        (gist.science section 2 logit equation; Paper-Notes "整体框架"),
+ * where c_t = sum_{s<=t} log f_s is the optional PaTH-FoX forget gate
+ * (Paper-Notes "PaTH-FoX 扩展" equation) and 0 without it. Keys j > i are
+ * masked. out_i = sum_j softmax_j(z_ij) v_j and lse_i = log sum_j exp(z_ij).
+ *
+ * Conventions shared by every entry point
+ * - Layout: contiguous row-major. q, k, v, w, out, dout and the gradients
+ *   are [B, H, L, d]; beta, log_f, lse, dbeta, dlog_f are [B, H, L] fp32.
+ *   Decode tensors q, k_new, v_new, w, out are [B, H, d]; decode beta is
+ *   [B, H] fp32; the caches are [B, H, capacity, d].
+ * - dtype: PATH_F32 or PATH_BF16 selects the element type of every
+ *   d-sized tensor (inputs, outputs, gradients, caches). beta, log_f, lse,
+ *   dbeta, dlog_f are always fp32. Arithmetic accumulates in fp32.
+ * - Pointers are DEVICE pointers unless stated otherwise. The caller owns
+ *   every buffer, including the workspace; the library allocates and frees
+ *   no device memory and keeps no state between calls (apart from the
+ *   host-side diagnostics at the end of this header). All work is
+ *   enqueued on `stream` (0 = legacy default stream); no call synchronises
+ *   the host.
+ * - Outputs and gradients must not alias inputs (except the decode caches,
+ *   which are updated in place by design).
+ * - Errors: arguments are validated on the host before anything is
+ *   launched; a failed check returns a status and launches nothing. A
+ *   launch failure returns PATH_ERR_CUDA (the CUDA error is left for
+ *   cudaGetLastError to report as usual). No call aborts, traps or throws.
+ * - Supported sizes: fwd/bwd d in {16, 32, 64, 128}; decode d in {64, 128};
+ *   B, H, L >= 1; B*H*L*d < 2^40 per tensor.
+ */
+#ifndef PATH_ATTN_H
+#define PATH_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *path_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    PATH_OK = 0,
+    PATH_ERR_INVALID_ARG = 1, /* null pointer, size <= 0, mismatched options */
+    PATH_ERR_UNSUPPORTED = 2, /* head dim or dtype this build does not handle */
+    PATH_ERR_WORKSPACE = 3,   /* workspace null or smaller than required */
+    PATH_ERR_CUDA = 4,        /* a kernel launch failed */
+    PATH_ERR_TIMEOUT = 5      /* reserved: a bounded device-side wait gave up */
+} path_status;
+
+typedef enum { PATH_F32 = 0, PATH_BF16 = 1 } path_dtype;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *path_status_string(path_status s);
+
+/*
+ * Workspace size in bytes that path_attn_fwd (for_bwd = 0) or path_attn_bwd
+ * (for_bwd != 0) needs for these sizes; 0 if the sizes are invalid or
+ * unsupported. The workspace is scratch: its contents on entry are ignored
+ * and on return are unspecified. Alignment: 256 bytes.
+ */
+size_t path_attn_workspace_bytes(int B, int H, int L, int d, path_dtype dt, int for_bwd);
+
+/*
+ * Forward pass.
+ * Computes out [B,H,L,d] (dtype dt) and lse [B,H,L] (fp32, natural log)
+ * from q, k, v, w [B,H,L,d] (dtype dt), beta [B,H,L] (fp32, used as given:
+ * the model layer's 2*sigmoid and any clipping happen before the call) and
+ * the optional log_f [B,H,L] (fp32; NULL = no forget gate).
+ * scale multiplies the bilinear PaTH term only; the gate is added unscaled.
+ * Blockwise algorithm: per-block UT transform T^{-1} = (I + strictLower(D W
+ * W^T))^{-1} D (Paper-Notes "训练策略", UT transform), boundary-adjusted
+ * queries/keys per block and block products (gist.science section 3
+ * "FlashAttention-Stijl Algoritme"), the full-matrix form
+ * lower(QK^T) - lower(QW^T) T^{-1} strictLower(WK^T) on each diagonal block
+ * (Paper-Notes "训练策略"), then online softmax and P.V.
+ */
+path_status path_attn_fwd(const void *q, const void *k, const void *v, const void *w,
+                          const float *beta, const float *log_f, float scale, int B, int H,
+                          int L, int d, path_dtype dt, void *out, float *lse, void *workspace,
+                          size_t workspace_bytes, path_stream_t stream);
+
+/*
+ * Backward pass of path_attn_fwd for the loss sum(out * dout).
+ * Inputs: the forward's inputs, its out and lse, and dout [B,H,L,d].
+ * Outputs: dq, dk, dv, dw [B,H,L,d] (dtype dt), dbeta [B,H,L] (fp32, w.r.t.
+ * beta as passed) and, iff log_f is non-NULL, dlog_f [B,H,L] (fp32; must be
+ * NULL iff log_f is NULL). Every output element is written (no accumulation
+ * into existing contents). The pages state no backward; it is the chain rule
+ * through the same blockwise algorithm as the forward.
+ */
+path_status path_attn_bwd(const void *q, const void *k, const void *v, const void *w,
+                          const float *beta, const float *log_f, float scale, int B, int H,
+                          int L, int d, path_dtype dt, const void *out, const float *lse,
+                          const void *dout, void *dq, void *dk, void *dv, void *dw,
+                          float *dbeta, float *dlog_f, void *workspace, size_t workspace_bytes,
+                          path_stream_t stream);
+
+/*
+ * Workspace size in bytes for path_decode_step; 0 if invalid/unsupported.
+ */
+size_t path_decode_workspace_bytes(int B, int H, int capacity, int d, path_dtype dt);
+
+/*
+ * One decode step (Paper-Notes "训练策略", inference paragraph; gist.science
+ * section 3 "Inferentie"): with n = n_cached valid rows in the caches,
+ *   1. every cached key j < n is updated in place, k_j <- k_j - beta w (w^T k_j)
+ *      (computed in fp32, stored back in dtype dt, rounded to nearest even);
+ *   2. k_new / v_new are written untransformed into row n of k_cache / v_cache;
+ *   3. out = softmax_j(scale * q^T k_j) V over the n+1 rows (the updated keys
+ *      as stored), written to out [B,H,d].
+ * After the call the caches hold n+1 rows; the caller advances n.
+ * Requires 0 <= n_cached and n_cached + 1 <= capacity (else
+ * PATH_ERR_INVALID_ARG). q, k_new, v_new, w: [B,H,d]; beta: [B,H] fp32.
+ */
+path_status path_decode_step(const void *q, const void *k_new, const void *v_new, const void *w,
+                             const float *beta, float scale, int B, int H, int d, int n_cached,
+                             int capacity, path_dtype dt, void *k_cache, void *v_cache, void *out,
+                             void *workspace, size_t workspace_bytes, path_stream_t stream);
+
+/*
+ * Diagnostics (host-side, process-wide; not needed for normal use).
+ *
+ * path_kernel_launch_count: number of CUDA kernels this library has launched
+ * in this process so far.
+ *
+ * path_profile_enable(on): while on, every internal stage of an entry point
+ * (UT prep, transport chain, attention main loop, ...) is bracketed by two CUDA
+ * events recorded on the call's stream. Returns the previous setting. Event
+ * creation is the only resource it uses; no device memory.
+ *
+ * path_profile_read(out, max_entries): waits for the recorded events,
+ * accumulates their elapsed times per stage name into out[0..n) and returns
+ * n (<= max_entries); the recorded events are released.
+ */
+typedef struct {
+    char name[32];
+    double total_ms;
+    int count;
+} path_stage_time;
+
+unsigned long long path_kernel_launch_count(void);
+int path_profile_enable(int on);
+int path_profile_read(path_stage_time *out, int max_entries);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PATH_ATTN_H */

@@ -1,0 +1,165 @@
+"""PaTH attention on B200 (sm_100a): thin Python binding of libpath_attn.so.
+
+The binding only marshals arguments: it checks dtypes, shapes and
+contiguity, allocates outputs and workspace with torch when the caller does
+not pass them, and calls the C ABI declared in ``include/path_attn.h`` on the
+current torch CUDA stream. Every step of the computation runs in the
+library's CUDA kernels; there is no CPU path. If the library is missing or no
+CUDA device is present, the calls raise.
+
+Entry points (same names as the C ABI):
+- ``path_attn_fwd(q, k, v, w, beta, log_f=None, scale=None) -> (out, lse)``
+- ``path_attn_bwd(q, k, v, w, beta, out, lse, dout, log_f=None, scale=None) -> dict``
+- ``path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=None) -> out``
+- ``path_attn_workspace_bytes``, ``path_decode_workspace_bytes``, ``path_status_string``
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpath_attn.so")
+
+PATH_F32, PATH_BF16 = 0, 1
+_DT = {torch.float32: PATH_F32, torch.bfloat16: PATH_BF16}
+_lib = None
+
+
+class PathError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {path_status_string(status)} (status {status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m softmax_attention_block_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp, i, f, sz = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
+                            ctypes.c_size_t)
+        L.path_status_string.argtypes = [i]
+        L.path_status_string.restype = ctypes.c_char_p
+        L.path_attn_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        L.path_attn_workspace_bytes.restype = sz
+        L.path_decode_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.path_decode_workspace_bytes.restype = sz
+        L.path_attn_fwd.argtypes = [vp, vp, vp, vp, fp, fp, f, i, i, i, i, i, vp, fp, vp, sz, vp]
+        L.path_attn_bwd.argtypes = [vp, vp, vp, vp, fp, fp, f, i, i, i, i, i, vp, fp, vp,
+                                    vp, vp, vp, vp, fp, fp, vp, sz, vp]
+        L.path_decode_step.argtypes = [vp, vp, vp, vp, fp, f, i, i, i, i, i, i, vp, vp, vp, vp,
+                                       sz, vp]
+        for fn in (L.path_attn_fwd, L.path_attn_bwd, L.path_decode_step):
+            fn.restype = i
+        _lib = L
+    return _lib
+
+
+def path_status_string(status: int) -> str:
+    return lib().path_status_string(int(status)).decode()
+
+
+def path_attn_workspace_bytes(B, H, L, d, dtype, for_bwd=False) -> int:
+    return int(lib().path_attn_workspace_bytes(B, H, L, d, _DT[dtype], int(bool(for_bwd))))
+
+
+def path_decode_workspace_bytes(B, H, capacity, d, dtype) -> int:
+    return int(lib().path_decode_workspace_bytes(B, H, capacity, d, _DT[dtype]))
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check_dev(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _workspace(nbytes, device, ws):
+    if ws is None:
+        return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+    if ws.numel() * ws.element_size() < nbytes:
+        raise ValueError("workspace too small")
+    return ws
+
+
+def _scale(scale, d):
+    return float(d ** -0.5 if scale is None else scale)
+
+
+def path_attn_fwd(q, k, v, w, beta, log_f=None, scale=None, out=None, lse=None, workspace=None):
+    """Forward pass. q, k, v, w: [B,H,L,d] (fp32 or bf16); beta, log_f: [B,H,L] fp32.
+    Returns (out [B,H,L,d], lse [B,H,L] fp32)."""
+    B, H, L, d = q.shape
+    dt = _DT[q.dtype]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    _check_dev(q, k, v, w, beta, log_f, out, lse)
+    nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, False)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().path_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(beta), _ptr(log_f),
+                             _scale(scale, d), B, H, L, d, dt, _ptr(out), _ptr(lse), _ptr(ws),
+                             nbytes, _stream())
+    if st:
+        raise PathError(st, "path_attn_fwd")
+    return out, lse
+
+
+def path_attn_bwd(q, k, v, w, beta, out, lse, dout, log_f=None, scale=None, grads=None,
+                  workspace=None):
+    """Backward of sum(out * dout). Returns dict dq, dk, dv, dw, dbeta[, dlog_f]."""
+    B, H, L, d = q.shape
+    dt = _DT[q.dtype]
+    if grads is None:
+        grads = {n: torch.empty_like(q) for n in ("dq", "dk", "dv", "dw")}
+        grads["dbeta"] = torch.empty_like(beta)
+        if log_f is not None:
+            grads["dlog_f"] = torch.empty_like(log_f)
+    dlf = grads.get("dlog_f") if log_f is not None else None
+    _check_dev(q, k, v, w, beta, log_f, out, lse, dout, *grads.values())
+    nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, True)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().path_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(beta), _ptr(log_f),
+                             _scale(scale, d), B, H, L, d, dt, _ptr(out), _ptr(lse), _ptr(dout),
+                             _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
+                             _ptr(grads["dw"]), _ptr(grads["dbeta"]), _ptr(dlf), _ptr(ws), nbytes,
+                             _stream())
+    if st:
+        raise PathError(st, "path_attn_bwd")
+    return grads
+
+
+def path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=None, out=None,
+                     workspace=None):
+    """One decode step; updates k_cache / v_cache ([B,H,cap,d]) in place. Returns out [B,H,d]."""
+    B, H, cap, d = k_cache.shape
+    dt = _DT[k_cache.dtype]
+    if out is None:
+        out = torch.empty_like(q)
+    _check_dev(q, k_new, v_new, w, beta, k_cache, v_cache, out)
+    nbytes = path_decode_workspace_bytes(B, H, cap, d, k_cache.dtype)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().path_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(w), _ptr(beta),
+                                _scale(scale, d), B, H, d, int(n_cached), cap, dt, _ptr(k_cache),
+                                _ptr(v_cache), _ptr(out), _ptr(ws), nbytes, _stream())
+    if st:
+        raise PathError(st, "path_decode_step")
+    return out

@@ -1,0 +1,65 @@
+// Attention main-loop kernels (transport chain, forward, backward) and the
+// forget-gate scans.
+#pragma once
+#include <type_traits>
+
+#include "common.cuh"
+
+namespace path {
+
+struct ChainArgs {
+    const void *Kt;  // [nh, Lp, d] boundary-adjusted keys
+    const void *Pm;  // [nh, nblk, d, d] block products
+    void *Khat;      // [nh, npairs, BT, d]; pair (I, J), J < I, at I(I-1)/2 + J
+    int nblk, nh;
+};
+
+struct FwdArgs {
+    const void *Qt, *Khat, *v;
+    const float *Sd;  // [nh, nblk, BT, BT]
+    const float *c;   // [nh, Lp] gate prefix or null
+    float scale;
+    int L, nblk, nh;
+    void *out;
+    float *lse;
+};
+
+struct BwdArgs {
+    const void *Qt, *Khat, *v, *Pm;
+    const float *Sd, *c;
+    float scale;
+    int L, nblk, nh;
+    const void *out, *dout;
+    const float *lse;
+    float *delta;    // [nh, Lp]
+    float *dQt;      // [nh, Lp, d]
+    float *dKt;      // [nh, Lp, d]
+    float *dPm;      // [nh, nblk, d, d], zeroed by the caller (accumulated)
+    float *dSd;      // [nh, nblk, BT, BT]
+    void *dv;        // [nh, L, d]
+    float *rowsum;   // [nh, Lp] or null
+    float *colsum;   // [nh, Lp] or null
+};
+
+cudaError_t chain_simt(const ChainArgs &c, int dt, int d, cudaStream_t st);
+cudaError_t attn_fwd_simt(const FwdArgs &a, int dt, int d, cudaStream_t st);
+cudaError_t attn_bwd_simt(const BwdArgs &a, int dt, int d, cudaStream_t st);
+cudaError_t gate_prefix(const float *logf, float *c, int L, int Lp, int nh, cudaStream_t st);
+cudaError_t gate_grad(const float *rowsum, const float *colsum, float *dlogf, int L, int Lp, int nh,
+                      cudaStream_t st);
+
+struct DecodeArgs {
+    const void *q, *k_new, *v_new, *w;  // [nh, d]
+    const float *beta;                  // [nh]
+    float scale;
+    int nh, n, capacity;
+    void *k_cache, *v_cache;            // [nh, capacity, d]
+    void *out;                          // [nh, d]
+    float *partial;                     // [nh, nchunk, d + 2]
+};
+
+constexpr int DECODE_CHUNK = 256;  // cached rows per CTA
+
+cudaError_t decode_step(const DecodeArgs &a, int dt, int d, cudaStream_t st);
+
+}  // namespace path

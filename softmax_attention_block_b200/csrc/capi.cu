@@ -1,0 +1,223 @@
+// C ABI of the PaTH attention library: argument validation, workspace
+// layout, and the launch sequence of each entry point.
+#include <math.h>
+
+#include "attn.cuh"
+#include "prep.cuh"
+#include "runtime.cuh"
+
+using namespace path;
+
+namespace {
+
+struct Layout {
+    int nh, L, d, nblk, Lp;
+    long long npairs;
+    size_t tsz;
+};
+
+Layout make_layout(int B, int H, int L, int d, path_dtype dt)
+{
+    Layout y;
+    y.nh = B * H;
+    y.L = L;
+    y.d = d;
+    y.nblk = ceil_div(L, BT);
+    y.Lp = y.nblk * BT;
+    y.npairs = (long long)y.nblk * (y.nblk - 1) / 2;
+    y.tsz = dt == PATH_F32 ? 4 : 2;
+    return y;
+}
+
+struct AttnWs {
+    float *c;
+    void *Qt, *Kt, *Pm, *Khat;
+    float *Sd;
+    PrepScratch prep;
+    // backward only
+    float *delta, *dQt, *dKt, *dPm, *dSd, *rowsum, *colsum;
+};
+
+// The single description of the workspace: used both to size and to carve it.
+size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &w)
+{
+    Carver c(base);
+    const size_t nh = y.nh, Lp = y.Lp, d = y.d, nb = y.nblk;
+    w.c = c.take<float>(nh * Lp);
+    w.Qt = c.take<char>(nh * Lp * d * y.tsz);
+    w.Kt = c.take<char>(nh * Lp * d * y.tsz);
+    w.Pm = c.take<char>(nh * nb * d * d * y.tsz);
+    w.Khat = c.take<char>(nh * (size_t)y.npairs * BT * d * y.tsz);
+    w.Sd = c.take<float>(nh * nb * BT * BT);
+    PrepDims D{y.nh, y.L, y.d, y.nblk, (int)dt};
+    carve_prep_scratch(c, D, bwd, w.prep);
+    if (bwd) {
+        w.delta = c.take<float>(nh * Lp);
+        w.dQt = c.take<float>(nh * Lp * d);
+        w.dKt = c.take<float>(nh * Lp * d);
+        w.dPm = c.take<float>(nh * nb * d * d);
+        w.dSd = c.take<float>(nh * nb * BT * BT);
+        w.rowsum = c.take<float>(nh * Lp);
+        w.colsum = c.take<float>(nh * Lp);
+    }
+    return c.bytes();
+}
+
+bool fwd_dims_ok(int B, int H, int L, int d)
+{
+    if (B <= 0 || H <= 0 || L <= 0) return false;
+    const long long elems = (long long)B * H * L * d;
+    return elems > 0 && elems < (1LL << 40);
+}
+
+bool head_dim_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+bool dtype_ok(path_dtype dt) { return dt == PATH_F32 || dt == PATH_BF16; }
+
+path_status launch_status(cudaError_t e) { return e == cudaSuccess ? PATH_OK : PATH_ERR_CUDA; }
+
+#define TRY(x)                                          \
+    do {                                                \
+        cudaError_t e_ = (x);                           \
+        if (e_ != cudaSuccess) return PATH_ERR_CUDA;    \
+    } while (0)
+
+// Shared by forward and backward: gate prefix, UT prep, transport chain.
+path_status run_prep_and_chain(const void *q, const void *k, const void *w, const float *beta,
+                               const float *log_f, const Layout &y, path_dtype dt, AttnWs &ws,
+                               cudaStream_t st)
+{
+    if (log_f) {
+        Stage s("gate_prefix", st);
+        TRY(gate_prefix(log_f, ws.c, y.L, y.Lp, y.nh, st));
+    }
+    PrepDims D{y.nh, y.L, y.d, y.nblk, (int)dt};
+    PrepInputs in{q, k, w, beta};
+    PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, (int)dt};
+    {
+        Stage s("ut_prep", st);
+        TRY(prep_forward(D, in, ws.prep, out, st));
+    }
+    ChainArgs ca{ws.Kt, ws.Pm, ws.Khat, y.nblk, y.nh};
+    {
+        Stage s("chain", st);
+        TRY(chain_simt(ca, (int)dt, y.d, st));
+    }
+    return PATH_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *path_status_string(path_status s)
+{
+    switch (s) {
+    case PATH_OK: return "ok";
+    case PATH_ERR_INVALID_ARG: return "invalid argument";
+    case PATH_ERR_UNSUPPORTED: return "unsupported size or dtype";
+    case PATH_ERR_WORKSPACE: return "workspace missing or too small";
+    case PATH_ERR_CUDA: return "CUDA launch failed";
+    case PATH_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+size_t path_attn_workspace_bytes(int B, int H, int L, int d, path_dtype dt, int for_bwd)
+{
+    if (!fwd_dims_ok(B, H, L, d) || !head_dim_supported(d) || !dtype_ok(dt)) return 0;
+    AttnWs w;
+    return carve_attn(nullptr, make_layout(B, H, L, d, dt), dt, for_bwd != 0, w);
+}
+
+path_status path_attn_fwd(const void *q, const void *k, const void *v, const void *w,
+                          const float *beta, const float *log_f, float scale, int B, int H, int L,
+                          int d, path_dtype dt, void *out, float *lse, void *workspace,
+                          size_t workspace_bytes, path_stream_t stream)
+{
+    if (!q || !k || !v || !w || !beta || !out || !lse) return PATH_ERR_INVALID_ARG;
+    if (!fwd_dims_ok(B, H, L, d) || !isfinite(scale)) return PATH_ERR_INVALID_ARG;
+    if (!head_dim_supported(d) || !dtype_ok(dt)) return PATH_ERR_UNSUPPORTED;
+    const Layout y = make_layout(B, H, L, d, dt);
+    AttnWs ws;
+    const size_t need = carve_attn(nullptr, y, dt, false, ws);
+    if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
+    carve_attn(workspace, y, dt, false, ws);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
+    if (s != PATH_OK) return s;
+    FwdArgs a{ws.Qt, ws.Khat, v, ws.Sd, log_f ? ws.c : nullptr, scale, y.L, y.nblk, y.nh, out, lse};
+    Stage s_attn("attn_fwd", st);
+    return launch_status(attn_fwd_simt(a, (int)dt, d, st));
+}
+
+path_status path_attn_bwd(const void *q, const void *k, const void *v, const void *w,
+                          const float *beta, const float *log_f, float scale, int B, int H, int L,
+                          int d, path_dtype dt, const void *out, const float *lse, const void *dout,
+                          void *dq, void *dk, void *dv, void *dw, float *dbeta, float *dlog_f,
+                          void *workspace, size_t workspace_bytes, path_stream_t stream)
+{
+    if (!q || !k || !v || !w || !beta || !out || !lse || !dout || !dq || !dk || !dv || !dw ||
+        !dbeta)
+        return PATH_ERR_INVALID_ARG;
+    if ((log_f == nullptr) != (dlog_f == nullptr)) return PATH_ERR_INVALID_ARG;
+    if (!fwd_dims_ok(B, H, L, d) || !isfinite(scale)) return PATH_ERR_INVALID_ARG;
+    if (!head_dim_supported(d) || !dtype_ok(dt)) return PATH_ERR_UNSUPPORTED;
+    const Layout y = make_layout(B, H, L, d, dt);
+    AttnWs ws;
+    const size_t need = carve_attn(nullptr, y, dt, true, ws);
+    if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
+    carve_attn(workspace, y, dt, true, ws);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
+    if (s != PATH_OK) return s;
+    TRY(cudaMemsetAsync(ws.dPm, 0, sizeof(float) * (size_t)y.nh * y.nblk * d * d, st));
+    BwdArgs a{ws.Qt,     ws.Khat,  v,        ws.Pm,  ws.Sd,  log_f ? ws.c : nullptr,
+              scale,     y.L,      y.nblk,   y.nh,   out,    dout,
+              lse,       ws.delta, ws.dQt,   ws.dKt, ws.dPm, ws.dSd,
+              dv,        ws.rowsum, ws.colsum};
+    TRY(attn_bwd_simt(a, (int)dt, d, st));
+    PrepDims D{y.nh, y.L, y.d, y.nblk, (int)dt};
+    PrepInputs in{q, k, w, beta};
+    PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta};
+    {
+        Stage s("ut_prep_bwd", st);
+        TRY(prep_backward(D, in, ws.prep, gr, st));
+    }
+    if (log_f) {
+        Stage s("gate_grad", st);
+        TRY(gate_grad(ws.rowsum, ws.colsum, dlog_f, y.L, y.Lp, y.nh, st));
+    }
+    return PATH_OK;
+}
+
+size_t path_decode_workspace_bytes(int B, int H, int capacity, int d, path_dtype dt)
+{
+    if (B <= 0 || H <= 0 || capacity <= 0 || (d != 64 && d != 128) || !dtype_ok(dt)) return 0;
+    const size_t nchunk = (size_t)ceil_div(capacity, DECODE_CHUNK);
+    return align_up((size_t)B * H * nchunk * (d + 2) * sizeof(float), 256);
+}
+
+path_status path_decode_step(const void *q, const void *k_new, const void *v_new, const void *w,
+                             const float *beta, float scale, int B, int H, int d, int n_cached,
+                             int capacity, path_dtype dt, void *k_cache, void *v_cache, void *out,
+                             void *workspace, size_t workspace_bytes, path_stream_t stream)
+{
+    if (!q || !k_new || !v_new || !w || !beta || !k_cache || !v_cache || !out)
+        return PATH_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || capacity <= 0 || n_cached < 0 || n_cached + 1 > capacity ||
+        !isfinite(scale))
+        return PATH_ERR_INVALID_ARG;
+    if ((d != 64 && d != 128) || !dtype_ok(dt)) return PATH_ERR_UNSUPPORTED;
+    // 16-byte vector access of q, w and the caches
+    const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(w) |
+                         reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache);
+    if (al & 15u) return PATH_ERR_INVALID_ARG;
+    const size_t need = path_decode_workspace_bytes(B, H, capacity, d, dt);
+    if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
+    DecodeArgs a{q, k_new, v_new, w, beta, scale, B * H, n_cached, capacity,
+                 k_cache, v_cache, out, static_cast<float *>(workspace)};
+    return launch_status(decode_step(a, (int)dt, d, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

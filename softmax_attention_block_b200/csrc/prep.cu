@@ -1,0 +1,471 @@
+// Per-block UT transform and boundary adjustment (forward), and its adjoint.
+//
+// Within one block of BT positions (rows of W, Q, K; beta; D = diag(beta)):
+//   A    = strictLower(D W W^T)          Tinv = (I + A)^{-1}      X = Tinv D
+//        (X is the T^{-1} of the UT transform, Paper-Notes "训练策略")
+//   What = X W                          P    = I - W^T What  (= H_e ... H_s)
+//   N    = strictLower(W K^T)           U    = X N
+//   Ktil = K - U^T W                    (row j: H_e ... H_{j+1} k_j)
+//   M    = lower(Q W^T)                 Qtil = Q - M What   (row i: H_s ... H_i q_i)
+//   Sd   = Q K^T - M U   on and below the diagonal: the full-matrix form
+//          lower(QK^T) - lower(QW^T) T^{-1} strictLower(WK^T) (Paper-Notes "训练策略")
+// Qtil / Ktil are the boundary-adjusted queries and keys of each block and P
+// the block product (gist.science section 3, "FlashAttention-Stijl Algoritme").
+#include "prep.cuh"
+#include "runtime.cuh"
+
+namespace path {
+
+namespace {
+
+// Tinv = (I + A)^{-1} for strictly lower A (forward substitution, one block
+// per CTA), and X = Tinv diag(beta).
+__global__ void __launch_bounds__(256) tri_inverse_kernel(const float *A, float *Tinv, float *X,
+                                                          const float *beta, int L, int nblk,
+                                                          int batch)
+{
+    extern __shared__ float sm[];
+    float *sA = sm;              // [BT][BT]
+    float *sT = sm + BT * BT;    // [BT][BT]
+    __shared__ float part[2][BT];
+    for (int z = blockIdx.x; z < batch; z += gridDim.x) {
+        const int h = z / nblk, blk = z % nblk;
+        const long long base = (long long)z * BT * BT;
+        for (int e = threadIdx.x; e < BT * BT; e += blockDim.x) {
+            sA[e] = A[base + e];
+            sT[e] = 0.f;
+        }
+        __syncthreads();
+        const int c = threadIdx.x % BT, half = threadIdx.x / BT;
+        if (half == 0) sT[c * BT + c] = 1.f;
+        __syncthreads();
+        for (int i = 1; i < BT; ++i) {
+            // row i, column c < i: -sum_{k=c}^{i-1} A[i][k] Tinv[k][c]; k split in two halves
+            float s = 0.f;
+            if (c < i) {
+                const int mid = (c + i) / 2;
+                const int k0 = half == 0 ? c : mid, k1 = half == 0 ? mid : i;
+                for (int k = k0; k < k1; ++k) s = fmaf(sA[i * BT + k], sT[k * BT + c], s);
+            }
+            part[half][c] = s;
+            __syncthreads();
+            if (half == 0 && c < i) sT[i * BT + c] = -(part[0][c] + part[1][c]);
+            __syncthreads();
+        }
+        for (int e = threadIdx.x; e < BT * BT; e += blockDim.x) {
+            const int col = e % BT;
+            const int pos = blk * BT + col;
+            const float b = pos < L ? beta[(long long)h * L + pos] : 0.f;
+            Tinv[base + e] = sT[e];
+            X[base + e] = sT[e] * b;
+        }
+        __syncthreads();
+    }
+}
+
+// dbeta[a] = sum_{b<a} dA[a][b] G[a][b] + sum_{a'} dX[a'][a] Tinv[a'][a]
+__global__ void dbeta_kernel(const float *dA, const float *G, const float *dX, const float *Tinv,
+                             float *dbeta, int L, int nblk, int batch)
+{
+    for (int z = blockIdx.x; z < batch; z += gridDim.x) {
+        const int h = z / nblk, blk = z % nblk;
+        const long long base = (long long)z * BT * BT;
+        const int a = threadIdx.x;
+        const int pos = blk * BT + a;
+        float s = 0.f;
+        for (int b = 0; b < a; ++b) s = fmaf(dA[base + a * BT + b], G[base + a * BT + b], s);
+        for (int r = 0; r < BT; ++r) s = fmaf(dX[base + r * BT + a], Tinv[base + r * BT + a], s);
+        if (pos < L) dbeta[(long long)h * L + pos] = s;
+    }
+}
+
+// out[a][b] = beta[a] * in[a][b] per block (beta = 0 past the sequence end)
+__global__ void scale_rows_kernel(const float *in, float *out, const float *beta, int L, int nblk,
+                                  int batch)
+{
+    for (int z = blockIdx.x; z < batch; z += gridDim.x) {
+        const int h = z / nblk, blk = z % nblk;
+        const long long base = (long long)z * BT * BT;
+        for (int e = threadIdx.x; e < BT * BT; e += blockDim.x) {
+            const int pos = blk * BT + e / BT;
+            const float b = pos < L ? beta[(long long)h * L + pos] : 0.f;
+            out[base + e] = b * in[base + e];
+        }
+    }
+}
+
+int grid_for(int batch) { return batch < 4096 ? batch : 4096; }
+
+}  // namespace
+
+cudaError_t scale_rows(const float *in, float *out, const float *beta, int L, int nblk, int batch,
+                       cudaStream_t st)
+{
+    scale_rows_kernel<<<grid_for(batch), 256, 0, st>>>(in, out, beta, L, nblk, batch);
+    count_launches();
+    return cudaGetLastError();
+}
+
+// --- operand builders -------------------------------------------------------
+static Operand user_rows(const void *p, int dt, int L, int d)  // [nh, L, d] user tensor
+{
+    Operand o;
+    o.p = p;
+    o.dt = dt;
+    o.sh = (long long)L * d;
+    o.sb = (long long)BT * d;
+    o.ld = d;
+    o.seq = L;
+    return o;
+}
+
+static Operand padded_rows(const void *p, int dt, int Lp, int d)  // [nh, Lp, d] workspace
+{
+    Operand o;
+    o.p = p;
+    o.dt = dt;
+    o.sh = (long long)Lp * d;
+    o.sb = (long long)BT * d;
+    o.ld = d;
+    return o;
+}
+
+static Operand blk_mat(const void *p, int dt, int nblk, int rows, int cols)  // [nh, nblk, rows, cols]
+{
+    Operand o;
+    o.p = p;
+    o.dt = dt;
+    o.sh = (long long)nblk * rows * cols;
+    o.sb = (long long)rows * cols;
+    o.ld = cols;
+    return o;
+}
+
+static Operand T_(Operand o)
+{
+    o.trans = 1;
+    return o;
+}
+
+static Operand masked(Operand o, int m)
+{
+    o.mask = m;
+    return o;
+}
+
+static void set_out(GemmArgs &g, void *p, int dt, long long sh, long long sb, int ldc, int c_seq)
+{
+    g.c = p;
+    g.cdt = dt;
+    g.csh = sh;
+    g.csb = sb;
+    g.ldc = ldc;
+    g.c_seq = c_seq;
+}
+
+static GemmArgs base_args(const PrepDims &D, int M, int N, int K)
+{
+    GemmArgs g;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.nblk = D.nblk;
+    g.batch = D.nh * D.nblk;
+    return g;
+}
+
+static void term(GemmArgs &g, Operand a, Operand b, float alpha)
+{
+    g.t[g.nterms].a = a;
+    g.t[g.nterms].b = b;
+    g.t[g.nterms].alpha = alpha;
+    ++g.nterms;
+}
+
+static void out_blk(GemmArgs &g, const PrepDims &D, float *p, int rows, int cols, int outmask = 0)
+{
+    set_out(g, p, F32, (long long)D.nblk * rows * cols, (long long)rows * cols, cols, -1);
+    g.outmask = outmask;
+}
+
+#define CK(x)                                 \
+    do {                                      \
+        cudaError_t e_ = (x);                 \
+        if (e_ != cudaSuccess) return e_;     \
+    } while (0)
+
+size_t prep_scratch_bytes(const PrepDims &D, bool backward)
+{
+    Carver c(nullptr);
+    PrepScratch s;
+    carve_prep_scratch(c, D, backward, s);
+    return c.bytes();
+}
+
+void carve_prep_scratch(Carver &c, const PrepDims &D, bool backward, PrepScratch &s)
+{
+    const size_t nb = (size_t)D.nh * D.nblk;
+    const size_t sq = nb * BT * BT, rd = nb * BT * D.d;
+    s.G = c.take<float>(sq);
+    s.A = c.take<float>(sq);
+    s.Tinv = c.take<float>(sq);
+    s.X = c.take<float>(sq);
+    s.N = c.take<float>(sq);
+    s.U = c.take<float>(sq);
+    s.M = c.take<float>(sq);
+    s.What = c.take<float>(rd);
+    if (backward) {
+        s.dM = c.take<float>(sq);
+        s.dU = c.take<float>(sq);
+        s.dN = c.take<float>(sq);
+        s.dX = c.take<float>(sq);
+        s.tmp = c.take<float>(sq);
+        s.dA = c.take<float>(sq);
+        s.dG = c.take<float>(sq);
+        s.dWhat = c.take<float>(rd);
+        s.dWacc = c.take<float>(rd);
+    }
+}
+
+// Shared first half of forward and backward: A, G, Tinv, X, What, N, U, M.
+static cudaError_t prep_core(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
+                             cudaStream_t st)
+{
+    const int L = D.L, d = D.d, nb = D.nblk;
+    const Operand W = user_rows(in.w, D.dt, L, d), K = user_rows(in.k, D.dt, L, d),
+                  Q = user_rows(in.q, D.dt, L, d);
+    {   // G = W W^T ; A = strictLower(D G)
+        GemmArgs g = base_args(D, BT, BT, d);
+        term(g, W, T_(W), 1.f);
+        out_blk(g, D, s.G, BT, BT);
+        CK(gemm_batched(g, st));
+        g.rowscale = in.beta;
+        g.rs_sh = L;
+        g.rs_sb = BT;
+        g.rs_seq = L;
+        out_blk(g, D, s.A, BT, BT, MASK_STRICT_LOWER);
+        CK(gemm_batched(g, st));
+    }
+    {
+        const int batch = D.nh * nb;
+        const size_t smem = 2 * BT * BT * sizeof(float);
+        CK(cudaFuncSetAttribute(tri_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem));
+        tri_inverse_kernel<<<grid_for(batch), 256, smem, st>>>(s.A, s.Tinv, s.X, in.beta, L, nb,
+                                                               batch);
+        count_launches();
+        CK(cudaGetLastError());
+    }
+    const Operand X = blk_mat(s.X, F32, nb, BT, BT);
+    {   // What = X W
+        GemmArgs g = base_args(D, BT, d, BT);
+        term(g, X, W, 1.f);
+        out_blk(g, D, s.What, BT, d);
+        CK(gemm_batched(g, st));
+    }
+    {   // N = strictLower(W K^T)
+        GemmArgs g = base_args(D, BT, BT, d);
+        term(g, W, T_(K), 1.f);
+        out_blk(g, D, s.N, BT, BT, MASK_STRICT_LOWER);
+        CK(gemm_batched(g, st));
+    }
+    {   // U = X N
+        GemmArgs g = base_args(D, BT, BT, BT);
+        term(g, X, blk_mat(s.N, F32, nb, BT, BT), 1.f);
+        out_blk(g, D, s.U, BT, BT);
+        CK(gemm_batched(g, st));
+    }
+    {   // M = lower(Q W^T)
+        GemmArgs g = base_args(D, BT, BT, d);
+        term(g, Q, T_(W), 1.f);
+        out_blk(g, D, s.M, BT, BT, MASK_LOWER);
+        CK(gemm_batched(g, st));
+    }
+    return cudaSuccess;
+}
+
+cudaError_t prep_forward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
+                         const PrepOutputs &out, cudaStream_t st)
+{
+    CK(prep_core(D, in, s, st));
+    const int L = D.L, d = D.d, nb = D.nblk, Lp = nb * BT;
+    const Operand W = user_rows(in.w, D.dt, L, d), K = user_rows(in.k, D.dt, L, d),
+                  Q = user_rows(in.q, D.dt, L, d);
+    const Operand U = blk_mat(s.U, F32, nb, BT, BT), M = blk_mat(s.M, F32, nb, BT, BT),
+                  What = blk_mat(s.What, F32, nb, BT, d);
+    {   // Ktil = K - U^T W
+        GemmArgs g = base_args(D, BT, d, BT);
+        term(g, T_(U), W, -1.f);
+        g.addend = K;
+        g.gamma = 1.f;
+        set_out(g, out.Kt, out.tdt, (long long)Lp * d, (long long)BT * d, d, -1);
+        CK(gemm_batched(g, st));
+    }
+    {   // Qtil = Q - M What
+        GemmArgs g = base_args(D, BT, d, BT);
+        term(g, M, What, -1.f);
+        g.addend = Q;
+        g.gamma = 1.f;
+        set_out(g, out.Qt, out.tdt, (long long)Lp * d, (long long)BT * d, d, -1);
+        CK(gemm_batched(g, st));
+    }
+    {   // P = I - W^T What
+        GemmArgs g = base_args(D, d, d, BT);
+        term(g, T_(W), What, -1.f);
+        g.add_identity = 1;
+        set_out(g, out.Pm, out.tdt, (long long)nb * d * d, (long long)d * d, d, -1);
+        CK(gemm_batched(g, st));
+    }
+    {   // Sd = Q K^T - M U (read only on and below the diagonal)
+        GemmArgs g = base_args(D, BT, BT, d);
+        term(g, Q, T_(K), 1.f);
+        set_out(g, out.Sd, F32, (long long)nb * BT * BT, (long long)BT * BT, BT, -1);
+        CK(gemm_batched(g, st));  // the second product has inner size BT: its own pass
+        GemmArgs g2 = base_args(D, BT, BT, BT);
+        term(g2, M, U, -1.f);
+        g2.addend = blk_mat(out.Sd, F32, nb, BT, BT);
+        g2.gamma = 1.f;
+        set_out(g2, out.Sd, F32, (long long)nb * BT * BT, (long long)BT * BT, BT, -1);
+        g2.outmask = MASK_LOWER;
+        CK(gemm_batched(g2, st));
+    }
+    return cudaSuccess;
+}
+
+cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
+                          const PrepGrads &gr, cudaStream_t st)
+{
+    CK(prep_core(D, in, s, st));
+    const int L = D.L, d = D.d, nb = D.nblk, Lp = nb * BT;
+    const Operand W = user_rows(in.w, D.dt, L, d), K = user_rows(in.k, D.dt, L, d),
+                  Q = user_rows(in.q, D.dt, L, d);
+    const Operand U = blk_mat(s.U, F32, nb, BT, BT), M = blk_mat(s.M, F32, nb, BT, BT),
+                  What = blk_mat(s.What, F32, nb, BT, d), X = blk_mat(s.X, F32, nb, BT, BT),
+                  Nm = blk_mat(s.N, F32, nb, BT, BT), Tinv = blk_mat(s.Tinv, F32, nb, BT, BT),
+                  G = blk_mat(s.G, F32, nb, BT, BT);
+    const Operand dSl = masked(blk_mat(gr.dSd, F32, nb, BT, BT), MASK_LOWER);
+    const Operand dQt = padded_rows(gr.dQt, F32, Lp, d), dKt = padded_rows(gr.dKt, F32, Lp, d);
+    const Operand dP = blk_mat(gr.dPm, F32, nb, d, d);
+    const Operand dM = blk_mat(s.dM, F32, nb, BT, BT), dU = blk_mat(s.dU, F32, nb, BT, BT),
+                  dN = blk_mat(s.dN, F32, nb, BT, BT), dX = blk_mat(s.dX, F32, nb, BT, BT),
+                  tmp = blk_mat(s.tmp, F32, nb, BT, BT), dA = blk_mat(s.dA, F32, nb, BT, BT),
+                  dGm = blk_mat(s.dG, F32, nb, BT, BT), dWhat = blk_mat(s.dWhat, F32, nb, BT, d),
+                  dWacc = blk_mat(s.dWacc, F32, nb, BT, d);
+    const long long ush = (long long)L * d, usb = (long long)BT * d;
+    {   // dM = lower(-dSl U^T - dQt What^T)
+        GemmArgs g = base_args(D, BT, BT, BT);
+        term(g, dSl, T_(U), -1.f);
+        out_blk(g, D, s.dM, BT, BT, MASK_LOWER);
+        CK(gemm_batched(g, st));
+        GemmArgs g2 = base_args(D, BT, BT, d);
+        term(g2, dQt, T_(What), -1.f);
+        g2.addend = dM;
+        g2.gamma = 1.f;
+        out_blk(g2, D, s.dM, BT, BT, MASK_LOWER);
+        CK(gemm_batched(g2, st));
+    }
+    {   // dq = dQt + dSl K + dM W
+        GemmArgs g = base_args(D, BT, d, BT);
+        term(g, dSl, K, 1.f);
+        term(g, dM, W, 1.f);
+        g.addend = dQt;
+        g.gamma = 1.f;
+        set_out(g, gr.dq, D.dt, ush, usb, d, L);
+        CK(gemm_batched(g, st));
+    }
+    {   // dU = -M^T dSl - W dKt^T
+        GemmArgs g = base_args(D, BT, BT, BT);
+        term(g, T_(M), dSl, -1.f);
+        out_blk(g, D, s.dU, BT, BT);
+        CK(gemm_batched(g, st));
+        GemmArgs g2 = base_args(D, BT, BT, d);
+        term(g2, W, T_(dKt), -1.f);
+        g2.addend = dU;
+        g2.gamma = 1.f;
+        out_blk(g2, D, s.dU, BT, BT);
+        CK(gemm_batched(g2, st));
+    }
+    {   // dN = strictLower(X^T dU)
+        GemmArgs g = base_args(D, BT, BT, BT);
+        term(g, T_(X), dU, 1.f);
+        out_blk(g, D, s.dN, BT, BT, MASK_STRICT_LOWER);
+        CK(gemm_batched(g, st));
+    }
+    {   // dk = dKt + dSl^T Q + dN^T W
+        GemmArgs g = base_args(D, BT, d, BT);
+        term(g, T_(dSl), Q, 1.f);
+        term(g, T_(dN), W, 1.f);
+        g.addend = dKt;
+        g.gamma = 1.f;
+        set_out(g, gr.dk, D.dt, ush, usb, d, L);
+        CK(gemm_batched(g, st));
+    }
+    {   // dWhat = -M^T dQt - W dP
+        GemmArgs g = base_args(D, BT, d, BT);
+        term(g, T_(M), dQt, -1.f);
+        out_blk(g, D, s.dWhat, BT, d);
+        CK(gemm_batched(g, st));
+        GemmArgs g2 = base_args(D, BT, d, d);
+        term(g2, W, dP, -1.f);
+        g2.addend = dWhat;
+        g2.gamma = 1.f;
+        out_blk(g2, D, s.dWhat, BT, d);
+        CK(gemm_batched(g2, st));
+    }
+    {   // dX = dU N^T + dWhat W^T
+        GemmArgs g = base_args(D, BT, BT, BT);
+        term(g, dU, T_(Nm), 1.f);
+        out_blk(g, D, s.dX, BT, BT);
+        CK(gemm_batched(g, st));
+        GemmArgs g2 = base_args(D, BT, BT, d);
+        term(g2, dWhat, T_(W), 1.f);
+        g2.addend = dX;
+        g2.gamma = 1.f;
+        out_blk(g2, D, s.dX, BT, BT);
+        CK(gemm_batched(g2, st));
+    }
+    {   // dA = strictLower(-(Tinv^T dX) X^T)   (adjoint of Tinv = (I + A)^{-1}, X = Tinv D)
+        GemmArgs g = base_args(D, BT, BT, BT);
+        term(g, T_(Tinv), dX, 1.f);
+        out_blk(g, D, s.tmp, BT, BT);
+        CK(gemm_batched(g, st));
+        GemmArgs g2 = base_args(D, BT, BT, BT);
+        term(g2, tmp, T_(X), -1.f);
+        out_blk(g2, D, s.dA, BT, BT, MASK_STRICT_LOWER);
+        CK(gemm_batched(g2, st));
+    }
+    // dG = strictLower(D dA): dA is strictly lower already, scale its rows by beta
+    CK(scale_rows(s.dA, s.dG, in.beta, L, nb, D.nh * nb, st));
+    {
+        const int batch = D.nh * nb;
+        dbeta_kernel<<<grid_for(batch), BT, 0, st>>>(s.dA, s.G, s.dX, s.Tinv, gr.dbeta, L, nb,
+                                                     batch);
+        count_launches();
+        CK(cudaGetLastError());
+    }
+    {   // dW = -U dKt + dN K + dM^T Q - What dP^T + X^T dWhat + (dG + dG^T) W
+        GemmArgs g = base_args(D, BT, d, BT);
+        term(g, U, dKt, -1.f);
+        term(g, dN, K, 1.f);
+        term(g, T_(dM), Q, 1.f);
+        out_blk(g, D, s.dWacc, BT, d);
+        CK(gemm_batched(g, st));
+        GemmArgs g2 = base_args(D, BT, d, d);
+        term(g2, What, T_(dP), -1.f);
+        g2.addend = dWacc;
+        g2.gamma = 1.f;
+        out_blk(g2, D, s.dWacc, BT, d);
+        CK(gemm_batched(g2, st));
+        GemmArgs g3 = base_args(D, BT, d, BT);
+        term(g3, T_(X), dWhat, 1.f);
+        term(g3, dGm, W, 1.f);
+        term(g3, T_(dGm), W, 1.f);
+        g3.addend = dWacc;
+        g3.gamma = 1.f;
+        set_out(g3, gr.dw, D.dt, ush, usb, d, L);
+        CK(gemm_batched(g3, st));
+    }
+    return cudaSuccess;
+}
+
+}  // namespace path

@@ -1,0 +1,47 @@
+// Per-block UT transform / boundary adjustment and its adjoint (see prep.cu).
+#pragma once
+#include "common.cuh"
+
+namespace path {
+
+struct PrepDims {
+    int nh, L, d, nblk, dt;  // dt: element type of q, k, w
+};
+
+struct PrepInputs {
+    const void *q, *k, *w;  // [nh, L, d]
+    const float *beta;      // [nh, L]
+};
+
+struct PrepOutputs {
+    void *Qt, *Kt;  // [nh, Lp, d] boundary-adjusted queries / keys (type tdt)
+    void *Pm;       // [nh, nblk, d, d] block products (type tdt)
+    float *Sd;      // [nh, nblk, BT, BT] diagonal-block bilinear logits (lower part)
+    int tdt;
+};
+
+struct PrepGrads {
+    const float *dQt, *dKt;  // [nh, Lp, d]
+    const float *dPm;        // [nh, nblk, d, d]
+    const float *dSd;        // [nh, nblk, BT, BT], zero above the diagonal
+    void *dq, *dk, *dw;      // [nh, L, d] (type dt)
+    float *dbeta;            // [nh, L]
+};
+
+struct PrepScratch {
+    float *G = nullptr, *A = nullptr, *Tinv = nullptr, *X = nullptr, *N = nullptr, *U = nullptr,
+          *M = nullptr, *What = nullptr;
+    float *dM = nullptr, *dU = nullptr, *dN = nullptr, *dX = nullptr, *tmp = nullptr,
+          *dA = nullptr, *dG = nullptr, *dWhat = nullptr, *dWacc = nullptr;
+};
+
+void carve_prep_scratch(Carver &c, const PrepDims &D, bool backward, PrepScratch &s);
+size_t prep_scratch_bytes(const PrepDims &D, bool backward);
+cudaError_t prep_forward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
+                         const PrepOutputs &out, cudaStream_t st);
+cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
+                          const PrepGrads &gr, cudaStream_t st);
+cudaError_t scale_rows(const float *in, float *out, const float *beta, int L, int nblk, int batch,
+                       cudaStream_t st);
+
+}  // namespace path

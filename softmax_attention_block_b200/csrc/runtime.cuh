@@ -1,0 +1,25 @@
+// Host-side diagnostics of the library: a process-wide count of kernel
+// launches and optional per-stage timing with CUDA events on the stage's own
+// stream (used by the benchmark to time one stage inside a full step).
+#pragma once
+#include <cuda_runtime.h>
+
+namespace path {
+
+void count_launches(int n = 1);
+
+// Brackets one stage of an entry point with events when profiling is on.
+class Stage {
+  public:
+    Stage(const char *name, cudaStream_t st);
+    ~Stage();
+    Stage(const Stage &) = delete;
+    Stage &operator=(const Stage &) = delete;
+
+  private:
+    const char *name_;
+    cudaStream_t st_;
+    cudaEvent_t e0_ = nullptr;
+};
+
+}  // namespace path

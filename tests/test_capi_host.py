@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function the header declares, sizes workspaces, and rejects invalid
+arguments with the documented status before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "path_attn.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+F32, BF16 = 0, 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import softmax_attention_block_b200 as P
+
+    if not os.path.exists(P.LIB_PATH):
+        from softmax_attention_block_b200 import build
+
+        build.build()
+    return P.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(path_[a-z_]+)\s*\(", text)))
+
+
+def test_header_symbols_exported(lib):
+    names = declared_functions()
+    assert "path_attn_fwd" in names and "path_decode_step" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in the header but not exported"
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.path_status_string(s)
+    assert lib.path_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(lib):
+    f = lib.path_attn_workspace_bytes
+    assert f(1, 1, 64, 16, F32, 0) > 0
+    assert f(8, 24, 4096, 64, BF16, 1) > f(8, 24, 4096, 64, BF16, 0) > 0
+    assert f(1, 1, 64, 48, BF16, 0) == 0  # unsupported head dim
+    assert f(0, 1, 64, 64, BF16, 0) == 0
+    assert f(1, 1, 0, 64, BF16, 0) == 0
+    assert f(1, 1, 64, 64, 7, 0) == 0
+    assert lib.path_decode_workspace_bytes(32, 32, 16448, 128, BF16) > 0
+    assert lib.path_decode_workspace_bytes(1, 1, 10, 96, BF16) == 0
+    assert f(1, 1, 64, 64, BF16, 0) % 256 == 0
+
+
+FAKE = 0x1000  # never dereferenced: every call below fails validation first
+
+
+def fwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, w=FAKE, beta=FAKE, log_f=None, scale=0.125, B=1, H=1,
+             L=64, d=64, dt=BF16, out=FAKE, lse=FAKE, ws=FAKE, wsb=1 << 40)
+    a.update(kw)
+    return lib.path_attn_fwd(a["q"], a["k"], a["v"], a["w"], a["beta"], a["log_f"], a["scale"],
+                             a["B"], a["H"], a["L"], a["d"], a["dt"], a["out"], a["lse"], a["ws"],
+                             a["wsb"], None)
+
+
+def test_fwd_rejects_bad_arguments(lib):
+    assert fwd(lib, q=None) == INVALID
+    assert fwd(lib, lse=None) == INVALID
+    assert fwd(lib, L=0) == INVALID
+    assert fwd(lib, B=-1) == INVALID
+    assert fwd(lib, scale=float("nan")) == INVALID
+    assert fwd(lib, d=48) == UNSUPPORTED
+    assert fwd(lib, dt=5) == UNSUPPORTED
+    assert fwd(lib, ws=None) == WORKSPACE
+    assert fwd(lib, wsb=100) == WORKSPACE
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    def bwd(**kw):
+        a = dict(log_f=None, dlog_f=None, dq=FAKE, L=64, d=64, wsb=1 << 40)
+        a.update(kw)
+        return lib.path_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, a["log_f"], 0.125, 1, 1, a["L"],
+                                 a["d"], BF16, FAKE, FAKE, FAKE, a["dq"], FAKE, FAKE, FAKE, FAKE,
+                                 a["dlog_f"], FAKE, a["wsb"], None)
+
+    assert bwd(dq=None) == INVALID
+    assert bwd(log_f=FAKE) == INVALID  # dlog_f must be given with log_f
+    assert bwd(dlog_f=FAKE) == INVALID
+    assert bwd(d=24) == UNSUPPORTED
+    assert bwd(wsb=10) == WORKSPACE
+
+
+def test_decode_rejects_bad_arguments(lib):
+    def dec(**kw):
+        a = dict(q=FAKE, n=10, cap=11, d=128, wsb=1 << 40, kc=FAKE)
+        a.update(kw)
+        return lib.path_decode_step(a["q"], FAKE, FAKE, FAKE, FAKE, 0.1, 2, 2, a["d"], a["n"],
+                                    a["cap"], BF16, a["kc"], FAKE, FAKE, FAKE, a["wsb"], None)
+
+    assert dec(n=11) == INVALID           # n_cached + 1 > capacity
+    assert dec(n=-1) == INVALID
+    assert dec(q=None) == INVALID
+    assert dec(kc=FAKE + 8) == INVALID     # caches must be 16-byte aligned
+    assert dec(d=32) == UNSUPPORTED
+    assert dec(wsb=4) == WORKSPACE
+
+
+def test_profile_toggle(lib):
+    prev = lib.path_profile_enable(1)
+    assert lib.path_profile_enable(prev) == 1

@@ -19,9 +19,13 @@
  *   are [B, H, L, d]; beta, log_f, lse, dbeta, dlog_f are [B, H, L] fp32.
  *   Decode tensors q, k_new, v_new, w, out are [B, H, d]; decode beta is
  *   [B, H] fp32; the caches are [B, H, capacity, d].
- * - dtype: PATH_F32 or PATH_BF16 selects the element type of every
- *   d-sized tensor (inputs, outputs, gradients, caches). beta, log_f, lse,
- *   dbeta, dlog_f are always fp32. Arithmetic accumulates in fp32.
+ * - dtype (path_dtype below) selects the element types of the d-sized
+ *   tensors. beta, log_f, lse, dbeta, dlog_f are always fp32. Arithmetic
+ *   accumulates in fp32; on the bf16 paths the computed boundary-adjusted
+ *   queries/keys and block products are held in fp16 for the tensor-core
+ *   products, which requires their entries to stay below 65504 in
+ *   magnitude (true whenever |q|, |k| do and beta * |w|^2 lies in [0, 2],
+ *   since then every H has norm <= 1).
  * - Pointers are DEVICE pointers unless stated otherwise. The caller owns
  *   every buffer, including the workspace; the library allocates and frees
  *   no device memory and keeps no state between calls (apart from the
@@ -54,10 +58,21 @@ typedef enum {
     PATH_ERR_UNSUPPORTED = 2, /* head dim or dtype this build does not handle */
     PATH_ERR_WORKSPACE = 3,   /* workspace null or smaller than required */
     PATH_ERR_CUDA = 4,        /* a kernel launch failed */
-    PATH_ERR_TIMEOUT = 5      /* reserved: a bounded device-side wait gave up */
+    PATH_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (path_attn_wait_status) */
 } path_status;
 
-typedef enum { PATH_F32 = 0, PATH_BF16 = 1 } path_dtype;
+/*
+ * Element types of one call:
+ *   PATH_F32          everything fp32.
+ *   PATH_BF16         q, k, v, w, out, dout, dq, dk, dv, dw (and decode
+ *                     caches) bf16.
+ *   PATH_BF16_F32OUT  q, k, v, w bf16; out, dout, dq, dk, dv, dw fp32
+ *                     (fwd/bwd only). Use it when gradients or outputs
+ *                     exceed what bf16 can hold to the needed absolute
+ *                     accuracy (bf16 keeps 8 significant bits), or for the
+ *                     forget-gate gradient, which depends on dout.out.
+ */
+typedef enum { PATH_F32 = 0, PATH_BF16 = 1, PATH_BF16_F32OUT = 2 } path_dtype;
 
 /* Human-readable name of a status code (static storage; never NULL). */
 const char *path_status_string(path_status s);
@@ -104,6 +119,17 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
                           const void *dout, void *dq, void *dk, void *dv, void *dw,
                           float *dbeta, float *dlog_f, void *workspace, size_t workspace_bytes,
                           path_stream_t stream);
+
+/*
+ * Device-side waits of the tensor-core kernels are bounded: if one gives up
+ * (a pipeline stage never completed), the kernel records it in the first
+ * bytes of the workspace, writes NaN to the rows it could not finish, frees
+ * its tensor memory and returns instead of hanging. This call waits for
+ * `stream`, then returns PATH_ERR_TIMEOUT if the last path_attn_fwd /
+ * path_attn_bwd that used `workspace` recorded such an event, else PATH_OK
+ * (PATH_ERR_CUDA if the read-back itself fails). It synchronises the host.
+ */
+path_status path_attn_wait_status(const void *workspace, path_stream_t stream);
 
 /*
  * Workspace size in bytes for path_decode_step; 0 if invalid/unsupported.

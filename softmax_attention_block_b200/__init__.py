@@ -23,8 +23,19 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpath_attn.so")
 
-PATH_F32, PATH_BF16 = 0, 1
+PATH_F32, PATH_BF16, PATH_BF16_F32OUT = 0, 1, 2
 _DT = {torch.float32: PATH_F32, torch.bfloat16: PATH_BF16}
+
+
+def _mode(in_dtype, out_dtype):
+    """path_dtype of a call from the input and output element types."""
+    if in_dtype == torch.float32 and out_dtype == torch.float32:
+        return PATH_F32
+    if in_dtype == torch.bfloat16 and out_dtype == torch.bfloat16:
+        return PATH_BF16
+    if in_dtype == torch.bfloat16 and out_dtype == torch.float32:
+        return PATH_BF16_F32OUT
+    raise ValueError(f"unsupported dtypes: inputs {in_dtype}, outputs {out_dtype}")
 _lib = None
 
 
@@ -55,7 +66,9 @@ def lib() -> ctypes.CDLL:
                                     vp, vp, vp, vp, fp, fp, vp, sz, vp]
         L.path_decode_step.argtypes = [vp, vp, vp, vp, fp, f, i, i, i, i, i, i, vp, vp, vp, vp,
                                        sz, vp]
-        for fn in (L.path_attn_fwd, L.path_attn_bwd, L.path_decode_step):
+        L.path_attn_wait_status.argtypes = [vp, vp]
+        L.path_kernel_launch_count.restype = ctypes.c_ulonglong
+        for fn in (L.path_attn_fwd, L.path_attn_bwd, L.path_decode_step, L.path_attn_wait_status):
             fn.restype = i
         _lib = L
     return _lib
@@ -65,8 +78,9 @@ def path_status_string(status: int) -> str:
     return lib().path_status_string(int(status)).decode()
 
 
-def path_attn_workspace_bytes(B, H, L, d, dtype, for_bwd=False) -> int:
-    return int(lib().path_attn_workspace_bytes(B, H, L, d, _DT[dtype], int(bool(for_bwd))))
+def path_attn_workspace_bytes(B, H, L, d, dtype, for_bwd=False, out_dtype=None) -> int:
+    mode = _mode(dtype, out_dtype or dtype)
+    return int(lib().path_attn_workspace_bytes(B, H, L, d, mode, int(bool(for_bwd))))
 
 
 def path_decode_workspace_bytes(B, H, capacity, d, dtype) -> int:
@@ -103,17 +117,19 @@ def _scale(scale, d):
     return float(d ** -0.5 if scale is None else scale)
 
 
-def path_attn_fwd(q, k, v, w, beta, log_f=None, scale=None, out=None, lse=None, workspace=None):
+def path_attn_fwd(q, k, v, w, beta, log_f=None, scale=None, out=None, lse=None, workspace=None,
+                  out_dtype=None):
     """Forward pass. q, k, v, w: [B,H,L,d] (fp32 or bf16); beta, log_f: [B,H,L] fp32.
+    out_dtype (default: q's dtype) may be torch.float32 with bf16 inputs.
     Returns (out [B,H,L,d], lse [B,H,L] fp32)."""
     B, H, L, d = q.shape
-    dt = _DT[q.dtype]
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    dt = _mode(q.dtype, out.dtype)
     if lse is None:
         lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
     _check_dev(q, k, v, w, beta, log_f, out, lse)
-    nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, False)
+    nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, False, out.dtype)
     ws = _workspace(nbytes, q.device, workspace)
     st = lib().path_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(beta), _ptr(log_f),
                              _scale(scale, d), B, H, L, d, dt, _ptr(out), _ptr(lse), _ptr(ws),
@@ -125,17 +141,21 @@ def path_attn_fwd(q, k, v, w, beta, log_f=None, scale=None, out=None, lse=None, 
 
 def path_attn_bwd(q, k, v, w, beta, out, lse, dout, log_f=None, scale=None, grads=None,
                   workspace=None):
-    """Backward of sum(out * dout). Returns dict dq, dk, dv, dw, dbeta[, dlog_f]."""
+    """Backward of sum(out * dout). out, dout and the returned dq, dk, dv, dw share
+    out's dtype. Returns dict dq, dk, dv, dw, dbeta[, dlog_f]."""
     B, H, L, d = q.shape
-    dt = _DT[q.dtype]
+    dt = _mode(q.dtype, out.dtype)
+    if dout.dtype != out.dtype:
+        raise ValueError("dout must have out's dtype")
     if grads is None:
-        grads = {n: torch.empty_like(q) for n in ("dq", "dk", "dv", "dw")}
+        grads = {n: torch.empty(q.shape, dtype=out.dtype, device=q.device)
+                 for n in ("dq", "dk", "dv", "dw")}
         grads["dbeta"] = torch.empty_like(beta)
         if log_f is not None:
             grads["dlog_f"] = torch.empty_like(log_f)
     dlf = grads.get("dlog_f") if log_f is not None else None
     _check_dev(q, k, v, w, beta, log_f, out, lse, dout, *grads.values())
-    nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, True)
+    nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, True, out.dtype)
     ws = _workspace(nbytes, q.device, workspace)
     st = lib().path_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(beta), _ptr(log_f),
                              _scale(scale, d), B, H, L, d, dt, _ptr(out), _ptr(lse), _ptr(dout),

@@ -41,9 +41,9 @@ struct BwdArgs {
     float *colsum;   // [nh, Lp] or null
 };
 
-cudaError_t chain_simt(const ChainArgs &c, int dt, int d, cudaStream_t st);
-cudaError_t attn_fwd_simt(const FwdArgs &a, int dt, int d, cudaStream_t st);
-cudaError_t attn_bwd_simt(const BwdArgs &a, int dt, int d, cudaStream_t st);
+cudaError_t chain_simt(const ChainArgs &c, Types t, int d, cudaStream_t st);
+cudaError_t attn_fwd_simt(const FwdArgs &a, Types t, int d, cudaStream_t st);
+cudaError_t attn_bwd_simt(const BwdArgs &a, Types t, int d, cudaStream_t st);
 cudaError_t gate_prefix(const float *logf, float *c, int L, int Lp, int nh, cudaStream_t st);
 cudaError_t gate_grad(const float *rowsum, const float *colsum, float *dlogf, int L, int Lp, int nh,
                       cudaStream_t st);

@@ -1,0 +1,373 @@
+// PaTH attention forward on 5th-generation tensor cores (sm_100a).
+//
+// One CTA per (128-row query tile I, head). Warp roles:
+//   warps 0-3  softmax: one query row per thread (TMEM lane = row)
+//   warp 4     producer: TMA loads of Qtil_I, then per key tile the transported
+//              keys Khat_{I,J}, the values V_J and the gate prefix c_J into a
+//              ring of NS stages
+//   warp 5     MMA issuer: S = Qtil Khat^T (fp16 operands, fp32 in TMEM,
+//              double-buffered) and O_tile = P V (bf16 operands)
+// The diagonal tile's logits come precomputed from the UT prep (the
+// full-matrix form of each block); tiles J < I come from S = Qtil Khat^T.
+// Softmax works in the log2 domain; the running max rescales the register
+// accumulator when each P.V tile is added (one tile behind the MMA).
+#include "attn.cuh"
+#include "attn_tc.cuh"
+#include "runtime.cuh"
+#include "tc.cuh"
+
+namespace path {
+
+namespace {
+
+using namespace tc;
+
+constexpr int NT = 192;
+constexpr int W_PROD = 4, W_MMA = 5;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+template <int D>
+struct Cfg {
+    static constexpr int PANELS = D / 64;
+    static constexpr int TILE = 128 * D * 2;  // bytes of one 128-row 16-bit tile
+    static constexpr int NS = D == 64 ? 3 : 2;
+    static constexpr int Q_OFF = 0;
+    static constexpr int ST_OFF = Q_OFF + TILE;
+    static constexpr int ST_BYTES = 2 * TILE + 1024;  // K, V, gate prefix (512 B)
+    static constexpr int P_OFF = ST_OFF + NS * ST_BYTES;
+    static constexpr int BAR_OFF = P_OFF + 128 * 128 * 2;
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;  // + alignment slack
+    static constexpr uint32_t TMEM_COLS = 512;       // S0 [0,128) S1 [128,256) O [256, 256+D)
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p)
+{
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void flag_error(int *err, int code)
+{
+    if (err) atomicCAS(err, 0, code);
+}
+
+template <typename TO>
+__device__ __forceinline__ void store_row(TO *dst, const float *v, int D, float scale);
+
+template <>
+__device__ __forceinline__ void store_row<float>(float *dst, const float *v, int D, float scale)
+{
+    for (int e = 0; e < D; e += 4)
+        *reinterpret_cast<float4 *>(dst + e) =
+            make_float4(v[e] * scale, v[e + 1] * scale, v[e + 2] * scale, v[e + 3] * scale);
+}
+
+template <>
+__device__ __forceinline__ void store_row<bf16>(bf16 *dst, const float *v, int D, float scale)
+{
+    for (int e = 0; e < D; e += 8) {
+        uint4 u;
+        __nv_bfloat162 *hh = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) hh[i] = __floats2bfloat162_rn(v[e + 2 * i] * scale, v[e + 2 * i + 1] * scale);
+        *reinterpret_cast<uint4 *>(dst + e) = u;
+    }
+}
+
+template <int D, bool FOX, typename TO>
+__global__ void __launch_bounds__(NT, 1)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                  const __grid_constant__ CUtensorMap mV, FwdTcArgs a)
+{
+    using C = Cfg<D>;
+    constexpr int NS = C::NS;
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = align1024(smraw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::BAR_OFF);
+    uint64_t *q_full = bars;
+    uint64_t *kv_full = bars + 1;
+    uint64_t *kv_empty = bars + 1 + NS;
+    uint64_t *s_full = bars + 1 + 2 * NS;
+    uint64_t *p_full = bars + 3 + 2 * NS;
+    uint64_t *o_full = bars + 4 + 2 * NS;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 5 + 2 * NS);
+    uint8_t *sQ = sm + C::Q_OFF;
+    uint8_t *sP = sm + C::P_OFF;
+    auto sK = [&](int s) { return sm + C::ST_OFF + s * C::ST_BYTES; };
+    auto sV = [&](int s) { return sm + C::ST_OFF + s * C::ST_BYTES + C::TILE; };
+    auto sC = [&](int s) { return reinterpret_cast<float *>(sm + C::ST_OFF + s * C::ST_BYTES + 2 * C::TILE); };
+
+    const int I = a.nblk - 1 - (int)blockIdx.x;  // longest rows of the causal triangle first
+    const int h = blockIdx.y;
+    const int niter = I + 1;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int Lp = a.nblk * BT;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        mbar_init(p_full, 128);
+        mbar_init(o_full, 1);
+        mbar_fence_init();
+    }
+    if (warp == W_MMA) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp == W_PROD) {
+        if (lane == 0) {
+            int issued = 0;
+            mbar_expect_tx(q_full, C::TILE);
+            for (int p = 0; p < C::PANELS; ++p)
+                tma_load_2d(sQ + p * 16384, &mQ, 64 * p, h * Lp + I * BT, q_full);
+            for (int it = 0; it < niter; ++it) {
+                const int s = it % NS;
+                if (it >= NS && !mbar_wait(&kv_empty[s], ((it / NS) - 1) & 1, WAIT_POLLS)) {
+                    flag_error(a.err, 1);
+                    break;
+                }
+                const int J = it == 0 ? I : I - it;
+                const uint32_t bytes = C::TILE + (it > 0 ? C::TILE : 0) + (FOX ? 512 : 0);
+                mbar_expect_tx(&kv_full[s], bytes);
+                if (it > 0) {
+                    const int row = (int)((h * a.npairs + (long long)I * (I - 1) / 2 + J) * BT);
+                    for (int p = 0; p < C::PANELS; ++p)
+                        tma_load_2d(sK(s) + p * 16384, &mK, 64 * p, row, &kv_full[s]);
+                }
+                for (int p = 0; p < C::PANELS; ++p)
+                    tma_load_3d(sV(s) + p * 16384, &mV, 64 * p, J * BT, h, &kv_full[s]);
+                if (FOX) bulk_load(sC(s), a.c + (long long)h * Lp + J * BT, 512, &kv_full[s]);
+                issued = it + 1;
+            }
+            // never leave while copies into this CTA's shared memory are in flight
+            for (int it = issued - NS > 0 ? issued - NS : 0; it < issued; ++it)
+                mbar_wait(&kv_full[it % NS], (it / NS) & 1, WAIT_POLLS);
+        }
+    } else if (warp == W_MMA) {
+        if (lane == 0) {
+            const uint32_t idS = idesc_f16(128, 128, AB_F16, 0, 0);
+            const uint32_t idO = idesc_f16(128, D, AB_BF16, 0, 1);
+            const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
+            bool ok = mbar_wait(q_full, 0, WAIT_POLLS) && mbar_wait(&kv_full[0], 0, WAIT_POLLS);
+            fence_after_sync();
+            for (int it = 0; ok && it < niter; ++it) {
+                if (it + 1 < niter) {  // S for the next tile, overlapping this tile's softmax
+                    const int n = it + 1, s = n % NS, b = n & 1;
+                    if (!mbar_wait(&kv_full[s], (n / NS) & 1, WAIT_POLLS)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_after_sync();
+                    const uint32_t k_addr = smem_u32(sK(s));
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+                        mma_ss(tbase + b * 128, desc_sw128(q_addr + off, 16, 1024),
+                               desc_sw128(k_addr + off, 16, 1024), idS, kk > 0);
+                    }
+                    commit(&s_full[b]);
+                }
+                if (!mbar_wait(p_full, it & 1, WAIT_POLLS)) {
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+                const int s = it % NS;
+                const uint32_t v_addr = smem_u32(sV(s));
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t aoff = (kk / 4) * 16384 + (kk % 4) * 32;
+                    mma_ss(tbase + 256, desc_sw128(p_addr + aoff, 16, 1024),
+                           desc_sw128(v_addr + kk * 2048, 16384, 1024), idO, kk > 0);
+                }
+                commit(o_full);
+                commit(&kv_empty[s]);
+            }
+            if (!ok) flag_error(a.err, 2);
+        }
+    } else {
+        // softmax: thread r owns query row r of the tile
+        const int r = threadIdx.x;
+        const int gi = I * BT + r;
+        const bool valid = gi < a.L;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const float k1 = a.scale_log2;
+        const float ci2 = FOX ? a.c[(long long)h * Lp + gi] * LOG2E : 0.f;
+        float acc[D];
+#pragma unroll
+        for (int e = 0; e < D; ++e) acc[e] = 0.f;
+        float m = -INFINITY, l = 0.f, mA = -INFINITY;
+        bool ok = true;
+        const float *sd = a.Sd + (((long long)h * a.nblk + I) * BT + r) * BT;
+        for (int it = 0; it < niter; ++it) {
+            const int s = it % NS, b = it & 1;
+            if (FOX && !mbar_wait(&kv_full[s], (it / NS) & 1, WAIT_POLLS)) {
+                ok = false;
+                break;
+            }
+            const float *cj = sC(s);
+            auto bias = [&](int j) { return FOX ? ci2 - cj[j] * LOG2E : 0.f; };
+            // pass 1: row max
+            float mrow = -INFINITY;
+            if (it == 0) {
+                for (int j = 0; j < BT; j += 4) {
+                    const float4 v4 = *reinterpret_cast<const float4 *>(sd + j);
+                    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (j + u <= r) mrow = fmaxf(mrow, fmaf(vv[u], k1, bias(j + u)));
+                }
+            } else {
+                if (!mbar_wait(&s_full[b], ((it - 1) >> 1) & 1, WAIT_POLLS)) {
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+#pragma unroll 1
+                for (int c0 = 0; c0 < BT; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tbase + b * 128 + c0 + lane_off, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) mrow = fmaxf(mrow, fmaf(v[j], k1, bias(c0 + j)));
+                }
+            }
+            const float m_new = fmaxf(m, mrow);
+            // add the previous tile's P.V (scaled to its max m) into the accumulator
+            if (it >= 1) {
+                if (!mbar_wait(o_full, (it - 1) & 1, WAIT_POLLS)) {
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+                const float corr = ex2(mA - m);
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tbase + 256 + c0 + lane_off, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
+                }
+                mA = m;
+            }
+            // pass 2: probabilities -> P (bf16, swizzled K-major) and row sum
+            float rowsum = 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BT; c0 += 32) {
+                float v[32];
+                if (it == 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = sd[c0 + j];
+                } else {
+                    tmem_ld32(tbase + b * 128 + c0 + lane_off, v);
+                    tmem_wait_ld();
+                }
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    uint4 u;
+                    __nv_bfloat162 *hh = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        float pp[2];
+#pragma unroll
+                        for (int t = 0; t < 2; ++t) {
+                            const int j = c0 + g * 8 + q2 * 2 + t;
+                            const float z = fmaf(v[g * 8 + q2 * 2 + t], k1, bias(j));
+                            pp[t] = (it > 0 || j <= r) ? ex2(z - m_new) : 0.f;
+                            rowsum += pp[t];
+                        }
+                        hh[q2] = __floats2bfloat162_rn(pp[0], pp[1]);
+                    }
+                    const int col = c0 + g * 8;
+                    *reinterpret_cast<uint4 *>(sP + (col >> 6) * 16384 + sw128_offset(r, col & 63)) = u;
+                }
+            }
+            l = fmaf(l, ex2(m - m_new), rowsum);
+            m = m_new;
+            fence_async_smem();
+            fence_before_sync();
+            mbar_arrive(p_full);
+        }
+        if (ok && mbar_wait(o_full, (niter - 1) & 1, WAIT_POLLS)) {
+            fence_after_sync();
+            const float corr = ex2(mA - m);
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                float v[32];
+                tmem_ld32(tbase + 256 + c0 + lane_off, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
+            }
+        } else {
+            ok = false;
+        }
+        if (!ok) flag_error(a.err, 3);
+        if (valid) {
+            TO *dst = static_cast<TO *>(a.out) + ((long long)h * a.L + gi) * D;
+            const float inv = ok ? 1.f / l : __int_as_float(0x7fc00000);
+            store_row<TO>(dst, acc, D, inv);
+            a.lse[(long long)h * a.L + gi] = ok ? (m + log2f(l)) * LN2 : __int_as_float(0x7fc00000);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == W_MMA) tmem_dealloc(tbase, C::TMEM_COLS);
+}
+
+template <int D, bool FOX, typename TO>
+cudaError_t launch(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mV,
+                   const FwdTcArgs &a, cudaStream_t st)
+{
+    auto k = fwd_tc_kernel<D, FOX, TO>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM);
+    if (e != cudaSuccess) return e;
+    k<<<dim3(a.nblk, a.nh), NT, Cfg<D>::SMEM, st>>>(mQ, mK, mV, a);
+    count_launches();
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attn_fwd_tc_supported(Types t, int d)
+{
+    return t.in == BF16 && t.mid == F16 && (d == 64 || d == 128);
+}
+
+cudaError_t attn_fwd_tc(const FwdArgs &f, Types t, int d, int *err, cudaStream_t st)
+{
+    const int Lp = f.nblk * BT;
+    const long long npairs = (long long)f.nblk * (f.nblk - 1) / 2;
+    CUtensorMap mQ, mK, mV;
+    if (!make_map_2d(&mQ, f.Qt, F16, d, (uint64_t)f.nh * Lp, 128)) return cudaErrorInvalidValue;
+    if (npairs > 0) {
+        if (!make_map_2d(&mK, f.Khat, F16, d, (uint64_t)f.nh * npairs * BT, 128))
+            return cudaErrorInvalidValue;
+    } else {
+        mK = mQ;  // no off-diagonal tiles: never read
+    }
+    if (!make_map_3d(&mV, f.v, BF16, d, f.L, f.nh, 128)) return cudaErrorInvalidValue;
+    FwdTcArgs a{f.Sd, f.c, f.scale * 1.4426950408889634f, f.L, f.nblk, f.nh, npairs, f.out, f.lse, err};
+    const bool fox = f.c != nullptr;
+    const bool f32 = t.out == F32;
+#define L_(D_, FOX_, TO_) return launch<D_, FOX_, TO_>(mQ, mK, mV, a, st)
+    if (d == 64) {
+        if (fox) { if (f32) L_(64, true, float); else L_(64, true, bf16); }
+        else { if (f32) L_(64, false, float); else L_(64, false, bf16); }
+    } else {
+        if (fox) { if (f32) L_(128, true, float); else L_(128, true, bf16); }
+        else { if (f32) L_(128, false, float); else L_(128, false, bf16); }
+    }
+#undef L_
+}
+
+}  // namespace path

@@ -33,7 +33,7 @@ __device__ void stage_rows(float *dst, int ldd, const T *src, int rows_valid)
 // Transport chain: Khat_{I,J} for every pair J < I.
 // grid (nblk - 1, nh), BT threads; thread r carries row r of block J.
 // ---------------------------------------------------------------------------
-template <typename T, int D>
+template <typename T, int D>  // T: intermediate (mid) type
 __global__ void __launch_bounds__(BT) chain_kernel(const T *Kt, const T *Pm, T *Khat, int nblk)
 {
     extern __shared__ float sm[];
@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(BT) chain_kernel(const T *Kt, const T *Pm, T *
 // ---------------------------------------------------------------------------
 // Forward. grid (2*nblk, nh), QR threads; thread i = query row.
 // ---------------------------------------------------------------------------
-template <typename T, int D>
+template <typename T, typename TM, typename TO, int D>  // input, mid (intermediate), output types
 __global__ void __launch_bounds__(QR) fwd_kernel(FwdArgs a)
 {
     extern __shared__ float sm[];
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(QR) fwd_kernel(FwdArgs a)
     const int li = half * QR + threadIdx.x;  // row within tile I
     const int gi = I * BT + li;
     const bool valid = gi < L;
-    const T *qt = static_cast<const T *>(a.Qt) + ((long long)h * Lp + gi) * D;
+    const TM *qt = static_cast<const TM *>(a.Qt) + ((long long)h * Lp + gi) * D;
     for (int e = 0; e < D; ++e) sQ[e * QR + threadIdx.x] = to_f(qt[e]);
     const float ci = (a.c && valid) ? a.c[(long long)h * Lp + gi] : 0.f;
     float m = -INFINITY, l = 0.f, o[D];
@@ -124,10 +124,10 @@ __global__ void __launch_bounds__(QR) fwd_kernel(FwdArgs a)
     // off-diagonal tiles, right to left
     const long long npairs = (long long)nblk * (nblk - 1) / 2;
     for (int J = I - 1; J >= 0; --J) {
-        const T *kh = static_cast<const T *>(a.Khat) + ((long long)h * npairs + pair_index(I, J)) * BT * D;
+        const TM *kh = static_cast<const TM *>(a.Khat) + ((long long)h * npairs + pair_index(I, J)) * BT * D;
         for (int k0 = 0; k0 < BT; k0 += KS) {
             __syncthreads();
-            stage_rows<T, D>(sK, D, kh + (long long)k0 * D, KS);
+            stage_rows<TM, D>(sK, D, kh + (long long)k0 * D, KS);
             stage_rows<T, D>(sV, D, V + (long long)(J * BT + k0) * D, KS);
             for (int u = threadIdx.x; u < KS; u += blockDim.x)
                 sC[u] = a.c ? a.c[(long long)h * Lp + J * BT + k0 + u] : 0.f;
@@ -146,8 +146,8 @@ __global__ void __launch_bounds__(QR) fwd_kernel(FwdArgs a)
     }
     if (!valid) return;
     const float inv = 1.f / l;
-    T *out = static_cast<T *>(a.out) + ((long long)h * L + gi) * D;
-    for (int e = 0; e < D; ++e) out[e] = from_f<T>(o[e] * inv);
+    TO *out = static_cast<TO *>(a.out) + ((long long)h * L + gi) * D;
+    for (int e = 0; e < D; ++e) out[e] = from_f<TO>(o[e] * inv);
     a.lse[(long long)h * L + gi] = m + __logf(l);
 }
 
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(QR) fwd_kernel(FwdArgs a)
 // Backward, query side: dQtil (off-diagonal pairs), dSd (diagonal tiles),
 // row sums of dZ. grid (2*nblk, nh), QR threads.
 // ---------------------------------------------------------------------------
-template <typename T, int D>
+template <typename T, typename TM, typename TO, int D>
 __global__ void __launch_bounds__(QR) bwd_q_kernel(BwdArgs a)
 {
     extern __shared__ float sm[];
@@ -169,8 +169,8 @@ __global__ void __launch_bounds__(QR) bwd_q_kernel(BwdArgs a)
     const int li = half * QR + threadIdx.x;
     const int gi = I * BT + li;
     const bool valid = gi < L;
-    const T *qt = static_cast<const T *>(a.Qt) + ((long long)h * Lp + gi) * D;
-    const T *dO = static_cast<const T *>(a.dout) + ((long long)h * L + (valid ? gi : 0)) * D;
+    const TM *qt = static_cast<const TM *>(a.Qt) + ((long long)h * Lp + gi) * D;
+    const TO *dO = static_cast<const TO *>(a.dout) + ((long long)h * L + (valid ? gi : 0)) * D;
     for (int e = 0; e < D; ++e) {
         sQ[e * QR + threadIdx.x] = to_f(qt[e]);
         sDO[e * QR + threadIdx.x] = valid ? to_f(dO[e]) : 0.f;
@@ -209,10 +209,10 @@ __global__ void __launch_bounds__(QR) bwd_q_kernel(BwdArgs a)
     }
     const long long npairs = (long long)nblk * (nblk - 1) / 2;
     for (int J = I - 1; J >= 0; --J) {
-        const T *kh = static_cast<const T *>(a.Khat) + ((long long)h * npairs + pair_index(I, J)) * BT * D;
+        const TM *kh = static_cast<const TM *>(a.Khat) + ((long long)h * npairs + pair_index(I, J)) * BT * D;
         for (int k0 = 0; k0 < BT; k0 += KS) {
             __syncthreads();
-            stage_rows<T, D>(sK, D, kh + (long long)k0 * D, KS);
+            stage_rows<TM, D>(sK, D, kh + (long long)k0 * D, KS);
             stage_rows<T, D>(sV, D, V + (long long)(J * BT + k0) * D, KS);
             for (int u = threadIdx.x; u < KS; u += blockDim.x)
                 sC[u] = a.c ? a.c[(long long)h * Lp + J * BT + k0 + u] : 0.f;
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(QR) bwd_q_kernel(BwdArgs a)
 // dP (atomically accumulated), column sums of dZ.
 // grid (2*nblk, nh), QR threads; thread j = key row.
 // ---------------------------------------------------------------------------
-template <typename T, int D>
+template <typename T, typename TM, typename TO, int D>
 __global__ void __launch_bounds__(QR) bwd_k_kernel(BwdArgs a)
 {
     extern __shared__ float sm[];
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(QR) bwd_k_kernel(BwdArgs a)
     const int t = threadIdx.x;
     float *kh = sKh + t * (D + 1), *vj = sVj + t * (D + 1), *ab = sAb + t * (D + 1);
     const T *V = static_cast<const T *>(a.v) + (long long)h * L * D;
-    const T *dOut = static_cast<const T *>(a.dout) + (long long)h * L * D;
+    const TO *dOut = static_cast<const TO *>(a.dout) + (long long)h * L * D;
     for (int e = 0; e < D; ++e) {
         vj[e] = valid ? to_f(V[(long long)gj * D + e]) : 0.f;
         ab[e] = 0.f;
@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(QR) bwd_k_kernel(BwdArgs a)
     float colsum = 0.f;
     const long long npairs = (long long)nblk * (nblk - 1) / 2;
     auto stage_queries = [&](int I, int q0) {
-        const T *qt = static_cast<const T *>(a.Qt) + ((long long)h * Lp + I * BT + q0) * D;
+        const TM *qt = static_cast<const TM *>(a.Qt) + ((long long)h * Lp + I * BT + q0) * D;
         const int rows = min(QR, L - (I * BT + q0));
         for (int e = t; e < QR * D; e += blockDim.x) {
             const int r = e / D, c = e % D;
@@ -289,12 +289,12 @@ __global__ void __launch_bounds__(QR) bwd_k_kernel(BwdArgs a)
     };
     for (int I = nblk - 1; I > J; --I) {
         __syncthreads();
-        const T *khat = static_cast<const T *>(a.Khat) +
+        const TM *khat = static_cast<const TM *>(a.Khat) +
                         ((long long)h * npairs + pair_index(I, J)) * BT * D + (long long)lj * D;
         for (int e = 0; e < D; ++e) kh[e] = to_f(khat[e]);
         if (I + 1 < nblk) {
             // dP_I += Abar_{I+1}^T Khat_{J,I}   and   Abar <- Abar_{I+1} P_I
-            const T *p = static_cast<const T *>(a.Pm) + ((long long)h * nblk + I) * D * D;
+            const TM *p = static_cast<const TM *>(a.Pm) + ((long long)h * nblk + I) * D * D;
             for (int e = t; e < D * D; e += blockDim.x) sP[e] = to_f(p[e]);
             __syncthreads();
             float *dpm = a.dPm + ((long long)h * nblk + I) * D * D;
@@ -361,8 +361,8 @@ __global__ void __launch_bounds__(QR) bwd_k_kernel(BwdArgs a)
         }
     }
     if (!valid) return;
-    T *dvo = static_cast<T *>(a.dv) + ((long long)h * L + gj) * D;
-    for (int e = 0; e < D; ++e) dvo[e] = from_f<T>(dv[e]);
+    TO *dvo = static_cast<TO *>(a.dv) + ((long long)h * L + gj) * D;
+    for (int e = 0; e < D; ++e) dvo[e] = from_f<TO>(dv[e]);
     if (a.colsum) a.colsum[(long long)h * Lp + gj] = colsum;
 }
 
@@ -432,69 +432,84 @@ cudaError_t run_chain(const ChainArgs &c, cudaStream_t st)
     return cudaGetLastError();
 }
 
-template <typename T, int D>
+template <typename T, typename TM, typename TO, int D>
 cudaError_t run_fwd(const FwdArgs &a, cudaStream_t st)
 {
     const size_t smem = (D * QR + 2 * KS * D + KS) * sizeof(float);
-    CK(set_smem(fwd_kernel<T, D>, smem));
-    fwd_kernel<T, D><<<dim3(2 * a.nblk, a.nh), QR, smem, st>>>(a);
+    CK(set_smem(fwd_kernel<T, TM, TO, D>, smem));
+    fwd_kernel<T, TM, TO, D><<<dim3(2 * a.nblk, a.nh), QR, smem, st>>>(a);
     count_launches();
     return cudaGetLastError();
 }
 
-template <typename T, int D>
+template <typename T, typename TM, typename TO, int D>
 cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
 {
     const int Lp = a.nblk * BT;
-    delta_kernel<T, D><<<512, 256, 0, st>>>(static_cast<const T *>(a.out),
-                                            static_cast<const T *>(a.dout), a.delta, a.L, Lp, a.nh);
+    delta_kernel<TO, D><<<512, 256, 0, st>>>(static_cast<const TO *>(a.out),
+                                             static_cast<const TO *>(a.dout), a.delta, a.L, Lp, a.nh);
     count_launches();
     CK(cudaGetLastError());
     const size_t smq = (2 * D * QR + 2 * KS * D + KS) * sizeof(float);
-    CK(set_smem(bwd_q_kernel<T, D>, smq));
+    CK(set_smem(bwd_q_kernel<T, TM, TO, D>, smq));
     {
         Stage s_q("attn_bwd_q", st);
-        bwd_q_kernel<T, D><<<dim3(2 * a.nblk, a.nh), QR, smq, st>>>(a);
+        bwd_q_kernel<T, TM, TO, D><<<dim3(2 * a.nblk, a.nh), QR, smq, st>>>(a);
         count_launches();
     }
     CK(cudaGetLastError());
     const size_t smk = (2 * QR * D + 3 * QR * (D + 1) + D * D + 3 * QR) * sizeof(float);
-    CK(set_smem(bwd_k_kernel<T, D>, smk));
+    CK(set_smem(bwd_k_kernel<T, TM, TO, D>, smk));
     {
         Stage s_k("attn_bwd_k", st);
-        bwd_k_kernel<T, D><<<dim3(2 * a.nblk, a.nh), QR, smk, st>>>(a);
+        bwd_k_kernel<T, TM, TO, D><<<dim3(2 * a.nblk, a.nh), QR, smk, st>>>(a);
         count_launches();
     }
     return cudaGetLastError();
 }
 
+template <int D, typename F>
+cudaError_t by_types(Types t, F &&f)
+{
+    using DD = std::integral_constant<int, D>;
+    if (t.in == F32) return f(float(), float(), float(), DD());
+    if (t.out == BF16) return f(bf16(), f16(), bf16(), DD());
+    return f(bf16(), f16(), float(), DD());
+}
+
 template <typename F>
-cudaError_t dispatch(int dt, int d, F &&f)
+cudaError_t dispatch(Types t, int d, F &&f)
 {
     switch (d) {
-    case 16: return dt == F32 ? f(float(), std::integral_constant<int, 16>()) : f(bf16(), std::integral_constant<int, 16>());
-    case 32: return dt == F32 ? f(float(), std::integral_constant<int, 32>()) : f(bf16(), std::integral_constant<int, 32>());
-    case 64: return dt == F32 ? f(float(), std::integral_constant<int, 64>()) : f(bf16(), std::integral_constant<int, 64>());
-    case 128: return dt == F32 ? f(float(), std::integral_constant<int, 128>()) : f(bf16(), std::integral_constant<int, 128>());
+    case 16: return by_types<16>(t, f);
+    case 32: return by_types<32>(t, f);
+    case 64: return by_types<64>(t, f);
+    case 128: return by_types<128>(t, f);
     }
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t chain_simt(const ChainArgs &c, int dt, int d, cudaStream_t st)
+cudaError_t chain_simt(const ChainArgs &c, Types t, int d, cudaStream_t st)
 {
-    return dispatch(dt, d, [&](auto t, auto dd) { return run_chain<decltype(t), decltype(dd)::value>(c, st); });
+    return dispatch(t, d, [&](auto, auto i, auto, auto dd) {
+        return run_chain<decltype(i), decltype(dd)::value>(c, st);
+    });
 }
 
-cudaError_t attn_fwd_simt(const FwdArgs &a, int dt, int d, cudaStream_t st)
+cudaError_t attn_fwd_simt(const FwdArgs &a, Types t, int d, cudaStream_t st)
 {
-    return dispatch(dt, d, [&](auto t, auto dd) { return run_fwd<decltype(t), decltype(dd)::value>(a, st); });
+    return dispatch(t, d, [&](auto x, auto i, auto o, auto dd) {
+        return run_fwd<decltype(x), decltype(i), decltype(o), decltype(dd)::value>(a, st);
+    });
 }
 
-cudaError_t attn_bwd_simt(const BwdArgs &a, int dt, int d, cudaStream_t st)
+cudaError_t attn_bwd_simt(const BwdArgs &a, Types t, int d, cudaStream_t st)
 {
-    return dispatch(dt, d, [&](auto t, auto dd) { return run_bwd<decltype(t), decltype(dd)::value>(a, st); });
+    return dispatch(t, d, [&](auto x, auto i, auto o, auto dd) {
+        return run_bwd<decltype(x), decltype(i), decltype(o), decltype(dd)::value>(a, st);
+    });
 }
 
 cudaError_t gate_prefix(const float *logf, float *c, int L, int Lp, int nh, cudaStream_t st)

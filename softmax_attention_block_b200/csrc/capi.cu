@@ -3,6 +3,7 @@
 #include <math.h>
 
 #include "attn.cuh"
+#include "attn_tc.cuh"
 #include "prep.cuh"
 #include "runtime.cuh"
 
@@ -25,11 +26,12 @@ Layout make_layout(int B, int H, int L, int d, path_dtype dt)
     y.nblk = ceil_div(L, BT);
     y.Lp = y.nblk * BT;
     y.npairs = (long long)y.nblk * (y.nblk - 1) / 2;
-    y.tsz = dt == PATH_F32 ? 4 : 2;
+    y.tsz = dtype_size(types_of(dt).mid);
     return y;
 }
 
 struct AttnWs {
+    int *err;  // device error word: first bounded wait that gave up (0 = none)
     float *c;
     void *Qt, *Kt, *Pm, *Khat;
     float *Sd;
@@ -43,13 +45,14 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
 {
     Carver c(base);
     const size_t nh = y.nh, Lp = y.Lp, d = y.d, nb = y.nblk;
+    w.err = c.take<int>(64);
     w.c = c.take<float>(nh * Lp);
     w.Qt = c.take<char>(nh * Lp * d * y.tsz);
     w.Kt = c.take<char>(nh * Lp * d * y.tsz);
     w.Pm = c.take<char>(nh * nb * d * d * y.tsz);
     w.Khat = c.take<char>(nh * (size_t)y.npairs * BT * d * y.tsz);
     w.Sd = c.take<float>(nh * nb * BT * BT);
-    PrepDims D{y.nh, y.L, y.d, y.nblk, (int)dt};
+    PrepDims D{y.nh, y.L, y.d, y.nblk, types_of(dt).in, types_of(dt).out};
     carve_prep_scratch(c, D, bwd, w.prep);
     if (bwd) {
         w.delta = c.take<float>(nh * Lp);
@@ -72,7 +75,12 @@ bool fwd_dims_ok(int B, int H, int L, int d)
 
 bool head_dim_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
-bool dtype_ok(path_dtype dt) { return dt == PATH_F32 || dt == PATH_BF16; }
+bool dtype_ok(path_dtype dt)
+{
+    return dt == PATH_F32 || dt == PATH_BF16 || dt == PATH_BF16_F32OUT;
+}
+
+bool decode_dtype_ok(path_dtype dt) { return dt == PATH_F32 || dt == PATH_BF16; }
 
 path_status launch_status(cudaError_t e) { return e == cudaSuccess ? PATH_OK : PATH_ERR_CUDA; }
 
@@ -81,6 +89,16 @@ path_status launch_status(cudaError_t e) { return e == cudaSuccess ? PATH_OK : P
         cudaError_t e_ = (x);                           \
         if (e_ != cudaSuccess) return PATH_ERR_CUDA;    \
     } while (0)
+
+// Tensor-core forward: bf16 inputs, d in {64, 128}, 16-byte aligned v (TMA),
+// row coordinates of the transported-key tiles within int range.
+bool use_tc_fwd(Types t, const Layout &y, const void *v)
+{
+    if (!attn_fwd_tc_supported(t, y.d)) return false;
+    if (reinterpret_cast<uintptr_t>(v) & 15u) return false;
+    return (long long)y.nh * (y.npairs + 1) * BT < (1LL << 31) &&
+           (long long)y.nh * y.Lp < (1LL << 31);
+}
 
 // Shared by forward and backward: gate prefix, UT prep, transport chain.
 path_status run_prep_and_chain(const void *q, const void *k, const void *w, const float *beta,
@@ -91,9 +109,10 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
         Stage s("gate_prefix", st);
         TRY(gate_prefix(log_f, ws.c, y.L, y.Lp, y.nh, st));
     }
-    PrepDims D{y.nh, y.L, y.d, y.nblk, (int)dt};
+    const Types t = types_of(dt);
+    PrepDims D{y.nh, y.L, y.d, y.nblk, t.in, t.out};
     PrepInputs in{q, k, w, beta};
-    PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, (int)dt};
+    PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, t.mid};
     {
         Stage s("ut_prep", st);
         TRY(prep_forward(D, in, ws.prep, out, st));
@@ -101,7 +120,7 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
     ChainArgs ca{ws.Kt, ws.Pm, ws.Khat, y.nblk, y.nh};
     {
         Stage s("chain", st);
-        TRY(chain_simt(ca, (int)dt, y.d, st));
+        TRY(chain_simt(ca, t, y.d, st));
     }
     return PATH_OK;
 }
@@ -144,11 +163,14 @@ path_status path_attn_fwd(const void *q, const void *k, const void *v, const voi
     if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
     carve_attn(workspace, y, dt, false, ws);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    TRY(cudaMemsetAsync(ws.err, 0, sizeof(int), st));
     path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
     if (s != PATH_OK) return s;
     FwdArgs a{ws.Qt, ws.Khat, v, ws.Sd, log_f ? ws.c : nullptr, scale, y.L, y.nblk, y.nh, out, lse};
+    const Types t = types_of(dt);
     Stage s_attn("attn_fwd", st);
-    return launch_status(attn_fwd_simt(a, (int)dt, d, st));
+    if (use_tc_fwd(t, y, v)) return launch_status(attn_fwd_tc(a, t, d, ws.err, st));
+    return launch_status(attn_fwd_simt(a, t, d, st));
 }
 
 path_status path_attn_bwd(const void *q, const void *k, const void *v, const void *w,
@@ -169,6 +191,7 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
     if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
     carve_attn(workspace, y, dt, true, ws);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    TRY(cudaMemsetAsync(ws.err, 0, sizeof(int), st));
     path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
     if (s != PATH_OK) return s;
     TRY(cudaMemsetAsync(ws.dPm, 0, sizeof(float) * (size_t)y.nh * y.nblk * d * d, st));
@@ -176,8 +199,8 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
               scale,     y.L,      y.nblk,   y.nh,   out,    dout,
               lse,       ws.delta, ws.dQt,   ws.dKt, ws.dPm, ws.dSd,
               dv,        ws.rowsum, ws.colsum};
-    TRY(attn_bwd_simt(a, (int)dt, d, st));
-    PrepDims D{y.nh, y.L, y.d, y.nblk, (int)dt};
+    TRY(attn_bwd_simt(a, types_of(dt), d, st));
+    PrepDims D{y.nh, y.L, y.d, y.nblk, types_of(dt).in, types_of(dt).out};
     PrepInputs in{q, k, w, beta};
     PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta};
     {
@@ -191,9 +214,20 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
     return PATH_OK;
 }
 
+path_status path_attn_wait_status(const void *workspace, path_stream_t stream)
+{
+    if (!workspace) return PATH_ERR_INVALID_ARG;
+    int code = 0;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&code, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return PATH_ERR_CUDA;
+    return code ? PATH_ERR_TIMEOUT : PATH_OK;
+}
+
 size_t path_decode_workspace_bytes(int B, int H, int capacity, int d, path_dtype dt)
 {
-    if (B <= 0 || H <= 0 || capacity <= 0 || (d != 64 && d != 128) || !dtype_ok(dt)) return 0;
+    if (B <= 0 || H <= 0 || capacity <= 0 || (d != 64 && d != 128) || !decode_dtype_ok(dt)) return 0;
     const size_t nchunk = (size_t)ceil_div(capacity, DECODE_CHUNK);
     return align_up((size_t)B * H * nchunk * (d + 2) * sizeof(float), 256);
 }
@@ -208,7 +242,7 @@ path_status path_decode_step(const void *q, const void *k_new, const void *v_new
     if (B <= 0 || H <= 0 || capacity <= 0 || n_cached < 0 || n_cached + 1 > capacity ||
         !isfinite(scale))
         return PATH_ERR_INVALID_ARG;
-    if ((d != 64 && d != 128) || !dtype_ok(dt)) return PATH_ERR_UNSUPPORTED;
+    if ((d != 64 && d != 128) || !decode_dtype_ok(dt)) return PATH_ERR_UNSUPPORTED;
     // 16-byte vector access of q, w and the caches
     const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(w) |
                          reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache);

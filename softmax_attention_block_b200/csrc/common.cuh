@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -14,11 +15,14 @@ namespace path {
 constexpr int BT = 128;
 
 typedef __nv_bfloat16 bf16;
+typedef __half f16;
 
-enum DType { F32 = 0, BF16 = 1 };
+// element types of device buffers
+enum DType { F32 = 0, BF16 = 1, F16 = 2 };
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(bf16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f(f16 x) { return __half2float(x); }
 
 template <typename T>
 __device__ __forceinline__ T from_f(float x);
@@ -26,19 +30,43 @@ template <>
 __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
+template <>
+__device__ __forceinline__ f16 from_f<f16>(float x) { return __float2half_rn(x); }
 
 __device__ __forceinline__ float load_as_f(const void *p, int dt, long long i)
 {
-    return dt == F32 ? static_cast<const float *>(p)[i]
-                     : __bfloat162float(static_cast<const bf16 *>(p)[i]);
+    if (dt == F32) return static_cast<const float *>(p)[i];
+    if (dt == BF16) return __bfloat162float(static_cast<const bf16 *>(p)[i]);
+    return __half2float(static_cast<const f16 *>(p)[i]);
 }
 
 __device__ __forceinline__ void store_from_f(void *p, int dt, long long i, float x)
 {
     if (dt == F32)
         static_cast<float *>(p)[i] = x;
-    else
+    else if (dt == BF16)
         static_cast<bf16 *>(p)[i] = __float2bfloat16_rn(x);
+    else
+        static_cast<f16 *>(p)[i] = __float2half_rn(x);
+}
+
+inline size_t dtype_size(int dt) { return dt == F32 ? 4 : 2; }
+
+// The three element types one call works with:
+//   in  - q, k, v, w (and the decode caches)
+//   mid - the computed boundary-adjusted queries/keys, block products and
+//         transported keys (fp16 on the bf16 paths: same tensor-core rate as
+//         bf16, three more mantissa bits)
+//   out - out, dout and the gradients dq, dk, dv, dw
+struct Types {
+    int in, mid, out;
+};
+
+inline Types types_of(path_dtype dt)
+{
+    if (dt == PATH_F32) return {F32, F32, F32};
+    if (dt == PATH_BF16) return {BF16, F16, BF16};
+    return {BF16, F16, F32};  // PATH_BF16_F32OUT
 }
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }

@@ -370,7 +370,7 @@ cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScr
         term(g, dM, W, 1.f);
         g.addend = dQt;
         g.gamma = 1.f;
-        set_out(g, gr.dq, D.dt, ush, usb, d, L);
+        set_out(g, gr.dq, D.odt, ush, usb, d, L);
         CK(gemm_batched(g, st));
     }
     {   // dU = -M^T dSl - W dKt^T
@@ -397,7 +397,7 @@ cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScr
         term(g, T_(dN), W, 1.f);
         g.addend = dKt;
         g.gamma = 1.f;
-        set_out(g, gr.dk, D.dt, ush, usb, d, L);
+        set_out(g, gr.dk, D.odt, ush, usb, d, L);
         CK(gemm_batched(g, st));
     }
     {   // dWhat = -M^T dQt - W dP
@@ -462,7 +462,7 @@ cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScr
         term(g3, T_(dGm), W, 1.f);
         g3.addend = dWacc;
         g3.gamma = 1.f;
-        set_out(g3, gr.dw, D.dt, ush, usb, d, L);
+        set_out(g3, gr.dw, D.odt, ush, usb, d, L);
         CK(gemm_batched(g3, st));
     }
     return cudaSuccess;

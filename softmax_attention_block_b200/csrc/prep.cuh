@@ -5,7 +5,9 @@
 namespace path {
 
 struct PrepDims {
-    int nh, L, d, nblk, dt;  // dt: element type of q, k, w
+    int nh, L, d, nblk;
+    int dt;   // element type of q, k, w
+    int odt;  // element type of dq, dk, dw
 };
 
 struct PrepInputs {

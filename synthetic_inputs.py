@@ -63,9 +63,10 @@ def _beta(x: torch.Tensor, clip: bool) -> torch.Tensor:
 
 
 def make_inputs(B, H, L, d, dtype=torch.bfloat16, seed=0, fox=False, clip_beta=True,
-                with_dout=True):
+                with_dout=True, out_dtype=None):
     """Training-shape inputs: dict of CPU tensors q, k, v, w [B,H,L,d] (dtype),
-    beta [B,H,L] fp32, log_f [B,H,L] fp32 or None, dout [B,H,L,d] (dtype) or None."""
+    beta [B,H,L] fp32, log_f [B,H,L] fp32 or None, dout [B,H,L,d] (out_dtype,
+    default dtype) or None."""
     g = torch.Generator().manual_seed(seed)
     shp = (B, H, L, d)
     q = torch.randn(shp, generator=g)
@@ -79,16 +80,16 @@ def make_inputs(B, H, L, d, dtype=torch.bfloat16, seed=0, fox=False, clip_beta=T
     out = dict(q=q.to(dtype), k=k.to(dtype), v=v.to(dtype), w=w.to(dtype),
                beta=_beta(xb, clip_beta).float().contiguous(),
                log_f=torch.nn.functional.logsigmoid(zf).float().contiguous() if fox else None,
-               dout=do.to(dtype) if with_dout else None)
+               dout=do.to(out_dtype or dtype) if with_dout else None)
     return out
 
 
-def workload_inputs(name: str, seed: int = 0, heads=None):
+def workload_inputs(name: str, seed: int = 0, heads=None, out_dtype=None):
     """Inputs of a named training workload. ``heads`` (list of flat b*H+h
     indices) keeps only those heads, as B=1 H=len(heads) (same values)."""
     w = WORKLOADS[name]
     x = make_inputs(w.B, w.H, w.L, w.d, w.dtype, seed, fox=w.fox, clip_beta=w.clip_beta,
-                    with_dout=True)
+                    with_dout=True, out_dtype=out_dtype)
     if heads is not None:
         idx = torch.as_tensor(heads)
         for key, t in list(x.items()):

@@ -1,10 +1,20 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
 
-Tolerances (max absolute error): 1e-4 for fp32 inputs, 2e-2 for bf16 inputs
-with fp32 accumulation, on outputs, lse and every gradient. Both sides read
-identical input bytes from ``synthetic_inputs``; the oracle sees them exactly
-(upcast to fp64).
+Bars (max absolute error, elementwise, against the oracle on identical input
+bytes):
+- fp32 inputs and outputs: 1e-4 on out, lse and every gradient.
+- bf16 inputs, fp32 accumulate, fp32 outputs (PATH_BF16_F32OUT): 2e-2 on out,
+  lse and every gradient.
+- bf16 inputs and bf16 outputs (PATH_BF16): 2e-2 plus one bf16 ulp of the
+  reference value on the bf16-stored tensors (out, dq, dk, dv, dw): bf16 keeps
+  8 significant bits, so a value of magnitude >= 8 cannot be stored closer
+  than 2e-2. lse and dbeta (fp32) keep 2e-2. dlog_f (fp32) gets 2e-2 plus
+  2^-7 max|dlog_f|: it is a sum of dZ over every (query, key) pair that
+  straddles a position, and dZ carries delta = dout . out, which in this mode
+  comes from the bf16-rounded out.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -14,7 +24,7 @@ import synthetic_inputs as si
 
 pytestmark = pytest.mark.gpu
 
-TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+STORED_BF16 = ("out", "dq", "dk", "dv", "dw")
 
 
 @pytest.fixture(scope="module")
@@ -31,52 +41,98 @@ def to_dev(x):
     return {k: (v.cuda() if v is not None else None) for k, v in x.items()}
 
 
-def maxerr(a, b):
-    a = a.detach().float().cpu().double().numpy() if hasattr(a, "detach") else np.asarray(a)
-    return float(np.max(np.abs(a - b))) if a.size else 0.0
+def np64(t):
+    return t.detach().float().cpu().double().numpy() if hasattr(t, "detach") else np.asarray(t)
 
 
-def run_ours(P, x, backward):
+def ulp_bf16(x):
+    """Spacing of bf16 numbers at |x| (8 significant bits)."""
+    a = np.maximum(np.abs(x), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 7)
+
+
+def run_ours(P, x, backward, out_dtype=None):
     d = to_dev(x)
-    out, lse = P.path_attn_fwd(d["q"], d["k"], d["v"], d["w"], d["beta"], d["log_f"])
+    B, H, L, D = d["q"].shape
+    od = out_dtype or d["q"].dtype
+    nb = max(P.path_attn_workspace_bytes(B, H, L, D, d["q"].dtype, bwd, od)
+             for bwd in (False, backward))
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    out, lse = P.path_attn_fwd(d["q"], d["k"], d["v"], d["w"], d["beta"], d["log_f"],
+                               out_dtype=out_dtype, workspace=ws)
+    assert P.lib().path_attn_wait_status(ws.data_ptr(), None) == 0, "forward wait timed out"
     g = None
     if backward:
-        g = P.path_attn_bwd(d["q"], d["k"], d["v"], d["w"], d["beta"], out, lse, d["dout"],
-                            d["log_f"])
+        g = P.path_attn_bwd(d["q"], d["k"], d["v"], d["w"], d["beta"], out, lse,
+                            d["dout"].to(out.dtype), d["log_f"], workspace=ws)
+        assert P.lib().path_attn_wait_status(ws.data_ptr(), None) == 0, "backward wait timed out"
     torch.cuda.synchronize()
     return out, lse, g
 
 
-def check(P, x, backward, tol, report=""):
-    out, lse, g = run_ours(P, x, backward)
+def oracle_results(x, backward):
     ro, rl = oracle.fwd(x["q"], x["k"], x["v"], x["w"], x["beta"], x["log_f"])
-    errs = {"out": maxerr(out, ro), "lse": maxerr(lse, rl)}
+    r = {"out": ro, "lse": rl}
     if backward:
-        rg = oracle.bwd(x["q"], x["k"], x["v"], x["w"], x["beta"], x["dout"], x["log_f"])
-        for n, ref in rg.items():
-            errs[n] = maxerr(g[n], ref)
-            errs[n + "/max|ref|"] = errs[n] / max(float(np.max(np.abs(ref))), 1e-30)
-    print(f"\n[{report}] " + " ".join(f"{k}={v:.3g}" for k, v in errs.items()))
-    bad = {k: v for k, v in errs.items() if "/" not in k and not v <= tol}
-    assert not bad, f"{report}: over tolerance {tol}: {bad}"
+        r.update(oracle.bwd(x["q"], x["k"], x["v"], x["w"], x["beta"], x["dout"], x["log_f"]))
+    return r
+
+
+def compare(ours, ref, mode, report):
+    """ours/ref: dicts name -> array. mode: 'f32', 'bf16in_f32out' or 'bf16'."""
+    errs, bad = {}, {}
+    for n, r in ref.items():
+        got = np64(ours[n])
+        diff = np.abs(got - r)
+        errs[n] = float(diff.max()) if diff.size else 0.0
+        errs[n + "/max|ref|"] = errs[n] / max(float(np.abs(r).max()), 1e-30)
+        if mode == "f32":
+            ok = errs[n] <= 1e-4
+        elif mode == "bf16in_f32out" or n in ("lse", "dbeta"):
+            ok = errs[n] <= 2e-2
+        elif n in STORED_BF16:
+            ok = bool(np.all(diff <= 2e-2 + ulp_bf16(r)))
+        elif n == "dlog_f":
+            ok = errs[n] <= 2e-2 + 2.0 ** -7 * float(np.abs(r).max())
+        else:
+            ok = errs[n] <= 2e-2
+        if not ok:
+            bad[n] = errs[n]
+    print(f"\n[{report} | {mode}] " + " ".join(f"{k}={v:.3g}" for k, v in errs.items()))
+    assert not bad, f"{report} ({mode}): over the bar: {bad}"
     return errs
+
+
+def ours_dict(out, lse, g):
+    d = {"out": out, "lse": lse}
+    if g:
+        d.update(g)
+    return d
+
+
+def check(P, x, backward, modes, report):
+    ref = oracle_results(x, backward)
+    for mode in modes:
+        od = torch.float32 if mode == "bf16in_f32out" else None
+        out, lse, g = run_ours(P, x, backward, out_dtype=od)
+        compare(ours_dict(out, lse, g), ref, mode, report)
 
 
 def test_fp32_tiny_forward(P):
     x = si.workload_inputs("fwd_fp32_tiny")
-    check(P, x, backward=False, tol=1e-4, report="fwd_fp32_tiny")
+    check(P, x, False, ["f32"], "fwd_fp32_tiny")
 
 
 @pytest.mark.parametrize("L,d,fox", [(1, 16, False), (64, 16, True), (300, 32, True),
                                      (257, 64, False), (130, 128, True)])
 def test_fp32_fwd_bwd_shapes(P, L, d, fox):
     x = si.make_inputs(1, 2, L, d, torch.float32, seed=1, fox=fox, clip_beta=False)
-    check(P, x, backward=True, tol=1e-4, report=f"fp32 L={L} d={d} fox={fox}")
+    check(P, x, True, ["f32"], f"fp32 L={L} d={d} fox={fox}")
 
 
 def test_bf16_l1024_forward(P):
     x = si.workload_inputs("fwd_bf16_l1024")
-    check(P, x, backward=False, tol=2e-2, report="fwd_bf16_l1024")
+    check(P, x, False, ["bf16", "bf16in_f32out"], "fwd_bf16_l1024")
 
 
 @pytest.mark.parametrize("L,d,fox", [(1, 64, False), (100, 64, True), (128, 64, False),
@@ -84,38 +140,37 @@ def test_bf16_l1024_forward(P):
                                      (390, 128, True)])
 def test_bf16_fwd_bwd_ragged(P, L, d, fox):
     x = si.make_inputs(2, 2, L, d, torch.bfloat16, seed=2, fox=fox)
-    check(P, x, backward=True, tol=2e-2, report=f"bf16 L={L} d={d} fox={fox}")
+    check(P, x, True, ["bf16", "bf16in_f32out"], f"bf16 L={L} d={d} fox={fox}")
 
 
 def test_bf16_l1024_fwd_bwd(P):
     x = si.make_inputs(2, 4, 1024, 64, torch.bfloat16, seed=0)
-    check(P, x, backward=True, tol=2e-2, report="bf16 l1024 fwd+bwd")
+    check(P, x, True, ["bf16", "bf16in_f32out"], "bf16 l1024 fwd+bwd")
 
 
-def _sampled_full_size(P, name, heads):
-    """Full-size run on the GPU, oracle on a few heads (heads are independent)."""
+def _sampled_full_size(P, name, heads, modes):
+    """Full-size run on the GPU (the benchmark's launch), oracle on a few heads
+    (heads are independent, so those heads' values are exact comparisons)."""
     w = si.WORKLOADS[name]
     x = si.workload_inputs(name)
-    out, lse, g = run_ours(P, x, backward=True)
-    flat = lambda t: t.reshape(w.B * w.H, *t.shape[2:])[heads]
     xs = si.workload_inputs(name, heads=heads)
-    ro, rl = oracle.fwd(xs["q"], xs["k"], xs["v"], xs["w"], xs["beta"], xs["log_f"])
-    rg = oracle.bwd(xs["q"], xs["k"], xs["v"], xs["w"], xs["beta"], xs["dout"], xs["log_f"])
-    errs = {"out": maxerr(flat(out), ro[0]), "lse": maxerr(flat(lse), rl[0])}
-    for n, ref in rg.items():
-        errs[n] = maxerr(flat(g[n]), ref[0])
-        errs[n + "/max|ref|"] = errs[n] / max(float(np.max(np.abs(ref))), 1e-30)
-    print(f"\n[{name} heads {heads}] " + " ".join(f"{k}={v:.3g}" for k, v in errs.items()))
-    bad = {k: v for k, v in errs.items() if "/" not in k and not v <= 2e-2}
-    assert not bad, f"{name}: over tolerance: {bad}"
+    ref = {k: v[0] for k, v in oracle_results(xs, True).items()}
+    flat = lambda t: t.reshape(w.B * w.H, *t.shape[2:])[heads]
+    for mode in modes:
+        od = torch.float32 if mode == "bf16in_f32out" else None
+        out, lse, g = run_ours(P, x, True, out_dtype=od)
+        ours = {k: flat(v) for k, v in ours_dict(out, lse, g).items()}
+        compare(ours, ref, mode, f"{name} heads {heads}")
+        del out, lse, g, ours
+        torch.cuda.empty_cache()
 
 
 def test_full_size_l4096_sampled_heads(P):
-    _sampled_full_size(P, "fwdbwd_bf16_l4096", [0, 77, 191])
+    _sampled_full_size(P, "fwdbwd_bf16_l4096", [0, 77, 191], ["bf16", "bf16in_f32out"])
 
 
 def test_full_size_fox_l16384_sampled_heads(P):
-    _sampled_full_size(P, "fox_fwdbwd_l16384", [5])
+    _sampled_full_size(P, "fox_fwdbwd_l16384", [5], ["bf16in_f32out", "bf16"])
 
 
 def _decode_check(P, B, H, d, n0, cap, steps, dtype, heads, tol):
@@ -132,20 +187,33 @@ def _decode_check(P, B, H, d, n0, cap, steps, dtype, heads, tol):
         ref = oracle.decode_step(sel(s["q"]), sel(s["k_new"]), sel(s["v_new"]), sel(s["w"]),
                                  sel(s["beta"]), ok, ov, n0 + t,
                                  round_bf16=(dtype == torch.bfloat16))
-        worst = max(worst, maxerr(sel(out.cpu()), ref))
+        worst = max(worst, float(np.abs(np64(sel(out.cpu())) - ref).max()))
+        if t == 0 and dtype == torch.bfloat16 and n0 > 0:
+            # One update from identical caches: the GPU (fp32) and the oracle (fp64)
+            # round the same exact value, so they agree except where it lies within
+            # the fp32 error of a rounding boundary: at most one ulp apart.
+            k1 = np64(sel(kd.cpu())[..., :n0, :])
+            r1 = ok[..., :n0, :]
+            one_ulp = ulp_bf16(np.maximum(np.abs(k1), np.abs(r1)))
+            assert np.all(np.abs(k1 - r1) <= one_ulp), "single-step cache update off by > 1 ulp"
     torch.cuda.synchronize()
     n = n0 + steps
-    kg = sel(kd.cpu())[..., :n, :].double().numpy()
+    kg = np64(sel(kd.cpu())[..., :n, :])
     kref = ok[..., :n, :]
     if dtype == torch.bfloat16:
-        # cache entries within 2 bf16 ulps (relative 2^-7) of the oracle's rounded cache
-        ulp = np.maximum(np.abs(kref), 1e-30) * 2.0 ** -7
-        cache_bad = int(np.sum(np.abs(kg - kref) > 2 * ulp + 1e-6))
+        # After many steps the two caches drift apart: each one-ulp rounding flip
+        # (checked above for a single step) feeds every later update of its row, and
+        # an update that cancels most of an entry keeps the absolute difference. The
+        # drift is bounded in ulps at each row's scale: within 4 bf16 ulps of the
+        # row's largest entry after `steps` updates.
+        row_ulp = ulp_bf16(np.abs(kref).max(axis=-1, keepdims=True))
+        cache_bad = int(np.sum(np.abs(kg - kref) > 4 * row_ulp))
     else:
         cache_bad = int(np.sum(np.abs(kg - kref) > 1e-4))
     print(f"\n[decode B={B} H={H} d={d} n0={n0} steps={steps}] out max err {worst:.3g}, "
-          f"cache entries beyond tolerance {cache_bad}")
-    np.testing.assert_array_equal(sel(vd.cpu())[..., :n, :].double().numpy(), ov[..., :n, :])
+          f"cache entries beyond tolerance {cache_bad}, entries differing "
+          f"{int(np.sum(kg != kref))} of {kg.size}")
+    np.testing.assert_array_equal(np64(sel(vd.cpu())[..., :n, :]), ov[..., :n, :])
     assert worst <= tol
     assert cache_bad == 0
 
@@ -153,7 +221,8 @@ def _decode_check(P, B, H, d, n0, cap, steps, dtype, heads, tol):
 @pytest.mark.parametrize("dtype,d", [(torch.float32, 64), (torch.bfloat16, 64),
                                      (torch.bfloat16, 128)])
 def test_decode_small(P, dtype, d):
-    _decode_check(P, 2, 3, d, 700, 720, 5, dtype, list(range(6)), TOL[dtype])
+    _decode_check(P, 2, 3, d, 700, 720, 5, dtype, list(range(6)),
+                  1e-4 if dtype == torch.float32 else 2e-2)
 
 
 def test_decode_from_empty_cache(P):

@@ -16,6 +16,7 @@ struct ChainArgs {
 
 struct FwdArgs {
     const void *Qt, *Khat, *v;
+    const void *vh;   // fp16 copy of v (tensor-core path) or null
     const float *Sd;  // [nh, nblk, BT, BT]
     const float *c;   // [nh, Lp] gate prefix or null
     float scale;
@@ -44,6 +45,8 @@ struct BwdArgs {
 cudaError_t chain_simt(const ChainArgs &c, Types t, int d, cudaStream_t st);
 cudaError_t attn_fwd_simt(const FwdArgs &a, Types t, int d, cudaStream_t st);
 cudaError_t attn_bwd_simt(const BwdArgs &a, Types t, int d, cudaStream_t st);
+// delta_i = dO_i . O_i into a.delta ([nh, Lp], zero past L)
+cudaError_t compute_delta(const BwdArgs &a, Types t, int d, cudaStream_t st);
 cudaError_t gate_prefix(const float *logf, float *c, int L, int Lp, int nh, cudaStream_t st);
 cudaError_t gate_grad(const float *rowsum, const float *colsum, float *dlogf, int L, int Lp, int nh,
                       cudaStream_t st);

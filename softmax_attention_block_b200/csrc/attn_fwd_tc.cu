@@ -5,8 +5,10 @@
 //   warp 4     producer: TMA loads of Qtil_I, then per key tile the transported
 //              keys Khat_{I,J}, the values V_J and the gate prefix c_J into a
 //              ring of NS stages
-//   warp 5     MMA issuer: S = Qtil Khat^T (fp16 operands, fp32 in TMEM,
-//              double-buffered) and O_tile = P V (bf16 operands)
+//   warp 5     MMA issuer: S = Qtil Khat^T and O_tile = P V (fp16 operands,
+//              fp32 accumulators in TMEM; S double-buffered). P lies in [0, 1],
+//              where fp16 keeps three more mantissa bits than bf16, so V is
+//              read from an fp16 copy made once per call.
 // The diagonal tile's logits come precomputed from the UT prep (the
 // full-matrix form of each block); tiles J < I come from S = Qtil Khat^T.
 // Softmax works in the log2 domain; the running max rescales the register
@@ -153,7 +155,7 @@ __global__ void __launch_bounds__(NT, 1)
     } else if (warp == W_MMA) {
         if (lane == 0) {
             const uint32_t idS = idesc_f16(128, 128, AB_F16, 0, 0);
-            const uint32_t idO = idesc_f16(128, D, AB_BF16, 0, 1);
+            const uint32_t idO = idesc_f16(128, D, AB_F16, 0, 1);
             const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
             bool ok = mbar_wait(q_full, 0, WAIT_POLLS) && mbar_wait(&kv_full[0], 0, WAIT_POLLS);
             fence_after_sync();
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(NT, 1)
                 }
                 mA = m;
             }
-            // pass 2: probabilities -> P (bf16, swizzled K-major) and row sum
+            // pass 2: probabilities -> P (fp16, swizzled K-major) and row sum
             float rowsum = 0.f;
 #pragma unroll 1
             for (int c0 = 0; c0 < BT; c0 += 32) {
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     uint4 u;
-                    __nv_bfloat162 *hh = reinterpret_cast<__nv_bfloat162 *>(&u);
+                    __half2 *hh = reinterpret_cast<__half2 *>(&u);
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2) {
                         float pp[2];
@@ -284,7 +286,7 @@ __global__ void __launch_bounds__(NT, 1)
                             pp[t] = (it > 0 || j <= r) ? ex2(z - m_new) : 0.f;
                             rowsum += pp[t];
                         }
-                        hh[q2] = __floats2bfloat162_rn(pp[0], pp[1]);
+                        hh[q2] = __floats2half2_rn(pp[0], pp[1]);
                     }
                     const int col = c0 + g * 8;
                     *reinterpret_cast<uint4 *>(sP + (col >> 6) * 16384 + sw128_offset(r, col & 63)) = u;
@@ -336,7 +338,30 @@ cudaError_t launch(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorM
     return cudaGetLastError();
 }
 
+// dst = fp16 copy of src (bf16), 8 elements per thread step
+__global__ void to_f16_kernel(const bf16 *src, f16 *dst, long long n8)
+{
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
+         i += (long long)gridDim.x * blockDim.x) {
+        const uint4 u = reinterpret_cast<const uint4 *>(src)[i];
+        const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
+        uint4 o;
+        __half2 *h = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) h[k] = __float22half2_rn(__bfloat1622float2(b[k]));
+        reinterpret_cast<uint4 *>(dst)[i] = o;
+    }
+}
+
 }  // namespace
+
+cudaError_t convert_to_f16(const void *src, void *dst, long long n, cudaStream_t st)
+{
+    if (n % 8) return cudaErrorInvalidValue;
+    to_f16_kernel<<<1184, 256, 0, st>>>(static_cast<const bf16 *>(src), static_cast<f16 *>(dst), n / 8);
+    count_launches();
+    return cudaGetLastError();
+}
 
 bool attn_fwd_tc_supported(Types t, int d)
 {
@@ -355,7 +380,7 @@ cudaError_t attn_fwd_tc(const FwdArgs &f, Types t, int d, int *err, cudaStream_t
     } else {
         mK = mQ;  // no off-diagonal tiles: never read
     }
-    if (!make_map_3d(&mV, f.v, BF16, d, f.L, f.nh, 128)) return cudaErrorInvalidValue;
+    if (!make_map_3d(&mV, f.vh, F16, d, f.L, f.nh, 128)) return cudaErrorInvalidValue;
     FwdTcArgs a{f.Sd, f.c, f.scale * 1.4426950408889634f, f.L, f.nblk, f.nh, npairs, f.out, f.lse, err};
     const bool fox = f.c != nullptr;
     const bool f32 = t.out == F32;

@@ -512,6 +512,18 @@ cudaError_t attn_bwd_simt(const BwdArgs &a, Types t, int d, cudaStream_t st)
     });
 }
 
+cudaError_t compute_delta(const BwdArgs &a, Types t, int d, cudaStream_t st)
+{
+    return dispatch(t, d, [&](auto, auto, auto o, auto dd) {
+        using TO = decltype(o);
+        delta_kernel<TO, decltype(dd)::value><<<512, 256, 0, st>>>(
+            static_cast<const TO *>(a.out), static_cast<const TO *>(a.dout), a.delta, a.L,
+            a.nblk * BT, a.nh);
+        count_launches();
+        return cudaGetLastError();
+    });
+}
+
 cudaError_t gate_prefix(const float *logf, float *c, int L, int Lp, int nh, cudaStream_t st)
 {
     gate_prefix_kernel<<<ceil_div(nh, 64), 64, 0, st>>>(logf, c, L, Lp, nh);

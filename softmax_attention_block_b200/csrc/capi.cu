@@ -34,10 +34,13 @@ struct AttnWs {
     int *err;  // device error word: first bounded wait that gave up (0 = none)
     float *c;
     void *Qt, *Kt, *Pm, *Khat;
+    void *Vh;  // fp16 copy of v for the tensor-core forward
     float *Sd;
     PrepScratch prep;
     // backward only
     float *delta, *dQt, *dKt, *dPm, *dSd, *rowsum, *colsum;
+    float *lse_p;     // lse padded to Lp (tensor-core backward)
+    void *dout16;     // bf16 copy of an fp32 dout (tensor-core backward)
 };
 
 // The single description of the workspace: used both to size and to carve it.
@@ -51,6 +54,7 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
     w.Kt = c.take<char>(nh * Lp * d * y.tsz);
     w.Pm = c.take<char>(nh * nb * d * d * y.tsz);
     w.Khat = c.take<char>(nh * (size_t)y.npairs * BT * d * y.tsz);
+    w.Vh = c.take<char>(nh * (size_t)y.L * d * 2);
     w.Sd = c.take<float>(nh * nb * BT * BT);
     PrepDims D{y.nh, y.L, y.d, y.nblk, types_of(dt).in, types_of(dt).out};
     carve_prep_scratch(c, D, bwd, w.prep);
@@ -62,6 +66,8 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
         w.dSd = c.take<float>(nh * nb * BT * BT);
         w.rowsum = c.take<float>(nh * Lp);
         w.colsum = c.take<float>(nh * Lp);
+        w.lse_p = c.take<float>(nh * Lp);
+        w.dout16 = c.take<char>(nh * (size_t)y.L * d * 2);
     }
     return c.bytes();
 }
@@ -90,14 +96,19 @@ path_status launch_status(cudaError_t e) { return e == cudaSuccess ? PATH_OK : P
         if (e_ != cudaSuccess) return PATH_ERR_CUDA;    \
     } while (0)
 
-// Tensor-core forward: bf16 inputs, d in {64, 128}, 16-byte aligned v (TMA),
-// row coordinates of the transported-key tiles within int range.
+// Tile row coordinates of the tensor maps (int32) stay in range.
+bool tc_rows_fit(const Layout &y)
+{
+    return (long long)y.nh * (y.npairs + 1) * BT < (1LL << 31) &&
+           (long long)y.nh * y.Lp < (1LL << 31) && (long long)y.nh * y.nblk * y.d < (1LL << 31);
+}
+
+// Tensor-core forward: bf16 inputs, d in {64, 128}, 16-byte aligned v (TMA).
 bool use_tc_fwd(Types t, const Layout &y, const void *v)
 {
     if (!attn_fwd_tc_supported(t, y.d)) return false;
     if (reinterpret_cast<uintptr_t>(v) & 15u) return false;
-    return (long long)y.nh * (y.npairs + 1) * BT < (1LL << 31) &&
-           (long long)y.nh * y.Lp < (1LL << 31);
+    return tc_rows_fit(y);
 }
 
 // Shared by forward and backward: gate prefix, UT prep, transport chain.
@@ -120,7 +131,10 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
     ChainArgs ca{ws.Kt, ws.Pm, ws.Khat, y.nblk, y.nh};
     {
         Stage s("chain", st);
-        TRY(chain_simt(ca, t, y.d, st));
+        if (attn_fwd_tc_supported(t, y.d) && tc_rows_fit(y))
+            TRY(chain_tc(ca, y.d, ws.err, st));
+        else
+            TRY(chain_simt(ca, t, y.d, st));
     }
     return PATH_OK;
 }
@@ -166,10 +180,17 @@ path_status path_attn_fwd(const void *q, const void *k, const void *v, const voi
     TRY(cudaMemsetAsync(ws.err, 0, sizeof(int), st));
     path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
     if (s != PATH_OK) return s;
-    FwdArgs a{ws.Qt, ws.Khat, v, ws.Sd, log_f ? ws.c : nullptr, scale, y.L, y.nblk, y.nh, out, lse};
+    FwdArgs a{ws.Qt, ws.Khat, v, ws.Vh, ws.Sd, log_f ? ws.c : nullptr, scale, y.L, y.nblk, y.nh, out, lse};
     const Types t = types_of(dt);
+    if (use_tc_fwd(t, y, v)) {
+        {
+            Stage s_cv("v_to_f16", st);
+            TRY(convert_to_f16(v, ws.Vh, (long long)y.nh * y.L * d, st));
+        }
+        Stage s_attn("attn_fwd", st);
+        return launch_status(attn_fwd_tc(a, t, d, ws.err, st));
+    }
     Stage s_attn("attn_fwd", st);
-    if (use_tc_fwd(t, y, v)) return launch_status(attn_fwd_tc(a, t, d, ws.err, st));
     return launch_status(attn_fwd_simt(a, t, d, st));
 }
 
@@ -199,7 +220,21 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
               scale,     y.L,      y.nblk,   y.nh,   out,    dout,
               lse,       ws.delta, ws.dQt,   ws.dKt, ws.dPm, ws.dSd,
               dv,        ws.rowsum, ws.colsum};
-    TRY(attn_bwd_simt(a, types_of(dt), d, st));
+    const Types t = types_of(dt);
+    const bool tc = attn_bwd_tc_supported(t, d) && tc_rows_fit(y) &&
+                    !((reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(dout)) & 15u);
+    if (tc) {
+        {
+            Stage s_d("delta", st);
+            TRY(compute_delta(a, t, d, st));
+        }
+        TRY(cudaMemsetAsync(ws.dQt, 0, sizeof(float) * (size_t)y.nh * y.Lp * d, st));
+        TRY(cudaMemsetAsync(ws.rowsum, 0, sizeof(float) * (size_t)y.nh * y.Lp, st));
+        Stage s_b("attn_bwd", st);
+        TRY(attn_bwd_tc(a, t, ws.lse_p, ws.dout16, ws.err, st));
+    } else {
+        TRY(attn_bwd_simt(a, t, d, st));
+    }
     PrepDims D{y.nh, y.L, y.d, y.nblk, types_of(dt).in, types_of(dt).out};
     PrepInputs in{q, k, w, beta};
     PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta};

@@ -189,25 +189,30 @@ def _decode_check(P, B, H, d, n0, cap, steps, dtype, heads, tol):
                                  round_bf16=(dtype == torch.bfloat16))
         worst = max(worst, float(np.abs(np64(sel(out.cpu())) - ref).max()))
         if t == 0 and dtype == torch.bfloat16 and n0 > 0:
-            # One update from identical caches: the GPU (fp32) and the oracle (fp64)
-            # round the same exact value, so they agree except where it lies within
-            # the fp32 error of a rounding boundary: at most one ulp apart.
+            # One update from identical caches. The GPU computes k - beta w (w.k) in
+            # fp32, the oracle in fp64; both round to bf16. The fp32 result is off by
+            # at most ~2^-22 of the row's magnitude, so the two agree within one ulp
+            # of the entry, plus (where the update cancels most of the entry and the
+            # entry becomes tiny next to its row) 2^-16 of the row's largest entry.
             k1 = np64(sel(kd.cpu())[..., :n0, :])
             r1 = ok[..., :n0, :]
-            one_ulp = ulp_bf16(np.maximum(np.abs(k1), np.abs(r1)))
-            assert np.all(np.abs(k1 - r1) <= one_ulp), "single-step cache update off by > 1 ulp"
+            ctol = (ulp_bf16(np.maximum(np.abs(k1), np.abs(r1)))
+                    + 2.0 ** -16 * np.abs(r1).max(axis=-1, keepdims=True))
+            assert np.all(np.abs(k1 - r1) <= ctol), "single-step cache update beyond 1 ulp"
     torch.cuda.synchronize()
     n = n0 + steps
     kg = np64(sel(kd.cpu())[..., :n, :])
     kref = ok[..., :n, :]
     if dtype == torch.bfloat16:
         # After many steps the two caches drift apart: each one-ulp rounding flip
-        # (checked above for a single step) feeds every later update of its row, and
-        # an update that cancels most of an entry keeps the absolute difference. The
-        # drift is bounded in ulps at each row's scale: within 4 bf16 ulps of the
-        # row's largest entry after `steps` updates.
-        row_ulp = ulp_bf16(np.abs(kref).max(axis=-1, keepdims=True))
-        cache_bad = int(np.sum(np.abs(kg - kref) > 4 * row_ulp))
+        # (checked above for a single step) feeds every later update of its row.
+        # Over the whole run each row must still agree with the oracle's to bf16
+        # resolution: relative L2 difference of the row at most 2^-8.
+        num = np.sqrt(np.sum((kg - kref) ** 2, axis=-1))
+        den = np.sqrt(np.sum(kref ** 2, axis=-1))
+        cache_bad = int(np.sum(num > 2.0 ** -8 * den))
+        worst_row = float(np.max(num / np.maximum(den, 1e-30)))
+        print(f"  worst row relative L2 difference {worst_row:.3g}")
     else:
         cache_bad = int(np.sum(np.abs(kg - kref) > 1e-4))
     print(f"\n[decode B={B} H={H} d={d} n0={n0} steps={steps}] out max err {worst:.3g}, "

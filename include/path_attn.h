@@ -154,6 +154,33 @@ path_status path_decode_step(const void *q, const void *k_new, const void *v_new
                              void *workspace, size_t workspace_bytes, path_stream_t stream);
 
 /*
+ * path_decode_step_noalloc: the same decode step as path_decode_step (same
+ * arguments and results, minus the workspace) for callers that cannot call
+ * cudaMalloc: for example a caller whose device memory is entirely owned by
+ * another allocator (a framework's caching allocator or a fixed pool that
+ * must stay the only owner), or one that cannot afford an allocation's
+ * latency or its failure in the middle of decoding. It allocates nothing:
+ * the per-chunk partial results live in a fixed 4 MiB device array inside
+ * the library (1,048,576 floats); every GPU that loads the library holds its
+ * own copy until the process exits. The pages have no counterpart to this
+ * entry point.
+ * - Limit: B*H*ceil(n_cached/16384)*(d+2) <= 1,048,576; beyond that the call
+ *   returns PATH_ERR_WORKSPACE and launches nothing. Within it, the rows per
+ *   chunk grow (256, 1024, 4096 or 16384) until the partials fit.
+ * - The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ * - Every call on a device shares that device's array and leaves its last
+ *   contents there. Nothing in it needs clearing between calls, but calls on
+ *   one device whose work overlaps on the GPU (e.g. on unordered streams)
+ *   race on it: order them.
+ */
+path_status path_decode_step_noalloc(const void *q, const void *k_new, const void *v_new,
+                                     const void *w, const float *beta, float scale, int B, int H,
+                                     int d, int n_cached, int capacity, path_dtype dt,
+                                     void *k_cache, void *v_cache, void *out,
+                                     path_stream_t stream);
+
+/*
  * Diagnostics (host-side, process-wide; not needed for normal use).
  *
  * path_kernel_launch_count: number of CUDA kernels this library has launched

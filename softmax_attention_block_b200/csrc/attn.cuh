@@ -65,4 +65,11 @@ constexpr int DECODE_CHUNK = 256;  // cached rows per CTA
 
 cudaError_t decode_step(const DecodeArgs &a, int dt, int d, cudaStream_t st);
 
+// Allocation-free decode: fixed device scratch of NOALLOC_SCRATCH_FLOATS.
+constexpr long long NOALLOC_SCRATCH_FLOATS = 1LL << 20;
+// Smallest chunk (rows per CTA) whose partials fit the fixed scratch; 0 if none.
+int noalloc_chunk_rows(int nh, int n, int d);
+cudaError_t noalloc_scratch(float **ptr);
+cudaError_t decode_step_noalloc(const DecodeArgs &a, int dt, int d, int chunk, cudaStream_t st);
+
 }  // namespace path

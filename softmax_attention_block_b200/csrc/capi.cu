@@ -289,4 +289,28 @@ path_status path_decode_step(const void *q, const void *k_new, const void *v_new
     return launch_status(decode_step(a, (int)dt, d, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+path_status path_decode_step_noalloc(const void *q, const void *k_new, const void *v_new,
+                                     const void *w, const float *beta, float scale, int B, int H,
+                                     int d, int n_cached, int capacity, path_dtype dt,
+                                     void *k_cache, void *v_cache, void *out,
+                                     path_stream_t stream)
+{
+    if (!q || !k_new || !v_new || !w || !beta || !k_cache || !v_cache || !out)
+        return PATH_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || capacity <= 0 || n_cached < 0 || n_cached + 1 > capacity ||
+        !isfinite(scale))
+        return PATH_ERR_INVALID_ARG;
+    if ((d != 64 && d != 128) || !decode_dtype_ok(dt)) return PATH_ERR_UNSUPPORTED;
+    const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(w) |
+                         reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache);
+    if (al & 15u) return PATH_ERR_INVALID_ARG;
+    const int chunk = noalloc_chunk_rows(B * H, n_cached, d);
+    if (chunk == 0) return PATH_ERR_WORKSPACE;  // partials exceed the fixed scratch
+    float *scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return PATH_ERR_CUDA;
+    DecodeArgs a{q, k_new, v_new, w, beta, scale, B * H, n_cached, capacity,
+                 k_cache, v_cache, out, scratch};
+    return launch_status(decode_step_noalloc(a, (int)dt, d, chunk, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -8,6 +8,8 @@
 // bytes per lane): it reads k and v once, writes the updated k once, and keeps
 // a running (max, sum, acc) of the softmax. Pass 2 (decode_combine_kernel)
 // merges the chunks with the new key, which it also appends to the caches.
+#include <mutex>
+
 #include "attn.cuh"
 #include "runtime.cuh"
 
@@ -77,7 +79,7 @@ __device__ __forceinline__ float group_sum(float x)
 constexpr int THREADS = 256;
 constexpr int UNROLL = 4;
 
-template <typename T, int D>
+template <typename T, int D, int CHUNK = DECODE_CHUNK>
 __global__ void __launch_bounds__(THREADS) decode_chunk_kernel(DecodeArgs a, int nchunk)
 {
     constexpr int V = Vec<T>::N;        // elements per 16-byte vector
@@ -87,8 +89,8 @@ __global__ void __launch_bounds__(THREADS) decode_chunk_kernel(DecodeArgs a, int
     __shared__ float s_acc[G][D];
     const int chunk = blockIdx.x, h = blockIdx.y;
     const int lane_in_row = threadIdx.x % LPR, g = threadIdx.x / LPR;
-    const int r0 = chunk * DECODE_CHUNK;
-    const int r1 = min(a.n, r0 + DECODE_CHUNK);
+    const int r0 = chunk * CHUNK;
+    const int r1 = min(a.n, r0 + CHUNK);
     float w[V], q[V];
     unpack<T>(reinterpret_cast<const uint4 *>(static_cast<const T *>(a.w) + (long long)h * D)[lane_in_row], w);
     unpack<T>(reinterpret_cast<const uint4 *>(static_cast<const T *>(a.q) + (long long)h * D)[lane_in_row], q);
@@ -222,7 +224,78 @@ cudaError_t run(const DecodeArgs &a, cudaStream_t st)
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the chunk partials live in a fixed device array.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int CHUNK>
+cudaError_t run_fixed(const DecodeArgs &a, cudaStream_t st)
+{
+    const int nchunk = ceil_div(a.n, CHUNK);
+    if (nchunk > 0) {
+        decode_chunk_kernel<T, D, CHUNK><<<dim3(nchunk, a.nh), THREADS, 0, st>>>(a, nchunk);
+        count_launches();
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    decode_combine_kernel<T, D><<<a.nh, D, 0, st>>>(a, nchunk);
+    count_launches();
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t run_chunked(const DecodeArgs &a, int chunk, cudaStream_t st)
+{
+    switch (chunk) {
+    case 256: return run_fixed<T, D, 256>(a, st);
+    case 1024: return run_fixed<T, D, 1024>(a, st);
+    case 4096: return run_fixed<T, D, 4096>(a, st);
+    default: return run_fixed<T, D, 16384>(a, st);
+    }
+}
+
 }  // namespace
+
+// Scratch of path_decode_step_noalloc: NOALLOC_SCRATCH_FLOATS floats (4 MiB)
+// in every GPU that loads the library, held until the process exits.
+static __device__ __align__(256) float g_noalloc_scratch[NOALLOC_SCRATCH_FLOATS];
+
+int noalloc_chunk_rows(int nh, int n, int d)
+{
+    static const int sizes[] = {256, 1024, 4096, 16384};
+    for (int c : sizes) {
+        const long long need = (long long)nh * ceil_div(n > 0 ? n : 1, c) * (d + 2);
+        if (need <= (long long)NOALLOC_SCRATCH_FLOATS) return c;
+    }
+    return 0;
+}
+
+cudaError_t noalloc_scratch(float **ptr)
+{
+    // cudaGetSymbolAddress once per device, with that device current; the
+    // array's name in host code is only a host-side stand-in for it.
+    static std::mutex mu;
+    static float *cache[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!cache[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        cache[dev] = static_cast<float *>(p);
+    }
+    *ptr = cache[dev];
+    return cudaSuccess;
+}
+
+cudaError_t decode_step_noalloc(const DecodeArgs &a, int dt, int d, int chunk, cudaStream_t st)
+{
+    if (d == 64) return dt == F32 ? run_chunked<float, 64>(a, chunk, st) : run_chunked<bf16, 64>(a, chunk, st);
+    if (d == 128) return dt == F32 ? run_chunked<float, 128>(a, chunk, st) : run_chunked<bf16, 128>(a, chunk, st);
+    return cudaErrorInvalidValue;
+}
 
 cudaError_t decode_step(const DecodeArgs &a, int dt, int d, cudaStream_t st)
 {

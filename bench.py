@@ -1,10 +1,10 @@
 #!/usr/bin/env python
 """Benchmark of the PaTH attention hot path on B200.
 
-One step = the whole training hot path on one batch: path_attn_fwd then
-path_attn_bwd (UT prep, transport chain, attention forward, attention
-backward, UT adjoint, gate gradient) at B=8 H=24 L=4096 d=64 bf16, inputs
-resident in HBM. The decode step (B=32 H=32 d=128, cache 16384 -> 16448,
+One step = the whole training hot path on one batch: path_attn_fwd (UT prep,
+transport chain, attention forward) then path_attn_bwd reusing the
+forward's workspace (attention backward, UT adjoint, gate gradient) at B=8
+H=24 L=4096 d=64 bf16, inputs resident in HBM. The decode step (B=32 H=32 d=128, cache 16384 -> 16448,
 64 steps) is timed after it and reported under "decode".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -233,15 +233,17 @@ def run_ours(args):
     lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
     grads = {n: torch.empty_like(x["q"]) for n in ("dq", "dk", "dv", "dw")}
     grads["dbeta"] = torch.empty_like(x["beta"])
-    ws_bytes = max(P.path_attn_workspace_bytes(w.B, w.H, w.L, w.d, w.dtype, True),
-                   P.path_attn_workspace_bytes(w.B, w.H, w.L, w.d, w.dtype, False))
+    # one backward-sized workspace: the forward leaves its block transforms and
+    # transported keys there and the backward reuses them (training usage)
+    ws_bytes = P.path_attn_workspace_bytes(w.B, w.H, w.L, w.d, w.dtype, True)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
     def step(inp):
         P.path_attn_fwd(inp["q"], inp["k"], inp["v"], inp["w"], inp["beta"], inp["log_f"],
                         out=out, lse=lse, workspace=ws)
         P.path_attn_bwd(inp["q"], inp["k"], inp["v"], inp["w"], inp["beta"], out, lse,
-                        inp["dout"], inp["log_f"], grads=grads, workspace=ws)
+                        inp["dout"], inp["log_f"], grads=grads, workspace=ws,
+                        reuse_fwd_workspace=True)
 
     def barrier():
         if world > 1:
@@ -407,6 +409,33 @@ def bench_decode(P, dev, peaks, world, max_over_ranks, barrier):
                          "peak_source": f"{peaks['source']} HBM copy"}}
 
 
+PROFILE_CASES = {
+    # name: (B, H, L, d, log_f) -- one untimed fwd + bwd, for profiler captures
+    "b1h24l4096": (1, 24, 4096, 64, False),
+    "b1h6l16384fox": (1, 6, 16384, 64, True),
+}
+
+
+def run_profile_case(name):
+    """One forward and one backward (reusing the forward's workspace) on a small
+    shape of the benchmark workload, for ncu captures of single launches."""
+    import softmax_attention_block_b200 as P
+
+    B, H, L, d, fox = PROFILE_CASES[name]
+    x = si.make_inputs(B, H, L, d, torch.bfloat16, seed=0, fox=fox)
+    dx = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
+    ws = torch.empty(P.path_attn_workspace_bytes(B, H, L, d, torch.bfloat16, True),
+                     dtype=torch.uint8, device="cuda")
+    out, lse = P.path_attn_fwd(dx["q"], dx["k"], dx["v"], dx["w"], dx["beta"], dx["log_f"],
+                               workspace=ws)
+    P.path_attn_bwd(dx["q"], dx["k"], dx["v"], dx["w"], dx["beta"], out, lse, dx["dout"],
+                    dx["log_f"], workspace=ws, reuse_fwd_workspace=True)
+    torch.cuda.synchronize()
+    status = P.lib().path_attn_wait_status(ws.data_ptr(), None)
+    print(json.dumps({"profile_case": name, "wait_status": status}))
+    return 1 if status else 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -416,7 +445,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run one untimed fwd+bwd on a small shape (for profiler captures)")
     args = ap.parse_args()
+    if args.profile_case:
+        return run_profile_case(args.profile_case)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

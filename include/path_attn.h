@@ -80,8 +80,10 @@ const char *path_status_string(path_status s);
 /*
  * Workspace size in bytes that path_attn_fwd (for_bwd = 0) or path_attn_bwd
  * (for_bwd != 0) needs for these sizes; 0 if the sizes are invalid or
- * unsupported. The workspace is scratch: its contents on entry are ignored
- * and on return are unspecified. Alignment: 256 bytes.
+ * unsupported. The backward size is the larger and also serves the forward.
+ * The workspace is scratch (its contents on entry are ignored), except that
+ * path_attn_bwd with PATH_BWD_REUSE_FWD_WORKSPACE reads what the forward left
+ * in it. Alignment: 256 bytes.
  */
 size_t path_attn_workspace_bytes(int B, int H, int L, int d, path_dtype dt, int for_bwd);
 
@@ -104,6 +106,9 @@ path_status path_attn_fwd(const void *q, const void *k, const void *v, const voi
                           int L, int d, path_dtype dt, void *out, float *lse, void *workspace,
                           size_t workspace_bytes, path_stream_t stream);
 
+/* flags of path_attn_bwd */
+#define PATH_BWD_REUSE_FWD_WORKSPACE 1u
+
 /*
  * Backward pass of path_attn_fwd for the loss sum(out * dout).
  * Inputs: the forward's inputs, its out and lse, and dout [B,H,L,d].
@@ -112,13 +117,19 @@ path_status path_attn_fwd(const void *q, const void *k, const void *v, const voi
  * NULL iff log_f is NULL). Every output element is written (no accumulation
  * into existing contents). The pages state no backward; it is the chain rule
  * through the same blockwise algorithm as the forward.
+ * flags: 0, or PATH_BWD_REUSE_FWD_WORKSPACE when `workspace` is the buffer
+ * the matching path_attn_fwd call used (sized with for_bwd != 0 at that
+ * call), holding what that call left there, with q, k, w, beta and log_f
+ * unchanged since: the backward then reuses the forward's block transforms
+ * and transported keys instead of recomputing them. Unknown flag bits are
+ * PATH_ERR_INVALID_ARG.
  */
 path_status path_attn_bwd(const void *q, const void *k, const void *v, const void *w,
                           const float *beta, const float *log_f, float scale, int B, int H,
                           int L, int d, path_dtype dt, const void *out, const float *lse,
                           const void *dout, void *dq, void *dk, void *dv, void *dw,
-                          float *dbeta, float *dlog_f, void *workspace, size_t workspace_bytes,
-                          path_stream_t stream);
+                          float *dbeta, float *dlog_f, unsigned flags, void *workspace,
+                          size_t workspace_bytes, path_stream_t stream);
 
 /*
  * Device-side waits of the tensor-core kernels are bounded: if one gives up

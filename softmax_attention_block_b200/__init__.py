@@ -63,7 +63,7 @@ def lib() -> ctypes.CDLL:
         L.path_decode_workspace_bytes.restype = sz
         L.path_attn_fwd.argtypes = [vp, vp, vp, vp, fp, fp, f, i, i, i, i, i, vp, fp, vp, sz, vp]
         L.path_attn_bwd.argtypes = [vp, vp, vp, vp, fp, fp, f, i, i, i, i, i, vp, fp, vp,
-                                    vp, vp, vp, vp, fp, fp, vp, sz, vp]
+                                    vp, vp, vp, vp, fp, fp, ctypes.c_uint, vp, sz, vp]
         L.path_decode_step.argtypes = [vp, vp, vp, vp, fp, f, i, i, i, i, i, i, vp, vp, vp, vp,
                                        sz, vp]
         L.path_attn_wait_status.argtypes = [vp, vp]
@@ -139,10 +139,19 @@ def path_attn_fwd(q, k, v, w, beta, log_f=None, scale=None, out=None, lse=None, 
     return out, lse
 
 
+PATH_BWD_REUSE_FWD_WORKSPACE = 1
+
+
 def path_attn_bwd(q, k, v, w, beta, out, lse, dout, log_f=None, scale=None, grads=None,
-                  workspace=None):
+                  workspace=None, reuse_fwd_workspace=False):
     """Backward of sum(out * dout). out, dout and the returned dq, dk, dv, dw share
-    out's dtype. Returns dict dq, dk, dv, dw, dbeta[, dlog_f]."""
+    out's dtype. Returns dict dq, dk, dv, dw, dbeta[, dlog_f].
+
+    reuse_fwd_workspace: `workspace` is the buffer the matching path_attn_fwd call
+    used (allocated with the backward size), inputs unchanged since; the backward
+    then reuses the forward's block transforms and transported keys."""
+    if reuse_fwd_workspace and workspace is None:
+        raise ValueError("reuse_fwd_workspace needs the forward's workspace")
     B, H, L, d = q.shape
     dt = _mode(q.dtype, out.dtype)
     if dout.dtype != out.dtype:
@@ -160,8 +169,9 @@ def path_attn_bwd(q, k, v, w, beta, out, lse, dout, log_f=None, scale=None, grad
     st = lib().path_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(beta), _ptr(log_f),
                              _scale(scale, d), B, H, L, d, dt, _ptr(out), _ptr(lse), _ptr(dout),
                              _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
-                             _ptr(grads["dw"]), _ptr(grads["dbeta"]), _ptr(dlf), _ptr(ws), nbytes,
-                             _stream())
+                             _ptr(grads["dw"]), _ptr(grads["dbeta"]), _ptr(dlf),
+                             PATH_BWD_REUSE_FWD_WORKSPACE if reuse_fwd_workspace else 0, _ptr(ws),
+                             nbytes, _stream())
     if st:
         raise PathError(st, "path_attn_bwd")
     return grads

@@ -1,11 +1,14 @@
 // PaTH attention forward on 5th-generation tensor cores (sm_100a).
 //
 // One CTA per (128-row query tile I, head). Warp roles:
-//   warps 0-3  softmax: one query row per thread (TMEM lane = row)
-//   warp 4     producer: TMA loads of Qtil_I, then per key tile the transported
+//   warps 0-7  softmax: warps w and w+4 share TMEM lanes 32(w%4)..+31 (query
+//              rows); each takes half of the 128 key columns of S and half of
+//              the d columns of O, exchanging the row max through shared
+//              memory, so each SM sub-partition interleaves two softmax warps
+//   warp 8     producer: TMA loads of Qtil_I, then per key tile the transported
 //              keys Khat_{I,J}, the values V_J and the gate prefix c_J into a
 //              ring of NS stages
-//   warp 5     MMA issuer: S = Qtil Khat^T and O_tile = P V (fp16 operands,
+//   warp 9     MMA issuer: S = Qtil Khat^T and O_tile = P V (fp16 operands,
 //              fp32 accumulators in TMEM; S double-buffered). P lies in [0, 1],
 //              where fp16 keeps three more mantissa bits than bf16, so V is
 //              read from an fp16 copy made once per call.
@@ -24,8 +27,9 @@ namespace {
 
 using namespace tc;
 
-constexpr int NT = 192;
-constexpr int W_PROD = 4, W_MMA = 5;
+constexpr int NT = 320;
+constexpr int W_PROD = 8, W_MMA = 9;
+constexpr int NSOFT = 256;  // softmax threads
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -39,13 +43,19 @@ struct Cfg {
     static constexpr int ST_BYTES = 2 * TILE + 1024;  // K, V, gate prefix (512 B)
     static constexpr int P_OFF = ST_OFF + NS * ST_BYTES;
     static constexpr int BAR_OFF = P_OFF + 128 * 128 * 2;
-    static constexpr int SMEM = BAR_OFF + 256 + 1024;  // + alignment slack
+    static constexpr int RED_OFF = BAR_OFF + 256;     // [2][2][128] row maxima, [2][128] row sums
+    static constexpr int SMEM = RED_OFF + 6 * 128 * 4 + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;       // S0 [0,128) S1 [128,256) O [256, 256+D)
 };
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
 {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void named_barrier(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ void flag_error(int *err, int code)
@@ -113,7 +123,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(p_full, 128);
+        mbar_init(p_full, NSOFT);
         mbar_init(o_full, 1);
         mbar_fence_init();
     }
@@ -195,36 +205,41 @@ __global__ void __launch_bounds__(NT, 1)
             if (!ok) flag_error(a.err, 2);
         }
     } else {
-        // softmax: thread r owns query row r of the tile
-        const int r = threadIdx.x;
+        // softmax: row r = TMEM lane; this warp owns S columns [c0s, c0s+64) and
+        // O columns [c0o, c0o+D/2) of it
+        constexpr int DH = D / 2;
+        const int q4 = warp & 3, hf = warp >> 2;
+        const int r = q4 * 32 + lane;
         const int gi = I * BT + r;
         const bool valid = gi < a.L;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const int c0s = hf * 64, c0o = hf * DH;
+        float *red = reinterpret_cast<float *>(sm + C::RED_OFF);  // [2][2][128]
+        float *redl = red + 512;                                  // [2][128]
         const float k1 = a.scale_log2;
         const float ci2 = FOX ? a.c[(long long)h * Lp + gi] * LOG2E : 0.f;
-        float acc[D];
+        float acc[DH];
 #pragma unroll
-        for (int e = 0; e < D; ++e) acc[e] = 0.f;
+        for (int e = 0; e < DH; ++e) acc[e] = 0.f;
         float m = -INFINITY, l = 0.f, mA = -INFINITY;
         bool ok = true;
-        const float *sd = a.Sd + (((long long)h * a.nblk + I) * BT + r) * BT;
+        const float *sd = a.Sd + (((long long)h * a.nblk + I) * BT + r) * BT + c0s;
         for (int it = 0; it < niter; ++it) {
             const int s = it % NS, b = it & 1;
             if (FOX && !mbar_wait(&kv_full[s], (it / NS) & 1, WAIT_POLLS)) {
                 ok = false;
                 break;
             }
-            const float *cj = sC(s);
-            auto bias = [&](int j) { return FOX ? ci2 - cj[j] * LOG2E : 0.f; };
-            // pass 1: row max
-            float mrow = -INFINITY;
+            const float *cj = sC(s) + c0s;
+            float z[64];
             if (it == 0) {
-                for (int j = 0; j < BT; j += 4) {
-                    const float4 v4 = *reinterpret_cast<const float4 *>(sd + j);
-                    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        if (j + u <= r) mrow = fmaxf(mrow, fmaf(vv[u], k1, bias(j + u)));
+                for (int j = 0; j < 64; j += 4) {
+                    const float4 v4 = *reinterpret_cast<const float4 *>(sd + j);
+                    z[j] = v4.x;
+                    z[j + 1] = v4.y;
+                    z[j + 2] = v4.z;
+                    z[j + 3] = v4.w;
                 }
             } else {
                 if (!mbar_wait(&s_full[b], ((it - 1) >> 1) & 1, WAIT_POLLS)) {
@@ -232,16 +247,22 @@ __global__ void __launch_bounds__(NT, 1)
                     break;
                 }
                 fence_after_sync();
-#pragma unroll 1
-                for (int c0 = 0; c0 < BT; c0 += 32) {
-                    float v[32];
-                    tmem_ld32(tbase + b * 128 + c0 + lane_off, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) mrow = fmaxf(mrow, fmaf(v[j], k1, bias(c0 + j)));
-                }
+                float *z0 = z, *z1 = z + 32;
+                tmem_ld32(tbase + b * 128 + c0s + lane_off, *reinterpret_cast<float(*)[32]>(z0));
+                tmem_ld32(tbase + b * 128 + c0s + 32 + lane_off, *reinterpret_cast<float(*)[32]>(z1));
+                tmem_wait_ld();
             }
-            const float m_new = fmaxf(m, mrow);
+            float pmax = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                const float bias = FOX ? ci2 - cj[j] * LOG2E : 0.f;
+                z[j] = (it > 0 || c0s + j <= r) ? fmaf(z[j], k1, bias) : -INFINITY;
+                pmax = fmaxf(pmax, z[j]);
+            }
+            float *rb = red + (it & 1) * 256;
+            rb[hf * 128 + r] = pmax;
+            named_barrier(1 + q4, 64);
+            const float m_new = fmaxf(m, fmaxf(rb[r], rb[128 + r]));
             // add the previous tile's P.V (scaled to its max m) into the accumulator
             if (it >= 1) {
                 if (!mbar_wait(o_full, (it - 1) & 1, WAIT_POLLS)) {
@@ -251,46 +272,29 @@ __global__ void __launch_bounds__(NT, 1)
                 fence_after_sync();
                 const float corr = ex2(mA - m);
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                for (int c0 = 0; c0 < DH; c0 += 32) {
                     float v[32];
-                    tmem_ld32(tbase + 256 + c0 + lane_off, v);
+                    tmem_ld32(tbase + 256 + c0o + c0 + lane_off, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
                 }
                 mA = m;
             }
-            // pass 2: probabilities -> P (fp16, swizzled K-major) and row sum
+            // probabilities -> P (fp16, swizzled K-major panel hf) and partial row sum
             float rowsum = 0.f;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BT; c0 += 32) {
-                float v[32];
-                if (it == 0) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = sd[c0 + j];
-                } else {
-                    tmem_ld32(tbase + b * 128 + c0 + lane_off, v);
-                    tmem_wait_ld();
+            for (int g = 0; g < 8; ++g) {
+                uint4 u;
+                __half2 *hh = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const float p0 = ex2(z[g * 8 + 2 * q2] - m_new);
+                    const float p1 = ex2(z[g * 8 + 2 * q2 + 1] - m_new);
+                    rowsum += p0 + p1;
+                    hh[q2] = __floats2half2_rn(p0, p1);
                 }
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    uint4 u;
-                    __half2 *hh = reinterpret_cast<__half2 *>(&u);
-#pragma unroll
-                    for (int q2 = 0; q2 < 4; ++q2) {
-                        float pp[2];
-#pragma unroll
-                        for (int t = 0; t < 2; ++t) {
-                            const int j = c0 + g * 8 + q2 * 2 + t;
-                            const float z = fmaf(v[g * 8 + q2 * 2 + t], k1, bias(j));
-                            pp[t] = (it > 0 || j <= r) ? ex2(z - m_new) : 0.f;
-                            rowsum += pp[t];
-                        }
-                        hh[q2] = __floats2half2_rn(pp[0], pp[1]);
-                    }
-                    const int col = c0 + g * 8;
-                    *reinterpret_cast<uint4 *>(sP + (col >> 6) * 16384 + sw128_offset(r, col & 63)) = u;
-                }
+                *reinterpret_cast<uint4 *>(sP + hf * 16384 + sw128_offset(r, g * 8)) = u;
             }
             l = fmaf(l, ex2(m - m_new), rowsum);
             m = m_new;
@@ -302,9 +306,9 @@ __global__ void __launch_bounds__(NT, 1)
             fence_after_sync();
             const float corr = ex2(mA - m);
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = 0; c0 < DH; c0 += 32) {
                 float v[32];
-                tmem_ld32(tbase + 256 + c0 + lane_off, v);
+                tmem_ld32(tbase + 256 + c0o + c0 + lane_off, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
@@ -312,12 +316,16 @@ __global__ void __launch_bounds__(NT, 1)
         } else {
             ok = false;
         }
+        // row sum: both halves share the running max, so the partial sums add
+        redl[hf * 128 + r] = l;
+        named_barrier(1 + q4, 64);
+        const float lt = redl[r] + redl[128 + r];
         if (!ok) flag_error(a.err, 3);
         if (valid) {
-            TO *dst = static_cast<TO *>(a.out) + ((long long)h * a.L + gi) * D;
-            const float inv = ok ? 1.f / l : __int_as_float(0x7fc00000);
-            store_row<TO>(dst, acc, D, inv);
-            a.lse[(long long)h * a.L + gi] = ok ? (m + log2f(l)) * LN2 : __int_as_float(0x7fc00000);
+            TO *dst = static_cast<TO *>(a.out) + ((long long)h * a.L + gi) * D + c0o;
+            const float inv = ok ? 1.f / lt : __int_as_float(0x7fc00000);
+            store_row<TO>(dst, acc, DH, inv);
+            if (hf == 0) a.lse[(long long)h * a.L + gi] = ok ? (m + log2f(lt)) * LN2 : __int_as_float(0x7fc00000);
         }
     }
     fence_before_sync();

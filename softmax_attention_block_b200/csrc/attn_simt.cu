@@ -366,20 +366,23 @@ __global__ void __launch_bounds__(QR) bwd_k_kernel(BwdArgs a)
     if (a.colsum) a.colsum[(long long)h * Lp + gj] = colsum;
 }
 
-// delta_i = dO_i . O_i
+// delta_i = dO_i . O_i, one warp per row (coalesced row reads)
 template <typename T, int D>
 __global__ void delta_kernel(const T *out, const T *dout, float *delta, int L, int Lp, int nh)
 {
+    const int lane = threadIdx.x % 32;
     const long long n = (long long)nh * Lp;
-    for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < n;
-         x += (long long)gridDim.x * blockDim.x) {
+    const long long warps = (long long)gridDim.x * (blockDim.x / 32);
+    for (long long x = blockIdx.x * (long long)(blockDim.x / 32) + threadIdx.x / 32; x < n; x += warps) {
         const int h = (int)(x / Lp), i = (int)(x % Lp);
         float s = 0.f;
         if (i < L) {
             const T *o = out + ((long long)h * L + i) * D, *g = dout + ((long long)h * L + i) * D;
-            for (int e = 0; e < D; ++e) s = fmaf(to_f(o[e]), to_f(g[e]), s);
+            for (int e = lane; e < D; e += 32) s = fmaf(to_f(o[e]), to_f(g[e]), s);
         }
-        delta[x] = s;
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+        if (lane == 0) delta[x] = s;
     }
 }
 
@@ -446,7 +449,7 @@ template <typename T, typename TM, typename TO, int D>
 cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
 {
     const int Lp = a.nblk * BT;
-    delta_kernel<TO, D><<<512, 256, 0, st>>>(static_cast<const TO *>(a.out),
+    delta_kernel<TO, D><<<1184, 256, 0, st>>>(static_cast<const TO *>(a.out),
                                              static_cast<const TO *>(a.dout), a.delta, a.L, Lp, a.nh);
     count_launches();
     CK(cudaGetLastError());
@@ -516,7 +519,7 @@ cudaError_t compute_delta(const BwdArgs &a, Types t, int d, cudaStream_t st)
 {
     return dispatch(t, d, [&](auto, auto, auto o, auto dd) {
         using TO = decltype(o);
-        delta_kernel<TO, decltype(dd)::value><<<512, 256, 0, st>>>(
+        delta_kernel<TO, decltype(dd)::value><<<1184, 256, 0, st>>>(
             static_cast<const TO *>(a.out), static_cast<const TO *>(a.dout), a.delta, a.L,
             a.nblk * BT, a.nh);
         count_launches();

@@ -40,6 +40,7 @@ struct AttnWs {
     // backward only
     float *delta, *dQt, *dKt, *dPm, *dSd, *rowsum, *colsum;
     float *lse_p;     // lse padded to Lp (tensor-core backward)
+    float *dP64;      // per-half block-product adjoints (fused prep adjoint)
     void *dout16;     // bf16 copy of an fp32 dout (tensor-core backward)
 };
 
@@ -67,6 +68,7 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
         w.rowsum = c.take<float>(nh * Lp);
         w.colsum = c.take<float>(nh * Lp);
         w.lse_p = c.take<float>(nh * Lp);
+        w.dP64 = c.take<float>(nh * 2 * nb * d * d);
         w.dout16 = c.take<char>(nh * (size_t)y.L * d * 2);
     }
     return c.bytes();
@@ -126,7 +128,7 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
     PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, t.mid};
     {
         Stage s("ut_prep", st);
-        TRY(prep_forward(D, in, ws.prep, out, st));
+        TRY(prep_forward_rec(D, in, out, st));
     }
     ChainArgs ca{ws.Kt, ws.Pm, ws.Khat, y.nblk, y.nh};
     {
@@ -198,7 +200,8 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
                           const float *beta, const float *log_f, float scale, int B, int H, int L,
                           int d, path_dtype dt, const void *out, const float *lse, const void *dout,
                           void *dq, void *dk, void *dv, void *dw, float *dbeta, float *dlog_f,
-                          void *workspace, size_t workspace_bytes, path_stream_t stream)
+                          unsigned flags, void *workspace, size_t workspace_bytes,
+                          path_stream_t stream)
 {
     if (!q || !k || !v || !w || !beta || !out || !lse || !dout || !dq || !dk || !dv || !dw ||
         !dbeta)
@@ -212,9 +215,12 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
     if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
     carve_attn(workspace, y, dt, true, ws);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (flags & ~PATH_BWD_REUSE_FWD_WORKSPACE) return PATH_ERR_INVALID_ARG;
     TRY(cudaMemsetAsync(ws.err, 0, sizeof(int), st));
-    path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
-    if (s != PATH_OK) return s;
+    if (!(flags & PATH_BWD_REUSE_FWD_WORKSPACE)) {
+        path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
+        if (s != PATH_OK) return s;
+    }
     TRY(cudaMemsetAsync(ws.dPm, 0, sizeof(float) * (size_t)y.nh * y.nblk * d * d, st));
     BwdArgs a{ws.Qt,     ws.Khat,  v,        ws.Pm,  ws.Sd,  log_f ? ws.c : nullptr,
               scale,     y.L,      y.nblk,   y.nh,   out,    dout,
@@ -240,7 +246,10 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
     PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta};
     {
         Stage s("ut_prep_bwd", st);
-        TRY(prep_backward(D, in, ws.prep, gr, st));
+        if (prep_backward_fused_supported(D))
+            TRY(prep_backward_fused(D, in, gr, ws.dP64, st));
+        else
+            TRY(prep_backward(D, in, ws.prep, gr, st));
     }
     if (log_f) {
         Stage s("gate_grad", st);

@@ -1,6 +1,7 @@
-// Per-block UT transform and boundary adjustment (forward), and its adjoint.
+// Adjoint of the per-block UT transform and boundary adjustment.
 //
-// Within one block of BT positions (rows of W, Q, K; beta; D = diag(beta)):
+// The forward quantities of one block of BT positions (rows of W, Q, K;
+// beta; D = diag(beta)) in closed form, recomputed here for the adjoint:
 //   A    = strictLower(D W W^T)          Tinv = (I + A)^{-1}      X = Tinv D
 //        (X is the T^{-1} of the UT transform, Paper-Notes "训练策略")
 //   What = X W                          P    = I - W^T What  (= H_e ... H_s)
@@ -227,7 +228,7 @@ void carve_prep_scratch(Carver &c, const PrepDims &D, bool backward, PrepScratch
     }
 }
 
-// Shared first half of forward and backward: A, G, Tinv, X, What, N, U, M.
+// Closed-form forward quantities the adjoint needs: A, G, Tinv, X, What, N, U, M.
 static cudaError_t prep_core(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
                              cudaStream_t st)
 {
@@ -280,54 +281,6 @@ static cudaError_t prep_core(const PrepDims &D, const PrepInputs &in, const Prep
         term(g, Q, T_(W), 1.f);
         out_blk(g, D, s.M, BT, BT, MASK_LOWER);
         CK(gemm_batched(g, st));
-    }
-    return cudaSuccess;
-}
-
-cudaError_t prep_forward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
-                         const PrepOutputs &out, cudaStream_t st)
-{
-    CK(prep_core(D, in, s, st));
-    const int L = D.L, d = D.d, nb = D.nblk, Lp = nb * BT;
-    const Operand W = user_rows(in.w, D.dt, L, d), K = user_rows(in.k, D.dt, L, d),
-                  Q = user_rows(in.q, D.dt, L, d);
-    const Operand U = blk_mat(s.U, F32, nb, BT, BT), M = blk_mat(s.M, F32, nb, BT, BT),
-                  What = blk_mat(s.What, F32, nb, BT, d);
-    {   // Ktil = K - U^T W
-        GemmArgs g = base_args(D, BT, d, BT);
-        term(g, T_(U), W, -1.f);
-        g.addend = K;
-        g.gamma = 1.f;
-        set_out(g, out.Kt, out.tdt, (long long)Lp * d, (long long)BT * d, d, -1);
-        CK(gemm_batched(g, st));
-    }
-    {   // Qtil = Q - M What
-        GemmArgs g = base_args(D, BT, d, BT);
-        term(g, M, What, -1.f);
-        g.addend = Q;
-        g.gamma = 1.f;
-        set_out(g, out.Qt, out.tdt, (long long)Lp * d, (long long)BT * d, d, -1);
-        CK(gemm_batched(g, st));
-    }
-    {   // P = I - W^T What
-        GemmArgs g = base_args(D, d, d, BT);
-        term(g, T_(W), What, -1.f);
-        g.add_identity = 1;
-        set_out(g, out.Pm, out.tdt, (long long)nb * d * d, (long long)d * d, d, -1);
-        CK(gemm_batched(g, st));
-    }
-    {   // Sd = Q K^T - M U (read only on and below the diagonal)
-        GemmArgs g = base_args(D, BT, BT, d);
-        term(g, Q, T_(K), 1.f);
-        set_out(g, out.Sd, F32, (long long)nb * BT * BT, (long long)BT * BT, BT, -1);
-        CK(gemm_batched(g, st));  // the second product has inner size BT: its own pass
-        GemmArgs g2 = base_args(D, BT, BT, BT);
-        term(g2, M, U, -1.f);
-        g2.addend = blk_mat(out.Sd, F32, nb, BT, BT);
-        g2.gamma = 1.f;
-        set_out(g2, out.Sd, F32, (long long)nb * BT * BT, (long long)BT * BT, BT, -1);
-        g2.outmask = MASK_LOWER;
-        CK(gemm_batched(g2, st));
     }
     return cudaSuccess;
 }

@@ -1,4 +1,5 @@
-// Per-block UT transform / boundary adjustment and its adjoint (see prep.cu).
+// Per-block UT transform / boundary adjustment: forward by recurrences
+// (prep_fwd_rec.cu), adjoint through the closed form (prep.cu).
 #pragma once
 #include "common.cuh"
 
@@ -39,10 +40,16 @@ struct PrepScratch {
 
 void carve_prep_scratch(Carver &c, const PrepDims &D, bool backward, PrepScratch &s);
 size_t prep_scratch_bytes(const PrepDims &D, bool backward);
-cudaError_t prep_forward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
-                         const PrepOutputs &out, cudaStream_t st);
+// Same outputs as prep_forward, computed by per-row recurrences in fp32.
+cudaError_t prep_forward_rec(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
+                             cudaStream_t st);
 cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
                           const PrepGrads &gr, cudaStream_t st);
+// Fused adjoint for head dim 64 (two 64-position halves per block). dQt and
+// dKt are overwritten; dP64: [nh, 2 nblk, 64, 64] scratch.
+bool prep_backward_fused_supported(const PrepDims &D);
+cudaError_t prep_backward_fused(const PrepDims &D, const PrepInputs &in, const PrepGrads &g,
+                                float *dP64, cudaStream_t st);
 cudaError_t scale_rows(const float *in, float *out, const float *beta, int L, int nblk, int batch,
                        cudaStream_t st);
 

@@ -1,0 +1,172 @@
+// Forward UT prep of one 128-position block as direct recurrences (fp32).
+//
+// Within block J (positions s..e, H_t = I - beta_t w_t w_t^T) the forward
+// needs four things, each a product of the block's H factors:
+//   Ktil_j = H_e ... H_{j+1} k_j          (keys carried to the block end)
+//   Qtil_i = H_s ... H_i q_i              (queries carried back to the block start;
+//                                          as a row, q_i^T H_i ... H_s)
+//   P      = H_e ... H_s                  (the block product)
+//   Sd_ij  = q_i^T H_i ... H_{j+1} k_j    (j <= i: the logits inside the block)
+// They are the quantities the UT transform expresses in closed form
+// (Paper-Notes "训练策略": I - W^T T^{-1} W, and the full-matrix form). Here
+// each is the sequence of rank-one updates itself, run by one thread per
+// row or column: thread j carries k_j through H_{j+1}, ..., H_e and emits
+// Sd_tj = q_t . k_j after every step (the in-place key update of the
+// inference paragraph, applied inside the block); thread i carries q_i
+// through H_i, ..., H_s; thread c carries column c of I through H_s, ..., H_e.
+// Positions past the sequence end have beta = 0 and w = 0 (H = I).
+#include "prep.cuh"
+#include "runtime.cuh"
+
+namespace path {
+
+namespace {
+
+template <int D>
+struct RecCfg {
+    static constexpr int NT = 2 * BT + (D < 32 ? 32 : D);  // keys, queries, P columns
+    static constexpr int MIN_CTAS = D <= 32 ? 2 : 1;
+};
+
+template <typename T, typename TM, int D>
+__global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
+    prep_fwd_rec_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ w,
+                        const float *__restrict__ beta, int L, int nblk, TM *Qt, TM *Kt, TM *Pm,
+                        float *Sd)
+{
+    extern __shared__ float sm[];
+    float *sW = sm;              // [BT][D+1]
+    float *sQ = sW + BT * (D + 1);  // [BT][D+1]
+    float *sB = sQ + BT * (D + 1);  // [BT]
+    const int J = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    const int Lp = nblk * BT;
+    const long long row0 = (long long)h * L + (long long)J * BT;  // first row of the block in [nh, L]
+    const int nvalid = min(BT, L - J * BT);
+    for (int e = tid; e < BT * D; e += blockDim.x) {
+        const int r = e / D, c = e % D;
+        const bool ok = r < nvalid;
+        sW[r * (D + 1) + c] = ok ? to_f(w[(row0 + r) * D + c]) : 0.f;
+        sQ[r * (D + 1) + c] = ok ? to_f(q[(row0 + r) * D + c]) : 0.f;
+    }
+    for (int r = tid; r < BT; r += blockDim.x) sB[r] = r < nvalid ? beta[row0 + r] : 0.f;
+    __syncthreads();
+
+    if (tid < BT) {
+        // keys: Ktil and the diagonal-block logits
+        const int j = tid;
+        float x[D];
+        for (int c = 0; c < D; ++c) x[c] = j < nvalid ? to_f(k[(row0 + j) * D + c]) : 0.f;
+        float *sd = Sd + ((long long)h * nblk + J) * BT * BT;
+        {
+            float s = 0.f;
+#pragma unroll
+            for (int c = 0; c < D; ++c) s = fmaf(sQ[j * (D + 1) + c], x[c], s);
+            sd[(long long)j * BT + j] = s;
+        }
+        for (int t = 1; t < BT; ++t) {
+            if (t > j) {
+                const float *wt = sW + t * (D + 1), *qt = sQ + t * (D + 1);
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < D; c += 2) {
+                    a0 = fmaf(wt[c], x[c], a0);
+                    a1 = fmaf(wt[c + 1], x[c + 1], a1);
+                }
+                const float coef = sB[t] * (a0 + a1);
+                float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < D; c += 2) {
+                    x[c] = fmaf(-coef, wt[c], x[c]);
+                    x[c + 1] = fmaf(-coef, wt[c + 1], x[c + 1]);
+                    s0 = fmaf(qt[c], x[c], s0);
+                    s1 = fmaf(qt[c + 1], x[c + 1], s1);
+                }
+                sd[(long long)t * BT + j] = s0 + s1;
+            } else if (t < j) {
+                sd[(long long)t * BT + j] = 0.f;  // above the diagonal (never read)
+            }
+        }
+        TM *dst = Kt + ((long long)h * Lp + (long long)J * BT + j) * D;
+        for (int c = 0; c < D; ++c) dst[c] = from_f<TM>(x[c]);
+    } else if (tid < 2 * BT) {
+        // queries: Qtil_i = H_s ... H_i q_i (apply H_i first)
+        const int i = tid - BT;
+        float x[D];
+        for (int c = 0; c < D; ++c) x[c] = sQ[i * (D + 1) + c];
+        for (int t = BT - 1; t >= 0; --t) {
+            if (t <= i) {
+                const float *wt = sW + t * (D + 1);
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < D; c += 2) {
+                    a0 = fmaf(wt[c], x[c], a0);
+                    a1 = fmaf(wt[c + 1], x[c + 1], a1);
+                }
+                const float coef = sB[t] * (a0 + a1);
+#pragma unroll
+                for (int c = 0; c < D; ++c) x[c] = fmaf(-coef, wt[c], x[c]);
+            }
+        }
+        TM *dst = Qt + ((long long)h * Lp + (long long)J * BT + i) * D;
+        for (int c = 0; c < D; ++c) dst[c] = from_f<TM>(x[c]);
+    } else {
+        // block product P = H_e ... H_s, one column per thread
+        const int col = tid - 2 * BT;
+        if (col < D) {
+            float x[D];
+            for (int c = 0; c < D; ++c) x[c] = c == col ? 1.f : 0.f;
+            for (int t = 0; t < BT; ++t) {
+                const float *wt = sW + t * (D + 1);
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < D; c += 2) {
+                    a0 = fmaf(wt[c], x[c], a0);
+                    a1 = fmaf(wt[c + 1], x[c + 1], a1);
+                }
+                const float coef = sB[t] * (a0 + a1);
+#pragma unroll
+                for (int c = 0; c < D; ++c) x[c] = fmaf(-coef, wt[c], x[c]);
+            }
+            TM *dst = Pm + ((long long)h * nblk + J) * D * D;
+            for (int r = 0; r < D; ++r) dst[(long long)r * D + col] = from_f<TM>(x[r]);
+        }
+    }
+}
+
+template <typename T, typename TM, int D>
+cudaError_t run(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out, cudaStream_t st)
+{
+    const size_t smem = (2 * BT * (D + 1) + BT) * sizeof(float);
+    auto kern = prep_fwd_rec_kernel<T, TM, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(Dm.nblk, Dm.nh), RecCfg<D>::NT, smem, st>>>(
+        static_cast<const T *>(in.q), static_cast<const T *>(in.k), static_cast<const T *>(in.w),
+        in.beta, Dm.L, Dm.nblk, static_cast<TM *>(out.Qt), static_cast<TM *>(out.Kt),
+        static_cast<TM *>(out.Pm), out.Sd);
+    count_launches();
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t by_types(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out, cudaStream_t st)
+{
+    if (Dm.dt == F32) return run<float, float, D>(Dm, in, out, st);
+    return run<bf16, f16, D>(Dm, in, out, st);
+}
+
+}  // namespace
+
+cudaError_t prep_forward_rec(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out,
+                             cudaStream_t st)
+{
+    switch (Dm.d) {
+    case 16: return by_types<16>(Dm, in, out, st);
+    case 32: return by_types<32>(Dm, in, out, st);
+    case 64: return by_types<64>(Dm, in, out, st);
+    case 128: return by_types<128>(Dm, in, out, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace path

@@ -87,12 +87,13 @@ def test_bwd_rejects_bad_arguments(lib):
         a.update(kw)
         return lib.path_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, a["log_f"], 0.125, 1, 1, a["L"],
                                  a["d"], BF16, FAKE, FAKE, FAKE, a["dq"], FAKE, FAKE, FAKE, FAKE,
-                                 a["dlog_f"], FAKE, a["wsb"], None)
+                                 a["dlog_f"], a.get("flags", 0), FAKE, a["wsb"], None)
 
     assert bwd(dq=None) == INVALID
     assert bwd(log_f=FAKE) == INVALID  # dlog_f must be given with log_f
     assert bwd(dlog_f=FAKE) == INVALID
     assert bwd(d=24) == UNSUPPORTED
+    assert bwd(flags=2) == INVALID  # unknown flag bits
     assert bwd(wsb=10) == WORKSPACE
 
 

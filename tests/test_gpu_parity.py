@@ -51,7 +51,7 @@ def ulp_bf16(x):
     return np.exp2(np.floor(np.log2(a)) - 7)
 
 
-def run_ours(P, x, backward, out_dtype=None):
+def run_ours(P, x, backward, out_dtype=None, reuse=False):
     d = to_dev(x)
     B, H, L, D = d["q"].shape
     od = out_dtype or d["q"].dtype
@@ -64,7 +64,8 @@ def run_ours(P, x, backward, out_dtype=None):
     g = None
     if backward:
         g = P.path_attn_bwd(d["q"], d["k"], d["v"], d["w"], d["beta"], out, lse,
-                            d["dout"].to(out.dtype), d["log_f"], workspace=ws)
+                            d["dout"].to(out.dtype), d["log_f"], workspace=ws,
+                            reuse_fwd_workspace=reuse)
         assert P.lib().path_attn_wait_status(ws.data_ptr(), None) == 0, "backward wait timed out"
     torch.cuda.synchronize()
     return out, lse, g
@@ -143,6 +144,23 @@ def test_bf16_fwd_bwd_ragged(P, L, d, fox):
     check(P, x, True, ["bf16", "bf16in_f32out"], f"bf16 L={L} d={d} fox={fox}")
 
 
+@pytest.mark.parametrize("fox", [False, True])
+def test_backward_reusing_forward_workspace(P, fox):
+    """A backward that reuses the forward's workspace gives the gradients of one
+    that recomputes the block transforms (to summation order), and both meet the bar."""
+    x = si.make_inputs(1, 3, 700, 64, torch.bfloat16, seed=4, fox=fox)
+    ref = oracle_results(x, True)
+    outs = []
+    for reuse in (False, True):
+        out, lse, g = run_ours(P, x, True, out_dtype=torch.float32, reuse=reuse)
+        compare(ours_dict(out, lse, g), ref, "bf16in_f32out", f"reuse={reuse} fox={fox}")
+        outs.append(g)
+    # dQtil accumulates across key tiles with fp32 atomics, so the two runs may
+    # differ in the last bits (summation order), not more
+    for n in outs[0]:
+        torch.testing.assert_close(outs[0][n], outs[1][n], rtol=1e-5, atol=1e-6, msg=n)
+
+
 def test_bf16_l1024_fwd_bwd(P):
     x = si.make_inputs(2, 4, 1024, 64, torch.bfloat16, seed=0)
     check(P, x, True, ["bf16", "bf16in_f32out"], "bf16 l1024 fwd+bwd")
@@ -179,6 +197,7 @@ def _decode_check(P, B, H, d, n0, cap, steps, dtype, heads, tol):
     sel = lambda t: t.reshape(B * H, *t.shape[2:])[heads].unsqueeze(0)
     ok = sel(kc).double().numpy().copy()
     ov = sel(vc).double().numpy().copy()
+    ok64, ov64 = ok.copy(), ov.copy()  # the same steps without rounding the cache
     worst = 0.0
     for t, s in enumerate(seq):
         sd = {k: v.cuda() for k, v in s.items()}
@@ -188,6 +207,9 @@ def _decode_check(P, B, H, d, n0, cap, steps, dtype, heads, tol):
                                  sel(s["beta"]), ok, ov, n0 + t,
                                  round_bf16=(dtype == torch.bfloat16))
         worst = max(worst, float(np.abs(np64(sel(out.cpu())) - ref).max()))
+        if dtype == torch.bfloat16:
+            oracle.decode_step(sel(s["q"]), sel(s["k_new"]), sel(s["v_new"]), sel(s["w"]),
+                               sel(s["beta"]), ok64, ov64, n0 + t)
         if t == 0 and dtype == torch.bfloat16 and n0 > 0:
             # One update from identical caches. The GPU computes k - beta w (w.k) in
             # fp32, the oracle in fp64; both round to bf16. The fp32 result is off by
@@ -204,15 +226,20 @@ def _decode_check(P, B, H, d, n0, cap, steps, dtype, heads, tol):
     kg = np64(sel(kd.cpu())[..., :n, :])
     kref = ok[..., :n, :]
     if dtype == torch.bfloat16:
-        # After many steps the two caches drift apart: each one-ulp rounding flip
-        # (checked above for a single step) feeds every later update of its row.
-        # Over the whole run each row must still agree with the oracle's to bf16
-        # resolution: relative L2 difference of the row at most 2^-8.
-        num = np.sqrt(np.sum((kg - kref) ** 2, axis=-1))
-        den = np.sqrt(np.sum(kref ** 2, axis=-1))
-        cache_bad = int(np.sum(num > 2.0 ** -8 * den))
-        worst_row = float(np.max(num / np.maximum(den, 1e-30)))
-        print(f"  worst row relative L2 difference {worst_row:.3g}")
+        # Over many steps the two bf16 caches drift apart: each rounding flip
+        # (one ulp, checked above for a single step) feeds every later update of
+        # its row, and rows that the updates shrink keep the absolute difference.
+        # The yardstick is the drift that bf16 rounding itself causes: the oracle's
+        # bf16 cache against the same steps in fp64. Each GPU row must be within
+        # twice that drift of the oracle's bf16 row, plus bf16 resolution (2^-8 of
+        # the row's norm).
+        rnorm = lambda a: np.sqrt(np.sum(a ** 2, axis=-1))
+        diff = rnorm(kg - kref)
+        drift = rnorm(kref - ok64[..., :n, :])
+        bound = 2.0 * drift + 2.0 ** -8 * rnorm(kref)
+        cache_bad = int(np.sum(diff > bound))
+        print(f"  worst row: diff / bound = {float(np.max(diff / bound)):.3g}; median rounding "
+              f"drift {float(np.median(drift / np.maximum(rnorm(kref), 1e-30))):.3g} of the row")
     else:
         cache_bad = int(np.sum(np.abs(kg - kref) > 1e-4))
     print(f"\n[decode B={B} H={H} d={d} n0={n0} steps={steps}] out max err {worst:.3g}, "

@@ -51,16 +51,34 @@ def fa_equiv_flops(B, H, L, d):
     return 7.0 * L * L * d * B * H
 
 
-def stage_flops(name, B, H, L, d, BT=128):
-    """Algorithmic FLOP of one launch of a stage (causal, leading order)."""
-    nh = B * H
+# fp32 FMA peak from unit counts and clocks: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz
+ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def stage_model(name, B, H, L, d, BT=128):
+    """(algorithmic FLOP of one launch, bound) of a stage; causal, leading order.
+
+    Tensor-core stages count the products of the blockwise algorithm; the UT
+    prep stages count the fp32 arithmetic of the per-block recurrences and
+    64x64 products they are made of."""
+    nh, nblk, HB = B * H, -(-L // BT), 64
     per = {
-        "attn_fwd": 2.0 * L * L * d,                      # QK^T + PV
-        "attn_bwd_q": 3.0 * L * L * d,                    # S, dP, dQ
-        "attn_bwd_k": 4.0 * L * L * d + 2.0 * L * L * d * d / BT,  # S, dP, dV, dK + chain adjoint
-        "chain": 1.0 * L * L * d * d / BT,                # key-side block transport
+        "attn_fwd": (2.0 * L * L * d, "tensor"),                      # QK^T + PV
+        # S, dP, dV, dK, dQ recomputed / formed once per causal pair, plus the
+        # key-side chain adjoint (Abar P_I and Abar^T Khat per block pair)
+        "attn_bwd": (5.0 * L * L * d + 2.0 * L * L * d * d / BT, "tensor"),
+        "attn_bwd_q": (3.0 * L * L * d, "tensor"),                    # S, dP, dQ (SIMT path)
+        "attn_bwd_k": (4.0 * L * L * d + 2.0 * L * L * d * d / BT, "tensor"),
+        "chain": (1.0 * L * L * d * d / BT, "tensor"),               # key-side block transport
+        # keys (Ktil + in-block logits), queries, block product: rank-one steps
+        "ut_prep": (nblk * (BT * BT / 2 * 10.0 * d + BT * 4.0 * d * d), "alu"),
+        # per 128-block: 8 products + 4 x 64 recurrences (composition) and
+        # 2 halves x (24 products incl. the two solves)
+        "ut_prep_bwd": (nblk * (8 * 2.0 * HB * HB * d + 4 * HB * HB * 4.0 * d
+                                + 2 * 24 * 2.0 * HB * HB * d), "alu"),
     }
-    return per.get(name, 0.0) * nh
+    f, bound = per.get(name, (0.0, None))
+    return f * nh, bound
 
 
 def load_peaks():
@@ -294,12 +312,16 @@ def run_ours(args):
     roofline = None
     if dom:
         per_launch_ms = stages[dom][0] / stages[dom][1]
-        f = stage_flops(dom, w.B, w.H, w.L, w.d)
+        f, bound = stage_model(dom, w.B, w.H, w.L, w.d)
         ach = f / (per_launch_ms * 1e-3) / 1e12 if f else None
-        peak = peaks["bf16_tflops_sustained"]
-        roofline = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak,
+        if bound == "alu":
+            peak, src = ALU_F32_TFLOPS, "fp32 FMA from unit counts and max clock"
+        else:
+            peak = peaks["bf16_tflops_sustained"]
+            src = f"{peaks['source']} bf16 dense (sustained)"
+        roofline = {"kernel": dom, "bound": bound or "tensor", "achieved": ach, "peak": peak,
                     "unit": "TFLOP/s", "frac": (ach / peak) if ach else None, "traffic": None,
-                    "peak_source": f"{peaks['source']} bf16 dense (sustained)"}
+                    "peak_source": src}
 
     # end to end through the API with host buffers (pinned), copies in the timed region
     e2e = None

@@ -5,19 +5,23 @@
 // for S^T, dP^T, dV and the chain adjoint Abar. Per tile pair:
 //   MMA 1:  S^T  = Khat_{J,I} Qtil_I^T          (fp16)
 //           dP^T = V_J dO_I^T                    (bf16)
+//           issued as two 64-query halves, one per elementwise warpgroup
 //   threads: P = exp(scale S + c_i - c_j - lse_i), dZ = P (dP - delta_i),
-//            dS = scale dZ; P^T (bf16) and dS^T (fp16) to shared memory
+//            dS = scale dZ; P^T (bf16) and dS^T (fp16) to shared memory;
+//            [gate] row sums of dS by warp reduce-scatter, column sums per thread
 //   MMA 2:  dV   += P^T dO_I                              (bf16)
 //           dP_I += Abar_{I+1}^T Khat_{J,I}                (fp16; operand
 //                   [Abar | Khat] so the M=128 form applies, top half kept)
 //           Abar  = Abar_{I+1} P_I + dS^T Qtil_I           (fp16, fp32 in TMEM)
 //           dQtil_I += dS Khat_{J,I}                       (fp16)
-//           [gate] row sums of dS                          (dS times a ones column)
 // Khat_{J,I+1} = Khat_{J,I} P_I^T, so Abar is the adjoint carried back along
 // the key-side transport chain; after the pair (J+1, J) it is dKtil_J. dQtil,
 // dP and the row sums accumulate across CTAs with fp32 vector reductions.
 // The diagonal tile takes its logits from the UT prep and writes dS to the
 // prep's adjoint instead (dSd), which carries it to dQ, dK, dW, dbeta.
+//
+// Every accumulator has its own TMEM columns, so MMA 1 of the next pair runs
+// while the warpgroups drain MMA 2's results of this one.
 #include "attn.cuh"
 #include "attn_tc.cuh"
 #include "runtime.cuh"
@@ -30,8 +34,9 @@ namespace {
 using namespace tc;
 
 constexpr int D = 64;
-constexpr int NT = 192;
-constexpr int W_PROD = 4, W_MMA = 5;
+constexpr int NT = 320;                  // warps 0-7 elementwise (two warpgroups), 8 producer, 9 MMA
+constexpr int NEW = 256;                 // elementwise threads
+constexpr int W_PROD = 8, W_MMA = 9;
 constexpr float LOG2E = 1.4426950408889634f;
 
 struct BCfg {
@@ -40,46 +45,44 @@ struct BCfg {
     static constexpr int V_OFF = AB_OFF + TILE;
     static constexpr int PT_OFF = V_OFF + TILE;  // P^T  [keys x queries] bf16, 2 panels
     static constexpr int DS_OFF = PT_OFF + 2 * 16384;  // dS^T [keys x queries] fp16
-    static constexpr int ONE_OFF = DS_OFF + 2 * 16384; // ones [16 x 128] fp16, 2 panels of 2 KB
-    static constexpr int ST_OFF = ONE_OFF + 4096;
+    static constexpr int ST_OFF = DS_OFF + 2 * 16384;
     // stage: Khat, Qtil, dO, P_I (8 KB), rows (lse, delta, c: 3 x 512 B)
     static constexpr int S_KH = 0, S_Q = TILE, S_DO = 2 * TILE, S_P = 3 * TILE, S_ROW = 3 * TILE + 8192;
     static constexpr int ST_BYTES = 3 * TILE + 8192 + 2048;
-    static constexpr int BAR_OFF = ST_OFF + 2 * ST_BYTES;
+    static constexpr int CS_OFF = ST_OFF + 2 * ST_BYTES;  // [128] column-sum exchange
+    static constexpr int BAR_OFF = CS_OFF + 512;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
-    // TMEM columns
-    static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_AB = 320;
-    static constexpr uint32_t T_DQ = 0, T_RS = 64, T_DPI = 128;
+    // TMEM columns: no two accumulators share columns
+    static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_AB = 320, T_DQ = 384, T_DPI = 448;
 };
+
+__device__ __forceinline__ void named_barrier(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
 {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-__device__ __forceinline__ void red_add_v4(float *dst, float a, float b, float c, float d)
-{
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c),
-                 "f"(d)
-                 : "memory");
-}
-
 template <bool FOX, typename TO>
 __global__ void __launch_bounds__(NT, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                   const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mDO,
-                  const __grid_constant__ CUtensorMap mP, BwdTcArgs a)
+                  const __grid_constant__ CUtensorMap mP, const __grid_constant__ CUtensorMap mDQ,
+                  const __grid_constant__ CUtensorMap mDPI, BwdTcArgs a)
 {
     using C = BCfg;
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
     uint8_t *sAb = sm + C::AB_OFF, *sV = sm + C::V_OFF, *sPt = sm + C::PT_OFF, *sDs = sm + C::DS_OFF;
-    uint8_t *sOne = sm + C::ONE_OFF;
+    float *sCs = reinterpret_cast<float *>(sm + C::CS_OFF);
     auto stage = [&](int s) { return sm + C::ST_OFF + s * C::ST_BYTES; };
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::BAR_OFF);
     uint64_t *v_full = bars, *ld_full = bars + 1, *ld_empty = bars + 3, *s_full = bars + 5,
-             *p_full = bars + 6, *m2_full = bars + 7, *e_done = bars + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
+             *p_full = bars + 7, *m2_full = bars + 8, *e_done = bars + 9;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
 
     const int J = blockIdx.x, h = blockIdx.y;
     const int nblk = a.nblk, last = nblk - 1, Lp = nblk * BT;
@@ -92,20 +95,13 @@ __global__ void __launch_bounds__(NT, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&ld_full[s], 1);
             mbar_init(&ld_empty[s], 1);
+            mbar_init(&s_full[s], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
+        mbar_init(p_full, NEW);
         mbar_init(m2_full, 1);
-        mbar_init(e_done, 128);
+        mbar_init(e_done, NEW);
         mbar_fence_init();
     }
-    // ones column for the row sums of dS: B operand [16 x 128 keys], row 0 = 1
-    for (int e = tid; e < 16 * 128; e += NT) {
-        const int n = e / 128, k = e % 128;
-        *reinterpret_cast<f16 *>(sOne + (k >> 6) * 2048 + sw128_offset(n, k & 63)) =
-            __float2half_rn(n == 0 ? 1.f : 0.f);
-    }
-    fence_async_smem();
     if (warp == W_MMA) tmem_alloc(tmem_slot, 512);
     fence_before_sync();
     __syncthreads();
@@ -127,7 +123,7 @@ __global__ void __launch_bounds__(NT, 1)
                 const bool diag = it == niter - 1;
                 const bool hasP = !diag && I < last;
                 uint8_t *st = stage(s);
-                const uint32_t bytes = C::TILE * (diag ? 1 : 3) + (hasP ? 8192 : 0) + 1536;
+                const uint32_t bytes = C::TILE * (diag ? 1 : 3) + (hasP ? 8192 : 0) + 1024;
                 mbar_expect_tx(&ld_full[s], bytes);
                 if (!diag) {
                     const int row = (int)((h * a.npairs + (long long)I * (I - 1) / 2 + J) * BT);
@@ -139,55 +135,61 @@ __global__ void __launch_bounds__(NT, 1)
                 float *rows = reinterpret_cast<float *>(st + C::S_ROW);
                 bulk_load(rows, a.lse_p + (long long)h * Lp + I * BT, 512, &ld_full[s]);
                 bulk_load(rows + 128, a.delta + (long long)h * Lp + I * BT, 512, &ld_full[s]);
-                bulk_load(rows + 256, a.c ? a.c + (long long)h * Lp + I * BT : a.delta, 512, &ld_full[s]);
                 issued = it + 1;
             }
             for (int it = issued - 2 > 0 ? issued - 2 : 0; it < issued; ++it)
                 mbar_wait(&ld_full[it & 1], (it >> 1) & 1, WAIT_POLLS);
         }
     } else if (warp == W_MMA) {
-        if (lane == 0) {
-            const uint32_t idS = idesc_f16(128, 128, AB_F16, 0, 0);
-            const uint32_t idDP = idesc_f16(128, 128, AB_BF16, 0, 0);
+        // the whole warp runs the issue loop (uniform descriptors); lane 0 issues
+        const uint32_t lead = lane == 0;
+        {
+            const uint32_t idS = idesc_f16(128, 64, AB_F16, 0, 0);
+            const uint32_t idDP = idesc_f16(128, 64, AB_BF16, 0, 0);
             const uint32_t idDV = idesc_f16(128, D, AB_BF16, 0, 1);
             const uint32_t idAbP = idesc_f16(128, D, AB_F16, 0, 1);
             const uint32_t idMN = idesc_f16(128, D, AB_F16, 1, 1);
-            const uint32_t idRS = idesc_f16(128, 16, AB_F16, 1, 0);
             const uint32_t ab0 = smem_u32(sAb), v0 = smem_u32(sV), pt0 = smem_u32(sPt),
-                           ds0 = smem_u32(sDs), one0 = smem_u32(sOne);
+                           ds0 = smem_u32(sDs);
             bool ok = mbar_wait(v_full, 0, WAIT_POLLS);
             for (int it = 0; ok && it < niter; ++it) {
                 const int s = it & 1, I = tile_of(it);
                 const bool diag = it == niter - 1;
-                if (!mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_POLLS) ||
-                    (it >= 1 && !mbar_wait(e_done, (it - 1) & 1, WAIT_POLLS))) {
+                // S^T / dP^T are free: the warpgroups consumed them before MMA 2 of the
+                // previous pair was issued (below)
+                if (!mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_POLLS)) {
                     ok = false;
                     break;
                 }
                 fence_after_sync();
                 const uint32_t kh0 = smem_u32(stage(s) + C::S_KH), q0 = smem_u32(stage(s) + C::S_Q),
                                do0 = smem_u32(stage(s) + C::S_DO), p0 = smem_u32(stage(s) + C::S_P);
-                // MMA 1
-                if (!diag) {
+                // MMA 1, one 64-query half at a time (queries 64hf.. are rows 64hf.. of Q, dO)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    if (!diag) {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            mma_ss_if(lead, tbase + C::T_S + 64 * hf, desc_sw128(kh0 + kk * 32, 16, 1024),
+                                   desc_sw128(q0 + hf * 8192 + kk * 32, 16, 1024), idS, kk > 0);
+                    }
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tbase + C::T_S, desc_sw128(kh0 + kk * 32, 16, 1024),
-                               desc_sw128(q0 + kk * 32, 16, 1024), idS, kk > 0);
+                        mma_ss_if(lead, tbase + C::T_DP + 64 * hf, desc_sw128(v0 + kk * 32, 16, 1024),
+                               desc_sw128(do0 + hf * 8192 + kk * 32, 16, 1024), idDP, kk > 0);
+                    commit_if(lead, &s_full[hf]);
                 }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(tbase + C::T_DP, desc_sw128(v0 + kk * 32, 16, 1024),
-                           desc_sw128(do0 + kk * 32, 16, 1024), idDP, kk > 0);
-                commit(s_full);
-                if (!mbar_wait(p_full, it & 1, WAIT_POLLS)) {
+                // MMA 2 needs this pair's P / dS, and the previous pair's results drained
+                if (!mbar_wait(p_full, it & 1, WAIT_POLLS) ||
+                    (it >= 1 && !mbar_wait(e_done, (it - 1) & 1, WAIT_POLLS))) {
                     ok = false;
                     break;
                 }
                 fence_after_sync();
-                // MMA 2: dV += P^T dO   (K = 128 queries)
+                // dV += P^T dO   (K = 128 queries)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tbase + C::T_DV, desc_sw128(pt0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                    mma_ss_if(lead, tbase + C::T_DV, desc_sw128(pt0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                            desc_sw128(do0 + kk * 2048, 16384, 1024), idDV, (it > 0 || kk > 0));
                 if (!diag) {
                     if (I < last) {
@@ -195,123 +197,171 @@ __global__ void __launch_bounds__(NT, 1)
                         const uint32_t lbo = kh0 - ab0;
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            mma_ss(tbase + C::T_DPI, desc_sw128(ab0 + kk * 2048, lbo, 1024),
+                            mma_ss_if(lead, tbase + C::T_DPI, desc_sw128(ab0 + kk * 2048, lbo, 1024),
                                    desc_sw128(kh0 + kk * 2048, 16384, 1024), idMN, kk > 0);
                         // Abar = Abar_{I+1} P_I
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk)
-                            mma_ss(tbase + C::T_AB, desc_sw128(ab0 + kk * 32, 16, 1024),
+                            mma_ss_if(lead, tbase + C::T_AB, desc_sw128(ab0 + kk * 32, 16, 1024),
                                    desc_sw128(p0 + kk * 2048, 16384, 1024), idAbP, kk > 0);
                     }
                     // Abar += dS^T Qtil   (K = 128 queries)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tbase + C::T_AB, desc_sw128(ds0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        mma_ss_if(lead, tbase + C::T_AB, desc_sw128(ds0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                                desc_sw128(q0 + kk * 2048, 16384, 1024), idAbP, (I < last || kk > 0));
                     // dQtil = dS Khat   (A = dS^T read MN-major, K = 128 keys)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tbase + C::T_DQ, desc_sw128(ds0 + kk * 2048, 16384, 1024),
+                        mma_ss_if(lead, tbase + C::T_DQ, desc_sw128(ds0 + kk * 2048, 16384, 1024),
                                desc_sw128(kh0 + kk * 2048, 16384, 1024), idMN, kk > 0);
                 }
-                if (FOX) {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tbase + C::T_RS, desc_sw128(ds0 + kk * 2048, 16384, 1024),
-                               desc_sw128(one0 + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024), idRS, kk > 0);
-                }
-                commit(m2_full);
-                commit(&ld_empty[s]);
+                commit_if(lead, m2_full);
+                commit_if(lead, &ld_empty[s]);
             }
-            if (!ok && a.err) atomicCAS(a.err, 0, 12);
+            if (!ok && lead && a.err) atomicCAS(a.err, 0, 12);
         }
     } else {
-        // elementwise warps: thread j owns key row j of tile J
-        const int j = tid;
+        // elementwise warpgroups: warpgroup g takes query columns [64g, 64g + 64);
+        // thread j owns key row j of tile J. Per query i the rows hold
+        // nb_i = (c_i - lse_i) log2(e) and scale * delta_i.
+        const int g = warp >> 2, j = tid & 127;
         const int gj = J * BT + j;
         const bool valid = gj < a.L;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const bool leader = j == 0;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const float k1 = a.scale * LOG2E;
         const float cj2 = FOX ? a.c[(long long)h * Lp + gj] * LOG2E : 0.f;
+        // fp32 staging of this warpgroup's 32 columns of dQtil / dP_I for the tile
+        // reductions, inside its own P^T / dS^T panel (free between MMA 2 and the
+        // next pair's probabilities)
+        uint8_t *stq = sPt + g * 16384, *stp = sDs + g * 16384;
         float colsum = 0.f;
         bool ok = true;
+        // Every thread runs every iteration and every named barrier; after a
+        // failed wait the work is skipped, never the barriers.
         for (int it = 0; it < niter; ++it) {
             const int s = it & 1, I = tile_of(it);
             const bool diag = it == niter - 1;
-            if (!mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_POLLS) ||
-                !mbar_wait(s_full, it & 1, WAIT_POLLS)) {
+            if (ok && (!mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_POLLS) ||
+                       !mbar_wait(&s_full[g], it & 1, WAIT_POLLS)))
                 ok = false;
-                break;
-            }
             fence_after_sync();
+            // the previous pair's tile reductions have finished reading the staging
+            if (it > 0) named_barrier(2 + g, 128);
             const float *rows = reinterpret_cast<const float *>(stage(s) + C::S_ROW);
             const float *sd = a.Sd + ((long long)h * nblk + J) * BT * BT;
             float *dsd = a.dSd + ((long long)h * nblk + J) * BT * BT;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BT; c0 += 32) {
-                float sv[32], dp[32];
-                if (!diag) tmem_ld32(tbase + C::T_S + c0 + lane_off, sv);
-                tmem_ld32(tbase + C::T_DP + c0 + lane_off, dp);
-                tmem_wait_ld();
+            auto load = [&](int c, float (&sv)[16], float (&dp)[16]) {
                 if (diag) {
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) sv[u] = sd[(c0 + u) * BT + j];
+                    for (int u = 0; u < 16; ++u) sv[u] = sd[(c + u) * BT + j];
+                } else {
+                    tmem_ld16(tbase + C::T_S + c + lane_off, sv);
                 }
-                float pv[32], dsv[32];
+                tmem_ld16(tbase + C::T_DP + c + lane_off, dp);
+            };
+            auto chunk = [&](int c, const float (&sv)[16], const float (&dp)[16]) {
+                float pv[16], dsv[16];
+                const float4 *nb4 = reinterpret_cast<const float4 *>(rows + c);
+                const float4 *sd4 = reinterpret_cast<const float4 *>(rows + 128 + c);
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const int i = c0 + u;
-                    const float lse2 = rows[i] * LOG2E;
-                    const float bias = FOX ? rows[256 + i] * LOG2E - cj2 : 0.f;
-                    float p = ex2(fmaf(sv[u], k1, bias) - lse2);
-                    if (diag && i < j) p = 0.f;
-                    const float dz = p * (dp[u] - rows[128 + i]);
-                    pv[u] = p;
-                    dsv[u] = a.scale * dz;
-                    // column sums from the same fp16 values the row-sum MMA adds up, so
-                    // the gate gradient's crossing sums cancel exactly
-                    if (FOX) colsum += __half2float(__float2half_rn(dsv[u]));
-                    if (diag) dsd[(long long)i * BT + j] = dsv[u];
-                }
+                for (int q = 0; q < 4; ++q) {
+                    const float4 nb = nb4[q], sdl = sd4[q];
+                    const float nbv[4] = {nb.x, nb.y, nb.z, nb.w}, sdv[4] = {sdl.x, sdl.y, sdl.z, sdl.w};
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    uint4 up, ud;
-                    __nv_bfloat162 *hp = reinterpret_cast<__nv_bfloat162 *>(&up);
-                    __half2 *hd = reinterpret_cast<__half2 *>(&ud);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        hp[k] = __floats2bfloat162_rn(pv[g * 8 + 2 * k], pv[g * 8 + 2 * k + 1]);
-                        hd[k] = __floats2half2_rn(dsv[g * 8 + 2 * k], dsv[g * 8 + 2 * k + 1]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int u = 4 * q + e, i = c + u;
+                        const float x = fmaf(sv[u], k1, FOX ? nbv[e] - cj2 : nbv[e]);
+                        float p = ex2(x);
+                        if (diag && i < j) p = 0.f;
+                        const float ds = p * fmaf(dp[u], a.scale, -sdv[e]);
+                        pv[u] = p;
+                        dsv[u] = ds;
+                        if (diag) dsd[(long long)i * BT + j] = ds;
                     }
-                    const int col = c0 + g * 8;
-                    const uint32_t off = (col >> 6) * 16384 + sw128_offset(j, col & 63);
-                    *reinterpret_cast<uint4 *>(sPt + off) = up;
-                    *reinterpret_cast<uint4 *>(sDs + off) = ud;
                 }
+                uint32_t pb[8], db[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const __nv_bfloat162 bb = __floats2bfloat162_rn(pv[2 * k], pv[2 * k + 1]);
+                    pb[k] = *reinterpret_cast<const uint32_t *>(&bb);
+                    const __half2 hh = __floats2half2_rn(dsv[2 * k], dsv[2 * k + 1]);
+                    db[k] = *reinterpret_cast<const uint32_t *>(&hh);
+                }
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const uint32_t off = (c >> 6) * 16384 + sw128_offset(j, (c & 63) + 8 * hf);
+                    *reinterpret_cast<uint4 *>(sPt + off) =
+                        make_uint4(pb[4 * hf], pb[4 * hf + 1], pb[4 * hf + 2], pb[4 * hf + 3]);
+                    *reinterpret_cast<uint4 *>(sDs + off) =
+                        make_uint4(db[4 * hf], db[4 * hf + 1], db[4 * hf + 2], db[4 * hf + 3]);
+                }
+                if (FOX) {
+                    // gate: row and column sums of the same fp16-rounded dS that the
+                    // MMAs read, so the crossing sums in the gate gradient cancel
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float2 f2 = __half22float2(*reinterpret_cast<const __half2 *>(&db[k]));
+                        dsv[2 * k] = f2.x;
+                        dsv[2 * k + 1] = f2.y;
+                        colsum += f2.x + f2.y;
+                    }
+                    // reduce-scatter over the warp's 32 keys: lanes 2m, 2m+1 end with query c + m
+#pragma unroll
+                    for (int o = 16, n = 16; o >= 2; o >>= 1, n >>= 1) {
+                        const bool up = lane & o;
+#pragma unroll
+                        for (int k = 0; k < n / 2; ++k) {
+                            const float send = up ? dsv[k] : dsv[k + n / 2];
+                            const float keep = up ? dsv[k + n / 2] : dsv[k];
+                            dsv[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                        }
+                    }
+                    dsv[0] += __shfl_xor_sync(0xffffffffu, dsv[0], 1);
+                    if (!(lane & 1))
+                        atomicAdd(a.rowsum + (long long)h * Lp + I * BT + c + (lane >> 1), dsv[0] / a.scale);
+                }
+            };
+            if (ok) {
+                // 16-column chunks; the next chunk's TMEM loads are in flight
+                // while the current one is computed
+                float sA[16], dA[16], sB[16], dB[16];
+                const int cb = 64 * g;
+                load(cb, sA, dA);
+                tmem_wait_ld_tied(sA, dA);
+                load(cb + 16, sB, dB);
+                chunk(cb, sA, dA);
+                tmem_wait_ld_tied(sB, dB);
+                load(cb + 32, sA, dA);
+                chunk(cb + 16, sB, dB);
+                tmem_wait_ld_tied(sA, dA);
+                load(cb + 48, sB, dB);
+                chunk(cb + 32, sA, dA);
+                tmem_wait_ld_tied(sB, dB);
+                chunk(cb + 48, sB, dB);
             }
             fence_async_smem();
             fence_before_sync();
             mbar_arrive(p_full);
-            if (!mbar_wait(m2_full, it & 1, WAIT_POLLS)) {
-                ok = false;
-                break;
-            }
+            if (ok && !mbar_wait(m2_full, it & 1, WAIT_POLLS)) ok = false;
             fence_after_sync();
-            if (!diag) {
-                // chain adjoint: operand for the next pair, or dKtil_J after pair (J+1, J)
-#pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
+            const bool drain = ok && !diag;
+            const int c0 = 32 * g;  // this warpgroup's 32 columns of each d-wide result
+            if (drain) {
+                {
+                    // chain adjoint: operand for the next pair, or dKtil_J after pair (J+1, J)
                     float v[32];
                     tmem_ld32(tbase + C::T_AB + c0 + lane_off, v);
                     tmem_wait_ld();
                     if (I > J + 1) {
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
+                        for (int q = 0; q < 4; ++q) {
                             uint4 u;
                             __half2 *hh = reinterpret_cast<__half2 *>(&u);
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) hh[k] = __floats2half2_rn(v[g * 8 + 2 * k], v[g * 8 + 2 * k + 1]);
-                            *reinterpret_cast<uint4 *>(sAb + sw128_offset(j, c0 + g * 8)) = u;
+                            for (int k = 0; k < 4; ++k) hh[k] = __floats2half2_rn(v[q * 8 + 2 * k], v[q * 8 + 2 * k + 1]);
+                            *reinterpret_cast<uint4 *>(sAb + sw128_offset(j, c0 + q * 8)) = u;
                         }
                     } else {
                         float *dk = a.dKt + ((long long)h * Lp + gj) * D + c0;
@@ -320,61 +370,59 @@ __global__ void __launch_bounds__(NT, 1)
                             *reinterpret_cast<float4 *>(dk + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
                     }
                 }
-                // dQtil rows of tile I (lane = query row)
-                float *dq = a.dQt + ((long long)h * Lp + I * BT + tid) * D;
-#pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                {
+                    // dQtil rows of tile I (lane = query row), staged 128B-swizzled
                     float v[32];
                     tmem_ld32(tbase + C::T_DQ + c0 + lane_off, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int u = 0; u < 32; u += 4) red_add_v4(dq + c0 + u, v[u], v[u + 1], v[u + 2], v[u + 3]);
+                    for (int k = 0; k < 8; ++k)
+                        *reinterpret_cast<float4 *>(stq + j * 128 + ((k ^ (j & 7)) << 4)) =
+                            make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
                 }
                 if (I < last) {
-                    // dP_I rows f = 0..63 live in lanes 0..63 (warps 0, 1)
+                    // dP_I rows f = 0..63 live in lanes 0..63 (warps 0, 1 of each warpgroup)
                     float v[32];
+                    tmem_ld32(tbase + C::T_DPI + c0 + lane_off, v);
+                    tmem_wait_ld();
+                    if (j < D) {
 #pragma unroll
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        tmem_ld32(tbase + C::T_DPI + c0 + lane_off, v);
-                        tmem_wait_ld();
-                        if (tid < D) {
-                            float *dpm = a.dPm + (((long long)h * nblk + I) * D + tid) * D + c0;
-#pragma unroll
-                            for (int u = 0; u < 32; u += 4) red_add_v4(dpm + u, v[u], v[u + 1], v[u + 2], v[u + 3]);
-                        }
+                        for (int k = 0; k < 8; ++k)
+                            *reinterpret_cast<float4 *>(stp + j * 128 + ((k ^ (j & 7)) << 4)) =
+                                make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
                     }
                 }
+                fence_async_smem();
             }
-            if (FOX) {
-                float v[32];
-                tmem_ld32(tbase + C::T_RS + lane_off, v);
-                tmem_wait_ld();
-                atomicAdd(a.rowsum + (long long)h * Lp + I * BT + tid, v[0] / a.scale);
+            named_barrier(2 + g, 128);
+            if (drain && leader) {
+                tma_reduce_add_2d(&mDQ, c0, h * Lp + I * BT, stq);
+                if (I < last) tma_reduce_add_2d(&mDPI, c0, (h * nblk + I) * D, stp);
+                bulk_commit();
             }
             fence_before_sync();
             mbar_arrive(e_done);
+            if (drain && leader) bulk_wait_read<0>();
         }
+        if (leader) bulk_wait_all();
         // the last tile has no off-diagonal pairs: its dKtil is zero
         if (ok && J == last) {
-            float *dk = a.dKt + ((long long)h * Lp + gj) * D;
-            for (int e = 0; e < D; e += 4) *reinterpret_cast<float4 *>(dk + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+            float *dk = a.dKt + ((long long)h * Lp + gj) * D + 32 * g;
+            for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4 *>(dk + e) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        // column sums: warpgroup 1 hands its half to warpgroup 0
+        if (g == 1) sCs[j] = colsum;
+        named_barrier(1, NEW);
         // dV_J
         if (ok) {
-            float dv[D];
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                float v[32];
-                tmem_ld32(tbase + C::T_DV + c0 + lane_off, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int u = 0; u < 32; ++u) dv[c0 + u] = v[u];
-            }
+            float v[32];
+            tmem_ld32(tbase + C::T_DV + 32 * g + lane_off, v);
+            tmem_wait_ld();
             if (valid) {
-                TO *dst = static_cast<TO *>(a.dv) + ((long long)h * a.L + gj) * D;
+                TO *dst = static_cast<TO *>(a.dv) + ((long long)h * a.L + gj) * D + 32 * g;
 #pragma unroll
-                for (int e = 0; e < D; ++e) dst[e] = from_f<TO>(dv[e]);
-                if (a.colsum) a.colsum[(long long)h * Lp + gj] = colsum / a.scale;
+                for (int e = 0; e < 32; ++e) dst[e] = from_f<TO>(v[e]);
+                if (a.colsum && g == 0) a.colsum[(long long)h * Lp + gj] = (colsum + sCs[j]) / a.scale;
             }
         } else if (a.err) {
             atomicCAS(a.err, 0, 13);
@@ -386,14 +434,17 @@ __global__ void __launch_bounds__(NT, 1)
     if (warp == W_MMA) tmem_dealloc(tbase, 512);
 }
 
-// padded lse for the tensor-core backward: rows past L get +inf (probability 0)
-__global__ void pad_lse_kernel(const float *lse, float *lse_p, int L, int Lp, int nh)
+// Per-query terms of the tensor-core backward: nb = (c - lse) log2(e) (+inf
+// lse past L gives nb = -inf, probability 0) and delta scaled in place.
+__global__ void row_terms_kernel(const float *lse, const float *c, float *nb, float *delta,
+                                 float scale, int L, int Lp, int nh)
 {
     const long long n = (long long)nh * Lp;
     for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < n;
          x += (long long)gridDim.x * blockDim.x) {
         const int h = (int)(x / Lp), i = (int)(x % Lp);
-        lse_p[x] = i < L ? lse[(long long)h * L + i] : INFINITY;
+        nb[x] = i < L ? ((c ? c[x] : 0.f) - lse[(long long)h * L + i]) * LOG2E : -INFINITY;
+        delta[x] *= scale;
     }
 }
 
@@ -411,7 +462,7 @@ cudaError_t launch(const CUtensorMap *m, const BwdTcArgs &a, cudaStream_t st)
     auto k = bwd_tc_kernel<FOX, TO>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BCfg::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<dim3(a.nblk, a.nh), NT, BCfg::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], a);
+    k<<<dim3(a.nblk, a.nh), NT, BCfg::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], a);
     count_launches();
     return cudaGetLastError();
 }
@@ -425,7 +476,8 @@ cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16
 {
     const int Lp = b.nblk * BT;
     const long long npairs = (long long)b.nblk * (b.nblk - 1) / 2;
-    pad_lse_kernel<<<592, 256, 0, st>>>(b.lse, lse_p, b.L, Lp, b.nh);
+    // delta is scratch of the backward: scaled here in place for the kernel below
+    row_terms_kernel<<<592, 256, 0, st>>>(b.lse, b.c, lse_p, b.delta, b.scale, b.L, Lp, b.nh);
     count_launches();
     const void *dob = b.dout;
     if (t.out == F32) {
@@ -437,7 +489,7 @@ cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    CUtensorMap m[5];
+    CUtensorMap m[7];
     if (!make_map_2d(&m[0], b.Qt, F16, D, (uint64_t)b.nh * Lp, 128)) return cudaErrorInvalidValue;
     if (npairs > 0) {
         if (!make_map_2d(&m[1], b.Khat, F16, D, (uint64_t)b.nh * npairs * BT, 128)) return cudaErrorInvalidValue;
@@ -446,7 +498,9 @@ cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16
     }
     if (!make_map_3d(&m[2], b.v, BF16, D, b.L, b.nh, 128) ||
         !make_map_3d(&m[3], dob, BF16, D, b.L, b.nh, 128) ||
-        !make_map_2d(&m[4], b.Pm, F16, D, (uint64_t)b.nh * b.nblk * D, D))
+        !make_map_2d(&m[4], b.Pm, F16, D, (uint64_t)b.nh * b.nblk * D, D) ||
+        !make_map_f32_2d(&m[5], b.dQt, D, (uint64_t)b.nh * Lp, 128) ||
+        !make_map_f32_2d(&m[6], b.dPm, D, (uint64_t)b.nh * b.nblk * D, 64))
         return cudaErrorInvalidValue;
     BwdTcArgs a{b.Sd, b.c, lse_p, b.delta, b.scale, b.L, b.nblk, b.nh, npairs,
                 b.dQt, b.dKt, b.dPm, b.dSd, b.dv, b.rowsum, b.colsum, err};

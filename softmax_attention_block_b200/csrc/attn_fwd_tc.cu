@@ -224,80 +224,80 @@ __global__ void __launch_bounds__(NT, 1)
         float m = -INFINITY, l = 0.f, mA = -INFINITY;
         bool ok = true;
         const float *sd = a.Sd + (((long long)h * a.nblk + I) * BT + r) * BT + c0s;
+        // Every thread runs every iteration and every named barrier; after a
+        // failed wait the work is skipped, never the barriers.
         for (int it = 0; it < niter; ++it) {
             const int s = it % NS, b = it & 1;
-            if (FOX && !mbar_wait(&kv_full[s], (it / NS) & 1, WAIT_POLLS)) {
-                ok = false;
-                break;
-            }
+            if (ok && FOX && !mbar_wait(&kv_full[s], (it / NS) & 1, WAIT_POLLS)) ok = false;
             const float *cj = sC(s) + c0s;
             float z[64];
-            if (it == 0) {
-#pragma unroll
-                for (int j = 0; j < 64; j += 4) {
-                    const float4 v4 = *reinterpret_cast<const float4 *>(sd + j);
-                    z[j] = v4.x;
-                    z[j + 1] = v4.y;
-                    z[j + 2] = v4.z;
-                    z[j + 3] = v4.w;
-                }
-            } else {
-                if (!mbar_wait(&s_full[b], ((it - 1) >> 1) & 1, WAIT_POLLS)) {
-                    ok = false;
-                    break;
-                }
-                fence_after_sync();
-                float *z0 = z, *z1 = z + 32;
-                tmem_ld32(tbase + b * 128 + c0s + lane_off, *reinterpret_cast<float(*)[32]>(z0));
-                tmem_ld32(tbase + b * 128 + c0s + 32 + lane_off, *reinterpret_cast<float(*)[32]>(z1));
-                tmem_wait_ld();
-            }
             float pmax = -INFINITY;
+            if (ok && it > 0 && !mbar_wait(&s_full[b], ((it - 1) >> 1) & 1, WAIT_POLLS)) ok = false;
+            if (ok) {
+                if (it == 0) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const float bias = FOX ? ci2 - cj[j] * LOG2E : 0.f;
-                z[j] = (it > 0 || c0s + j <= r) ? fmaf(z[j], k1, bias) : -INFINITY;
-                pmax = fmaxf(pmax, z[j]);
+                    for (int j = 0; j < 64; j += 4) {
+                        const float4 v4 = *reinterpret_cast<const float4 *>(sd + j);
+                        z[j] = v4.x;
+                        z[j + 1] = v4.y;
+                        z[j + 2] = v4.z;
+                        z[j + 3] = v4.w;
+                    }
+                } else {
+                    fence_after_sync();
+                    float *z0 = z, *z1 = z + 32;
+                    tmem_ld32(tbase + b * 128 + c0s + lane_off, *reinterpret_cast<float(*)[32]>(z0));
+                    tmem_ld32(tbase + b * 128 + c0s + 32 + lane_off, *reinterpret_cast<float(*)[32]>(z1));
+                    tmem_wait_ld();
+                }
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    const float bias = FOX ? ci2 - cj[j] * LOG2E : 0.f;
+                    z[j] = (it > 0 || c0s + j <= r) ? fmaf(z[j], k1, bias) : -INFINITY;
+                    pmax = fmaxf(pmax, z[j]);
+                }
             }
             float *rb = red + (it & 1) * 256;
             rb[hf * 128 + r] = pmax;
             named_barrier(1 + q4, 64);
             const float m_new = fmaxf(m, fmaxf(rb[r], rb[128 + r]));
             // add the previous tile's P.V (scaled to its max m) into the accumulator
-            if (it >= 1) {
+            if (ok && it >= 1) {
                 if (!mbar_wait(o_full, (it - 1) & 1, WAIT_POLLS)) {
                     ok = false;
-                    break;
-                }
-                fence_after_sync();
-                const float corr = ex2(mA - m);
+                } else {
+                    fence_after_sync();
+                    const float corr = ex2(mA - m);
 #pragma unroll
-                for (int c0 = 0; c0 < DH; c0 += 32) {
-                    float v[32];
-                    tmem_ld32(tbase + 256 + c0o + c0 + lane_off, v);
-                    tmem_wait_ld();
+                    for (int c0 = 0; c0 < DH; c0 += 32) {
+                        float v[32];
+                        tmem_ld32(tbase + 256 + c0o + c0 + lane_off, v);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
+                        for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
+                    }
+                    mA = m;
                 }
-                mA = m;
             }
-            // probabilities -> P (fp16, swizzled K-major panel hf) and partial row sum
-            float rowsum = 0.f;
+            if (ok) {
+                // probabilities -> P (fp16, swizzled K-major panel hf) and partial row sum
+                float rowsum = 0.f;
 #pragma unroll
-            for (int g = 0; g < 8; ++g) {
-                uint4 u;
-                __half2 *hh = reinterpret_cast<__half2 *>(&u);
+                for (int g = 0; g < 8; ++g) {
+                    uint4 u;
+                    __half2 *hh = reinterpret_cast<__half2 *>(&u);
 #pragma unroll
-                for (int q2 = 0; q2 < 4; ++q2) {
-                    const float p0 = ex2(z[g * 8 + 2 * q2] - m_new);
-                    const float p1 = ex2(z[g * 8 + 2 * q2 + 1] - m_new);
-                    rowsum += p0 + p1;
-                    hh[q2] = __floats2half2_rn(p0, p1);
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const float p0 = ex2(z[g * 8 + 2 * q2] - m_new);
+                        const float p1 = ex2(z[g * 8 + 2 * q2 + 1] - m_new);
+                        rowsum += p0 + p1;
+                        hh[q2] = __floats2half2_rn(p0, p1);
+                    }
+                    *reinterpret_cast<uint4 *>(sP + hf * 16384 + sw128_offset(r, g * 8)) = u;
                 }
-                *reinterpret_cast<uint4 *>(sP + hf * 16384 + sw128_offset(r, g * 8)) = u;
+                l = fmaf(l, ex2(m - m_new), rowsum);
+                m = m_new;
             }
-            l = fmaf(l, ex2(m - m_new), rowsum);
-            m = m_new;
             fence_async_smem();
             fence_before_sync();
             mbar_arrive(p_full);

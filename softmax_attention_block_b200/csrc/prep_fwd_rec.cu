@@ -26,7 +26,42 @@ template <int D>
 struct RecCfg {
     static constexpr int NT = 2 * BT + (D < 32 ? 32 : D);  // keys, queries, P columns
     static constexpr int MIN_CTAS = D <= 32 ? 2 : 1;
+    static constexpr int LDS = D + 4;  // shared row stride: 16-byte rows for vector reads
 };
+
+// Dot product of row t of a shared [BT][D + 4] matrix with x. Every thread of
+// the warp reads the same row: broadcast 16-byte loads.
+template <int D>
+__device__ __forceinline__ float row_dot(const float *sm, int t, const float (&x)[D])
+{
+    const float4 *p = reinterpret_cast<const float4 *>(sm + t * RecCfg<D>::LDS);
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {
+        const float4 v = p[c];
+        s0 = fmaf(v.x, x[4 * c], s0);
+        s1 = fmaf(v.y, x[4 * c + 1], s1);
+        s2 = fmaf(v.z, x[4 * c + 2], s2);
+        s3 = fmaf(v.w, x[4 * c + 3], s3);
+    }
+    return (s0 + s1) + (s2 + s3);
+}
+
+// x <- H_t x = x - beta_t w_t (w_t . x)
+template <int D>
+__device__ __forceinline__ void apply_h(float (&x)[D], const float *sW, const float *sB, int t)
+{
+    const float coef = sB[t] * row_dot<D>(sW, t, x);
+    const float4 *p = reinterpret_cast<const float4 *>(sW + t * RecCfg<D>::LDS);
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {
+        const float4 v = p[c];
+        x[4 * c] = fmaf(-coef, v.x, x[4 * c]);
+        x[4 * c + 1] = fmaf(-coef, v.y, x[4 * c + 1]);
+        x[4 * c + 2] = fmaf(-coef, v.z, x[4 * c + 2]);
+        x[4 * c + 3] = fmaf(-coef, v.w, x[4 * c + 3]);
+    }
+}
 
 template <typename T, typename TM, int D>
 __global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
@@ -34,10 +69,11 @@ __global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
                         const float *__restrict__ beta, int L, int nblk, TM *Qt, TM *Kt, TM *Pm,
                         float *Sd)
 {
-    extern __shared__ float sm[];
-    float *sW = sm;              // [BT][D+1]
-    float *sQ = sW + BT * (D + 1);  // [BT][D+1]
-    float *sB = sQ + BT * (D + 1);  // [BT]
+    constexpr int LDS = RecCfg<D>::LDS;
+    extern __shared__ __align__(16) float sm[];
+    float *sW = sm;              // [BT][D+4]
+    float *sQ = sW + BT * LDS;   // [BT][D+4]
+    float *sB = sQ + BT * LDS;   // [BT]
     const int J = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
     const int Lp = nblk * BT;
     const long long row0 = (long long)h * L + (long long)J * BT;  // first row of the block in [nh, L]
@@ -45,8 +81,8 @@ __global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
     for (int e = tid; e < BT * D; e += blockDim.x) {
         const int r = e / D, c = e % D;
         const bool ok = r < nvalid;
-        sW[r * (D + 1) + c] = ok ? to_f(w[(row0 + r) * D + c]) : 0.f;
-        sQ[r * (D + 1) + c] = ok ? to_f(q[(row0 + r) * D + c]) : 0.f;
+        sW[r * LDS + c] = ok ? to_f(w[(row0 + r) * D + c]) : 0.f;
+        sQ[r * LDS + c] = ok ? to_f(q[(row0 + r) * D + c]) : 0.f;
     }
     for (int r = tid; r < BT; r += blockDim.x) sB[r] = r < nvalid ? beta[row0 + r] : 0.f;
     __syncthreads();
@@ -55,79 +91,45 @@ __global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
         // keys: Ktil and the diagonal-block logits
         const int j = tid;
         float x[D];
+#pragma unroll
         for (int c = 0; c < D; ++c) x[c] = j < nvalid ? to_f(k[(row0 + j) * D + c]) : 0.f;
         float *sd = Sd + ((long long)h * nblk + J) * BT * BT;
-        {
-            float s = 0.f;
-#pragma unroll
-            for (int c = 0; c < D; ++c) s = fmaf(sQ[j * (D + 1) + c], x[c], s);
-            sd[(long long)j * BT + j] = s;
-        }
-        for (int t = 1; t < BT; ++t) {
+        sd[(long long)j * BT + j] = row_dot<D>(sQ, j, x);
+        // the step index is the same for the whole warp (broadcast rows);
+        // lanes with t <= j only write the zero above the diagonal
+        for (int t = (j & ~31) + 1; t < BT; ++t) {
             if (t > j) {
-                const float *wt = sW + t * (D + 1), *qt = sQ + t * (D + 1);
-                float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-                for (int c = 0; c < D; c += 2) {
-                    a0 = fmaf(wt[c], x[c], a0);
-                    a1 = fmaf(wt[c + 1], x[c + 1], a1);
-                }
-                const float coef = sB[t] * (a0 + a1);
-                float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-                for (int c = 0; c < D; c += 2) {
-                    x[c] = fmaf(-coef, wt[c], x[c]);
-                    x[c + 1] = fmaf(-coef, wt[c + 1], x[c + 1]);
-                    s0 = fmaf(qt[c], x[c], s0);
-                    s1 = fmaf(qt[c + 1], x[c + 1], s1);
-                }
-                sd[(long long)t * BT + j] = s0 + s1;
+                apply_h<D>(x, sW, sB, t);
+                sd[(long long)t * BT + j] = row_dot<D>(sQ, t, x);
             } else if (t < j) {
                 sd[(long long)t * BT + j] = 0.f;  // above the diagonal (never read)
             }
         }
+        for (int t = 0; t < (j & ~31); ++t) sd[(long long)t * BT + j] = 0.f;
         TM *dst = Kt + ((long long)h * Lp + (long long)J * BT + j) * D;
+#pragma unroll
         for (int c = 0; c < D; ++c) dst[c] = from_f<TM>(x[c]);
     } else if (tid < 2 * BT) {
         // queries: Qtil_i = H_s ... H_i q_i (apply H_i first)
         const int i = tid - BT;
         float x[D];
-        for (int c = 0; c < D; ++c) x[c] = sQ[i * (D + 1) + c];
-        for (int t = BT - 1; t >= 0; --t) {
-            if (t <= i) {
-                const float *wt = sW + t * (D + 1);
-                float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                for (int c = 0; c < D; c += 2) {
-                    a0 = fmaf(wt[c], x[c], a0);
-                    a1 = fmaf(wt[c + 1], x[c + 1], a1);
-                }
-                const float coef = sB[t] * (a0 + a1);
-#pragma unroll
-                for (int c = 0; c < D; ++c) x[c] = fmaf(-coef, wt[c], x[c]);
-            }
-        }
+        for (int c = 0; c < D; ++c) x[c] = sQ[i * LDS + c];
+        for (int t = (i | 31); t >= 0; --t)
+            if (t <= i) apply_h<D>(x, sW, sB, t);
         TM *dst = Qt + ((long long)h * Lp + (long long)J * BT + i) * D;
+#pragma unroll
         for (int c = 0; c < D; ++c) dst[c] = from_f<TM>(x[c]);
     } else {
         // block product P = H_e ... H_s, one column per thread
         const int col = tid - 2 * BT;
         if (col < D) {
             float x[D];
+#pragma unroll
             for (int c = 0; c < D; ++c) x[c] = c == col ? 1.f : 0.f;
-            for (int t = 0; t < BT; ++t) {
-                const float *wt = sW + t * (D + 1);
-                float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-                for (int c = 0; c < D; c += 2) {
-                    a0 = fmaf(wt[c], x[c], a0);
-                    a1 = fmaf(wt[c + 1], x[c + 1], a1);
-                }
-                const float coef = sB[t] * (a0 + a1);
-#pragma unroll
-                for (int c = 0; c < D; ++c) x[c] = fmaf(-coef, wt[c], x[c]);
-            }
+            for (int t = 0; t < BT; ++t) apply_h<D>(x, sW, sB, t);
             TM *dst = Pm + ((long long)h * nblk + J) * D * D;
+#pragma unroll
             for (int r = 0; r < D; ++r) dst[(long long)r * D + col] = from_f<TM>(x[r]);
         }
     }
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
 template <typename T, typename TM, int D>
 cudaError_t run(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out, cudaStream_t st)
 {
-    const size_t smem = (2 * BT * (D + 1) + BT) * sizeof(float);
+    const size_t smem = (2 * BT * RecCfg<D>::LDS + BT) * sizeof(float);
     auto kern = prep_fwd_rec_kernel<T, TM, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -67,6 +67,33 @@ __device__ __forceinline__ void mma_ss(uint32_t tmem_d, uint64_t adesc, uint64_t
         : "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// mma_ss issued by the threads with `issue` != 0 only. Called by a whole
+// converged warp with warp-uniform operands and `issue` set on one lane, so
+// the descriptors stay uniform values and the warp never diverges.
+__device__ __forceinline__ void mma_ss_if(uint32_t issue, uint32_t tmem_d, uint64_t adesc,
+                                          uint64_t bdesc, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %5, 0;\n\t"
+        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        :
+        : "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(issue));
+}
+
+// commit() by the threads with `issue` != 0 only (the lane that issued the MMAs).
+__device__ __forceinline__ void commit_if(uint32_t issue, uint64_t *bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred q;\n\t"
+        "setp.ne.b32 q, %1, 0;\n\t"
+        "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n"
+        :
+        : "r"(smem_u32(bar)), "r"(issue)
+        : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 operation this thread issued has completed.
 __device__ __forceinline__ void commit(uint64_t *bar)
 {
@@ -128,6 +155,35 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32])
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 16 consecutive fp32 columns of this thread's lane (same addressing as tmem_ld32).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16])
+{
+    uint32_t *u = reinterpret_cast<uint32_t *>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+          "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
+          "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr));
+}
+
+// Waits for this thread's TMEM loads; the registers of `a` and `b` are tied to
+// the wait, so no use of them can be scheduled before it (needed when loads
+// stay in flight while other registers are being used).
+__device__ __forceinline__ void tmem_wait_ld_tied(float (&a)[16], float (&b)[16])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]),
+                   "+f"(a[6]), "+f"(a[7]), "+f"(a[8]), "+f"(a[9]), "+f"(a[10]), "+f"(a[11]),
+                   "+f"(a[12]), "+f"(a[13]), "+f"(a[14]), "+f"(a[15]), "+f"(b[0]), "+f"(b[1]),
+                   "+f"(b[2]), "+f"(b[3]), "+f"(b[4]), "+f"(b[5]), "+f"(b[6]), "+f"(b[7]),
+                   "+f"(b[8]), "+f"(b[9]), "+f"(b[10]), "+f"(b[11]), "+f"(b[12]), "+f"(b[13]),
+                   "+f"(b[14]), "+f"(b[15])
+                 :
+                 : "memory");
+}
 
 // --- mbarriers --------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
@@ -247,6 +303,17 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int 
         : "memory");
 }
 
+// Shared -> global element-wise fp32 add of a tile through a tensor map
+// (128B-swizzled source; the map's element type decides the arithmetic).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, int x, int y, const void *src)
+{
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];"
+        :
+        : "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(src))
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Wait until at most N committed store groups still read shared memory.
@@ -273,6 +340,10 @@ __device__ __forceinline__ float ex2(float x)
 // driver rejects the map (alignment, strides).
 bool make_map_2d(CUtensorMap *m, const void *base, int dt, uint64_t cols, uint64_t rows,
                  uint32_t box_rows);
+// fp32 [rows][cols] with a box of 32 columns (128 bytes) x `box_rows` rows,
+// 128-byte swizzled (for tile reductions into fp32 accumulators).
+bool make_map_f32_2d(CUtensorMap *m, const float *base, uint64_t cols, uint64_t rows,
+                     uint32_t box_rows);
 // 3-D [outer][rows][cols] with rows beyond `rows` read as zero.
 bool make_map_3d(CUtensorMap *m, const void *base, int dt, uint64_t cols, uint64_t rows,
                  uint64_t outer, uint32_t box_rows);

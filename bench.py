@@ -53,6 +53,8 @@ def fa_equiv_flops(B, H, L, d):
 
 # fp32 FMA peak from unit counts and clocks: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz
 ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# dense TF32 / BF16 nominal ratio (1.1 / 2.25 PFLOP/s), to derive a TF32 peak
+TF32_PER_BF16 = 1.1 / 2.25
 
 
 def stage_model(name, B, H, L, d, BT=128):
@@ -60,7 +62,7 @@ def stage_model(name, B, H, L, d, BT=128):
 
     Tensor-core stages count the products of the blockwise algorithm; the UT
     prep stages count the fp32 arithmetic of the per-block recurrences and
-    64x64 products they are made of."""
+    64x64 products they are made of ("tf32": products on TF32 tensor cores)."""
     nh, nblk, HB = B * H, -(-L // BT), 64
     per = {
         "attn_fwd": (2.0 * L * L * d, "tensor"),                      # QK^T + PV
@@ -72,13 +74,23 @@ def stage_model(name, B, H, L, d, BT=128):
         "chain": (1.0 * L * L * d * d / BT, "tensor"),               # key-side block transport
         # keys (Ktil + in-block logits), queries, block product: rank-one steps
         "ut_prep": (nblk * (BT * BT / 2 * 10.0 * d + BT * 4.0 * d * d), "alu"),
-        # per 128-block: 8 products + 4 x 64 recurrences (composition) and
-        # 2 halves x (24 products incl. the two solves)
+        # per 128-block: 8 products of 64x64 by 64xd, and 4 x 64 rank-one steps
+        "ut_adj_compose": (nblk * (8 * 2.0 * HB * HB * d + 4 * HB * HB * 4.0 * d), "tf32"),
+        # per 64-half: 22 products and two 64x128 triangular solves
+        "ut_adj64": (2 * nblk * (22 * 2.0 * HB * HB * d + 2 * HB * HB * 128.0), "tf32"),
         "ut_prep_bwd": (nblk * (8 * 2.0 * HB * HB * d + 4 * HB * HB * 4.0 * d
                                 + 2 * 24 * 2.0 * HB * HB * d), "alu"),
     }
     f, bound = per.get(name, (0.0, None))
     return f * nh, bound
+
+
+# DRAM bytes (read + write) per launch of a kernel, from an ncu capture of the
+# B=1 H=24 L=4096 d=64 case (profiles/ summaries), scaled to the benchmark's
+# B=8 by the heads processed; None where the kernel changed since the capture.
+DRAM_BYTES_B1H24 = {
+    "attn_bwd": 326.980352e6 + 96.854272e6,
+}
 
 
 def load_peaks():
@@ -316,12 +328,19 @@ def run_ours(args):
         ach = f / (per_launch_ms * 1e-3) / 1e12 if f else None
         if bound == "alu":
             peak, src = ALU_F32_TFLOPS, "fp32 FMA from unit counts and max clock"
+        elif bound == "tf32":
+            peak = peaks["bf16_tflops_sustained"] * TF32_PER_BF16
+            src = f"{peaks['source']} bf16 dense (sustained) x nominal tf32/bf16 ratio"
+            bound = "tensor"
         else:
             peak = peaks["bf16_tflops_sustained"]
             src = f"{peaks['source']} bf16 dense (sustained)"
+        traffic = DRAM_BYTES_B1H24.get(dom)
+        if traffic is not None:
+            traffic *= (w.B * w.H) / 24.0
         roofline = {"kernel": dom, "bound": bound or "tensor", "achieved": ach, "peak": peak,
-                    "unit": "TFLOP/s", "frac": (ach / peak) if ach else None, "traffic": None,
-                    "peak_source": src}
+                    "unit": "TFLOP/s", "frac": (ach / peak) if ach else None, "traffic": traffic,
+                    "traffic_unit": "bytes per launch", "peak_source": src}
 
     # end to end through the API with host buffers (pinned), copies in the timed region
     e2e = None

@@ -471,24 +471,28 @@ cudaError_t launch(const CUtensorMap *m, const BwdTcArgs &a, cudaStream_t st)
 
 bool attn_bwd_tc_supported(Types t, int d) { return t.in == BF16 && t.mid == F16 && d == 64; }
 
-cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16, int *err,
-                        cudaStream_t st)
+cudaError_t attn_bwd_tc_prepare(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16,
+                                cudaStream_t st)
 {
     const int Lp = b.nblk * BT;
-    const long long npairs = (long long)b.nblk * (b.nblk - 1) / 2;
-    // delta is scratch of the backward: scaled here in place for the kernel below
+    // delta is scratch of the backward: scaled here in place for the kernel
     row_terms_kernel<<<592, 256, 0, st>>>(b.lse, b.c, lse_p, b.delta, b.scale, b.L, Lp, b.nh);
     count_launches();
-    const void *dob = b.dout;
     if (t.out == F32) {
         const long long n = (long long)b.nh * b.L * D;
         f32_to_bf16_kernel<<<1184, 256, 0, st>>>(static_cast<const float *>(b.dout),
                                                  static_cast<bf16 *>(dout_bf16), n);
         count_launches();
-        dob = dout_bf16;
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16, int *err,
+                        cudaStream_t st)
+{
+    const int Lp = b.nblk * BT;
+    const long long npairs = (long long)b.nblk * (b.nblk - 1) / 2;
+    const void *dob = t.out == F32 ? dout_bf16 : b.dout;
     CUtensorMap m[7];
     if (!make_map_2d(&m[0], b.Qt, F16, D, (uint64_t)b.nh * Lp, 128)) return cudaErrorInvalidValue;
     if (npairs > 0) {

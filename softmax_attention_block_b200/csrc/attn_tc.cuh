@@ -27,7 +27,10 @@ struct BwdTcArgs {
 };
 
 bool attn_bwd_tc_supported(Types t, int d);
-// lse_p: [nh, Lp] scratch; dout_bf16: [nh, L, d] scratch (used when dout is fp32)
+// lse_p: [nh, Lp] scratch; dout_bf16: [nh, L, d] scratch (used when dout is fp32).
+// attn_bwd_tc_prepare (per-query terms, bf16 dout) runs first on the same stream.
+cudaError_t attn_bwd_tc_prepare(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16,
+                                cudaStream_t st);
 cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16, int *err,
                         cudaStream_t st);
 

@@ -233,6 +233,7 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
         {
             Stage s_d("delta", st);
             TRY(compute_delta(a, t, d, st));
+            TRY(attn_bwd_tc_prepare(a, t, ws.lse_p, ws.dout16, st));
         }
         TRY(cudaMemsetAsync(ws.dQt, 0, sizeof(float) * (size_t)y.nh * y.Lp * d, st));
         TRY(cudaMemsetAsync(ws.rowsum, 0, sizeof(float) * (size_t)y.nh * y.Lp, st));
@@ -244,12 +245,11 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
     PrepDims D{y.nh, y.L, y.d, y.nblk, types_of(dt).in, types_of(dt).out};
     PrepInputs in{q, k, w, beta};
     PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta};
-    {
+    if (prep_backward_fused_supported(D)) {
+        TRY(prep_backward_fused(D, in, gr, ws.dP64, st));  // times its two kernels itself
+    } else {
         Stage s("ut_prep_bwd", st);
-        if (prep_backward_fused_supported(D))
-            TRY(prep_backward_fused(D, in, gr, ws.dP64, st));
-        else
-            TRY(prep_backward(D, in, ws.prep, gr, st));
+        TRY(prep_backward(D, in, ws.prep, gr, st));
     }
     if (log_f) {
         Stage s("gate_grad", st);

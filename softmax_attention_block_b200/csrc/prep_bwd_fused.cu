@@ -689,17 +689,23 @@ cudaError_t run(const PrepDims &Dm, const PrepInputs &in, const PrepGrads &g, fl
     const T *q = static_cast<const T *>(in.q), *k = static_cast<const T *>(in.k),
             *w = static_cast<const T *>(in.w);
     const bool vec = rows_vec_aligned<T>(q) && rows_vec_aligned<T>(k) && rows_vec_aligned<T>(w);
-    kc<<<dim3(Dm.nblk, Dm.nh), NT, smc, st>>>(q, k, w, in.beta, Dm.L, Dm.nblk, vec,
-                                              const_cast<float *>(g.dQt), const_cast<float *>(g.dKt),
-                                              g.dPm, g.dSd, dP64);
-    count_launches();
+    {
+        Stage s_c("ut_adj_compose", st);
+        kc<<<dim3(Dm.nblk, Dm.nh), NT, smc, st>>>(q, k, w, in.beta, Dm.L, Dm.nblk, vec,
+                                                  const_cast<float *>(g.dQt),
+                                                  const_cast<float *>(g.dKt), g.dPm, g.dSd, dP64);
+        count_launches();
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    ku<<<dim3(2 * Dm.nblk, Dm.nh), NT, smu, st>>>(q, k, w, in.beta, Dm.L, Dm.nblk, vec, g.dQt,
-                                                  g.dKt, dP64, g.dSd, static_cast<TO *>(g.dq),
-                                                  static_cast<TO *>(g.dk), static_cast<TO *>(g.dw),
-                                                  g.dbeta);
-    count_launches();
+    {
+        Stage s_u("ut_adj64", st);
+        ku<<<dim3(2 * Dm.nblk, Dm.nh), NT, smu, st>>>(q, k, w, in.beta, Dm.L, Dm.nblk, vec, g.dQt,
+                                                      g.dKt, dP64, g.dSd, static_cast<TO *>(g.dq),
+                                                      static_cast<TO *>(g.dk),
+                                                      static_cast<TO *>(g.dw), g.dbeta);
+        count_launches();
+    }
     return cudaGetLastError();
 }
 

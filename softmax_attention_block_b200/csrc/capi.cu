@@ -128,7 +128,10 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
     PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, t.mid};
     {
         Stage s("ut_prep", st);
-        TRY(prep_forward_rec(D, in, out, st));
+        if (prep_forward_tc_supported(D))
+            TRY(prep_forward_tc(D, in, out, st));
+        else
+            TRY(prep_forward_rec(D, in, out, st));
     }
     ChainArgs ca{ws.Kt, ws.Pm, ws.Khat, y.nblk, y.nh};
     {

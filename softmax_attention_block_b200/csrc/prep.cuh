@@ -40,9 +40,14 @@ struct PrepScratch {
 
 void carve_prep_scratch(Carver &c, const PrepDims &D, bool backward, PrepScratch &s);
 size_t prep_scratch_bytes(const PrepDims &D, bool backward);
-// Same outputs as prep_forward, computed by per-row recurrences in fp32.
+// Qtil, Ktil, P, Sd of every 128-block, computed by per-row recurrences in fp32.
 cudaError_t prep_forward_rec(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
                              cudaStream_t st);
+// The same outputs for head dim 64, by the UT transform of each 64-position half on
+// the tensor cores (split TF32) and a 128-level composition.
+bool prep_forward_tc_supported(const PrepDims &D);
+cudaError_t prep_forward_tc(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
+                            cudaStream_t st);
 cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
                           const PrepGrads &gr, cudaStream_t st);
 // Fused adjoint for head dim 64 (two 64-position halves per block). dQt and

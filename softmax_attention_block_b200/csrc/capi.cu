@@ -41,6 +41,7 @@ struct AttnWs {
     float *delta, *dQt, *dKt, *dPm, *dSd, *rowsum, *colsum;
     float *lse_p;     // lse padded to Lp (tensor-core backward)
     float *dP64;      // per-half block-product adjoints (fused prep adjoint)
+    float *halves = nullptr;  // 64-half quantities of the tensor-core prep (head dim 64)
     void *dout16;     // bf16 copy of an fp32 dout (tensor-core backward)
 };
 
@@ -69,6 +70,7 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
         w.colsum = c.take<float>(nh * Lp);
         w.lse_p = c.take<float>(nh * Lp);
         w.dP64 = c.take<float>(nh * 2 * nb * d * d);
+        w.halves = c.take<float>(prep_forward_tc_supported(D) ? nh * nb * 4 * 64 * 64 : 0);
         w.dout16 = c.take<char>(nh * (size_t)y.L * d * 2);
     }
     return c.bytes();
@@ -125,7 +127,7 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
     const Types t = types_of(dt);
     PrepDims D{y.nh, y.L, y.d, y.nblk, t.in, t.out};
     PrepInputs in{q, k, w, beta};
-    PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, t.mid};
+    PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, t.mid, ws.halves};
     {
         Stage s("ut_prep", st);
         if (prep_forward_tc_supported(D))
@@ -180,7 +182,11 @@ path_status path_attn_fwd(const void *q, const void *k, const void *v, const voi
     AttnWs ws;
     const size_t need = carve_attn(nullptr, y, dt, false, ws);
     if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
-    carve_attn(workspace, y, dt, false, ws);
+    // a workspace sized for the backward also receives what a backward that
+    // reuses it needs beyond the forward's own buffers
+    const bool for_bwd = workspace_bytes >= carve_attn(nullptr, y, dt, true, ws);
+    carve_attn(workspace, y, dt, for_bwd, ws);
+    if (!for_bwd) ws.halves = nullptr;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     TRY(cudaMemsetAsync(ws.err, 0, sizeof(int), st));
     path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
@@ -247,7 +253,7 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
     }
     PrepDims D{y.nh, y.L, y.d, y.nblk, types_of(dt).in, types_of(dt).out};
     PrepInputs in{q, k, w, beta};
-    PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta};
+    PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta, ws.halves};
     if (prep_backward_fused_supported(D)) {
         TRY(prep_backward_fused(D, in, gr, ws.dP64, st));  // times its two kernels itself
     } else {

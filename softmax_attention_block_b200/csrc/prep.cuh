@@ -21,6 +21,9 @@ struct PrepOutputs {
     void *Pm;       // [nh, nblk, d, d] block products (type tdt)
     float *Sd;      // [nh, nblk, BT, BT] diagonal-block bilinear logits (lower part)
     int tdt;
+    // optional (head dim 64, tensor-core prep): per block the 64-half quantities
+    // Ktil_a, Qtil_b, P_a, P_b ([nh, nblk, 4, 64, 64] fp32) for the backward
+    float *halves = nullptr;
 };
 
 struct PrepGrads {
@@ -29,6 +32,7 @@ struct PrepGrads {
     const float *dSd;        // [nh, nblk, BT, BT], zero above the diagonal
     void *dq, *dk, *dw;      // [nh, L, d] (type dt)
     float *dbeta;            // [nh, L]
+    const float *halves = nullptr;  // PrepOutputs::halves of the forward (fused adjoint)
 };
 
 struct PrepScratch {

@@ -10,8 +10,8 @@
 //      Qtil[b] = Qtil_b P_a,  Ktil[a] = Ktil_a P_b^T,  P = P_b P_a,
 //      Sd[b, a] = Qtil_b Ktil_a^T     (Sd[a, a], Sd[b, b] are the halves' own),
 //    so the 128-level adjoints become per-half ones by a few 64x64 products.
-//    The halves' quantities are recomputed by the same rank-one recurrences
-//    as the forward prep (64 steps).
+//    The halves' quantities are the ones the forward's UT prep computed and
+//    left in the workspace.
 // 2. ut_adj64: per 64-position half, the UT transform in closed form
 //    (Paper-Notes "训练策略": T^{-1} = (I + strictLower(D W W^T))^{-1} D):
 //      A = strictLower(D W W^T), N = strictLower(W K^T), M = lower(Q W^T),
@@ -31,57 +31,15 @@ namespace {
 
 using namespace ut64;
 
-constexpr int WLD = D + 4;  // row stride of the recurrences' W (halves 4 floats apart)
-
-// Column c of a row of the recurrences' W: the two 32-column halves sit 36
-// floats apart, so the two lanes of a row read different banks.
-__device__ __forceinline__ int wx(int t, int c) { return t * WLD + c + (c >= 32 ? 4 : 0); }
-
-// x <- H_t x = x - beta_t w_t (w_t . x) on this lane's 32 columns (half p of
-// the row; the partner lane holds the other half), or x unchanged when !on.
-// Every lane of the warp calls it with the same t (it shuffles).
-__device__ __forceinline__ void apply_h_half(float (&x)[32], const float *sW, const float *sB, int t,
-                                             int p, bool on = true)
-{
-    const float4 *wt = reinterpret_cast<const float4 *>(sW + wx(t, 32 * p));
-    float w[32];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const float4 v = wt[c];
-        w[4 * c] = v.x;
-        w[4 * c + 1] = v.y;
-        w[4 * c + 2] = v.z;
-        w[4 * c + 3] = v.w;
-    }
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-    for (int c = 0; c < 32; c += 4) {
-        a0 = fmaf(w[c], x[c], a0);
-        a1 = fmaf(w[c + 1], x[c + 1], a1);
-        a2 = fmaf(w[c + 2], x[c + 2], a2);
-        a3 = fmaf(w[c + 3], x[c + 3], a3);
-    }
-    float dot = (a0 + a1) + (a2 + a3);
-    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-    const float coef = on ? sB[t] * dot : 0.f;
-#pragma unroll
-    for (int c = 0; c < 32; ++c) x[c] = fmaf(-coef, w[c], x[c]);
-}
-
 // ---------------------------------------------------------------------------
 // 1. 128-level adjoints -> per-half adjoints (in place for dQt / dKt)
 // ---------------------------------------------------------------------------
-template <typename T>
-__global__ void __launch_bounds__(NT) compose_adj_kernel(const T *q, const T *k, const T *w,
-                                                         const float *beta, int L, int nblk,
-                                                         bool vec, float *dQt, float *dKt,
-                                                         const float *dPm, const float *dSd,
-                                                         float *dP64)
+__global__ void __launch_bounds__(NT) compose_adj_kernel(const float *halves, int nblk, float *dQt,
+                                                         float *dKt, const float *dPm,
+                                                         const float *dSd, float *dP64)
 {
     extern __shared__ __align__(16) float sm[];
-    float *sW = sm;               // [128][WLD]
-    float *sBt = sW + BT * WLD;   // [128]
-    float *sKa = sBt + BT;        // Ktil_a
+    float *sKa = sm;              // Ktil_a
     float *sQb = sKa + MAT;       // Qtil_b
     float *sPa = sQb + MAT;       // P_a
     float *sPb = sPa + MAT;       // P_b
@@ -89,68 +47,21 @@ __global__ void __launch_bounds__(NT) compose_adj_kernel(const T *q, const T *k,
     float *sDQb = sDX + MAT;      // dQtil[b]
     float *sDKa = sDQb + MAT;     // dKtil[a]
     float *sDP = sDKa + MAT;      // dP
-    const int J = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    const int J = blockIdx.x, h = blockIdx.y;
     const int Lp = nblk * BT;
-    const long long row0 = (long long)h * L + (long long)J * BT;
-    const int nvalid = min(BT, L - J * BT);
+    const float *hv = halves + ((long long)h * nblk + J) * 4 * MAT;
     const float *dsd = dSd + ((long long)h * nblk + J) * BT * BT;
     const long long prow = (long long)h * Lp + (long long)J * BT;
+    // the halves' own quantities, as the forward's UT prep left them
+    cp_rows(sKa, hv, HB);
+    cp_rows(sQb, hv + MAT, HB);
+    cp_rows(sPa, hv + 2 * MAT, HB);
+    cp_rows(sPb, hv + 3 * MAT, HB);
     cp_rows(sDX, dsd + (long long)HB * BT, BT);
     cp_rows(sDQb, dQt + (prow + HB) * D, D);
     cp_rows(sDKa, dKt + prow * D, D);
     cp_rows(sDP, dPm + ((long long)h * nblk + J) * D * D, D);
-    {
-        float4 wv[BT * D / 4 / NT];
-#pragma unroll
-        for (int j = 0; j < BT * D / 4 / NT; ++j) {
-            const int e = tid + j * NT, r = e >> 4, c = (e & 15) * 4;
-            wv[j] = r < nvalid ? ld4(w + row0 * D, D, r, c, vec) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int j = 0; j < BT * D / 4 / NT; ++j) {
-            const int e = tid + j * NT, r = e >> 4, c = (e & 15) * 4;
-            *reinterpret_cast<float4 *>(sW + wx(r, c)) = wv[j];
-        }
-    }
-    for (int r = tid; r < BT; r += NT) sBt[r] = r < nvalid ? beta[row0 + r] : 0.f;
     cp_async_wait_all();
-    __syncthreads();
-    // the halves' own quantities, by recurrence; lane pair (2r, 2r+1) of role g
-    // holds row or column r, 32 columns each; the step index is warp-uniform
-    {
-        const int g = tid >> 7, r = (tid & 127) >> 1, p = tid & 1, rw = r & ~15;
-        float x[32];
-        if (g == 0) {  // key r of half a carried to the end of half a
-#pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-                const float4 v = r < nvalid ? ld4(k + row0 * D, D, r, 32 * p + c, vec)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                x[c] = v.x, x[c + 1] = v.y, x[c + 2] = v.z, x[c + 3] = v.w;
-            }
-            for (int t = rw + 1; t < HB; ++t) apply_h_half(x, sW, sBt, t, p, t > r);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) sKa[sx(r, 32 * p + c)] = x[c];
-        } else if (g == 1) {  // query 64+r of half b carried back to the start of half b
-            const int i = HB + r;
-#pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-                const float4 v = i < nvalid ? ld4(q + row0 * D, D, i, 32 * p + c, vec)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                x[c] = v.x, x[c + 1] = v.y, x[c + 2] = v.z, x[c + 3] = v.w;
-            }
-            for (int t = HB + rw + 15; t >= HB; --t) apply_h_half(x, sW, sBt, t, p, t <= i);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) sQb[sx(r, 32 * p + c)] = x[c];
-        } else {  // column r of P_a (g == 2) or P_b (g == 3)
-            const int t0 = g == 2 ? 0 : HB;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) x[c] = 32 * p + c == r ? 1.f : 0.f;
-            for (int t = t0; t < t0 + HB; ++t) apply_h_half(x, sW, sBt, t, p);
-            float *dst = g == 2 ? sPa : sPb;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) dst[sx(32 * p + c, r)] = x[c];
-        }
-    }
     __syncthreads();
     // each product goes straight from registers to global memory; every read
     // of dQt / dKt (the copies above) completed before the barrier above
@@ -327,9 +238,9 @@ template <typename T, typename TO>
 cudaError_t run(const PrepDims &Dm, const PrepInputs &in, const PrepGrads &g, float *dP64,
                 cudaStream_t st)
 {
-    const size_t smc = (BT * WLD + BT + 8 * MAT) * sizeof(float);
+    const size_t smc = 8 * MAT * sizeof(float);
     const size_t smu = (14 * MAT + HB) * sizeof(float);
-    auto kc = compose_adj_kernel<T>;
+    auto kc = compose_adj_kernel;
     auto ku = ut_adj64_kernel<T, TO>;
     cudaError_t e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smc);
     if (e == cudaSuccess)
@@ -340,8 +251,7 @@ cudaError_t run(const PrepDims &Dm, const PrepInputs &in, const PrepGrads &g, fl
     const bool vec = rows_vec_aligned<T>(q) && rows_vec_aligned<T>(k) && rows_vec_aligned<T>(w);
     {
         Stage s_c("ut_adj_compose", st);
-        kc<<<dim3(Dm.nblk, Dm.nh), NT, smc, st>>>(q, k, w, in.beta, Dm.L, Dm.nblk, vec,
-                                                  const_cast<float *>(g.dQt),
+        kc<<<dim3(Dm.nblk, Dm.nh), NT, smc, st>>>(g.halves, Dm.nblk, const_cast<float *>(g.dQt),
                                                   const_cast<float *>(g.dKt), g.dPm, g.dSd, dP64);
         count_launches();
     }
@@ -361,6 +271,7 @@ cudaError_t run(const PrepDims &Dm, const PrepInputs &in, const PrepGrads &g, fl
 }  // namespace
 
 bool prep_backward_fused_supported(const PrepDims &Dm) { return Dm.d == D; }
+
 
 // dQt and dKt are overwritten (used as scratch for the per-half adjoints).
 // All workspace buffers handed in (dQt, dKt, dPm, dSd, dP64) are 16-byte aligned.

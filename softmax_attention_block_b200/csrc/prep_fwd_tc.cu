@@ -72,7 +72,7 @@ template <typename T, typename TM>
 __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k, const T *w,
                                                          const float *beta, int L, int nblk,
                                                          bool vec, TM *Qt, TM *Kt, TM *Pm,
-                                                         float *Sd)
+                                                         float *Sd, float *halves)
 {
     constexpr bool EX = std::is_same<T, bf16>::value;  // W, Q, K exact in tf32
     extern __shared__ __align__(16) float sm[];
@@ -165,6 +165,18 @@ __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k,
             put_identity_plus(half == 0 ? sPa : sPb, f);
         }
     }
+    if (halves) {
+        // Ktil_a, Qtil_b, P_a, P_b for the backward's composition adjoint
+        float *dst = halves + ((long long)h * nblk + J) * 4 * MAT;
+        const float *src[4] = {sKa, sQb, sPa, sPb};
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            for (int e = tid; e < MAT / 4; e += NT) {
+                const int r = e >> 4, c = (e & 15) * 4;
+                *reinterpret_cast<float4 *>(dst + m * MAT + r * HB + c) =
+                    *reinterpret_cast<const float4 *>(src[m] + sx(r, c));
+            }
+    }
     // compose the 128-block
     {
         Frag f;
@@ -200,7 +212,7 @@ cudaError_t run(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out
     const bool vec = rows_vec_aligned<T>(q) && rows_vec_aligned<T>(k) && rows_vec_aligned<T>(w);
     kern<<<dim3(Dm.nblk, Dm.nh), NT, smem, st>>>(q, k, w, in.beta, Dm.L, Dm.nblk, vec,
                                                  static_cast<TM *>(out.Qt), static_cast<TM *>(out.Kt),
-                                                 static_cast<TM *>(out.Pm), out.Sd);
+                                                 static_cast<TM *>(out.Pm), out.Sd, out.halves);
     count_launches();
     return cudaGetLastError();
 }

@@ -34,6 +34,8 @@ using namespace ut64;
 // ---------------------------------------------------------------------------
 // 1. 128-level adjoints -> per-half adjoints (in place for dQt / dKt)
 // ---------------------------------------------------------------------------
+// SPLIT: split-TF32 products (fp32 inputs); otherwise single TF32 (bf16 inputs).
+template <bool SPLIT>
 __global__ void __launch_bounds__(NT) compose_adj_kernel(const float *halves, int nblk, float *dQt,
                                                          float *dKt, const float *dPm,
                                                          const float *dSd, float *dP64)
@@ -67,26 +69,26 @@ __global__ void __launch_bounds__(NT) compose_adj_kernel(const float *halves, in
     // of dQt / dKt (the copies above) completed before the barrier above
     {  // dQtil_b = dQtil[b] P_a^T + dSd[b,a] Ktil_a
         Frag f;
-        mm<false, true>(f, sDQb, sPa);
-        mm<false, false>(f, sDX, sKa);
+        mm<false, true, false, false, SPLIT>(f, sDQb, sPa);
+        mm<false, false, false, false, SPLIT>(f, sDX, sKa);
         put_rows(dQt + (prow + HB) * D, D, f, nullptr, nullptr, HB);
     }
     {  // dKtil_a = dKtil[a] P_b + dSd[b,a]^T Qtil_b
         Frag f;
-        mm<false, false>(f, sDKa, sPb);
-        mm<true, false>(f, sDX, sQb);
+        mm<false, false, false, false, SPLIT>(f, sDKa, sPb);
+        mm<true, false, false, false, SPLIT>(f, sDX, sQb);
         put_rows(dKt + prow * D, D, f, nullptr, nullptr, HB);
     }
     {  // dP_a = Qtil_b^T dQtil[b] + P_b^T dP
         Frag f;
-        mm<true, false>(f, sQb, sDQb);
-        mm<true, false>(f, sPb, sDP);
+        mm<true, false, false, false, SPLIT>(f, sQb, sDQb);
+        mm<true, false, false, false, SPLIT>(f, sPb, sDP);
         put_rows(dP64 + ((long long)h * 2 * nblk + 2 * J) * D * D, D, f, nullptr, nullptr, HB);
     }
     {  // dP_b = dKtil[a]^T Ktil_a + dP P_a^T
         Frag f;
-        mm<true, false>(f, sDKa, sKa);
-        mm<false, true>(f, sDP, sPa);
+        mm<true, false, false, false, SPLIT>(f, sDKa, sKa);
+        mm<false, true, false, false, SPLIT>(f, sDP, sPa);
         put_rows(dP64 + ((long long)h * 2 * nblk + 2 * J + 1) * D * D, D, f, nullptr, nullptr, HB);
     }
 }
@@ -107,6 +109,9 @@ __global__ void __launch_bounds__(NT) ut_adj64_kernel(const T *q, const T *k, co
           *sDP = sDK + MAT, *sDS = sDP + MAT, *sDWh = sDS + MAT, *sDU = sDWh + MAT,
           *sB = sDU + MAT;
     constexpr bool EX = std::is_same<T, bf16>::value;  // W, Q, K exact in tf32
+    // bf16 inputs: single-TF32 products (the precision of the fp16
+    // intermediates of this path); fp32 inputs: split TF32 (near fp32)
+    constexpr bool SPLIT = !EX;
     const int blk = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
     const int J = blk / 2, half = blk % 2;
     const int Lp = nblk * BT;
@@ -134,18 +139,18 @@ __global__ void __launch_bounds__(NT) ut_adj64_kernel(const T *q, const T *k, co
     // forward quantities
     {
         Frag f;
-        mm<false, true, EX, EX>(f, sW, sW);
+        mm<false, true, EX, EX, SPLIT>(f, sW, sW);
         put(sA, f, 1.f, false, OUT_STRICT, sB);  // A = strictLower(D W W^T)
     }
     diag_inverse(sA);
     {
         Frag f;
-        mm<false, true, EX, EX>(f, sW, sK);
+        mm<false, true, EX, EX, SPLIT>(f, sW, sK);
         put(sN, f, 1.f, false, OUT_STRICT);  // N = strictLower(W K^T)
     }
     {
         Frag f;
-        mm<false, true, EX, EX>(f, sQ, sW);
+        mm<false, true, EX, EX, SPLIT>(f, sQ, sW);
         put(sM, f, 1.f, false, OUT_LOWER);  // M = lower(Q W^T)
     }
     // [What | U] = (I + A)^{-1} D [W | N]: forward substitution, 128 right-hand sides
@@ -155,44 +160,44 @@ __global__ void __launch_bounds__(NT) ut_adj64_kernel(const T *q, const T *k, co
         sU[sx(r, c)] = sB[r] * sN[sx(r, c)];
     }
     __syncthreads();
-    tri_solve<false>(sA, sWh, sU);
+    tri_solve<false, SPLIT>(sA, sWh, sU);
     // adjoint
     {
         Frag f;
-        mm<true, false>(f, sM, sDQ);
-        mm<false, false, EX, false>(f, sW, sDP);
+        mm<true, false, false, false, SPLIT>(f, sM, sDQ);
+        mm<false, false, EX, false, SPLIT>(f, sW, sDP);
         put(sDWh, f, -1.f, false, OUT_ALL);  // dWhat = -M^T dQtil - W dP
     }
     {
         Frag f;
-        mm<false, true, EX, false>(f, sW, sDK);
-        mm<true, false>(f, sM, sDS);
+        mm<false, true, EX, false, SPLIT>(f, sW, sDK);
+        mm<true, false, false, false, SPLIT>(f, sM, sDS);
         put(sDU, f, -1.f, false, OUT_ALL);  // dU = -W dKtil^T - M^T dSd
     }
     {
         Frag f;
-        mm<false, true>(f, sDQ, sWh);
-        mm<false, true>(f, sDS, sU);
+        mm<false, true, false, false, SPLIT>(f, sDQ, sWh);
+        mm<false, true, false, false, SPLIT>(f, sDS, sU);
         put(sM, f, -1.f, false, OUT_LOWER);  // dM = lower(-dQtil What^T - dSd U^T), over M
     }
     {  // dq = dQtil + dSd K + dM W
         Frag f;
-        mm<false, false, false, EX>(f, sDS, sK);
-        mm<false, false, false, EX>(f, sM, sW);
+        mm<false, false, false, EX, SPLIT>(f, sDS, sK);
+        mm<false, false, false, EX, SPLIT>(f, sM, sW);
         put_rows(dq + row0 * D, D, f, sDQ, nullptr, nvalid);
     }
     // dR = (I + A)^{-T} [dWhat | dU]: backward substitution (its barriers also
     // order the dq reads of sDQ before sDQ is overwritten below)
-    tri_solve<true>(sA, sDWh, sDU);
+    tri_solve<true, SPLIT>(sA, sDWh, sDU);
     {  // dA = strictLower(-(dR_w What^T + dR_n U^T))   (into sDQ)
         Frag f;
-        mm<false, true>(f, sDWh, sWh);
-        mm<false, true>(f, sDU, sU);
+        mm<false, true, false, false, SPLIT>(f, sDWh, sWh);
+        mm<false, true, false, false, SPLIT>(f, sDU, sU);
         put(sDQ, f, -1.f, false, OUT_STRICT);
     }
     {  // G = W W^T over A (free after the solves)
         Frag f;
-        mm<false, true, EX, EX>(f, sW, sW);
+        mm<false, true, EX, EX, SPLIT>(f, sW, sW);
         put(sA, f, 1.f, false, OUT_ALL);
     }
     // dbeta_a = dR_w[a].W[a] + dR_n[a].N[a] + sum_{b<a} dA[a][b] G[a][b]; eight lanes per row
@@ -217,18 +222,18 @@ __global__ void __launch_bounds__(NT) ut_adj64_kernel(const T *q, const T *k, co
     scale_rows_mask(sDQ, sB, OUT_STRICT);
     {  // dk = dKtil + dSd^T Q + dN^T W
         Frag f;
-        mm<true, false, false, EX>(f, sDS, sQ);
-        mm<true, false, false, EX>(f, sDU, sW);
+        mm<true, false, false, EX, SPLIT>(f, sDS, sQ);
+        mm<true, false, false, EX, SPLIT>(f, sDU, sW);
         put_rows(dk + row0 * D, D, f, sDK, nullptr, nvalid);
     }
     {  // dw = D dR_w - U dKtil - What dP^T + dM^T Q + dN K + (dG + dG^T) W
         Frag f;
-        mm<false, false>(f, sU, sDK, -1.f);
-        mm<false, true>(f, sWh, sDP, -1.f);
-        mm<true, false, false, EX>(f, sM, sQ);
-        mm<false, false, false, EX>(f, sDU, sK);
-        mm<false, false, false, EX>(f, sDQ, sW);
-        mm<true, false, false, EX>(f, sDQ, sW);
+        mm<false, false, false, false, SPLIT>(f, sU, sDK, -1.f);
+        mm<false, true, false, false, SPLIT>(f, sWh, sDP, -1.f);
+        mm<true, false, false, EX, SPLIT>(f, sM, sQ);
+        mm<false, false, false, EX, SPLIT>(f, sDU, sK);
+        mm<false, false, false, EX, SPLIT>(f, sDQ, sW);
+        mm<true, false, false, EX, SPLIT>(f, sDQ, sW);
         put_rows(dw + row0 * D, D, f, sDWh, sB, nvalid);
     }
 }
@@ -240,7 +245,7 @@ cudaError_t run(const PrepDims &Dm, const PrepInputs &in, const PrepGrads &g, fl
 {
     const size_t smc = 8 * MAT * sizeof(float);
     const size_t smu = (14 * MAT + HB) * sizeof(float);
-    auto kc = compose_adj_kernel;
+    auto kc = compose_adj_kernel<std::is_same<T, float>::value>;
     auto ku = ut_adj64_kernel<T, TO>;
     cudaError_t e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smc);
     if (e == cudaSuccess)

@@ -75,6 +75,9 @@ __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k,
                                                          float *Sd, float *halves)
 {
     constexpr bool EX = std::is_same<T, bf16>::value;  // W, Q, K exact in tf32
+    // bf16 inputs: single-TF32 products (the precision of the fp16 outputs of
+    // this path); fp32 inputs: split TF32 (near fp32)
+    constexpr bool SPLIT = !EX;
     extern __shared__ __align__(16) float sm[];
     // working set of one half, then what the composition keeps
     float *sW = sm, *sQw = sW + MAT, *sKw = sQw + MAT, *sA = sKw + MAT, *sM = sA + MAT,
@@ -106,18 +109,18 @@ __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k,
         __syncthreads();
         {
             Frag f;
-            mm<false, true, EX, EX>(f, sW, sW);
+            mm<false, true, EX, EX, SPLIT>(f, sW, sW);
             put(sA, f, 1.f, false, OUT_STRICT, sB);  // A = strictLower(D W W^T)
         }
         diag_inverse(sA);
         {
             Frag f;
-            mm<false, true, EX, EX>(f, sW, sK);
+            mm<false, true, EX, EX, SPLIT>(f, sW, sK);
             put(sU, f, 1.f, false, OUT_STRICT, sB);  // D N, N = strictLower(W K^T)
         }
         {
             Frag f;
-            mm<false, true, EX, EX>(f, sQ, sW);
+            mm<false, true, EX, EX, SPLIT>(f, sQ, sW);
             put(sM, f, 1.f, false, OUT_LOWER);  // M = lower(Q W^T)
         }
         for (int e = tid; e < MAT; e += NT) {
@@ -125,12 +128,12 @@ __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k,
             sWh[sx(r, c)] = sB[r] * sW[sx(r, c)];
         }
         __syncthreads();
-        tri_solve<false>(sA, sWh, sU);  // [What | U] = (I + A)^{-1} D [W | N]
+        tri_solve<false, SPLIT>(sA, sWh, sU);  // [What | U] = (I + A)^{-1} D [W | N]
         {
             // Sd_hh = lower(Q K^T - M U); the block above the diagonal is zero
             Frag f;
-            mm<false, true, EX, EX>(f, sQ, sK);
-            mm<false, false>(f, sM, sU, -1.f);
+            mm<false, true, EX, EX, SPLIT>(f, sQ, sK);
+            mm<false, false, false, false, SPLIT>(f, sM, sU, -1.f);
             store_frag(sd + (long long)(half * HB) * BT + half * HB, BT, f, nullptr, false, OUT_LOWER);
             if (half == 0) {
                 for (int e = tid; e < MAT; e += NT) sd[(long long)(e / HB) * BT + HB + e % HB] = 0.f;
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k,
         {
             // Qtil_h = Q - M What (in place for half b: after every read of Q above)
             Frag f;
-            mm<false, false>(f, sM, sWh, -1.f);
+            mm<false, false, false, false, SPLIT>(f, sM, sWh, -1.f);
             if (half == 0) {
                 store_frag(Qt + prow * D, D, f, sQ, false, OUT_ALL);
             } else {
@@ -150,7 +153,7 @@ __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k,
         {
             // Ktil_h = K - U^T W (in place for half a: after every read of K above)
             Frag f;
-            mm<true, false, false, EX>(f, sU, sW, -1.f);
+            mm<true, false, false, EX, SPLIT>(f, sU, sW, -1.f);
             if (half == 0) {
                 __syncthreads();
                 put(sK, f, 1.f, true, OUT_ALL);
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k,
         {
             // P_h = I - W^T What
             Frag f;
-            mm<true, false, EX, false>(f, sW, sWh, -1.f);
+            mm<true, false, EX, false, SPLIT>(f, sW, sWh, -1.f);
             put_identity_plus(half == 0 ? sPa : sPb, f);
         }
     }
@@ -180,22 +183,22 @@ __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k,
     // compose the 128-block
     {
         Frag f;
-        mm<false, false>(f, sQb, sPa);
+        mm<false, false, false, false, SPLIT>(f, sQb, sPa);
         store_frag(Qt + (prow + HB) * D, D, f, nullptr, false, OUT_ALL);  // Qtil_b P_a
     }
     {
         Frag f;
-        mm<false, true>(f, sKa, sPb);
+        mm<false, true, false, false, SPLIT>(f, sKa, sPb);
         store_frag(Kt + prow * D, D, f, nullptr, false, OUT_ALL);  // Ktil_a P_b^T
     }
     {
         Frag f;
-        mm<false, false>(f, sPb, sPa);
+        mm<false, false, false, false, SPLIT>(f, sPb, sPa);
         store_frag(Pm + ((long long)h * nblk + J) * D * D, D, f, nullptr, false, OUT_ALL);
     }
     {
         Frag f;
-        mm<false, true>(f, sQb, sKa);
+        mm<false, true, false, false, SPLIT>(f, sQb, sKa);
         store_frag(sd + (long long)HB * BT, BT, f, nullptr, false, OUT_ALL);  // Qtil_b Ktil_a^T
     }
 }

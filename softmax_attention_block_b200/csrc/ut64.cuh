@@ -172,10 +172,12 @@ __device__ __forceinline__ void ldsm_x4(float (&r)[4], unsigned addr)
 }
 
 // f += sgn * op(A) op(B) over the full k = 64; A, B shared (layout sx),
-// op = transpose if TA / TB. EA / EB: the operand's values are exact in tf32
-// (bf16 data), so its low part is zero and those products are skipped.
-// Row-major fragments (A as is, B transposed) come by ldmatrix. No barrier.
-template <bool TA, bool TB, bool EA = false, bool EB = false>
+// op = transpose if TA / TB. SPLIT: split TF32 (near fp32); otherwise every
+// operand is rounded to TF32 once (one product per pair, fp16-class
+// accuracy). EA / EB: the operand's values are exact in tf32 (bf16 data), so
+// its low part is zero and those products are skipped. Row-major fragments
+// (A as is, B transposed) come by ldmatrix. No barrier.
+template <bool TA, bool TB, bool EA = false, bool EB = false, bool SPLIT = true>
 __device__ void mm(Frag &f, const float *A, const float *B, float sgn = 1.f)
 {
     const int lane = threadIdx.x & 31, g = lane >> 2, tg = lane & 3;
@@ -184,7 +186,7 @@ __device__ void mm(Frag &f, const float *A, const float *B, float sgn = 1.f)
     const int arow = m0 + lr + 8 * (lm & 1), acol = 4 * (lm >> 1);  // blocks a0..a3
     const int brow = n0 + lr + 8 * (lm >> 1), bcol = 4 * (lm & 1);  // b0, b1 of n-tile 0, then 1
     const unsigned abase = smem_u32(A), bbase = smem_u32(B);
-    constexpr int UNROLL = EA || EB ? 8 : 4;  // bounded by the registers of the fully split form
+    constexpr int UNROLL = EA || EB || !SPLIT ? 8 : 4;  // bounded by the registers of the split form
 #pragma unroll UNROLL
     for (int k0 = 0; k0 < HB; k0 += 8) {
         float af[4];
@@ -212,8 +214,11 @@ __device__ void mm(Frag &f, const float *A, const float *B, float sgn = 1.f)
         if (EA) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) ah[i] = __float_as_uint(af[i]), al[i] = 0u;
-        } else {
+        } else if (SPLIT) {
             split_a(af, ah, al);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ah[i] = to_tf32(af[i]), al[i] = 0u;
         }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -222,11 +227,13 @@ __device__ void mm(Frag &f, const float *A, const float *B, float sgn = 1.f)
             for (int i = 0; i < 2; ++i) {
                 if (EB)
                     bh[i] = __float_as_uint(bq[2 * nt + i]), bl[i] = 0u;
-                else
+                else if (SPLIT)
                     split_tf32(bq[2 * nt + i], bh[i], bl[i]);
+                else
+                    bh[i] = to_tf32(bq[2 * nt + i]), bl[i] = 0u;
             }
-            if (!EA) mma_tf32(f.v[nt], al, bh);
-            if (!EB) mma_tf32(f.v[nt], ah, bl);
+            if (SPLIT && !EA) mma_tf32(f.v[nt], al, bh);
+            if (SPLIT && !EB) mma_tf32(f.v[nt], ah, bl);
             mma_tf32(f.v[nt], ah, bh);
         }
     }
@@ -312,7 +319,7 @@ __device__ void diag_inverse(float *sA)
 // Z_c - sum over solved chunks k of A_ck X_k, then X_c = T_c (that) with
 // T_c the block inverse (transposed for the transposed system), both on the
 // tensor cores.
-template <bool TRANS>
+template <bool TRANS, bool SPLIT = true>
 __device__ void tri_solve(const float *sA, float *Z0, float *Z1)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tg = lane & 3;
@@ -323,10 +330,16 @@ __device__ void tri_solve(const float *sA, float *Z0, float *Z1)
     auto chunk_mma = [&](float (&acc)[4], int r0, int k0) {
         const float af[4] = {sys(r0 + g, k0 + tg), sys(r0 + g + 8, k0 + tg), sys(r0 + g, k0 + tg + 4),
                              sys(r0 + g + 8, k0 + tg + 4)};
-        uint32_t ah[4], al[4];
-        split_a(af, ah, al);
         const float bf[2] = {Z[sx(k0 + tg, c0 + g)], Z[sx(k0 + tg + 4, c0 + g)]};
-        mma3(acc, ah, al, bf);
+        if (SPLIT) {
+            uint32_t ah[4], al[4];
+            split_a(af, ah, al);
+            mma3(acc, ah, al, bf);
+        } else {
+            const uint32_t ah[4] = {to_tf32(af[0]), to_tf32(af[1]), to_tf32(af[2]), to_tf32(af[3])};
+            const uint32_t bh[2] = {to_tf32(bf[0]), to_tf32(bf[1])};
+            mma_tf32(acc, ah, bh);
+        }
     };
     for (int cb = 0; cb < 4; ++cb) {
         const int r0 = TRANS ? (3 - cb) * 16 : cb * 16;

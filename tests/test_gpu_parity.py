@@ -155,10 +155,16 @@ def test_backward_reusing_forward_workspace(P, fox):
         out, lse, g = run_ours(P, x, True, out_dtype=torch.float32, reuse=reuse)
         compare(ours_dict(out, lse, g), ref, "bf16in_f32out", f"reuse={reuse} fox={fox}")
         outs.append(g)
-    # dQtil accumulates across key tiles with fp32 atomics, so the two runs may
-    # differ in the last bits (summation order), not more
+    # dQtil and dP_I accumulate across key tiles by fp32 reductions whose order
+    # varies from run to run; the bf16-input path rounds the UT adjoint's
+    # operands to TF32 (11 significant bits), where such a last-bit difference
+    # can flip a rounding. So the two runs agree to that resolution, not more.
     for n in outs[0]:
-        torch.testing.assert_close(outs[0][n], outs[1][n], rtol=1e-5, atol=1e-6, msg=n)
+        a, b = outs[0][n].float(), outs[1][n].float()
+        tol = 2.0 ** -9 * float(a.abs().max()) + 1e-6
+        diff = float((a - b).abs().max())
+        print(f"[reuse vs recompute | {n}] max diff {diff:.3g} (bound {tol:.3g})")
+        assert diff <= tol, (n, diff, tol)
 
 
 def test_bf16_l1024_fwd_bwd(P):

@@ -5,7 +5,8 @@
 // for S^T, dP^T, dV and the chain adjoint Abar. Per tile pair:
 //   MMA 1:  S^T  = Khat_{J,I} Qtil_I^T          (fp16)
 //           dP^T = V_J dO_I^T                    (bf16)
-//           issued as two 64-query halves, one per elementwise warpgroup
+//           issued as soon as the previous pair's S^T / dP^T are consumed, ahead
+//           of that pair's MMA 2
 //   threads: P = exp(scale S + c_i - c_j - lse_i), dZ = P (dP - delta_i),
 //            dS = scale dZ; P^T (bf16) and dS^T (fp16) to shared memory;
 //            [gate] row sums of dS by warp reduce-scatter, column sums per thread
@@ -21,7 +22,7 @@
 // prep's adjoint instead (dSd), which carries it to dQ, dK, dW, dbeta.
 //
 // Every accumulator has its own TMEM columns, so MMA 1 of the next pair runs
-// while the warpgroups drain MMA 2's results of this one.
+// while MMA 2 of this one and the drain of its results proceed.
 #include "attn.cuh"
 #include "attn_tc.cuh"
 #include "runtime.cuh"
@@ -34,9 +35,12 @@ namespace {
 using namespace tc;
 
 constexpr int D = 64;
-constexpr int NT = 320;                  // warps 0-7 elementwise (two warpgroups), 8 producer, 9 MMA
-constexpr int NEW = 256;                 // elementwise threads
-constexpr int W_PROD = 8, W_MMA = 9;
+// warps 0-7: softmax (two warpgroups, one per 64-query half); 8-11: drain of
+// MMA 2's results; 12: TMA producer; 13: MMA issue; 14-15: idle
+constexpr int NT = 512;
+constexpr int NEW = 256;                 // softmax threads
+constexpr int NDR = 128;                 // drain threads
+constexpr int W_DRAIN0 = 8, W_PROD = 12, W_MMA = 13;
 constexpr float LOG2E = 1.4426950408889634f;
 
 struct BCfg {
@@ -95,11 +99,11 @@ __global__ void __launch_bounds__(NT, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&ld_full[s], 1);
             mbar_init(&ld_empty[s], 1);
-            mbar_init(&s_full[s], 1);
         }
+        mbar_init(s_full, 1);
         mbar_init(p_full, NEW);
         mbar_init(m2_full, 1);
-        mbar_init(e_done, NEW);
+        mbar_init(e_done, NDR);
         mbar_fence_init();
     }
     if (warp == W_MMA) tmem_alloc(tmem_slot, 512);
@@ -144,48 +148,49 @@ __global__ void __launch_bounds__(NT, 1)
         // the whole warp runs the issue loop (uniform descriptors); lane 0 issues
         const uint32_t lead = lane == 0;
         {
-            const uint32_t idS = idesc_f16(128, 64, AB_F16, 0, 0);
-            const uint32_t idDP = idesc_f16(128, 64, AB_BF16, 0, 0);
+            const uint32_t idS = idesc_f16(128, 128, AB_F16, 0, 0);
+            const uint32_t idDP = idesc_f16(128, 128, AB_BF16, 0, 0);
             const uint32_t idDV = idesc_f16(128, D, AB_BF16, 0, 1);
             const uint32_t idAbP = idesc_f16(128, D, AB_F16, 0, 1);
             const uint32_t idMN = idesc_f16(128, D, AB_F16, 1, 1);
             const uint32_t ab0 = smem_u32(sAb), v0 = smem_u32(sV), pt0 = smem_u32(sPt),
                            ds0 = smem_u32(sDs);
-            bool ok = mbar_wait(v_full, 0, WAIT_POLLS);
+            // MMA 1 of pair it: S^T = Khat Qtil^T (not on the diagonal), dP^T = V dO^T
+            auto mma1 = [&](int it) -> bool {
+                const int s = it & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_POLLS)))
+                    return false;
+                fence_after_sync();
+                const uint32_t kh0 = smem_u32(stage(s) + C::S_KH), q0 = smem_u32(stage(s) + C::S_Q),
+                               do0 = smem_u32(stage(s) + C::S_DO);
+                if (it != niter - 1) {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss_if(lead, tbase + C::T_S, desc_sw128(kh0 + kk * 32, 16, 1024),
+                                  desc_sw128(q0 + kk * 32, 16, 1024), idS, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss_if(lead, tbase + C::T_DP, desc_sw128(v0 + kk * 32, 16, 1024),
+                              desc_sw128(do0 + kk * 32, 16, 1024), idDP, kk > 0);
+                commit_if(lead, s_full);
+                return true;
+            };
+            bool ok = __all_sync(0xffffffffu, mbar_wait(v_full, 0, WAIT_POLLS)) && mma1(0);
             for (int it = 0; ok && it < niter; ++it) {
                 const int s = it & 1, I = tile_of(it);
                 const bool diag = it == niter - 1;
-                // S^T / dP^T are free: the warpgroups consumed them before MMA 2 of the
-                // previous pair was issued (below)
-                if (!mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_POLLS)) {
+                // MMA 2 needs this pair's P / dS in shared memory, and overwrites the
+                // previous pair's results: drained by then?
+                const bool ready = mbar_wait(p_full, it & 1, WAIT_POLLS) &&
+                                   (it == 0 || mbar_wait(e_done, (it - 1) & 1, WAIT_POLLS));
+                if (!__all_sync(0xffffffffu, ready)) {  // the warp stays converged
                     ok = false;
                     break;
                 }
                 fence_after_sync();
                 const uint32_t kh0 = smem_u32(stage(s) + C::S_KH), q0 = smem_u32(stage(s) + C::S_Q),
                                do0 = smem_u32(stage(s) + C::S_DO), p0 = smem_u32(stage(s) + C::S_P);
-                // MMA 1, one 64-query half at a time (queries 64hf.. are rows 64hf.. of Q, dO)
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    if (!diag) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            mma_ss_if(lead, tbase + C::T_S + 64 * hf, desc_sw128(kh0 + kk * 32, 16, 1024),
-                                   desc_sw128(q0 + hf * 8192 + kk * 32, 16, 1024), idS, kk > 0);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss_if(lead, tbase + C::T_DP + 64 * hf, desc_sw128(v0 + kk * 32, 16, 1024),
-                               desc_sw128(do0 + hf * 8192 + kk * 32, 16, 1024), idDP, kk > 0);
-                    commit_if(lead, &s_full[hf]);
-                }
-                // MMA 2 needs this pair's P / dS, and the previous pair's results drained
-                if (!mbar_wait(p_full, it & 1, WAIT_POLLS) ||
-                    (it >= 1 && !mbar_wait(e_done, (it - 1) & 1, WAIT_POLLS))) {
-                    ok = false;
-                    break;
-                }
-                fence_after_sync();
                 // dV += P^T dO   (K = 128 queries)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -216,43 +221,43 @@ __global__ void __launch_bounds__(NT, 1)
                         mma_ss_if(lead, tbase + C::T_DQ, desc_sw128(ds0 + kk * 2048, 16384, 1024),
                                desc_sw128(kh0 + kk * 2048, 16384, 1024), idMN, kk > 0);
                 }
-                commit_if(lead, m2_full);
-                commit_if(lead, &ld_empty[s]);
+                commit_if(lead, m2_full);  // the drain frees the stage after using it
+                // the next pair's MMA 1 (S^T / dP^T were consumed before this MMA 2);
+                // its completion also orders the next softmax's P / dS writes after
+                // this MMA 2's reads
+                if (it + 1 < niter && !mma1(it + 1)) {
+                    ok = false;
+                    break;
+                }
             }
             if (!ok && lead && a.err) atomicCAS(a.err, 0, 12);
         }
-    } else {
-        // elementwise warpgroups: warpgroup g takes query columns [64g, 64g + 64);
+    } else if (warp < W_DRAIN0) {
+        // softmax warpgroups: warpgroup g takes query columns [64g, 64g + 64);
         // thread j owns key row j of tile J. Per query i the rows hold
         // nb_i = (c_i - lse_i) log2(e) and scale * delta_i.
         const int g = warp >> 2, j = tid & 127;
         const int gj = J * BT + j;
-        const bool valid = gj < a.L;
-        const bool leader = j == 0;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const float k1 = a.scale * LOG2E;
         const float cj2 = FOX ? a.c[(long long)h * Lp + gj] * LOG2E : 0.f;
-        // fp32 staging of this warpgroup's 32 columns of dQtil / dP_I for the tile
-        // reductions, inside its own P^T / dS^T panel (free between MMA 2 and the
-        // next pair's probabilities)
-        uint8_t *stq = sPt + g * 16384, *stp = sDs + g * 16384;
         float colsum = 0.f;
         bool ok = true;
-        // Every thread runs every iteration and every named barrier; after a
-        // failed wait the work is skipped, never the barriers.
         for (int it = 0; it < niter; ++it) {
             const int s = it & 1, I = tile_of(it);
             const bool diag = it == niter - 1;
+            // s_full also orders this pair's P / dS writes after the previous MMA 2
             if (ok && (!mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_POLLS) ||
-                       !mbar_wait(&s_full[g], it & 1, WAIT_POLLS)))
+                       !mbar_wait(s_full, it & 1, WAIT_POLLS)))
                 ok = false;
+            ok = __all_sync(0xffffffffu, ok);  // shuffles and TMEM loads below are warp-wide
             fence_after_sync();
-            // the previous pair's tile reductions have finished reading the staging
-            if (it > 0) named_barrier(2 + g, 128);
             const float *rows = reinterpret_cast<const float *>(stage(s) + C::S_ROW);
             const float *sd = a.Sd + ((long long)h * nblk + J) * BT * BT;
             float *dsd = a.dSd + ((long long)h * nblk + J) * BT * BT;
-            auto load = [&](int c, float (&sv)[16], float (&dp)[16]) {
+#pragma unroll 1
+            for (int c = 64 * g; ok && c < 64 * g + 64; c += 16) {
+                float sv[16], dp[16];
                 if (diag) {
 #pragma unroll
                     for (int u = 0; u < 16; ++u) sv[u] = sd[(c + u) * BT + j];
@@ -260,8 +265,7 @@ __global__ void __launch_bounds__(NT, 1)
                     tmem_ld16(tbase + C::T_S + c + lane_off, sv);
                 }
                 tmem_ld16(tbase + C::T_DP + c + lane_off, dp);
-            };
-            auto chunk = [&](int c, const float (&sv)[16], const float (&dp)[16]) {
+                tmem_wait_ld_tied(sv, dp);
                 float pv[16], dsv[16];
                 const float4 *nb4 = reinterpret_cast<const float4 *>(rows + c);
                 const float4 *sd4 = reinterpret_cast<const float4 *>(rows + 128 + c);
@@ -322,34 +326,39 @@ __global__ void __launch_bounds__(NT, 1)
                     if (!(lane & 1))
                         atomicAdd(a.rowsum + (long long)h * Lp + I * BT + c + (lane >> 1), dsv[0] / a.scale);
                 }
-            };
-            if (ok) {
-                // 16-column chunks; the next chunk's TMEM loads are in flight
-                // while the current one is computed
-                float sA[16], dA[16], sB[16], dB[16];
-                const int cb = 64 * g;
-                load(cb, sA, dA);
-                tmem_wait_ld_tied(sA, dA);
-                load(cb + 16, sB, dB);
-                chunk(cb, sA, dA);
-                tmem_wait_ld_tied(sB, dB);
-                load(cb + 32, sA, dA);
-                chunk(cb + 16, sB, dB);
-                tmem_wait_ld_tied(sA, dA);
-                load(cb + 48, sB, dB);
-                chunk(cb + 32, sA, dA);
-                tmem_wait_ld_tied(sB, dB);
-                chunk(cb + 48, sB, dB);
             }
             fence_async_smem();
             fence_before_sync();
             mbar_arrive(p_full);
+        }
+        // column sums: warpgroup 1 hands its half to warpgroup 0
+        if (g == 1) sCs[j] = colsum;
+        named_barrier(1, NEW);
+        if (!ok && a.err) atomicCAS(a.err, 0, 13);
+        if (ok && g == 0 && a.colsum && gj < a.L) a.colsum[(long long)h * Lp + gj] = (colsum + sCs[j]) / a.scale;
+    } else if (warp < W_PROD) {
+        // drain warpgroup: thread j = lane j of TMEM (key row for Abar and dV, query
+        // row for dQtil, row f < 64 of dP_I); all 64 columns of each result.
+        // dQtil and dP_I leave through fp32 staging (128B-swizzled boxes of 32
+        // columns) in this pair's operand stage, free once MMA 2 has completed,
+        // and bulk tensor reduce-add; the stage goes back to the producer after the
+        // reductions have read it.
+        const int j = tid - 32 * W_DRAIN0;
+        const int gj = J * BT + j;
+        const bool leader = j == 0;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        bool ok = true;
+        for (int it = 0; it < niter; ++it) {
+            const int s = it & 1, I = tile_of(it);
+            const bool diag = it == niter - 1;
             if (ok && !mbar_wait(m2_full, it & 1, WAIT_POLLS)) ok = false;
+            ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-wide
             fence_after_sync();
+            uint8_t *stq = stage(s), *stp = stage(s) + 2 * 16384;  // dQtil: 2 x 16 KB, dP_I: 2 x 8 KB
             const bool drain = ok && !diag;
-            const int c0 = 32 * g;  // this warpgroup's 32 columns of each d-wide result
             if (drain) {
-                {
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
                     // chain adjoint: operand for the next pair, or dKtil_J after pair (J+1, J)
                     float v[32];
                     tmem_ld32(tbase + C::T_AB + c0 + lane_off, v);
@@ -370,62 +379,75 @@ __global__ void __launch_bounds__(NT, 1)
                             *reinterpret_cast<float4 *>(dk + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
                     }
                 }
-                {
-                    // dQtil rows of tile I (lane = query row), staged 128B-swizzled
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    // dQtil rows of tile I (lane = query row)
                     float v[32];
                     tmem_ld32(tbase + C::T_DQ + c0 + lane_off, v);
                     tmem_wait_ld();
+                    uint8_t *box = stq + (c0 >> 5) * 16384 + j * 128;
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        *reinterpret_cast<float4 *>(stq + j * 128 + ((k ^ (j & 7)) << 4)) =
+                        *reinterpret_cast<float4 *>(box + ((k ^ (j & 7)) << 4)) =
                             make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
                 }
                 if (I < last) {
-                    // dP_I rows f = 0..63 live in lanes 0..63 (warps 0, 1 of each warpgroup)
-                    float v[32];
-                    tmem_ld32(tbase + C::T_DPI + c0 + lane_off, v);
-                    tmem_wait_ld();
-                    if (j < D) {
+                    // dP_I rows f = 0..63 live in lanes 0..63 (the first two warps)
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        float v[32];
+                        tmem_ld32(tbase + C::T_DPI + c0 + lane_off, v);
+                        tmem_wait_ld();
+                        if (j < D) {
+                            uint8_t *box = stp + (c0 >> 5) * 8192 + j * 128;
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            *reinterpret_cast<float4 *>(stp + j * 128 + ((k ^ (j & 7)) << 4)) =
-                                make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                            for (int k = 0; k < 8; ++k)
+                                *reinterpret_cast<float4 *>(box + ((k ^ (j & 7)) << 4)) =
+                                    make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                        }
                     }
                 }
                 fence_async_smem();
             }
-            named_barrier(2 + g, 128);
-            if (drain && leader) {
-                tma_reduce_add_2d(&mDQ, c0, h * Lp + I * BT, stq);
-                if (I < last) tma_reduce_add_2d(&mDPI, c0, (h * nblk + I) * D, stp);
-                bulk_commit();
-            }
+            // TMEM results read and Abar written: MMA 2 of the next pair may go
             fence_before_sync();
             mbar_arrive(e_done);
-            if (drain && leader) bulk_wait_read<0>();
+            named_barrier(2, NDR);  // every staging row written
+            if (leader) {
+                if (drain) {
+                    tma_reduce_add_2d(&mDQ, 0, h * Lp + I * BT, stq);
+                    tma_reduce_add_2d(&mDQ, 32, h * Lp + I * BT, stq + 16384);
+                    if (I < last) {
+                        tma_reduce_add_2d(&mDPI, 0, (h * nblk + I) * D, stp);
+                        tma_reduce_add_2d(&mDPI, 32, (h * nblk + I) * D, stp + 8192);
+                    }
+                    bulk_commit();
+                    bulk_wait_read<0>();
+                }
+                mbar_arrive(&ld_empty[s]);  // the producer may refill this stage
+            }
         }
         if (leader) bulk_wait_all();
         // the last tile has no off-diagonal pairs: its dKtil is zero
         if (ok && J == last) {
-            float *dk = a.dKt + ((long long)h * Lp + gj) * D + 32 * g;
-            for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4 *>(dk + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+            float *dk = a.dKt + ((long long)h * Lp + gj) * D;
+            for (int e = 0; e < D; e += 4) *reinterpret_cast<float4 *>(dk + e) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        // column sums: warpgroup 1 hands its half to warpgroup 0
-        if (g == 1) sCs[j] = colsum;
-        named_barrier(1, NEW);
-        // dV_J
+        // dV_J, complete after the last MMA 2 (waited for above)
         if (ok) {
-            float v[32];
-            tmem_ld32(tbase + C::T_DV + 32 * g + lane_off, v);
-            tmem_wait_ld();
-            if (valid) {
-                TO *dst = static_cast<TO *>(a.dv) + ((long long)h * a.L + gj) * D + 32 * g;
+            TO *dst = static_cast<TO *>(a.dv) + ((long long)h * a.L + gj) * D;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                float v[32];
+                tmem_ld32(tbase + C::T_DV + c0 + lane_off, v);  // warp-wide; rows past L drop
+                tmem_wait_ld();
+                if (gj < a.L) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) dst[e] = from_f<TO>(v[e]);
-                if (a.colsum && g == 0) a.colsum[(long long)h * Lp + gj] = (colsum + sCs[j]) / a.scale;
+                    for (int e = 0; e < 32; ++e) dst[c0 + e] = from_f<TO>(v[e]);
+                }
             }
         } else if (a.err) {
-            atomicCAS(a.err, 0, 13);
+            atomicCAS(a.err, 0, 14);
         }
     }
     fence_before_sync();

@@ -15,7 +15,9 @@
 // The diagonal tile's logits come precomputed from the UT prep (the
 // full-matrix form of each block); tiles J < I come from S = Qtil Khat^T.
 // Softmax works in the log2 domain; the running max rescales the register
-// accumulator when each P.V tile is added (one tile behind the MMA).
+// accumulator when each P.V tile is added. At head dim 64 P and the P.V tiles
+// are double-buffered: a tile's P.V is added two tiles later and S runs two
+// tiles ahead, so the softmax never waits for the P.V just issued.
 #include "attn.cuh"
 #include "attn_tc.cuh"
 #include "runtime.cuh"
@@ -38,14 +40,17 @@ struct Cfg {
     static constexpr int PANELS = D / 64;
     static constexpr int TILE = 128 * D * 2;  // bytes of one 128-row 16-bit tile
     static constexpr int NS = D == 64 ? 3 : 2;
+    // P buffers in shared memory and P.V tiles in TMEM: with two, a tile's P.V is
+    // folded into the accumulator two tiles later and S runs two tiles ahead
+    static constexpr int PB = D == 64 ? 2 : 1;
     static constexpr int Q_OFF = 0;
     static constexpr int ST_OFF = Q_OFF + TILE;
     static constexpr int ST_BYTES = 2 * TILE + 1024;  // K, V, gate prefix (512 B)
     static constexpr int P_OFF = ST_OFF + NS * ST_BYTES;
-    static constexpr int BAR_OFF = P_OFF + 128 * 128 * 2;
+    static constexpr int BAR_OFF = P_OFF + PB * 128 * 128 * 2;
     static constexpr int RED_OFF = BAR_OFF + 256;     // [2][2][128] row maxima, [2][128] row sums
     static constexpr int SMEM = RED_OFF + 6 * 128 * 4 + 1024;  // + alignment slack
-    static constexpr uint32_t TMEM_COLS = 512;       // S0 [0,128) S1 [128,256) O [256, 256+D)
+    static constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128) S1 [128,256) O_b [256 + b D, 256 + (b+1) D)
 };
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
@@ -101,8 +106,8 @@ __global__ void __launch_bounds__(NT, 1)
     uint64_t *kv_empty = bars + 1 + NS;
     uint64_t *s_full = bars + 1 + 2 * NS;
     uint64_t *p_full = bars + 3 + 2 * NS;
-    uint64_t *o_full = bars + 4 + 2 * NS;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 5 + 2 * NS);
+    uint64_t *o_full = bars + 4 + 2 * NS;  // [PB]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 + 2 * NS + C::PB);
     uint8_t *sQ = sm + C::Q_OFF;
     uint8_t *sP = sm + C::P_OFF;
     auto sK = [&](int s) { return sm + C::ST_OFF + s * C::ST_BYTES; };
@@ -124,7 +129,7 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
         mbar_init(p_full, NSOFT);
-        mbar_init(o_full, 1);
+        for (int b = 0; b < C::PB; ++b) mbar_init(&o_full[b], 1);
         mbar_fence_init();
     }
     if (warp == W_MMA) tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -169,38 +174,62 @@ __global__ void __launch_bounds__(NT, 1)
             const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
             bool ok = mbar_wait(q_full, 0, WAIT_POLLS) && mbar_wait(&kv_full[0], 0, WAIT_POLLS);
             fence_after_sync();
-            for (int it = 0; ok && it < niter; ++it) {
-                if (it + 1 < niter) {  // S for the next tile, overlapping this tile's softmax
-                    const int n = it + 1, s = n % NS, b = n & 1;
-                    if (!mbar_wait(&kv_full[s], (n / NS) & 1, WAIT_POLLS)) {
+            // S = Qtil Khat^T of tile n into S buffer n & 1 (tile 0, the diagonal,
+            // takes its logits from the UT prep)
+            auto issue_s = [&](int n) -> bool {
+                const int s = n % NS, b = n & 1;
+                if (!mbar_wait(&kv_full[s], (n / NS) & 1, WAIT_POLLS)) return false;
+                fence_after_sync();
+                const uint32_t k_addr = smem_u32(sK(s));
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+                    mma_ss(tbase + b * 128, desc_sw128(q_addr + off, 16, 1024),
+                           desc_sw128(k_addr + off, 16, 1024), idS, kk > 0);
+                }
+                commit(&s_full[b]);
+                return true;
+            };
+            // O_tile(it) = P(it) V(it) into P.V buffer it % PB
+            auto issue_pv = [&](int it) {
+                const int s = it % NS, pb = it % C::PB;
+                const uint32_t v_addr = smem_u32(sV(s)), pa = p_addr + pb * 32768;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t aoff = (kk / 4) * 16384 + (kk % 4) * 32;
+                    mma_ss(tbase + 256 + pb * D, desc_sw128(pa + aoff, 16, 1024),
+                           desc_sw128(v_addr + kk * 2048, 16384, 1024), idO, kk > 0);
+                }
+                commit(&o_full[pb]);
+                commit(&kv_empty[s]);
+            };
+            if (NS >= 3) {
+                // S two tiles ahead: S(it + 2) reuses the S buffer of tile it right
+                // after tile it's softmax, and its keys were loaded a tile earlier
+                for (int n = 1; ok && n <= 2 && n < niter; ++n) ok = issue_s(n);
+                for (int it = 0; ok && it < niter; ++it) {
+                    if (!mbar_wait(p_full, it & 1, WAIT_POLLS)) {
                         ok = false;
                         break;
                     }
                     fence_after_sync();
-                    const uint32_t k_addr = smem_u32(sK(s));
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-                        mma_ss(tbase + b * 128, desc_sw128(q_addr + off, 16, 1024),
-                               desc_sw128(k_addr + off, 16, 1024), idS, kk > 0);
+                    issue_pv(it);
+                    if (it >= 1 && it + 2 < niter && !issue_s(it + 2)) ok = false;
+                }
+            } else {
+                // S one tile ahead, overlapping this tile's softmax
+                for (int it = 0; ok && it < niter; ++it) {
+                    if (it + 1 < niter && !issue_s(it + 1)) {
+                        ok = false;
+                        break;
                     }
-                    commit(&s_full[b]);
+                    if (!mbar_wait(p_full, it & 1, WAIT_POLLS)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_after_sync();
+                    issue_pv(it);
                 }
-                if (!mbar_wait(p_full, it & 1, WAIT_POLLS)) {
-                    ok = false;
-                    break;
-                }
-                fence_after_sync();
-                const int s = it % NS;
-                const uint32_t v_addr = smem_u32(sV(s));
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t aoff = (kk / 4) * 16384 + (kk % 4) * 32;
-                    mma_ss(tbase + 256, desc_sw128(p_addr + aoff, 16, 1024),
-                           desc_sw128(v_addr + kk * 2048, 16384, 1024), idO, kk > 0);
-                }
-                commit(o_full);
-                commit(&kv_empty[s]);
             }
             if (!ok) flag_error(a.err, 2);
         }
@@ -222,6 +251,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
         for (int e = 0; e < DH; ++e) acc[e] = 0.f;
         float m = -INFINITY, l = 0.f, mA = -INFINITY;
+        float mh0 = -INFINITY, mh1 = -INFINITY;  // row max of the tiles in P.V buffers 0, 1
         bool ok = true;
         const float *sd = a.Sd + (((long long)h * a.nblk + I) * BT + r) * BT + c0s;
         // Every thread runs every iteration and every named barrier; after a
@@ -233,6 +263,7 @@ __global__ void __launch_bounds__(NT, 1)
             float z[64];
             float pmax = -INFINITY;
             if (ok && it > 0 && !mbar_wait(&s_full[b], ((it - 1) >> 1) & 1, WAIT_POLLS)) ok = false;
+            ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-wide
             if (ok) {
                 if (it == 0) {
 #pragma unroll
@@ -261,26 +292,31 @@ __global__ void __launch_bounds__(NT, 1)
             rb[hf * 128 + r] = pmax;
             named_barrier(1 + q4, 64);
             const float m_new = fmaxf(m, fmaxf(rb[r], rb[128 + r]));
-            // add the previous tile's P.V (scaled to its max m) into the accumulator
-            if (ok && it >= 1) {
-                if (!mbar_wait(o_full, (it - 1) & 1, WAIT_POLLS)) {
-                    ok = false;
-                } else {
+            // fold the P.V of tile it - PB (scaled to that tile's max) into the
+            // accumulator; its P buffer is then free for this tile's probabilities
+            if (it >= C::PB) {
+                const int t = it - C::PB, pb = t % C::PB;
+                if (ok && !mbar_wait(&o_full[pb], (t / C::PB) & 1, WAIT_POLLS)) ok = false;
+                ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-wide
+                if (ok) {
                     fence_after_sync();
-                    const float corr = ex2(mA - m);
+                    const float mt = pb == 0 ? mh0 : mh1;
+                    const float corr = ex2(mA - mt);
 #pragma unroll
                     for (int c0 = 0; c0 < DH; c0 += 32) {
                         float v[32];
-                        tmem_ld32(tbase + 256 + c0o + c0 + lane_off, v);
+                        tmem_ld32(tbase + 256 + pb * D + c0o + c0 + lane_off, v);
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
                     }
-                    mA = m;
+                    mA = mt;
                 }
             }
             if (ok) {
-                // probabilities -> P (fp16, swizzled K-major panel hf) and partial row sum
+                // probabilities -> P buffer it % PB (fp16, swizzled K-major panel hf)
+                // and partial row sum
+                uint8_t *pbuf = sP + (it % C::PB) * 32768 + hf * 16384;
                 float rowsum = 0.f;
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
@@ -293,28 +329,38 @@ __global__ void __launch_bounds__(NT, 1)
                         rowsum += p0 + p1;
                         hh[q2] = __floats2half2_rn(p0, p1);
                     }
-                    *reinterpret_cast<uint4 *>(sP + hf * 16384 + sw128_offset(r, g * 8)) = u;
+                    *reinterpret_cast<uint4 *>(pbuf + sw128_offset(r, g * 8)) = u;
                 }
                 l = fmaf(l, ex2(m - m_new), rowsum);
                 m = m_new;
+                if (it % C::PB == 0)
+                    mh0 = m_new;
+                else
+                    mh1 = m_new;
             }
             fence_async_smem();
             fence_before_sync();
             mbar_arrive(p_full);
         }
-        if (ok && mbar_wait(o_full, (niter - 1) & 1, WAIT_POLLS)) {
-            fence_after_sync();
-            const float corr = ex2(mA - m);
+        // the last PB tiles' P.V
+        for (int t = niter - C::PB > 0 ? niter - C::PB : 0; t < niter; ++t) {
+            const int pb = t % C::PB;
+            if (ok && !mbar_wait(&o_full[pb], (t / C::PB) & 1, WAIT_POLLS)) ok = false;
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                fence_after_sync();
+                const float mt = pb == 0 ? mh0 : mh1;
+                const float corr = ex2(mA - mt);
 #pragma unroll
-            for (int c0 = 0; c0 < DH; c0 += 32) {
-                float v[32];
-                tmem_ld32(tbase + 256 + c0o + c0 + lane_off, v);
-                tmem_wait_ld();
+                for (int c0 = 0; c0 < DH; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tbase + 256 + pb * D + c0o + c0 + lane_off, v);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
+                    for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
+                }
+                mA = mt;
             }
-        } else {
-            ok = false;
         }
         // row sum: both halves share the running max, so the partial sums add
         redl[hf * 128 + r] = l;

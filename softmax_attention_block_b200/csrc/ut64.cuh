@@ -99,9 +99,9 @@ struct Rows {
 // fp32 accumulation, which keeps the products close to fp32 accuracy.
 __device__ __forceinline__ uint32_t to_tf32(float x)
 {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    // nearest TF32 value (ties away from zero) by integer arithmetic on the
+    // ALU pipe: add half of the 13 dropped mantissa bits' range, then clear them
+    return (__float_as_uint(x) + 0x1000u) & 0xffffe000u;
 }
 
 __device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)

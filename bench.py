@@ -89,7 +89,7 @@ def stage_model(name, B, H, L, d, BT=128):
 # B=1 H=24 L=4096 d=64 case (profiles/ summaries), scaled to the benchmark's
 # B=8 by the heads processed; None where the kernel changed since the capture.
 DRAM_BYTES_B1H24 = {
-    "attn_bwd": 326.980352e6 + 96.854272e6,
+    "attn_bwd": 325.6e6 + 97.7e6,
 }
 
 
@@ -495,12 +495,30 @@ PROFILE_CASES = {
     "b1h24l4096": (1, 24, 4096, 64, False),
     "b1h6l16384fox": (1, 6, 16384, 64, True),
 }
+# name: (B, H, d, cached rows) -- two untimed decode steps on a 16K-row cache
+DECODE_PROFILE_CASES = {
+    "decode_b2h32c16k": (2, 32, 128, 16384),
+}
 
 
 def run_profile_case(name):
     """One forward and one backward (reusing the forward's workspace) on a small
-    shape of the benchmark workload, for ncu captures of single launches."""
+    shape of the benchmark workload, for ncu captures of single launches; or two
+    decode steps on a smaller batch of the decode workload."""
     import softmax_attention_block_b200 as P
+
+    if name in DECODE_PROFILE_CASES:
+        B, H, d, n0 = DECODE_PROFILE_CASES[name]
+        kc, vc, seq = si.make_decode_inputs(B, H, d, n0, n0 + 2, 2, torch.bfloat16, seed=0)
+        kd, vd = kc.cuda(), vc.cuda()
+        out = torch.empty((B, H, d), dtype=torch.bfloat16, device="cuda")
+        for t, s in enumerate(seq):
+            s = {k: v.cuda() for k, v in s.items()}
+            P.path_decode_step(s["q"], s["k_new"], s["v_new"], s["w"], s["beta"], kd, vd, n0 + t,
+                               out=out)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": name, "ok": bool(torch.isfinite(out.float()).all())}))
+        return 0
 
     B, H, L, d, fox = PROFILE_CASES[name]
     x = si.make_inputs(B, H, L, d, torch.bfloat16, seed=0, fox=fox)
@@ -526,7 +544,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES) + sorted(DECODE_PROFILE_CASES),
                     help="run one untimed fwd+bwd on a small shape (for profiler captures)")
     args = ap.parse_args()
     if args.profile_case:

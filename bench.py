@@ -72,16 +72,23 @@ def stage_model(name, B, H, L, d, BT=128):
         "attn_bwd_q": (3.0 * L * L * d, "tensor"),                    # S, dP, dQ (SIMT path)
         "attn_bwd_k": (4.0 * L * L * d + 2.0 * L * L * d * d / BT, "tensor"),
         "chain": (1.0 * L * L * d * d / BT, "tensor"),               # key-side block transport
-        # keys (Ktil + in-block logits), queries, block product: rank-one steps
-        "ut_prep": (nblk * (BT * BT / 2 * 10.0 * d + BT * 4.0 * d * d), "alu"),
-        # per 128-block: 8 products of 64x64 by 64xd, and 4 x 64 rank-one steps
-        "ut_adj_compose": (nblk * (8 * 2.0 * HB * HB * d + 4 * HB * HB * 4.0 * d), "tf32"),
+        # head dim 64 (tensor-core prep): per 64-half 8 products 64x64xd and a
+        # 64x128 triangular solve, then 4 products composing the 128-block;
+        # other head dims: rank-one recurrences (keys with in-block logits,
+        # queries, block product)
+        "ut_prep": ((2 * (8 * 2.0 * HB * HB * d + HB * HB * 128.0) + 4 * 2.0 * HB * HB * d, "tf32")
+                    if d == 64 else (BT * BT / 2 * 10.0 * d + BT * 4.0 * d * d, "alu")),
+        # per 128-block: 8 products of 64x64 by 64xd (the halves' quantities come
+        # from the forward's UT prep)
+        "ut_adj_compose": (nblk * 8 * 2.0 * HB * HB * d, "tf32"),
         # per 64-half: 22 products and two 64x128 triangular solves
         "ut_adj64": (2 * nblk * (22 * 2.0 * HB * HB * d + 2 * HB * HB * 128.0), "tf32"),
         "ut_prep_bwd": (nblk * (8 * 2.0 * HB * HB * d + 4 * HB * HB * 4.0 * d
                                 + 2 * 24 * 2.0 * HB * HB * d), "alu"),
     }
     f, bound = per.get(name, (0.0, None))
+    if name == "ut_prep":
+        f *= nblk
     return f * nh, bound
 
 

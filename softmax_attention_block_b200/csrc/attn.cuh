@@ -61,7 +61,7 @@ struct DecodeArgs {
     float *partial;                     // [nh, nchunk, d + 2]
 };
 
-constexpr int DECODE_CHUNK = 256;  // cached rows per CTA
+constexpr int DECODE_CHUNK = 1024;  // cached rows per CTA
 
 cudaError_t decode_step(const DecodeArgs &a, int dt, int d, cudaStream_t st);
 

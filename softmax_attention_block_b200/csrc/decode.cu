@@ -77,7 +77,7 @@ __device__ __forceinline__ float group_sum(float x)
 }
 
 constexpr int THREADS = 256;
-constexpr int UNROLL = 4;
+constexpr int UNROLL = 8;  // rows in flight per row group (loads issued before the math)
 
 template <typename T, int D, int CHUNK = DECODE_CHUNK>
 __global__ void __launch_bounds__(THREADS) decode_chunk_kernel(DecodeArgs a, int nchunk)

@@ -263,6 +263,14 @@ def test_decode_small(P, dtype, d):
                   1e-4 if dtype == torch.float32 else 2e-2)
 
 
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 64), (torch.bfloat16, 128)])
+def test_decode_multi_chunk_ragged(P, dtype, d):
+    """Caches of several split chunks with a ragged last one (the chunk length is
+    a power of two; 2500 rows cross two boundaries at any of them up to 1024)."""
+    _decode_check(P, 1, 3, d, 2500, 2510, 4, dtype, [0, 1, 2],
+                  1e-4 if dtype == torch.float32 else 2e-2)
+
+
 def test_decode_from_empty_cache(P):
     _decode_check(P, 1, 2, 64, 0, 40, 30, torch.float32, [0, 1], 1e-4)
 

@@ -23,6 +23,8 @@
 //
 // Every accumulator has its own TMEM columns, so MMA 1 of the next pair runs
 // while MMA 2 of this one and the drain of its results proceed.
+#include <type_traits>
+
 #include "attn.cuh"
 #include "attn_tc.cuh"
 #include "runtime.cuh"
@@ -255,10 +257,12 @@ __global__ void __launch_bounds__(NT, 1)
             const float *rows = reinterpret_cast<const float *>(stage(s) + C::S_ROW);
             const float *sd = a.Sd + ((long long)h * nblk + J) * BT * BT;
             float *dsd = a.dSd + ((long long)h * nblk + J) * BT * BT;
-#pragma unroll 1
-            for (int c = 64 * g; ok && c < 64 * g + 64; c += 16) {
+            // one 16-column chunk; the diagonal tile (logits from the UT prep, causal
+            // mask, dS also to the prep's adjoint) is its own instantiation
+            auto chunk = [&](auto dg, int c) {
+                constexpr bool DG = decltype(dg)::value;
                 float sv[16], dp[16];
-                if (diag) {
+                if (DG) {
 #pragma unroll
                     for (int u = 0; u < 16; ++u) sv[u] = sd[(c + u) * BT + j];
                 } else {
@@ -278,11 +282,11 @@ __global__ void __launch_bounds__(NT, 1)
                         const int u = 4 * q + e, i = c + u;
                         const float x = fmaf(sv[u], k1, FOX ? nbv[e] - cj2 : nbv[e]);
                         float p = ex2(x);
-                        if (diag && i < j) p = 0.f;
+                        if (DG && i < j) p = 0.f;
                         const float ds = p * fmaf(dp[u], a.scale, -sdv[e]);
                         pv[u] = p;
                         dsv[u] = ds;
-                        if (diag) dsd[(long long)i * BT + j] = ds;
+                        if (DG) dsd[(long long)i * BT + j] = ds;
                     }
                 }
                 uint32_t pb[8], db[8];
@@ -326,6 +330,13 @@ __global__ void __launch_bounds__(NT, 1)
                     if (!(lane & 1))
                         atomicAdd(a.rowsum + (long long)h * Lp + I * BT + c + (lane >> 1), dsv[0] / a.scale);
                 }
+            };
+#pragma unroll 1
+            for (int c = 64 * g; ok && c < 64 * g + 64; c += 16) {
+                if (diag)
+                    chunk(std::true_type{}, c);
+                else
+                    chunk(std::false_type{}, c);
             }
             fence_async_smem();
             fence_before_sync();

@@ -281,11 +281,20 @@ __global__ void __launch_bounds__(NT, 1)
                     tmem_ld32(tbase + b * 128 + c0s + 32 + lane_off, *reinterpret_cast<float(*)[32]>(z1));
                     tmem_wait_ld();
                 }
+                if (it == 0) {  // the diagonal tile: causal mask
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const float bias = FOX ? ci2 - cj[j] * LOG2E : 0.f;
-                    z[j] = (it > 0 || c0s + j <= r) ? fmaf(z[j], k1, bias) : -INFINITY;
-                    pmax = fmaxf(pmax, z[j]);
+                    for (int j = 0; j < 64; ++j) {
+                        const float bias = FOX ? ci2 - cj[j] * LOG2E : 0.f;
+                        z[j] = c0s + j <= r ? fmaf(z[j], k1, bias) : -INFINITY;
+                        pmax = fmaxf(pmax, z[j]);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) {
+                        const float bias = FOX ? ci2 - cj[j] * LOG2E : 0.f;
+                        z[j] = fmaf(z[j], k1, bias);
+                        pmax = fmaxf(pmax, z[j]);
+                    }
                 }
             }
             float *rb = red + (it & 1) * 256;

@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(NT, 1)
              *p_full = bars + 7, *m2_full = bars + 8, *e_done = bars + 9;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
 
+    // key tiles along x: the CTAs of one head run together and share its Q, dO
+    // tiles in L2 (heads along x, longest tiles first, measured slower)
     const int J = blockIdx.x, h = blockIdx.y;
     const int nblk = a.nblk, last = nblk - 1, Lp = nblk * BT;
     const int niter = last - J + 1;  // off-diagonal tiles last..J+1, then the diagonal

@@ -114,8 +114,10 @@ __global__ void __launch_bounds__(NT, 1)
     auto sV = [&](int s) { return sm + C::ST_OFF + s * C::ST_BYTES + C::TILE; };
     auto sC = [&](int s) { return reinterpret_cast<float *>(sm + C::ST_OFF + s * C::ST_BYTES + 2 * C::TILE); };
 
-    const int I = a.nblk - 1 - (int)blockIdx.x;  // longest rows of the causal triangle first
-    const int h = blockIdx.y;
+    // heads along x: blocks start in launch order, so every head's longest rows of
+    // the causal triangle start first
+    const int I = a.nblk - 1 - (int)blockIdx.y;
+    const int h = blockIdx.x;
     const int niter = I + 1;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int Lp = a.nblk * BT;
@@ -396,7 +398,7 @@ cudaError_t launch(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorM
     auto k = fwd_tc_kernel<D, FOX, TO>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<dim3(a.nblk, a.nh), NT, Cfg<D>::SMEM, st>>>(mQ, mK, mV, a);
+    k<<<dim3(a.nh, a.nblk), NT, Cfg<D>::SMEM, st>>>(mQ, mK, mV, a);
     count_launches();
     return cudaGetLastError();
 }

@@ -39,7 +39,9 @@
  *   launch failure returns PATH_ERR_CUDA (the CUDA error is left for
  *   cudaGetLastError to report as usual). No call aborts, traps or throws.
  * - Supported sizes: fwd/bwd d in {16, 32, 64, 128}; decode d in {64, 128};
- *   B, H, L >= 1; B*H*L*d < 2^40 per tensor.
+ *   B, H, L >= 1; B*H*L*d < 2^40 per tensor; B*H <= 65535 and
+ *   ceil(L / 128) <= 65535 (launch grid dimensions): beyond those the calls
+ *   return PATH_ERR_UNSUPPORTED and the workspace queries 0.
  */
 #ifndef PATH_ATTN_H
 #define PATH_ATTN_H

@@ -85,6 +85,12 @@ bool fwd_dims_ok(int B, int H, int L, int d)
 
 bool head_dim_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
+// Heads and 128-row blocks index launch grid dimensions limited to 65535.
+bool grid_ok(int B, int H, int L)
+{
+    return (long long)B * H <= 65535 && (L + BT - 1) / BT <= 65535;
+}
+
 bool dtype_ok(path_dtype dt)
 {
     return dt == PATH_F32 || dt == PATH_BF16 || dt == PATH_BF16_F32OUT;
@@ -165,7 +171,8 @@ const char *path_status_string(path_status s)
 
 size_t path_attn_workspace_bytes(int B, int H, int L, int d, path_dtype dt, int for_bwd)
 {
-    if (!fwd_dims_ok(B, H, L, d) || !head_dim_supported(d) || !dtype_ok(dt)) return 0;
+    if (!fwd_dims_ok(B, H, L, d) || !head_dim_supported(d) || !dtype_ok(dt) || !grid_ok(B, H, L))
+        return 0;
     AttnWs w;
     return carve_attn(nullptr, make_layout(B, H, L, d, dt), dt, for_bwd != 0, w);
 }
@@ -177,7 +184,7 @@ path_status path_attn_fwd(const void *q, const void *k, const void *v, const voi
 {
     if (!q || !k || !v || !w || !beta || !out || !lse) return PATH_ERR_INVALID_ARG;
     if (!fwd_dims_ok(B, H, L, d) || !isfinite(scale)) return PATH_ERR_INVALID_ARG;
-    if (!head_dim_supported(d) || !dtype_ok(dt)) return PATH_ERR_UNSUPPORTED;
+    if (!head_dim_supported(d) || !dtype_ok(dt) || !grid_ok(B, H, L)) return PATH_ERR_UNSUPPORTED;
     const Layout y = make_layout(B, H, L, d, dt);
     AttnWs ws;
     const size_t need = carve_attn(nullptr, y, dt, false, ws);
@@ -217,7 +224,7 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
         return PATH_ERR_INVALID_ARG;
     if ((log_f == nullptr) != (dlog_f == nullptr)) return PATH_ERR_INVALID_ARG;
     if (!fwd_dims_ok(B, H, L, d) || !isfinite(scale)) return PATH_ERR_INVALID_ARG;
-    if (!head_dim_supported(d) || !dtype_ok(dt)) return PATH_ERR_UNSUPPORTED;
+    if (!head_dim_supported(d) || !dtype_ok(dt) || !grid_ok(B, H, L)) return PATH_ERR_UNSUPPORTED;
     const Layout y = make_layout(B, H, L, d, dt);
     AttnWs ws;
     const size_t need = carve_attn(nullptr, y, dt, true, ws);
@@ -280,7 +287,9 @@ path_status path_attn_wait_status(const void *workspace, path_stream_t stream)
 
 size_t path_decode_workspace_bytes(int B, int H, int capacity, int d, path_dtype dt)
 {
-    if (B <= 0 || H <= 0 || capacity <= 0 || (d != 64 && d != 128) || !decode_dtype_ok(dt)) return 0;
+    if (B <= 0 || H <= 0 || capacity <= 0 || (d != 64 && d != 128) || !decode_dtype_ok(dt) ||
+        !grid_ok(B, H, 1))
+        return 0;
     const size_t nchunk = (size_t)ceil_div(capacity, DECODE_CHUNK);
     return align_up((size_t)B * H * nchunk * (d + 2) * sizeof(float), 256);
 }
@@ -295,7 +304,7 @@ path_status path_decode_step(const void *q, const void *k_new, const void *v_new
     if (B <= 0 || H <= 0 || capacity <= 0 || n_cached < 0 || n_cached + 1 > capacity ||
         !isfinite(scale))
         return PATH_ERR_INVALID_ARG;
-    if ((d != 64 && d != 128) || !decode_dtype_ok(dt)) return PATH_ERR_UNSUPPORTED;
+    if ((d != 64 && d != 128) || !decode_dtype_ok(dt) || !grid_ok(B, H, 1)) return PATH_ERR_UNSUPPORTED;
     // 16-byte vector access of q, w and the caches
     const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(w) |
                          reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache);
@@ -318,7 +327,7 @@ path_status path_decode_step_noalloc(const void *q, const void *k_new, const voi
     if (B <= 0 || H <= 0 || capacity <= 0 || n_cached < 0 || n_cached + 1 > capacity ||
         !isfinite(scale))
         return PATH_ERR_INVALID_ARG;
-    if ((d != 64 && d != 128) || !decode_dtype_ok(dt)) return PATH_ERR_UNSUPPORTED;
+    if ((d != 64 && d != 128) || !decode_dtype_ok(dt) || !grid_ok(B, H, 1)) return PATH_ERR_UNSUPPORTED;
     const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(w) |
                          reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache);
     if (al & 15u) return PATH_ERR_INVALID_ARG;

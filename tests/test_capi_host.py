@@ -81,6 +81,20 @@ def test_fwd_rejects_bad_arguments(lib):
     assert fwd(lib, wsb=100) == WORKSPACE
 
 
+def test_grid_limits_unsupported(lib):
+    # heads and 128-row blocks index launch grid dimensions (at most 65535)
+    assert fwd(lib, B=256, H=256) == UNSUPPORTED
+    assert fwd(lib, L=65536 * 128 + 1, d=16) == UNSUPPORTED
+    f = lib.path_attn_workspace_bytes
+    assert f(256, 256, 64, 64, BF16, 1) == 0
+    assert f(1, 1, 65536 * 128 + 1, 16, BF16, 0) == 0
+    assert f(255, 257, 64, 64, BF16, 1) > 0  # 65535 heads
+    assert lib.path_decode_workspace_bytes(256, 256, 100, 128, BF16) == 0
+    st = lib.path_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, 256, 256, 128, 10, 11, BF16,
+                              FAKE, FAKE, FAKE, FAKE, 1 << 40, None)
+    assert st == UNSUPPORTED
+
+
 def test_bwd_rejects_bad_arguments(lib):
     def bwd(**kw):
         a = dict(log_f=None, dlog_f=None, dq=FAKE, L=64, d=64, wsb=1 << 40)

@@ -80,33 +80,39 @@ __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k,
     constexpr bool SPLIT = !EX;
     extern __shared__ __align__(16) float sm[];
     // working set of one half, then what the composition keeps
-    float *sW = sm, *sQw = sW + MAT, *sKw = sQw + MAT, *sA = sKw + MAT, *sM = sA + MAT,
+    float *sWa = sm, *sQw = sWa + MAT, *sKw = sQw + MAT, *sA = sKw + MAT, *sM = sA + MAT,
           *sWh = sM + MAT, *sU = sWh + MAT, *sKa = sU + MAT, *sPa = sKa + MAT, *sQb = sPa + MAT,
-          *sPb = sQb + MAT, *sB = sPb + MAT;
+          *sPb = sQb + MAT, *sWb = sPb + MAT, *sBa = sWb + MAT, *sBb = sBa + HB;
     const int J = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
     const int Lp = nblk * BT;
     const long long prow = (long long)h * Lp + (long long)J * BT;  // block's first row in [nh, Lp]
     float *sd = Sd + ((long long)h * nblk + J) * BT * BT;
 
+    // both halves' inputs up front (half a keeps its keys, -> Ktil_a, in sKa and
+    // half b its queries, -> Qtil_b, in sQb), so half b's loads are not exposed
 #pragma unroll 1
     for (int half = 0; half < 2; ++half) {
         const int pos0 = J * BT + half * HB;
         const int nvalid = max(0, min(HB, L - pos0));
         const long long row0 = (long long)h * L + pos0;
-        // half a keeps its keys (-> Ktil_a) in sKa, half b its queries (-> Qtil_b) in sQb
+        Rows<T> rw, rq, rk;
+        rw.ld(w + row0 * D, nvalid, vec);
+        rq.ld(q + row0 * D, nvalid, vec);
+        rk.ld(k + row0 * D, nvalid, vec);
+        rw.st(half == 0 ? sWa : sWb);
+        rq.st(half == 0 ? sQw : sQb);
+        rk.st(half == 0 ? sKa : sKw);
+        float *sB = half == 0 ? sBa : sBb;
+        for (int r = tid; r < HB; r += NT) sB[r] = r < nvalid ? beta[row0 + r] : 0.f;
+    }
+    __syncthreads();
+
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
         float *sK = half == 0 ? sKa : sKw;
         float *sQ = half == 0 ? sQw : sQb;
-        {
-            Rows<T> rw, rq, rk;
-            rw.ld(w + row0 * D, nvalid, vec);
-            rq.ld(q + row0 * D, nvalid, vec);
-            rk.ld(k + row0 * D, nvalid, vec);
-            rw.st(sW);
-            rq.st(sQ);
-            rk.st(sK);
-        }
-        for (int r = tid; r < HB; r += NT) sB[r] = r < nvalid ? beta[row0 + r] : 0.f;
-        __syncthreads();
+        float *sW = half == 0 ? sWa : sWb;
+        float *sB = half == 0 ? sBa : sBb;
         {
             Frag f;
             mm<false, true, EX, EX, SPLIT>(f, sW, sW);
@@ -206,7 +212,7 @@ __global__ void __launch_bounds__(NT) prep_fwd_tc_kernel(const T *q, const T *k,
 template <typename T, typename TM>
 cudaError_t run(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out, cudaStream_t st)
 {
-    const size_t smem = (11 * MAT + HB) * sizeof(float);
+    const size_t smem = (12 * MAT + 2 * HB) * sizeof(float);
     auto kern = prep_fwd_tc_kernel<T, TM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

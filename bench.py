@@ -245,6 +245,32 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- our arm
+def make_collectives(world, device):
+    """The benchmark's only collectives, host-side timing plumbing (no data path):
+    a barrier around the timed region and the max over ranks of a device time,
+    a float64 all-reduce on `device` (the GPU under NCCL, the CPU under gloo)."""
+    import torch.distributed as dist
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, max_over_ranks
+
+
+def whole_job_rate(world, units_per_rank, ms_per_step_max):
+    """Weak scaling: every rank runs the full workload, so the job processes
+    world x units per step in the slowest rank's time."""
+    return world * units_per_rank / (ms_per_step_max * 1e-3)
+
+
 def run_ours(args):
     import torch.distributed as dist
     import softmax_attention_block_b200 as P
@@ -282,16 +308,7 @@ def run_ours(args):
                         inp["dout"], inp["log_f"], grads=grads, workspace=ws,
                         reuse_fwd_workspace=True)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = make_collectives(world, dev)
 
     for _ in range(args.warmup):
         step(x)
@@ -318,8 +335,8 @@ def run_ours(args):
     stages = read_profile()
     ms_step = ms_total / args.steps
     flops = algorithmic_flops(w.B, w.H, w.L, w.d)
-    value = world * flops / (ms_step * 1e-3) / 1e12
-    tokens = world * w.B * w.L / (ms_step * 1e-3)
+    value = whole_job_rate(world, flops, ms_step) / 1e12
+    tokens = whole_job_rate(world, w.B * w.L, ms_step)
 
     # dominant stage -> roofline against the measured bf16 dense peak
     stage_rows = {n: {"ms_per_launch": t / c, "launches": c, "share": 0.0}
@@ -416,7 +433,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier()
         ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / args.steps
-        e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": whole_job_rate(world, flops, ms_e2e) / 1e12, "unit": UNIT,
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "pipeline": f"{w.B} per-sequence chunks; copies in, compute, copies out on 3 streams"}
         del host, hout, ws1
@@ -441,7 +458,7 @@ def run_ours(args):
                        "tensor is 100.7 MB; 126 MB L2)",
                        "parallelism": f"{world} rank(s), full workload per rank"},
             "tokens_per_s": tokens,
-            "tflops_fa_equiv": world * fa_equiv_flops(w.B, w.H, w.L, w.d) / (ms_step * 1e-3) / 1e12,
+            "tflops_fa_equiv": whole_job_rate(world, fa_equiv_flops(w.B, w.H, w.L, w.d), ms_step) / 1e12,
             "pct_bf16_peak": value / world / peaks["bf16_tflops_sustained"],
             "stages": stage_rows, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk, "decode": decode}
@@ -485,7 +502,7 @@ def bench_decode(P, dev, peaks, world, max_over_ranks, barrier):
     nh = w.B * w.H
     n_avg = w.n0 + (w.steps - 1) / 2.0
     bytes_step = 3.0 * nh * n_avg * w.d * 2  # read K, write K, read V (bf16)
-    gbs = world * bytes_step / (ms * 1e-3) / 1e9
+    gbs = whole_job_rate(world, bytes_step, ms) / 1e9
     chunk_ms = stages.get("decode_chunks", (0.0, 1))
     per_launch = chunk_ms[0] / max(chunk_ms[1], 1)
     ach = bytes_step / (per_launch * 1e-3) / 1e9 if per_launch else None

@@ -12,7 +12,9 @@ Definitions it follows (all from the pages' problem statement):
   Paper-Notes "整体框架" / "PaTH-FoX 扩展");
 - ``H_s = I - beta_s w_s w_s^T`` (gist.science section 2; Paper-Notes "关键设计");
 - forward by the in-place key-cache update (Paper-Notes "训练策略",
-  inference paragraph), backward by the per-query adjoint chain.
+  inference paragraph), backward by the per-query adjoint chain;
+- decode (optionally with the gate's per-key bias carried in place) and the
+  cache a prefill leaves behind, by the same in-place update.
 
 Parity is pinned by ``tests/test_oracle_pins.py`` against explicit matrix
 products, a library attention routine, closed forms, finite differences and
@@ -86,10 +88,14 @@ class Oracle:
                                         dp, dp, dp, dp, dp, dp, dp]
         lib.path_oracle_decode_step.argtypes = [dp, dp, dp, dp, dp, d, i, i, i, i, i, i,
                                                 dp, dp, dp]
+        lib.path_oracle_decode_step_gated.argtypes = [dp, dp, dp, dp, dp, dp, d, i, i, i, i, i,
+                                                      i, dp, dp, dp, dp]
+        lib.path_oracle_prefill_cache.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, dp, dp, dp]
         lib.path_oracle_round_bf16.argtypes = [d]
         lib.path_oracle_round_bf16.restype = d
         for f in (lib.path_oracle_fwd, lib.path_oracle_scores, lib.path_oracle_bwd,
-                  lib.path_oracle_decode_step):
+                  lib.path_oracle_decode_step, lib.path_oracle_decode_step_gated,
+                  lib.path_oracle_prefill_cache):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -141,25 +147,51 @@ class Oracle:
         return g
 
     def decode_step(self, q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=None,
-                    round_bf16=False):
+                    round_bf16=False, log_f=None, g_cache=None):
         """One decode step; k_cache/v_cache (fp64 numpy [B,H,cap,d]) are updated IN PLACE.
 
-        Returns out [B,H,d] (fp64)."""
-        q, k_new, v_new, w, beta = map(_f64, (q, k_new, v_new, w, beta))
-        for c in (k_cache, v_cache):
+        With the forget gate, log_f [B,H] is log f of the new position and
+        g_cache (fp64 numpy [B,H,cap]) the cached gate biases, also updated in
+        place. Returns out [B,H,d] (fp64)."""
+        q, k_new, v_new, w, beta, log_f = map(_f64, (q, k_new, v_new, w, beta, log_f))
+        caches = (k_cache, v_cache) + ((g_cache,) if log_f is not None else ())
+        for c in caches:
             if not (isinstance(c, np.ndarray) and c.dtype == np.float64 and c.flags.c_contiguous):
-                raise TypeError("k_cache / v_cache must be C-contiguous fp64 numpy arrays")
+                raise TypeError("caches must be C-contiguous fp64 numpy arrays")
         B, H, cap, d = k_cache.shape
         if scale is None:
             scale = d ** -0.5
         out = np.empty((B, H, d))
-        rc = self.lib.path_oracle_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(w),
-                                              _ptr(beta), float(scale), B, H, d, int(n_cached),
-                                              cap, int(bool(round_bf16)), _ptr(k_cache),
-                                              _ptr(v_cache), _ptr(out))
+        if log_f is None:
+            rc = self.lib.path_oracle_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(w),
+                                                  _ptr(beta), float(scale), B, H, d,
+                                                  int(n_cached), cap, int(bool(round_bf16)),
+                                                  _ptr(k_cache), _ptr(v_cache), _ptr(out))
+        else:
+            rc = self.lib.path_oracle_decode_step_gated(
+                _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(w), _ptr(beta), _ptr(log_f),
+                float(scale), B, H, d, int(n_cached), cap, int(bool(round_bf16)), _ptr(k_cache),
+                _ptr(v_cache), _ptr(g_cache), _ptr(out))
         if rc:
             raise ValueError("oracle decode_step: invalid arguments")
         return out
+
+    def prefill_cache(self, k, v, w, beta, log_f=None, capacity=None):
+        """The decode cache after positions 0..L-1: (k_cache, v_cache, g_cache), fp64
+        [B,H,cap,d], [B,H,cap,d], [B,H,cap] (g_cache None without the gate); rows past L
+        are zero."""
+        k, v, w, beta, log_f = map(_f64, (k, v, w, beta, log_f))
+        B, H, L, d = _dims(k)
+        cap = L if capacity is None else int(capacity)
+        kc = np.zeros((B, H, cap, d))
+        vc = np.zeros((B, H, cap, d))
+        gc = np.zeros((B, H, cap)) if log_f is not None else None
+        rc = self.lib.path_oracle_prefill_cache(_ptr(k), _ptr(v), _ptr(w), _ptr(beta),
+                                                _ptr(log_f), B, H, L, d, cap, _ptr(kc),
+                                                _ptr(vc), _ptr(gc))
+        if rc:
+            raise ValueError("oracle prefill_cache: invalid arguments")
+        return kc, vc, gc
 
     def round_bf16(self, x: float) -> float:
         """The oracle's double -> bfloat16 rounding (nearest, ties to even)."""
@@ -189,6 +221,10 @@ def bwd(*a, **kw):
 
 def decode_step(*a, **kw):
     return default().decode_step(*a, **kw)
+
+
+def prefill_cache(*a, **kw):
+    return default().prefill_cache(*a, **kw)
 
 
 def round_bf16(x):

@@ -39,6 +39,15 @@
  * Decode: one step of the in-place key update, append, then one-query
  * softmax attention over the n+1 keys; optionally rounding each updated key
  * to bfloat16 (round to nearest, ties to even) as a bf16 cache must hold it.
+ * With the forget gate, each cached key also carries g_j = c_t - c_j, the
+ * gate's logit bias for the current position t: a step adds log f_t to every
+ * cached g_j and appends g_t = 0 (the PaTH-FoX logit term c_i - c_j, carried
+ * in the same in-place manner as the keys).
+ *
+ * Prefill cache: the decode rule replayed over positions 0..L-1 without the
+ * attention, i.e. the cache a decoder holds after position L-1: row j of the
+ * key cache is H_{L-1} ... H_{j+1} k_j, row j of the value cache is v_j, and
+ * g_j = c_{L-1} - c_j.
  *
  * All arrays are contiguous row-major fp64: q, k, v, w, out, grads
  * [B,H,L,d]; beta, log_f, lse, dbeta, dlog_f [B,H,L]. log_f may be NULL
@@ -353,6 +362,42 @@ double path_oracle_round_bf16(double x)
 }
 
 /*
+ * One decode step of one head. K / V [capacity,d] hold n valid rows; g (NULL
+ * without the gate) holds their gate biases and logf_t is log f_t.
+ */
+static void decode_head(const double *q_t, const double *k_new, const double *v_new,
+                        const double *w_t, double beta_t, const double *logf_t, double scale,
+                        int d, int n, int round_bf16, double *K, double *V, double *g,
+                        double *o)
+{
+    for (int j = 0; j < n; ++j) {
+        double *k_j = K + (size_t)j * d;
+        apply_h(k_j, w_t, beta_t, d);
+        if (round_bf16)
+            for (int e = 0; e < d; ++e) k_j[e] = path_oracle_round_bf16(k_j[e]);
+        if (g) g[j] += *logf_t;
+    }
+    memcpy(K + (size_t)n * d, k_new, sizeof(double) * d);
+    memcpy(V + (size_t)n * d, v_new, sizeof(double) * d);
+    if (g) g[n] = 0.0;
+    double *z = malloc(sizeof(double) * (n + 1));
+    double m = -INFINITY;
+    for (int j = 0; j <= n; ++j) {
+        z[j] = scale * dot(q_t, K + (size_t)j * d, d) + (g ? g[j] : 0.0);
+        m = z[j] > m ? z[j] : m;
+    }
+    double ssum = 0.0;
+    for (int j = 0; j <= n; ++j) ssum += exp(z[j] - m);
+    for (int e = 0; e < d; ++e) o[e] = 0.0;
+    for (int j = 0; j <= n; ++j) {
+        const double pj = exp(z[j] - m) / ssum;
+        const double *v_j = V + (size_t)j * d;
+        for (int e = 0; e < d; ++e) o[e] += pj * v_j[e];
+    }
+    free(z);
+}
+
+/*
  * One decode step for every head. k_cache / v_cache [B,H,capacity,d] hold
  * n_cached valid rows. Rows 0..n-1 of k_cache are multiplied in place by
  * H_t = I - beta w w^T (rounded to bf16 when round_bf16 != 0), then row n of
@@ -368,37 +413,73 @@ int path_oracle_decode_step(const double *q, const double *k_new,
     if (B <= 0 || H <= 0 || d <= 0 || n_cached < 0 || n_cached + 1 > capacity)
         return 1;
     const int nh = B * H;
-    const int n = n_cached;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < nh; ++h)
+        decode_head(q + (size_t)h * d, k_new + (size_t)h * d, v_new + (size_t)h * d,
+                    w + (size_t)h * d, beta[h], NULL, scale, d, n_cached, round_bf16,
+                    k_cache + (size_t)h * capacity * d, v_cache + (size_t)h * capacity * d,
+                    NULL, out + (size_t)h * d);
+    return 0;
+}
+
+/*
+ * The decode step with the forget gate: as path_oracle_decode_step, and
+ * g_cache [B,H,capacity] holds the cached keys' gate biases: g_j += log_f
+ * (log_f [B,H], log f_t of the new position) for j < n, g_n = 0, and the
+ * logits are scale q.k_j + g_j.
+ */
+int path_oracle_decode_step_gated(const double *q, const double *k_new,
+                                  const double *v_new, const double *w,
+                                  const double *beta, const double *log_f,
+                                  double scale, int B, int H, int d, int n_cached,
+                                  int capacity, int round_bf16, double *k_cache,
+                                  double *v_cache, double *g_cache, double *out)
+{
+    if (B <= 0 || H <= 0 || d <= 0 || n_cached < 0 || n_cached + 1 > capacity ||
+        !log_f || !g_cache)
+        return 1;
+    const int nh = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < nh; ++h)
+        decode_head(q + (size_t)h * d, k_new + (size_t)h * d, v_new + (size_t)h * d,
+                    w + (size_t)h * d, beta[h], log_f + h, scale, d, n_cached, round_bf16,
+                    k_cache + (size_t)h * capacity * d, v_cache + (size_t)h * capacity * d,
+                    g_cache + (size_t)h * capacity, out + (size_t)h * d);
+    return 0;
+}
+
+/*
+ * The cache after a prefill of positions 0..L-1, by replaying the in-place
+ * update position by position: before position t is appended, each key
+ * already held is multiplied by H_t and each gate bias grows by log f_t.
+ * k, v, w [B,H,L,d]; beta, log_f [B,H,L] (log_f may be NULL; g_cache is then
+ * untouched). Writes rows 0..L-1 of k_cache, v_cache [B,H,capacity,d] and
+ * g_cache [B,H,capacity].
+ */
+int path_oracle_prefill_cache(const double *k, const double *v, const double *w,
+                              const double *beta, const double *log_f, int B, int H,
+                              int L, int d, int capacity, double *k_cache,
+                              double *v_cache, double *g_cache)
+{
+    if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || L > capacity || (log_f && !g_cache))
+        return 1;
+    const int nh = B * H;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int h = 0; h < nh; ++h) {
+        const size_t in0 = (size_t)h * L;
         double *K = k_cache + (size_t)h * capacity * d;
         double *V = v_cache + (size_t)h * capacity * d;
-        const double *w_t = w + (size_t)h * d;
-        const double *q_t = q + (size_t)h * d;
-        for (int j = 0; j < n; ++j) {
-            double *k_j = K + (size_t)j * d;
-            apply_h(k_j, w_t, beta[h], d);
-            if (round_bf16)
-                for (int e = 0; e < d; ++e) k_j[e] = path_oracle_round_bf16(k_j[e]);
+        double *g = log_f ? g_cache + (size_t)h * capacity : NULL;
+        for (int t = 0; t < L; ++t) {
+            const double *w_t = w + (in0 + t) * d;
+            for (int j = t - 1; j >= 0; --j) {
+                apply_h(K + (size_t)j * d, w_t, beta[in0 + t], d);
+                if (g) g[j] += log_f[in0 + t];
+            }
+            memcpy(K + (size_t)t * d, k + (in0 + t) * d, sizeof(double) * d);
+            memcpy(V + (size_t)t * d, v + (in0 + t) * d, sizeof(double) * d);
+            if (g) g[t] = 0.0;
         }
-        memcpy(K + (size_t)n * d, k_new + (size_t)h * d, sizeof(double) * d);
-        memcpy(V + (size_t)n * d, v_new + (size_t)h * d, sizeof(double) * d);
-        double *z = malloc(sizeof(double) * (n + 1));
-        double m = -INFINITY;
-        for (int j = 0; j <= n; ++j) {
-            z[j] = scale * dot(q_t, K + (size_t)j * d, d);
-            m = z[j] > m ? z[j] : m;
-        }
-        double ssum = 0.0;
-        for (int j = 0; j <= n; ++j) ssum += exp(z[j] - m);
-        double *o = out + (size_t)h * d;
-        for (int e = 0; e < d; ++e) o[e] = 0.0;
-        for (int j = 0; j <= n; ++j) {
-            const double pj = exp(z[j] - m) / ssum;
-            const double *v_j = V + (size_t)j * d;
-            for (int e = 0; e < d; ++e) o[e] += pj * v_j[e];
-        }
-        free(z);
     }
     return 0;
 }

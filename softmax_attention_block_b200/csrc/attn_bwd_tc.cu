@@ -5,8 +5,8 @@
 // for S^T, dP^T, dV and the chain adjoint Abar. Per tile pair:
 //   MMA 1:  S^T  = Khat_{J,I} Qtil_I^T          (fp16)
 //           dP^T = V_J dO_I^T                    (bf16)
-//           issued as soon as the previous pair's S^T / dP^T are consumed, ahead
-//           of that pair's MMA 2
+//           issued right after the previous pair's MMA 2, whose launch waits for
+//           the softmax to have consumed that pair's S^T / dP^T
 //   threads: P = exp(scale S + c_i - c_j - lse_i), dZ = P (dP - delta_i),
 //            dS = scale dZ; P^T (bf16) and dS^T (fp16) to shared memory;
 //            [gate] row sums of dS by warp reduce-scatter, column sums per thread
@@ -16,13 +16,14 @@
 //           Abar  = Abar_{I+1} P_I + dS^T Qtil_I           (fp16, fp32 in TMEM)
 //           dQtil_I += dS Khat_{J,I}                       (fp16)
 // Khat_{J,I+1} = Khat_{J,I} P_I^T, so Abar is the adjoint carried back along
-// the key-side transport chain; after the pair (J+1, J) it is dKtil_J. dQtil,
-// dP and the row sums accumulate across CTAs with fp32 vector reductions.
+// the key-side transport chain; after the pair (J+1, J) it is dKtil_J. dQtil
+// and dP are staged in shared memory by the drain warps and accumulate across
+// CTAs by TMA tensor reduce-add; the gate's row sums by fp32 atomics.
 // The diagonal tile takes its logits from the UT prep and writes dS to the
 // prep's adjoint instead (dSd), which carries it to dQ, dK, dW, dbeta.
 //
-// Every accumulator has its own TMEM columns, so MMA 1 of the next pair runs
-// while MMA 2 of this one and the drain of its results proceed.
+// Every accumulator has its own TMEM columns, so MMA 1 of the next pair and
+// the softmax on its results run while the drain empties this pair's MMA 2.
 #include <type_traits>
 
 #include "attn.cuh"

@@ -6,7 +6,9 @@ identity and full-matrix form printed on the Paper-Notes page ("训练策略"),
 a library attention routine (torch SDPA) where PaTH reduces to plain causal
 softmax attention, closed forms for repeated w, norm preservation of H at
 beta = 2, finite differences and autograd of an explicit-matrix formulation
-for every gradient, gradient invariants, and decode replay. The mutation
+for every gradient, gradient invariants, decode replay (with and without the
+gate's per-key bias), and the cache a prefill leaves (explicit products, the
+forward's last row, decode continuing the forward). The mutation
 tests at the end plant mistakes in a copy of the oracle source and check that
 a pin catches each one.
 """
@@ -351,6 +353,75 @@ def test_decode_bf16_cache_is_rounded_update(orc):
     np.testing.assert_array_equal(kb[:, :, n], kn)
 
 
+def test_gated_decode_replay_equals_forward_rows(orc):
+    """PaTH-FoX decode: each cached key carries its gate bias c_t - c_j, grown in
+    place by log f_t at every step (Paper-Notes "PaTH-FoX 扩展" logit term, carried
+    like the in-place key update of "训练策略"); replay reproduces the forward."""
+    rng = np.random.default_rng(19)
+    q, k, v, w, beta, logf = rand_case(rng, B=2, H=2, L=21, d=6, fox=True)
+    out, _ = orc.fwd(q, k, v, w, beta, logf, scale=0.5)
+    kc, vc, gc = np.zeros((2, 2, 21, 6)), np.zeros((2, 2, 21, 6)), np.zeros((2, 2, 21))
+    for t in range(21):
+        o = orc.decode_step(q[:, :, t], k[:, :, t], v[:, :, t], w[:, :, t], beta[:, :, t], kc, vc,
+                            t, scale=0.5, log_f=logf[:, :, t], g_cache=gc)
+        np.testing.assert_allclose(o, out[:, :, t], rtol=1e-11, atol=1e-13)
+
+
+# ---------------------------------------------------------------- prefill cache pins
+def test_prefill_cache_equals_explicit_products(orc):
+    """Row j of the cache after positions 0..L-1 is H_{L-1} ... H_{j+1} k_j, and its gate
+    bias is the sum of log f_s over s = j+1..L-1 (Paper-Notes "训练策略", inference
+    paragraph; "PaTH-FoX 扩展")."""
+    rng = np.random.default_rng(20)
+    B, H, L, d, cap = 2, 2, 11, 5, 14
+    q, k, v, w, beta, logf = rand_case(rng, B=B, H=H, L=L, d=d, fox=True)
+    kc, vc, gc = orc.prefill_cache(k, v, w, beta, logf, capacity=cap)
+    for b in range(B):
+        for h in range(H):
+            M = np.eye(d)  # H_{L-1} ... H_{j+1}, built by right-multiplying as j decreases
+            for j in range(L - 1, -1, -1):
+                np.testing.assert_allclose(kc[b, h, j], M @ k[b, h, j], rtol=1e-12, atol=1e-13)
+                assert gc[b, h, j] == pytest.approx(math.fsum(logf[b, h, j + 1:]), rel=1e-12,
+                                                    abs=1e-13)
+                M = M @ householder(w[b, h, j], beta[b, h, j])
+    np.testing.assert_array_equal(vc[:, :, :L], v)
+    assert not kc[:, :, L:].any() and not vc[:, :, L:].any() and not gc[:, :, L:].any()
+    kc2, _, gc2 = orc.prefill_cache(k, v, w, beta, None, capacity=cap)
+    np.testing.assert_array_equal(kc2, kc)
+    assert gc2 is None
+
+
+def test_prefill_cache_last_row_attention_is_forward_row(orc):
+    """Softmax attention of q_{L-1} over the prefill cache (logits scale q.k_j + g_j, a
+    library softmax) gives the forward's last output row and log-sum-exp."""
+    rng = np.random.default_rng(21)
+    q, k, v, w, beta, logf = rand_case(rng, B=1, H=3, L=13, d=4, fox=True)
+    out, lse = orc.fwd(q, k, v, w, beta, logf, scale=0.7)
+    kc, vc, gc = orc.prefill_cache(k, v, w, beta, logf)
+    z = torch.from_numpy(0.7 * np.einsum("bhd,bhjd->bhj", q[:, :, -1], kc) + gc)
+    p = torch.softmax(z, -1).numpy()
+    np.testing.assert_allclose(np.einsum("bhj,bhjd->bhd", p, vc), out[:, :, -1], rtol=1e-11,
+                               atol=1e-13)
+    np.testing.assert_allclose(torch.logsumexp(z, -1).numpy(), lse[:, :, -1], rtol=1e-11)
+
+
+@pytest.mark.parametrize("fox", [False, True])
+def test_decode_after_prefill_continues_the_forward(orc, fox):
+    """A prefill of the first L0 positions followed by decode steps reproduces the
+    forward rows L0.. of the whole sequence."""
+    rng = np.random.default_rng(22)
+    L0, L = 9, 14
+    q, k, v, w, beta, logf = rand_case(rng, B=2, H=2, L=L, d=5, fox=fox)
+    out, _ = orc.fwd(q, k, v, w, beta, logf, scale=0.6)
+    head = lambda a: None if a is None else a[:, :, :L0]
+    kc, vc, gc = orc.prefill_cache(head(k), head(v), head(w), head(beta), head(logf), capacity=L)
+    for t in range(L0, L):
+        o = orc.decode_step(q[:, :, t], k[:, :, t], v[:, :, t], w[:, :, t], beta[:, :, t], kc, vc,
+                            t, scale=0.6, log_f=None if logf is None else logf[:, :, t],
+                            g_cache=gc)
+        np.testing.assert_allclose(o, out[:, :, t], rtol=1e-11, atol=1e-13)
+
+
 # ---------------------------------------------------------------- planted mistakes
 MUTATIONS = [
     # (name, regex on the source, replacement, pin that must fail)
@@ -363,6 +434,11 @@ MUTATIONS = [
     ("dc_key_sign", r"a->dc\[j\] -= dz", "a->dc[j] += dz", "grad"),
     ("g_transport_sign", r"g\[e\] -= b \* gu \* u\[e\]", "g[e] += b * gu * u[e]", "grad"),
     ("round_ties_away", r"nearbyint\(x / ulp\)", "round(x / ulp)", "round"),
+    ("decode_gate_not_carried", r"if \(g\) g\[j\] \+= \*logf_t;", ";", "gated_decode"),
+    ("prefill_skips_newest_key", r"for \(int j = t - 1; j >= 0; --j\)",
+     "for (int j = t - 2; j >= 0; --j)", "prefill"),
+    ("prefill_gate_sign", r"if \(g\) g\[j\] \+= log_f\[in0 \+ t\];",
+     "if (g) g[j] -= log_f[in0 + t];", "prefill"),
 ]
 
 
@@ -398,6 +474,25 @@ def _pin_passes(orc, pin):
             grads = torch.autograd.grad(loss, ts)
             for n, ref in zip(["dq", "dk", "dv", "dw", "dbeta", "dlog_f"], grads):
                 np.testing.assert_allclose(g[n], ref.numpy(), rtol=1e-9, atol=1e-11)
+        elif pin == "gated_decode":
+            q, k, v, w, beta, logf = rand_case(rng, B=1, H=1, L=7, d=4, fox=True)
+            z = explicit_scores(q[0, 0], k[0, 0], w[0, 0], beta[0, 0], logf[0, 0], 1.0)
+            kc, vc, gc = np.zeros((1, 1, 7, 4)), np.zeros((1, 1, 7, 4)), np.zeros((1, 1, 7))
+            for t in range(7):
+                o = orc.decode_step(q[:, :, t], k[:, :, t], v[:, :, t], w[:, :, t],
+                                    beta[:, :, t], kc, vc, t, scale=1.0, log_f=logf[:, :, t],
+                                    g_cache=gc)
+                p = torch.softmax(torch.from_numpy(z[t, :t + 1]), -1).numpy()
+                np.testing.assert_allclose(o[0, 0], p @ v[0, 0, :t + 1], rtol=1e-10, atol=1e-12)
+        elif pin == "prefill":
+            q, k, v, w, beta, logf = rand_case(rng, B=1, H=1, L=7, d=4, fox=True)
+            kc, _, gc = orc.prefill_cache(k, v, w, beta, logf)
+            M = np.eye(4)
+            for j in range(6, -1, -1):
+                np.testing.assert_allclose(kc[0, 0, j], M @ k[0, 0, j], rtol=1e-10, atol=1e-12)
+                np.testing.assert_allclose(gc[0, 0, j], logf[0, 0, j + 1:].sum(), rtol=1e-10,
+                                           atol=1e-12)
+                M = M @ householder(w[0, 0, j], beta[0, 0, j])
         elif pin == "round":
             x = np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8)], dtype=np.float32)
             ref = torch.from_numpy(x).to(torch.bfloat16).double().numpy()

@@ -5,7 +5,9 @@ One step = the whole training hot path on one batch: path_attn_fwd (UT prep,
 transport chain, attention forward) then path_attn_bwd reusing the
 forward's workspace (attention backward, UT adjoint, gate gradient) at B=8
 H=24 L=4096 d=64 bf16, inputs resident in HBM. The decode step (B=32 H=32 d=128, cache 16384 -> 16448,
-64 steps) is timed after it and reported under "decode".
+64 steps) is timed after it and reported under "decode" (with the forget gate's per-key
+bias under "decode.gated"), and a prefill of the same sequences (forward plus the decode
+cache it leaves) under "prefill".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -438,6 +440,8 @@ def run_ours(args):
                "pipeline": f"{w.B} per-sequence chunks; copies in, compute, copies out on 3 streams"}
         del host, hout, ws1
 
+    prefill = None if args.no_prefill else bench_prefill(P, x, w, ws, peaks, world,
+                                                           max_over_ranks, barrier, args.steps)
     del x, out, lse, grads, ws
     torch.cuda.empty_cache()
     decode = None if args.no_decode else bench_decode(P, dev, peaks, world, max_over_ranks,
@@ -461,12 +465,58 @@ def run_ours(args):
             "tflops_fa_equiv": whole_job_rate(world, fa_equiv_flops(w.B, w.H, w.L, w.d), ms_step) / 1e12,
             "pct_bf16_peak": value / world / peaks["bf16_tflops_sustained"],
             "stages": stage_rows, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches, "clocks": clk, "decode": decode}
+            "gpu_launches": launches, "clocks": clk, "decode": decode, "prefill": prefill}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def bench_prefill(P, x, w, ws, peaks, world, max_over_ranks, barrier, steps):
+    """Prefill of the headline sequences (forward + the decode cache it leaves), timed
+    as a whole and, for the cache kernel, per launch against the HBM copy peak."""
+    cap = w.L + 64
+    kc = torch.empty((w.B, w.H, cap, w.d), dtype=w.dtype, device=x["q"].device)
+    vc = torch.empty_like(kc)
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=x["q"].device)
+
+    def call():
+        P.path_attn_prefill(x["q"], x["k"], x["v"], x["w"], x["beta"], cap, x["log_f"], out=out,
+                            lse=lse, k_cache=kc, v_cache=vc, workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    P.lib().path_profile_enable(1)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    P.lib().path_profile_enable(0)
+    stages = read_profile()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / steps
+    nh = w.B * w.H
+    # cache kernel, per launch: read the transported key tiles (fp16), P_last (fp16) and
+    # v; write the key and value caches (bf16)
+    bytes_launch = nh * (w.L * w.d * 2 * 4 + w.d * w.d * 2)
+    t, c = stages.get("prefill_cache", (0.0, 1))
+    per_launch = t / max(c, 1)
+    ach = bytes_launch / (per_launch * 1e-3) / 1e9 if per_launch else None
+    del kc, vc, out, lse
+    return {"workload": f"prefill {WORKLOAD}, cache capacity {cap}",
+            "value": whole_job_rate(world, w.B * w.L, ms), "unit": "tokens/s",
+            "ms_per_call": ms, "cache_kernel_ms": per_launch,
+            "roofline": {"kernel": "prefill_cache", "bound": "hbm", "achieved": ach,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"] if ach else None, "traffic": None,
+                         "algorithmic_bytes": bytes_launch,
+                         "peak_source": f"{peaks['source']} HBM copy"}}
 
 
 def bench_decode(P, dev, peaks, world, max_over_ranks, barrier):
@@ -506,12 +556,44 @@ def bench_decode(P, dev, peaks, world, max_over_ranks, barrier):
     chunk_ms = stages.get("decode_chunks", (0.0, 1))
     per_launch = chunk_ms[0] / max(chunk_ms[1], 1)
     ach = bytes_step / (per_launch * 1e-3) / 1e9 if per_launch else None
+    # the same steps with the forget gate (PaTH-FoX decode): the cached gate biases
+    # ([B,H,cap] fp32) are read and written in place beside the keys
+    gen = torch.Generator().manual_seed(1)
+    lfs = [torch.nn.functional.logsigmoid(3.0 + torch.randn((w.B, w.H), generator=gen)).to(dev)
+           for _ in range(w.steps)]
+    gc = torch.zeros((w.B, w.H, cap), dtype=torch.float32, device=dev)
+    for t in range(3):
+        s = sd[t]
+        P.path_decode_step(s["q"], s["k_new"], s["v_new"], s["w"], s["beta"], kd, vd, w.n0 + t,
+                           out=out, workspace=ws, log_f=lfs[t], g_cache=gc)
+    torch.cuda.synchronize()
+    barrier()
+    P.lib().path_profile_enable(1)
+    e0.record(stream)
+    for t, s in enumerate(sd):
+        P.path_decode_step(s["q"], s["k_new"], s["v_new"], s["w"], s["beta"], kd, vd, w.n0 + t,
+                           out=out, workspace=ws, log_f=lfs[t], g_cache=gc)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    P.lib().path_profile_enable(0)
+    gstages = read_profile()
+    gms = max_over_ranks(e0.elapsed_time(e1)) / w.steps
+    gbytes = bytes_step + 2.0 * nh * n_avg * 4  # + read and write the gate biases
+    gt, gcnt = gstages.get("decode_chunks", (0.0, 1))
+    gper = gt / max(gcnt, 1)
+    gach = gbytes / (gper * 1e-3) / 1e9 if gper else None
+    gated = {"value": whole_job_rate(world, gbytes, gms) / 1e9, "unit": "GB/s",
+             "us_per_step": gms * 1e3, "bytes_per_step": gbytes,
+             "roofline": {"kernel": "decode_chunks (gated)", "bound": "hbm", "achieved": gach,
+                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": gach / peaks["hbm_gbs"] if gach else None, "traffic": None}}
     return {"workload": DECODE, "value": gbs, "unit": "GB/s", "us_per_step": ms * 1e3,
             "bytes_per_step": bytes_step,
             "roofline": {"kernel": "decode_chunks", "bound": "hbm", "achieved": ach,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / peaks["hbm_gbs"] if ach else None, "traffic": None,
-                         "peak_source": f"{peaks['source']} HBM copy"}}
+                         "peak_source": f"{peaks['source']} HBM copy"},
+            "gated": gated}
 
 
 PROFILE_CASES = {
@@ -522,6 +604,10 @@ PROFILE_CASES = {
 # name: (B, H, d, cached rows) -- two untimed decode steps on a 16K-row cache
 DECODE_PROFILE_CASES = {
     "decode_b2h32c16k": (2, 32, 128, 16384),
+}
+# name: (B, H, L, d) -- one untimed prefill (forward + decode cache)
+PREFILL_PROFILE_CASES = {
+    "prefill_b4h24l4096": (4, 24, 4096, 64),
 }
 
 
@@ -542,6 +628,16 @@ def run_profile_case(name):
                                out=out)
         torch.cuda.synchronize()
         print(json.dumps({"profile_case": name, "ok": bool(torch.isfinite(out.float()).all())}))
+        return 0
+
+    if name in PREFILL_PROFILE_CASES:
+        B, H, L, d = PREFILL_PROFILE_CASES[name]
+        x = si.make_inputs(B, H, L, d, torch.bfloat16, seed=0)
+        dx = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
+        out, lse, kc, vc, _ = P.path_attn_prefill(dx["q"], dx["k"], dx["v"], dx["w"], dx["beta"],
+                                                  L + 64)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": name, "ok": bool(torch.isfinite(kc.float()).all())}))
         return 0
 
     B, H, L, d, fox = PROFILE_CASES[name]
@@ -567,8 +663,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES) + sorted(DECODE_PROFILE_CASES),
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES) + sorted(DECODE_PROFILE_CASES)
+                    + sorted(PREFILL_PROFILE_CASES),
                     help="run one untimed fwd+bwd on a small shape (for profiler captures)")
     args = ap.parse_args()
     if args.profile_case:

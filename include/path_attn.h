@@ -194,6 +194,52 @@ path_status path_decode_step_noalloc(const void *q, const void *k_new, const voi
                                      path_stream_t stream);
 
 /*
+ * PaTH-FoX decode step: path_decode_step with the forget gate. Each cached
+ * key j carries its gate bias g_j = c_t - c_j (the "PaTH-FoX 扩展" logit term
+ * of the Paper-Notes page, for the position t being decoded), updated in
+ * place like the keys:
+ *   1. keys as in path_decode_step, and g_j <- g_j + log_f for j < n;
+ *   2. k_new / v_new into row n, and g_n = 0;
+ *   3. out = softmax_j(scale * q^T k_j + g_j) V over the n+1 rows.
+ * log_f: [B,H] fp32, log f_t of the position being decoded (<= 0 for a
+ * forget gate, not checked). g_cache: [B,H,capacity] fp32, rows 0..n-1 as
+ * the previous step or path_attn_prefill left them; after the call rows
+ * 0..n. The workspace is sized by path_decode_workspace_bytes. Everything
+ * else, including the errors, as path_decode_step; log_f or g_cache NULL is
+ * PATH_ERR_INVALID_ARG.
+ */
+path_status path_decode_step_gated(const void *q, const void *k_new, const void *v_new,
+                                   const void *w, const float *beta, const float *log_f,
+                                   float scale, int B, int H, int d, int n_cached, int capacity,
+                                   path_dtype dt, void *k_cache, void *v_cache, float *g_cache,
+                                   void *out, void *workspace, size_t workspace_bytes,
+                                   path_stream_t stream);
+
+/*
+ * Prefill: path_attn_fwd over positions 0..L-1 (same arguments, results and
+ * workspace, sized by path_attn_workspace_bytes with for_bwd = 0 or 1), and
+ * the decode cache those positions leave, ready for path_decode_step (or
+ * path_decode_step_gated with the gate) at n_cached = L:
+ *   k_cache row j = H_{L-1} ... H_{j+1} k_j  (the in-place key update of the
+ *                   Paper-Notes "训练策略" inference paragraph, applied for
+ *                   every later position; computed blockwise from the
+ *                   forward's transported keys and block products),
+ *   v_cache row j = v_j,
+ *   g_cache row j = c_{L-1} - c_j = sum of log_f over positions j+1..L-1.
+ * k_cache, v_cache: [B,H,capacity,d] in the input element type (fp32 for
+ * PATH_F32, bf16 for PATH_BF16 and PATH_BF16_F32OUT), 16-byte aligned;
+ * g_cache: [B,H,capacity] fp32, NULL iff log_f is NULL. Only rows 0..L-1 are
+ * written. Requires d in {64, 128} (the decode head dims; else
+ * PATH_ERR_UNSUPPORTED) and L <= capacity (else PATH_ERR_INVALID_ARG). The
+ * caches must not alias the inputs.
+ */
+path_status path_attn_prefill(const void *q, const void *k, const void *v, const void *w,
+                              const float *beta, const float *log_f, float scale, int B, int H,
+                              int L, int d, path_dtype dt, void *out, float *lse, void *k_cache,
+                              void *v_cache, float *g_cache, int capacity, void *workspace,
+                              size_t workspace_bytes, path_stream_t stream);
+
+/*
  * Diagnostics (host-side, process-wide; not needed for normal use).
  *
  * path_kernel_launch_count: number of CUDA kernels this library has launched

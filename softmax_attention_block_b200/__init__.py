@@ -10,7 +10,10 @@ CUDA device is present, the calls raise.
 Entry points (same names as the C ABI):
 - ``path_attn_fwd(q, k, v, w, beta, log_f=None, scale=None) -> (out, lse)``
 - ``path_attn_bwd(q, k, v, w, beta, out, lse, dout, log_f=None, scale=None) -> dict``
-- ``path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=None) -> out``
+- ``path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=None,
+  log_f=None, g_cache=None) -> out`` (with ``log_f``: ``path_decode_step_gated``)
+- ``path_attn_prefill(q, k, v, w, beta, capacity, log_f=None, scale=None)
+  -> (out, lse, k_cache, v_cache, g_cache)``
 - ``path_attn_workspace_bytes``, ``path_decode_workspace_bytes``, ``path_status_string``
 """
 from __future__ import annotations
@@ -66,9 +69,14 @@ def lib() -> ctypes.CDLL:
                                     vp, vp, vp, vp, fp, fp, ctypes.c_uint, vp, sz, vp]
         L.path_decode_step.argtypes = [vp, vp, vp, vp, fp, f, i, i, i, i, i, i, vp, vp, vp, vp,
                                        sz, vp]
+        L.path_decode_step_gated.argtypes = [vp, vp, vp, vp, fp, fp, f, i, i, i, i, i, i, vp,
+                                             vp, fp, vp, vp, sz, vp]
+        L.path_attn_prefill.argtypes = [vp, vp, vp, vp, fp, fp, f, i, i, i, i, i, vp, fp, vp, vp,
+                                        fp, i, vp, sz, vp]
         L.path_attn_wait_status.argtypes = [vp, vp]
         L.path_kernel_launch_count.restype = ctypes.c_ulonglong
-        for fn in (L.path_attn_fwd, L.path_attn_bwd, L.path_decode_step, L.path_attn_wait_status):
+        for fn in (L.path_attn_fwd, L.path_attn_bwd, L.path_decode_step,
+                   L.path_decode_step_gated, L.path_attn_prefill, L.path_attn_wait_status):
             fn.restype = i
         _lib = L
     return _lib
@@ -178,18 +186,68 @@ def path_attn_bwd(q, k, v, w, beta, out, lse, dout, log_f=None, scale=None, grad
 
 
 def path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=None, out=None,
-                     workspace=None):
-    """One decode step; updates k_cache / v_cache ([B,H,cap,d]) in place. Returns out [B,H,d]."""
+                     workspace=None, log_f=None, g_cache=None):
+    """One decode step; updates k_cache / v_cache ([B,H,cap,d]) in place. Returns out [B,H,d].
+
+    With the forget gate, log_f [B,H] fp32 is log f of the new position and g_cache
+    [B,H,cap] fp32 the cached keys' gate biases, also updated in place
+    (path_decode_step_gated)."""
     B, H, cap, d = k_cache.shape
     dt = _DT[k_cache.dtype]
     if out is None:
         out = torch.empty_like(q)
-    _check_dev(q, k_new, v_new, w, beta, k_cache, v_cache, out)
+    if (log_f is None) != (g_cache is None):
+        raise ValueError("log_f and g_cache go together")
+    _check_dev(q, k_new, v_new, w, beta, k_cache, v_cache, out, log_f, g_cache)
     nbytes = path_decode_workspace_bytes(B, H, cap, d, k_cache.dtype)
     ws = _workspace(nbytes, q.device, workspace)
-    st = lib().path_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(w), _ptr(beta),
-                                _scale(scale, d), B, H, d, int(n_cached), cap, dt, _ptr(k_cache),
-                                _ptr(v_cache), _ptr(out), _ptr(ws), nbytes, _stream())
+    if log_f is None:
+        st = lib().path_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(w), _ptr(beta),
+                                    _scale(scale, d), B, H, d, int(n_cached), cap, dt,
+                                    _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(ws), nbytes,
+                                    _stream())
+        where = "path_decode_step"
+    else:
+        st = lib().path_decode_step_gated(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(w), _ptr(beta),
+                                          _ptr(log_f), _scale(scale, d), B, H, d, int(n_cached),
+                                          cap, dt, _ptr(k_cache), _ptr(v_cache), _ptr(g_cache),
+                                          _ptr(out), _ptr(ws), nbytes, _stream())
+        where = "path_decode_step_gated"
     if st:
-        raise PathError(st, "path_decode_step")
+        raise PathError(st, where)
     return out
+
+
+def path_attn_prefill(q, k, v, w, beta, capacity, log_f=None, scale=None, out=None, lse=None,
+                      k_cache=None, v_cache=None, g_cache=None, workspace=None, out_dtype=None):
+    """Forward over positions 0..L-1 plus the decode cache it leaves.
+
+    Returns (out, lse, k_cache, v_cache, g_cache): out / lse as path_attn_fwd; the
+    caches [B,H,capacity,d] in q's dtype with rows 0..L-1 written (k_cache row j =
+    H_{L-1} ... H_{j+1} k_j, v_cache row j = v_j); g_cache [B,H,capacity] fp32 (row j =
+    c_{L-1} - c_j) with the forget gate, else None. Caches the call allocates are
+    zero past row L-1."""
+    B, H, L, d = q.shape
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    dt = _mode(q.dtype, out.dtype)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    if k_cache is None:
+        k_cache = torch.zeros((B, H, capacity, d), dtype=q.dtype, device=q.device)
+    if v_cache is None:
+        v_cache = torch.zeros((B, H, capacity, d), dtype=q.dtype, device=q.device)
+    if log_f is not None and g_cache is None:
+        g_cache = torch.zeros((B, H, capacity), dtype=torch.float32, device=q.device)
+    if log_f is None:
+        g_cache = None
+    _check_dev(q, k, v, w, beta, log_f, out, lse, k_cache, v_cache, g_cache)
+    nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, False, out.dtype)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().path_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(beta), _ptr(log_f),
+                                 _scale(scale, d), B, H, L, d, dt, _ptr(out), _ptr(lse),
+                                 _ptr(k_cache), _ptr(v_cache), _ptr(g_cache), int(capacity),
+                                 _ptr(ws), nbytes, _stream())
+    if st:
+        raise PathError(st, "path_attn_prefill")
+    return out, lse, k_cache, v_cache, g_cache

@@ -59,11 +59,30 @@ struct DecodeArgs {
     void *k_cache, *v_cache;            // [nh, capacity, d]
     void *out;                          // [nh, d]
     float *partial;                     // [nh, nchunk, d + 2]
+    // forget gate (both null without it): log f_t per head [nh], and each
+    // cached key's logit bias c_t - c_j [nh, capacity], carried in place
+    const float *log_f = nullptr;
+    float *g_cache = nullptr;
 };
 
 constexpr int DECODE_CHUNK = 1024;  // cached rows per CTA
 
 cudaError_t decode_step(const DecodeArgs &a, int dt, int d, cudaStream_t st);
+
+// The decode cache a prefill of positions 0..L-1 leaves, from the forward's
+// transported keys and block products.
+struct CacheArgs {
+    const void *Kt;    // [nh, Lp, d] boundary-adjusted keys (mid type)
+    const void *Khat;  // [nh, npairs, BT, d] transported key tiles (mid type)
+    const void *Pm;    // [nh, nblk, d, d] block products (mid type)
+    const void *v;     // [nh, L, d] (input type)
+    const float *c;    // [nh, Lp] gate prefix, or null
+    int L, nblk, nh, capacity;
+    void *k_cache, *v_cache;  // [nh, capacity, d] (input type), rows 0..L-1 written
+    float *g_cache;           // [nh, capacity], rows 0..L-1 written; null without the gate
+};
+
+cudaError_t prefill_cache(const CacheArgs &a, Types t, int d, cudaStream_t st);
 
 // Allocation-free decode: fixed device scratch of NOALLOC_SCRATCH_FLOATS.
 constexpr long long NOALLOC_SCRATCH_FLOATS = 1LL << 20;

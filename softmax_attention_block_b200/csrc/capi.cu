@@ -152,6 +152,37 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
     return PATH_OK;
 }
 
+// path_attn_fwd after argument validation: carves `workspace` into ws and
+// enqueues the forward.
+path_status run_forward(const void *q, const void *k, const void *v, const void *w,
+                        const float *beta, const float *log_f, float scale, const Layout &y,
+                        path_dtype dt, void *out, float *lse, void *workspace,
+                        size_t workspace_bytes, AttnWs &ws, cudaStream_t st)
+{
+    const size_t need = carve_attn(nullptr, y, dt, false, ws);
+    if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
+    // a workspace sized for the backward also receives what a backward that
+    // reuses it needs beyond the forward's own buffers
+    const bool for_bwd = workspace_bytes >= carve_attn(nullptr, y, dt, true, ws);
+    carve_attn(workspace, y, dt, for_bwd, ws);
+    if (!for_bwd) ws.halves = nullptr;
+    TRY(cudaMemsetAsync(ws.err, 0, sizeof(int), st));
+    path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
+    if (s != PATH_OK) return s;
+    FwdArgs a{ws.Qt, ws.Khat, v, ws.Vh, ws.Sd, log_f ? ws.c : nullptr, scale, y.L, y.nblk, y.nh, out, lse};
+    const Types t = types_of(dt);
+    if (use_tc_fwd(t, y, v)) {
+        {
+            Stage s_cv("v_to_f16", st);
+            TRY(convert_to_f16(v, ws.Vh, (long long)y.nh * y.L * y.d, st));
+        }
+        Stage s_attn("attn_fwd", st);
+        return launch_status(attn_fwd_tc(a, t, y.d, ws.err, st));
+    }
+    Stage s_attn("attn_fwd", st);
+    return launch_status(attn_fwd_simt(a, t, y.d, st));
+}
+
 }  // namespace
 
 extern "C" {
@@ -185,31 +216,36 @@ path_status path_attn_fwd(const void *q, const void *k, const void *v, const voi
     if (!q || !k || !v || !w || !beta || !out || !lse) return PATH_ERR_INVALID_ARG;
     if (!fwd_dims_ok(B, H, L, d) || !isfinite(scale)) return PATH_ERR_INVALID_ARG;
     if (!head_dim_supported(d) || !dtype_ok(dt) || !grid_ok(B, H, L)) return PATH_ERR_UNSUPPORTED;
-    const Layout y = make_layout(B, H, L, d, dt);
     AttnWs ws;
-    const size_t need = carve_attn(nullptr, y, dt, false, ws);
-    if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
-    // a workspace sized for the backward also receives what a backward that
-    // reuses it needs beyond the forward's own buffers
-    const bool for_bwd = workspace_bytes >= carve_attn(nullptr, y, dt, true, ws);
-    carve_attn(workspace, y, dt, for_bwd, ws);
-    if (!for_bwd) ws.halves = nullptr;
+    return run_forward(q, k, v, w, beta, log_f, scale, make_layout(B, H, L, d, dt), dt, out, lse,
+                       workspace, workspace_bytes, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+path_status path_attn_prefill(const void *q, const void *k, const void *v, const void *w,
+                              const float *beta, const float *log_f, float scale, int B, int H,
+                              int L, int d, path_dtype dt, void *out, float *lse, void *k_cache,
+                              void *v_cache, float *g_cache, int capacity, void *workspace,
+                              size_t workspace_bytes, path_stream_t stream)
+{
+    if (!q || !k || !v || !w || !beta || !out || !lse || !k_cache || !v_cache)
+        return PATH_ERR_INVALID_ARG;
+    if ((log_f == nullptr) != (g_cache == nullptr)) return PATH_ERR_INVALID_ARG;
+    if (!fwd_dims_ok(B, H, L, d) || !isfinite(scale) || capacity < L) return PATH_ERR_INVALID_ARG;
+    if ((d != 64 && d != 128) || !dtype_ok(dt) || !grid_ok(B, H, L)) return PATH_ERR_UNSUPPORTED;
+    // 16-byte vector access of v and the caches
+    const uintptr_t al = reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(k_cache) |
+                         reinterpret_cast<uintptr_t>(v_cache);
+    if (al & 15u) return PATH_ERR_INVALID_ARG;
+    const Layout y = make_layout(B, H, L, d, dt);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    TRY(cudaMemsetAsync(ws.err, 0, sizeof(int), st));
-    path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
+    AttnWs ws;
+    path_status s = run_forward(q, k, v, w, beta, log_f, scale, y, dt, out, lse, workspace,
+                                workspace_bytes, ws, st);
     if (s != PATH_OK) return s;
-    FwdArgs a{ws.Qt, ws.Khat, v, ws.Vh, ws.Sd, log_f ? ws.c : nullptr, scale, y.L, y.nblk, y.nh, out, lse};
-    const Types t = types_of(dt);
-    if (use_tc_fwd(t, y, v)) {
-        {
-            Stage s_cv("v_to_f16", st);
-            TRY(convert_to_f16(v, ws.Vh, (long long)y.nh * y.L * d, st));
-        }
-        Stage s_attn("attn_fwd", st);
-        return launch_status(attn_fwd_tc(a, t, d, ws.err, st));
-    }
-    Stage s_attn("attn_fwd", st);
-    return launch_status(attn_fwd_simt(a, t, d, st));
+    CacheArgs ca{ws.Kt, ws.Khat, ws.Pm, v, log_f ? ws.c : nullptr, y.L, y.nblk, y.nh, capacity,
+                 k_cache, v_cache, g_cache};
+    Stage s_c("prefill_cache", st);
+    return launch_status(prefill_cache(ca, types_of(dt), d, st));
 }
 
 path_status path_attn_bwd(const void *q, const void *k, const void *v, const void *w,
@@ -313,6 +349,30 @@ path_status path_decode_step(const void *q, const void *k_new, const void *v_new
     if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
     DecodeArgs a{q, k_new, v_new, w, beta, scale, B * H, n_cached, capacity,
                  k_cache, v_cache, out, static_cast<float *>(workspace)};
+    return launch_status(decode_step(a, (int)dt, d, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+path_status path_decode_step_gated(const void *q, const void *k_new, const void *v_new,
+                                   const void *w, const float *beta, const float *log_f,
+                                   float scale, int B, int H, int d, int n_cached, int capacity,
+                                   path_dtype dt, void *k_cache, void *v_cache, float *g_cache,
+                                   void *out, void *workspace, size_t workspace_bytes,
+                                   path_stream_t stream)
+{
+    if (!q || !k_new || !v_new || !w || !beta || !log_f || !k_cache || !v_cache || !g_cache ||
+        !out)
+        return PATH_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || capacity <= 0 || n_cached < 0 || n_cached + 1 > capacity ||
+        !isfinite(scale))
+        return PATH_ERR_INVALID_ARG;
+    if ((d != 64 && d != 128) || !decode_dtype_ok(dt) || !grid_ok(B, H, 1)) return PATH_ERR_UNSUPPORTED;
+    const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(w) |
+                         reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache);
+    if (al & 15u) return PATH_ERR_INVALID_ARG;
+    const size_t need = path_decode_workspace_bytes(B, H, capacity, d, dt);
+    if (!workspace || workspace_bytes < need) return PATH_ERR_WORKSPACE;
+    DecodeArgs a{q, k_new, v_new, w, beta, scale, B * H, n_cached, capacity,
+                 k_cache, v_cache, out, static_cast<float *>(workspace), log_f, g_cache};
     return launch_status(decode_step(a, (int)dt, d, reinterpret_cast<cudaStream_t>(stream)));
 }
 

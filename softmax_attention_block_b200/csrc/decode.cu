@@ -1,7 +1,9 @@
 // Decode step: fused in-place key update + one-query attention over the
 // cache, split over chunks of rows (Paper-Notes "训练策略", inference
 // paragraph: cached keys are updated in place by H_t, after which decoding
-// is plain softmax attention).
+// is plain softmax attention). With the forget gate (Paper-Notes "PaTH-FoX
+// 扩展": the logit gains c_t - c_j), each cached key also carries that bias,
+// updated in place by the same pass: g_j += log f_t, and the new key's is 0.
 //
 // Pass 1 (decode_chunk_kernel): each CTA streams DECODE_CHUNK cached rows of
 // one head. A group of d/V lanes owns one row at a time (V elements of 16
@@ -79,7 +81,7 @@ __device__ __forceinline__ float group_sum(float x)
 constexpr int THREADS = 256;
 constexpr int UNROLL = 8;  // rows in flight per row group (loads issued before the math)
 
-template <typename T, int D, int CHUNK = DECODE_CHUNK>
+template <typename T, int D, bool GATE, int CHUNK = DECODE_CHUNK>
 __global__ void __launch_bounds__(THREADS) decode_chunk_kernel(DecodeArgs a, int nchunk)
 {
     constexpr int V = Vec<T>::N;        // elements per 16-byte vector
@@ -95,6 +97,8 @@ __global__ void __launch_bounds__(THREADS) decode_chunk_kernel(DecodeArgs a, int
     unpack<T>(reinterpret_cast<const uint4 *>(static_cast<const T *>(a.w) + (long long)h * D)[lane_in_row], w);
     unpack<T>(reinterpret_cast<const uint4 *>(static_cast<const T *>(a.q) + (long long)h * D)[lane_in_row], q);
     const float beta = a.beta[h];
+    const float lf = GATE ? a.log_f[h] : 0.f;
+    float *gc = GATE ? a.g_cache + (long long)h * a.capacity : nullptr;
     uint4 *K = reinterpret_cast<uint4 *>(static_cast<T *>(a.k_cache) + (long long)h * a.capacity * D);
     const uint4 *Vc = reinterpret_cast<const uint4 *>(static_cast<const T *>(a.v_cache) + (long long)h * a.capacity * D);
     float m = -INFINITY, l = 0.f, acc[V];
@@ -104,12 +108,15 @@ __global__ void __launch_bounds__(THREADS) decode_chunk_kernel(DecodeArgs a, int
     // every lane reaches every group shuffle; rows past the chunk are masked.
     for (int rb = r0; rb < r1; rb += G * UNROLL) {
         uint4 kv[UNROLL], vv[UNROLL];
+        float gv[UNROLL];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
             const int r = rb + u * G + g;
+            gv[u] = 0.f;
             if (r < r1) {
                 kv[u] = K[(long long)r * LPR + lane_in_row];
                 vv[u] = Vc[(long long)r * LPR + lane_in_row];
+                if (GATE) gv[u] = gc[r];
             } else {
                 kv[u] = make_uint4(0u, 0u, 0u, 0u);
                 vv[u] = make_uint4(0u, 0u, 0u, 0u);
@@ -135,8 +142,13 @@ __global__ void __launch_bounds__(THREADS) decode_chunk_kernel(DecodeArgs a, int
 #pragma unroll
             for (int i = 0; i < V; ++i) s = fmaf(q[i], k[i], s);
             s = group_sum<LPR>(s);
+            float bias = 0.f;
+            if (GATE) {
+                bias = gv[u] + lf;
+                if (valid && lane_in_row == 0) gc[r] = bias;
+            }
             if (valid) {
-                const float z = a.scale * s;
+                const float z = fmaf(a.scale, s, bias);
                 const float mn = fmaxf(m, z);
                 const float corr = __expf(m - mn);
                 const float p = __expf(z - mn);
@@ -206,6 +218,16 @@ __global__ void decode_combine_kernel(DecodeArgs a, int nchunk)
     const long long row = ((long long)h * a.capacity + a.n) * D + e;
     static_cast<T *>(a.k_cache)[row] = kn[e];
     static_cast<T *>(a.v_cache)[row] = vn[e];
+    if (a.g_cache && e == 0) a.g_cache[(long long)h * a.capacity + a.n] = 0.f;
+}
+
+template <typename T, int D, int CHUNK>
+void launch_chunks(const DecodeArgs &a, int nchunk, cudaStream_t st)
+{
+    if (a.g_cache)
+        decode_chunk_kernel<T, D, true, CHUNK><<<dim3(nchunk, a.nh), THREADS, 0, st>>>(a, nchunk);
+    else
+        decode_chunk_kernel<T, D, false, CHUNK><<<dim3(nchunk, a.nh), THREADS, 0, st>>>(a, nchunk);
 }
 
 template <typename T, int D>
@@ -214,7 +236,7 @@ cudaError_t run(const DecodeArgs &a, cudaStream_t st)
     const int nchunk = ceil_div(a.n, DECODE_CHUNK);
     if (nchunk > 0) {
         Stage s("decode_chunks", st);
-        decode_chunk_kernel<T, D><<<dim3(nchunk, a.nh), THREADS, 0, st>>>(a, nchunk);
+        launch_chunks<T, D, DECODE_CHUNK>(a, nchunk, st);
         count_launches();
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
@@ -232,7 +254,7 @@ cudaError_t run_fixed(const DecodeArgs &a, cudaStream_t st)
 {
     const int nchunk = ceil_div(a.n, CHUNK);
     if (nchunk > 0) {
-        decode_chunk_kernel<T, D, CHUNK><<<dim3(nchunk, a.nh), THREADS, 0, st>>>(a, nchunk);
+        launch_chunks<T, D, CHUNK>(a, nchunk, st);
         count_launches();
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;

@@ -129,3 +129,39 @@ def test_decode_rejects_bad_arguments(lib):
 def test_profile_toggle(lib):
     prev = lib.path_profile_enable(1)
     assert lib.path_profile_enable(prev) == 1
+
+
+def test_gated_decode_rejects_bad_arguments(lib):
+    def dec(**kw):
+        a = dict(log_f=FAKE, g=FAKE, n=10, cap=11, d=128, wsb=1 << 40)
+        a.update(kw)
+        return lib.path_decode_step_gated(FAKE, FAKE, FAKE, FAKE, FAKE, a["log_f"], 0.1, 2, 2,
+                                          a["d"], a["n"], a["cap"], BF16, FAKE, FAKE, a["g"],
+                                          FAKE, FAKE, a["wsb"], None)
+
+    assert dec(log_f=None) == INVALID
+    assert dec(g=None) == INVALID
+    assert dec(n=11) == INVALID
+    assert dec(d=16) == UNSUPPORTED
+    assert dec(wsb=4) == WORKSPACE
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    def pre(**kw):
+        a = dict(q=FAKE, v=FAKE, log_f=None, g=None, L=64, d=64, cap=64, kc=FAKE, ws=FAKE,
+                 wsb=1 << 40)
+        a.update(kw)
+        return lib.path_attn_prefill(a["q"], FAKE, a["v"], FAKE, FAKE, a["log_f"], 0.125, 1, 1,
+                                     a["L"], a["d"], BF16, FAKE, FAKE, a["kc"], FAKE, a["g"],
+                                     a["cap"], a["ws"], a["wsb"], None)
+
+    assert pre(q=None) == INVALID
+    assert pre(kc=None) == INVALID
+    assert pre(log_f=FAKE) == INVALID       # g_cache must come with log_f
+    assert pre(g=FAKE) == INVALID
+    assert pre(cap=63) == INVALID           # L > capacity
+    assert pre(kc=FAKE + 8) == INVALID      # caches must be 16-byte aligned
+    assert pre(v=FAKE + 4) == INVALID
+    assert pre(d=32) == UNSUPPORTED         # decode head dims only
+    assert pre(ws=None) == WORKSPACE
+    assert pre(wsb=100) == WORKSPACE

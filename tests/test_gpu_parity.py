@@ -284,3 +284,99 @@ def test_launch_counter_advances(P):
     x = si.make_inputs(1, 1, 200, 64, torch.bfloat16, seed=5)
     run_ours(P, x, backward=True)
     assert P.lib().path_kernel_launch_count() > before
+
+
+# ---------------------------------------------------------------- prefill -> decode
+def _cache_bar(got, ref, dtype):
+    """fp32 caches: 1e-4. bf16 caches: 2e-2 plus one bf16 ulp of the reference, the
+    stored-bf16 rule above (the keys are carried in fp16 through the forward's block
+    products and stored in bf16)."""
+    diff = np.abs(got - ref)
+    if dtype == torch.float32:
+        return bool(np.all(diff <= 1e-4)), float(diff.max())
+    return bool(np.all(diff <= 2e-2 + ulp_bf16(ref))), float(diff.max())
+
+
+def _prefill_check(P, x, cap, heads=None):
+    dd = to_dev(x)
+    dtype = dd["q"].dtype
+    out, lse, kc, vc, gc = P.path_attn_prefill(dd["q"], dd["k"], dd["v"], dd["w"], dd["beta"],
+                                               cap, dd["log_f"])
+    torch.cuda.synchronize()
+    B, H, L, d = dd["q"].shape
+    pick = (lambda t: t) if heads is None else (
+        lambda t: t.reshape(B * H, *t.shape[2:])[heads].unsqueeze(0))
+    xs = x if heads is None else {k: (None if v is None else pick(v)) for k, v in x.items()}
+    rk, rv, rg = oracle.prefill_cache(xs["k"], xs["v"], xs["w"], xs["beta"], xs["log_f"],
+                                      capacity=cap)
+    ref = oracle_results(xs, False)
+    mode = "f32" if dtype == torch.float32 else "bf16"
+    compare({"out": pick(out), "lse": pick(lse)}, ref, mode, f"prefill fwd L={L} d={d}")
+    ok_k, ek = _cache_bar(np64(pick(kc.cpu()))[..., :L, :], rk[..., :L, :], dtype)
+    np.testing.assert_array_equal(np64(pick(vc.cpu()))[..., :L, :], rv[..., :L, :])
+    eg = 0.0
+    if rg is not None:
+        eg = float(np.abs(np64(pick(gc.cpu()))[..., :L] - rg[..., :L]).max())
+    print(f"\n[prefill cache L={L} d={d} {dtype}] k max err {ek:.3g}, g max err {eg:.3g}")
+    assert ok_k, f"key cache beyond the bar (max err {ek:.3g})"
+    if rg is not None:
+        # g_j = c_{L-1} - c_j from prefix sums kept in fp64 and stored in fp32: two
+        # fp32 roundings of |c| and one of the difference, so |err| <= 3 2^-24 max|c|
+        cmax = float(np.abs(np.cumsum(np64(xs["log_f"]), axis=-1)).max())
+        assert eg <= 4 * 2.0 ** -24 * cmax + 1e-12, (eg, cmax)
+    # rows past L are left as the caller had them (zero here)
+    assert not kc[..., L:, :].any() and not vc[..., L:, :].any()
+    if gc is not None:
+        assert not gc[..., L:].any()
+
+
+@pytest.mark.parametrize("dtype,d,L,fox", [(torch.float32, 64, 300, False),
+                                           (torch.float32, 128, 130, True),
+                                           (torch.bfloat16, 64, 1, False),
+                                           (torch.bfloat16, 64, 100, True),
+                                           (torch.bfloat16, 64, 700, True),
+                                           (torch.bfloat16, 128, 390, False)])
+def test_prefill_cache_matches_oracle(P, dtype, d, L, fox):
+    x = si.make_inputs(2, 2, L, d, dtype, seed=6, fox=fox,
+                       clip_beta=dtype == torch.bfloat16)
+    _prefill_check(P, x, L + 9)
+
+
+def test_prefill_cache_full_size_sampled_heads(P):
+    """The headline shape (32 key blocks, so 31 chained block products before the
+    last one), oracle on sampled heads."""
+    x = si.workload_inputs("fwdbwd_bf16_l4096")
+    _prefill_check(P, x, 4096 + 64, heads=[0, 191])
+
+
+@pytest.mark.parametrize("dtype,d,fox,L0", [(torch.float32, 64, True, 333),
+                                            (torch.bfloat16, 64, True, 333),
+                                            (torch.bfloat16, 128, False, 333),
+                                            (torch.bfloat16, 64, True, 2100)])
+def test_decode_after_prefill_continues_the_forward(P, dtype, d, fox, L0):
+    """Prefill of the first L0 positions, then (gated) decode steps: the decode outputs
+    are the forward rows L0.. of the whole sequence (oracle). L0 = 2100 puts the
+    decode over three split chunks, the last one ragged."""
+    steps = 4
+    x = si.make_inputs(1, 2, L0 + steps, d, dtype, seed=7, fox=fox,
+                       clip_beta=dtype == torch.bfloat16)
+    ref_out, _ = oracle.fwd(x["q"], x["k"], x["v"], x["w"], x["beta"], x["log_f"])
+    dd = to_dev(x)
+    head = lambda t: None if t is None else t[:, :, :L0].contiguous()
+    col = lambda t, i: None if t is None else t[:, :, i].contiguous()
+    _, _, kc, vc, gc = P.path_attn_prefill(head(dd["q"]), head(dd["k"]), head(dd["v"]),
+                                           head(dd["w"]), head(dd["beta"]), L0 + steps,
+                                           head(dd["log_f"]))
+    worst, ok = 0.0, True
+    for t in range(L0, L0 + steps):
+        o = P.path_decode_step(col(dd["q"], t), col(dd["k"], t), col(dd["v"], t),
+                               col(dd["w"], t), col(dd["beta"], t), kc, vc, t,
+                               log_f=col(dd["log_f"], t), g_cache=gc)
+        r = ref_out[:, :, t]
+        diff = np.abs(np64(o.cpu()) - r)
+        worst = max(worst, float(diff.max()))
+        bar = 1e-4 if dtype == torch.float32 else 2e-2 + ulp_bf16(r)
+        ok = ok and bool(np.all(diff <= bar))
+    torch.cuda.synchronize()
+    print(f"\n[prefill + decode L0={L0} d={d} {dtype} fox={fox}] out max err {worst:.3g}")
+    assert ok

@@ -380,3 +380,43 @@ def test_decode_after_prefill_continues_the_forward(P, dtype, d, fox, L0):
     torch.cuda.synchronize()
     print(f"\n[prefill + decode L0={L0} d={d} {dtype} fox={fox}] out max err {worst:.3g}")
     assert ok
+
+
+def test_hand_worked_example(P):
+    """The hand-derived example of tests/golden (d = 2, zero-padded to the kernels' head
+    dims: zero columns leave every logit and the first two output columns unchanged),
+    forward and prefill cache against the hand values themselves."""
+    import json
+    import os
+
+    with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                           "hand_worked_d2_l3.json")) as f:
+        g = json.load(f)
+
+    def pad(key, d):
+        a = torch.tensor(g[key], dtype=torch.float32)
+        return torch.nn.functional.pad(a, (0, d - a.shape[-1]))[None, None].contiguous().cuda()
+
+    beta = torch.tensor(g["beta"], dtype=torch.float32)[None, None].cuda()
+    lf = torch.tensor(g["log_f"], dtype=torch.float32)[None, None].cuda()
+    vv = np.array(g["v"], dtype=np.float64)
+    for gated in (False, True):
+        z = np.array([[-np.inf if x is None else x for x in r]
+                      for r in g["logits_gated" if gated else "logits"]])
+        p = np.exp(z - z.max(axis=1, keepdims=True))
+        ro = (p / p.sum(axis=1, keepdims=True)) @ vv
+        for d in (16, 64):
+            q, k, v, w = (pad(n, d) for n in ("q", "k", "v", "w"))
+            log_f = lf if gated else None
+            if d == 64:
+                out, _, kc, vc, gc = P.path_attn_prefill(q, k, v, w, beta, 3, log_f,
+                                                         scale=g["scale"])
+                torch.cuda.synchronize()
+                np.testing.assert_allclose(np64(kc.cpu())[0, 0, :, :2], g["k_cache"], atol=1e-5)
+                assert not kc[..., 2:].any()
+                if gated:
+                    np.testing.assert_allclose(np64(gc.cpu())[0, 0], g["g_cache"], atol=1e-5)
+            else:
+                out, _ = P.path_attn_fwd(q, k, v, w, beta, log_f, scale=g["scale"])
+                torch.cuda.synchronize()
+            np.testing.assert_allclose(np64(out.cpu())[0, 0, :, :2], ro, atol=1e-5)

@@ -98,8 +98,9 @@ def stage_model(name, B, H, L, d, BT=128):
 # B=1 H=24 L=4096 d=64 case (profiles/ summaries), scaled to the benchmark's
 # B=8 by the heads processed; None where the kernel changed since the capture.
 DRAM_BYTES_B1H24 = {
-    "attn_bwd": 325.6e6 + 97.7e6,
+    "attn_bwd": 325.6e6 + 95.3e6,
 }
+DRAM_BYTES_PREFILL_CACHE_B4H24 = 157.2e6
 
 
 def load_peaks():
@@ -508,14 +509,16 @@ def bench_prefill(P, x, w, ws, peaks, world, max_over_ranks, barrier, steps):
     t, c = stages.get("prefill_cache", (0.0, 1))
     per_launch = t / max(c, 1)
     ach = bytes_launch / (per_launch * 1e-3) / 1e9 if per_launch else None
+    # DRAM bytes of one launch from the ncu capture at B=4 (profiles/), scaled by heads
+    traffic = DRAM_BYTES_PREFILL_CACHE_B4H24 * (w.B * w.H) / 96.0
     del kc, vc, out, lse
     return {"workload": f"prefill {WORKLOAD}, cache capacity {cap}",
             "value": whole_job_rate(world, w.B * w.L, ms), "unit": "tokens/s",
             "ms_per_call": ms, "cache_kernel_ms": per_launch,
             "roofline": {"kernel": "prefill_cache", "bound": "hbm", "achieved": ach,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": ach / peaks["hbm_gbs"] if ach else None, "traffic": None,
-                         "algorithmic_bytes": bytes_launch,
+                         "frac": ach / peaks["hbm_gbs"] if ach else None, "traffic": traffic,
+                         "traffic_unit": "bytes per launch", "algorithmic_bytes": bytes_launch,
                          "peak_source": f"{peaks['source']} HBM copy"}}
 
 

@@ -7,7 +7,8 @@ forward's workspace (attention backward, UT adjoint, gate gradient) at B=8
 H=24 L=4096 d=64 bf16, inputs resident in HBM. The decode step (B=32 H=32 d=128, cache 16384 -> 16448,
 64 steps) is timed after it and reported under "decode" (with the forget gate's per-key
 bias under "decode.gated"), and a prefill of the same sequences (forward plus the decode
-cache it leaves) under "prefill".
+cache it leaves) under "prefill", and fwd+bwd at head dim 128 (B=8 H=12, the same model
+width) under "d128".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -447,6 +448,8 @@ def run_ours(args):
     torch.cuda.empty_cache()
     decode = None if args.no_decode else bench_decode(P, dev, peaks, world, max_over_ranks,
                                                        barrier)
+    d128 = None if args.no_d128 else bench_d128(P, dev, peaks, world, max_over_ranks, barrier,
+                                                 2)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -466,7 +469,8 @@ def run_ours(args):
             "tflops_fa_equiv": whole_job_rate(world, fa_equiv_flops(w.B, w.H, w.L, w.d), ms_step) / 1e12,
             "pct_bf16_peak": value / world / peaks["bf16_tflops_sustained"],
             "stages": stage_rows, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches, "clocks": clk, "decode": decode, "prefill": prefill}
+            "gpu_launches": launches, "clocks": clk, "decode": decode, "prefill": prefill,
+            "d128": d128}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -520,6 +524,59 @@ def bench_prefill(P, x, w, ws, peaks, world, max_over_ranks, barrier, steps):
                          "frac": ach / peaks["hbm_gbs"] if ach else None, "traffic": traffic,
                          "traffic_unit": "bytes per launch", "algorithmic_bytes": bytes_launch,
                          "peak_source": f"{peaks['source']} HBM copy"}}
+
+
+D128 = (8, 12, 4096, 128)  # B, H, L, d: the headline model width (24 x 64) as 12 x 128
+
+
+def d128_flops(B, H, L, d):
+    """Algorithmic FLOP of one fwd+bwd at any head dim, by the headline convention with
+    its transport terms kept in d: forward 2 L^2 d + L^2 d^2 / 64, backward
+    5 L^2 d + 3 L^2 d^2 / 64 (both 64-position blocks); 11 L^2 d at d = 64."""
+    return B * H * (7.0 * L * L * d + 4.0 * L * L * d * d / 64)
+
+
+def bench_d128(P, dev, peaks, world, max_over_ranks, barrier, steps):
+    """fwd+bwd at head dim 128 (same model width as the headline), per stage."""
+    B, H, L, d = D128
+    xc = si.make_inputs(B, H, L, d, torch.bfloat16, seed=0)
+    x = {k: (v.to(dev) if v is not None else None) for k, v in xc.items()}
+    del xc
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    grads = {n: torch.empty_like(x["q"]) for n in ("dq", "dk", "dv", "dw")}
+    grads["dbeta"] = torch.empty_like(x["beta"])
+    ws = torch.empty(P.path_attn_workspace_bytes(B, H, L, d, torch.bfloat16, True),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        P.path_attn_fwd(x["q"], x["k"], x["v"], x["w"], x["beta"], None, out=out, lse=lse,
+                        workspace=ws)
+        P.path_attn_bwd(x["q"], x["k"], x["v"], x["w"], x["beta"], out, lse, x["dout"], None,
+                        grads=grads, workspace=ws, reuse_fwd_workspace=True)
+
+    step()
+    torch.cuda.synchronize()
+    barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    P.lib().path_profile_enable(1)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    P.lib().path_profile_enable(0)
+    stages = read_profile()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / steps
+    fl = d128_flops(B, H, L, d)
+    del x, out, lse, grads, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"bf16 fwd+bwd B={B} H={H} L={L} d={d}",
+            "value": whole_job_rate(world, fl, ms) / 1e12, "unit": UNIT, "ms_per_step": ms,
+            "flop_convention": "7 L^2 d + 4 L^2 d^2 / 64 per head (11 L^2 d at d = 64)",
+            "pct_bf16_peak": whole_job_rate(1, fl, ms) / 1e12 / peaks["bf16_tflops_sustained"],
+            "stages_ms": {n: t / c for n, (t, c) in stages.items()}}
 
 
 def bench_decode(P, dev, peaks, world, max_over_ranks, barrier):
@@ -667,6 +724,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-d128", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES) + sorted(DECODE_PROFILE_CASES)
                     + sorted(PREFILL_PROFILE_CASES),

@@ -99,14 +99,37 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
+def _expect(name, t, shape, dtype):
+    """The library reads and writes these buffers by size alone: check what it will assume."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+
+
 def _check_dev(*ts):
+    ts = [t for t in ts if t is not None]
     for t in ts:
-        if t is None:
-            continue
         if not t.is_cuda:
             raise ValueError("all tensors must be CUDA tensors")
         if not t.is_contiguous():
             raise ValueError("all tensors must be contiguous")
+        if t.device != ts[0].device:
+            raise ValueError("all tensors must be on one device")
+
+
+def _check_attn_inputs(q, k, v, w, beta, log_f):
+    if q.dim() != 4:
+        raise ValueError("q must be [B,H,L,d]")
+    if q.dtype not in _DT:
+        raise ValueError(f"q: dtype {q.dtype}, expected float32 or bfloat16")
+    B, H, L, d = q.shape
+    for n, t in (("k", k), ("v", v), ("w", w)):
+        _expect(n, t, q.shape, q.dtype)
+    _expect("beta", beta, (B, H, L), torch.float32)
+    _expect("log_f", log_f, (B, H, L), torch.float32)
 
 
 def _stream():
@@ -130,13 +153,16 @@ def path_attn_fwd(q, k, v, w, beta, log_f=None, scale=None, out=None, lse=None, 
     """Forward pass. q, k, v, w: [B,H,L,d] (fp32 or bf16); beta, log_f: [B,H,L] fp32.
     out_dtype (default: q's dtype) may be torch.float32 with bf16 inputs.
     Returns (out [B,H,L,d], lse [B,H,L] fp32)."""
+    _check_attn_inputs(q, k, v, w, beta, log_f)
     B, H, L, d = q.shape
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     dt = _mode(q.dtype, out.dtype)
     if lse is None:
         lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
-    _check_dev(q, k, v, w, beta, log_f, out, lse)
+    _expect("out", out, q.shape, out.dtype)
+    _expect("lse", lse, (B, H, L), torch.float32)
+    _check_dev(q, k, v, w, beta, log_f, out, lse, workspace)
     nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, False, out.dtype)
     ws = _workspace(nbytes, q.device, workspace)
     st = lib().path_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(beta), _ptr(log_f),
@@ -160,18 +186,28 @@ def path_attn_bwd(q, k, v, w, beta, out, lse, dout, log_f=None, scale=None, grad
     then reuses the forward's block transforms and transported keys."""
     if reuse_fwd_workspace and workspace is None:
         raise ValueError("reuse_fwd_workspace needs the forward's workspace")
+    _check_attn_inputs(q, k, v, w, beta, log_f)
     B, H, L, d = q.shape
     dt = _mode(q.dtype, out.dtype)
     if dout.dtype != out.dtype:
         raise ValueError("dout must have out's dtype")
+    _expect("out", out, q.shape, out.dtype)
+    _expect("dout", dout, q.shape, out.dtype)
+    _expect("lse", lse, (B, H, L), torch.float32)
     if grads is None:
         grads = {n: torch.empty(q.shape, dtype=out.dtype, device=q.device)
                  for n in ("dq", "dk", "dv", "dw")}
         grads["dbeta"] = torch.empty_like(beta)
         if log_f is not None:
             grads["dlog_f"] = torch.empty_like(log_f)
+    for n in ("dq", "dk", "dv", "dw"):
+        _expect(n, grads[n], q.shape, out.dtype)
+    _expect("dbeta", grads["dbeta"], (B, H, L), torch.float32)
     dlf = grads.get("dlog_f") if log_f is not None else None
-    _check_dev(q, k, v, w, beta, log_f, out, lse, dout, *grads.values())
+    if log_f is not None and dlf is None:
+        raise ValueError("grads needs dlog_f when log_f is given")
+    _expect("dlog_f", dlf, (B, H, L), torch.float32)
+    _check_dev(q, k, v, w, beta, log_f, out, lse, dout, workspace, *grads.values())
     nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, True, out.dtype)
     ws = _workspace(nbytes, q.device, workspace)
     st = lib().path_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(beta), _ptr(log_f),
@@ -192,13 +228,21 @@ def path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale
     With the forget gate, log_f [B,H] fp32 is log f of the new position and g_cache
     [B,H,cap] fp32 the cached keys' gate biases, also updated in place
     (path_decode_step_gated)."""
+    if k_cache.dim() != 4 or k_cache.dtype not in _DT:
+        raise ValueError("k_cache must be [B,H,capacity,d], float32 or bfloat16")
     B, H, cap, d = k_cache.shape
     dt = _DT[k_cache.dtype]
     if out is None:
         out = torch.empty_like(q)
     if (log_f is None) != (g_cache is None):
         raise ValueError("log_f and g_cache go together")
-    _check_dev(q, k_new, v_new, w, beta, k_cache, v_cache, out, log_f, g_cache)
+    _expect("v_cache", v_cache, k_cache.shape, k_cache.dtype)
+    for n, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("w", w), ("out", out)):
+        _expect(n, t, (B, H, d), k_cache.dtype)
+    _expect("beta", beta, (B, H), torch.float32)
+    _expect("log_f", log_f, (B, H), torch.float32)
+    _expect("g_cache", g_cache, (B, H, cap), torch.float32)
+    _check_dev(q, k_new, v_new, w, beta, k_cache, v_cache, out, log_f, g_cache, workspace)
     nbytes = path_decode_workspace_bytes(B, H, cap, d, k_cache.dtype)
     ws = _workspace(nbytes, q.device, workspace)
     if log_f is None:
@@ -227,12 +271,19 @@ def path_attn_prefill(q, k, v, w, beta, capacity, log_f=None, scale=None, out=No
     H_{L-1} ... H_{j+1} k_j, v_cache row j = v_j); g_cache [B,H,capacity] fp32 (row j =
     c_{L-1} - c_j) with the forget gate, else None. Caches the call allocates are
     zero past row L-1."""
+    _check_attn_inputs(q, k, v, w, beta, log_f)
     B, H, L, d = q.shape
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     dt = _mode(q.dtype, out.dtype)
     if lse is None:
         lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    _expect("out", out, q.shape, out.dtype)
+    _expect("lse", lse, (B, H, L), torch.float32)
+    _expect("k_cache", k_cache, (B, H, capacity, d), q.dtype)
+    _expect("v_cache", v_cache, (B, H, capacity, d), q.dtype)
+    if log_f is not None:
+        _expect("g_cache", g_cache, (B, H, capacity), torch.float32)
     if k_cache is None:
         k_cache = torch.zeros((B, H, capacity, d), dtype=q.dtype, device=q.device)
     if v_cache is None:
@@ -241,7 +292,7 @@ def path_attn_prefill(q, k, v, w, beta, capacity, log_f=None, scale=None, out=No
         g_cache = torch.zeros((B, H, capacity), dtype=torch.float32, device=q.device)
     if log_f is None:
         g_cache = None
-    _check_dev(q, k, v, w, beta, log_f, out, lse, k_cache, v_cache, g_cache)
+    _check_dev(q, k, v, w, beta, log_f, out, lse, k_cache, v_cache, g_cache, workspace)
     nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, False, out.dtype)
     ws = _workspace(nbytes, q.device, workspace)
     st = lib().path_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(beta), _ptr(log_f),

@@ -20,6 +20,8 @@ import tempfile
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 import oracle
 
@@ -420,6 +422,67 @@ def test_decode_after_prefill_continues_the_forward(orc, fox):
                             t, scale=0.6, log_f=None if logf is None else logf[:, :, t],
                             g_cache=gc)
         np.testing.assert_allclose(o, out[:, :, t], rtol=1e-11, atol=1e-13)
+
+
+# ---------------------------------------------------------------- randomized pins
+# The fixed-seed pins above, over random shapes, beta in [0, 2], unnormalised w
+# and gate on / off (hypothesis draws the case; numpy draws the values from its seed).
+CASES = st.tuples(st.integers(1, 9), st.integers(1, 5), st.floats(0.0, 2.0),
+                  st.booleans(), st.booleans(), st.integers(0, 2 ** 31 - 1))
+
+
+@settings(max_examples=40, deadline=None)
+@given(CASES)
+def test_random_scores_equal_explicit_products(case):
+    L, d, beta_hi, unit_w, fox, seed = case
+    rng = np.random.default_rng(seed)
+    q, k, v, w, beta, logf = rand_case(rng, B=1, H=1, L=L, d=d, beta_hi=beta_hi, unit_w=unit_w,
+                                       fox=fox)
+    z = oracle.scores(q, k, w, beta, logf, scale=0.9)[0, 0]
+    ref = explicit_scores(q[0, 0], k[0, 0], w[0, 0], beta[0, 0],
+                          None if logf is None else logf[0, 0], 0.9)
+    np.testing.assert_allclose(z, ref, rtol=1e-10, atol=1e-10)
+
+
+@settings(max_examples=25, deadline=None)
+@given(CASES)
+def test_random_decode_and_prefill_agree_with_forward(case):
+    L, d, beta_hi, unit_w, fox, seed = case
+    rng = np.random.default_rng(seed)
+    q, k, v, w, beta, logf = rand_case(rng, B=1, H=2, L=L, d=d, beta_hi=beta_hi, unit_w=unit_w,
+                                       fox=fox)
+    out, _ = oracle.fwd(q, k, v, w, beta, logf, scale=0.7)
+    kc, vc, gc = np.zeros((1, 2, L, d)), np.zeros((1, 2, L, d)), np.zeros((1, 2, L))
+    for t in range(L):
+        o = oracle.decode_step(q[:, :, t], k[:, :, t], v[:, :, t], w[:, :, t], beta[:, :, t],
+                               kc, vc, t, scale=0.7,
+                               log_f=None if logf is None else logf[:, :, t],
+                               g_cache=gc if fox else None)
+        np.testing.assert_allclose(o, out[:, :, t], rtol=1e-9, atol=1e-11)
+    pk, pv, pg = oracle.prefill_cache(k, v, w, beta, logf)
+    np.testing.assert_allclose(pk, kc, rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(pv, vc)
+    if fox:
+        np.testing.assert_allclose(pg, gc, rtol=1e-12, atol=1e-13)
+
+
+@settings(max_examples=15, deadline=None)
+@given(CASES)
+def test_random_gradient_invariants(case):
+    L, d, beta_hi, unit_w, fox, seed = case
+    rng = np.random.default_rng(seed)
+    q, k, v, w, beta, logf = rand_case(rng, B=1, H=1, L=L, d=d, beta_hi=beta_hi, unit_w=unit_w,
+                                       fox=fox)
+    dout = rng.standard_normal(q.shape)
+    g = oracle.bwd(q, k, v, w, beta, dout, logf, scale=0.8)
+    # scaling q by s and k by 1/s leaves every logit unchanged: sum q.dq = sum k.dk
+    assert math.isclose(float(np.sum(q * g["dq"])), float(np.sum(k * g["dk"])),
+                        rel_tol=1e-8, abs_tol=1e-9)
+    # H depends on w only through beta w w^T: sum w.dw = 2 sum beta dbeta
+    assert math.isclose(float(np.sum(w * g["dw"])), float(2 * np.sum(beta * g["dbeta"])),
+                        rel_tol=1e-8, abs_tol=1e-9)
+    # the rows of softmax sum to one: sum over keys of dv is sum over queries of dout
+    np.testing.assert_allclose(g["dv"].sum(axis=-2), dout.sum(axis=-2), rtol=1e-9, atol=1e-10)
 
 
 # ---------------------------------------------------------------- planted mistakes

@@ -165,3 +165,29 @@ def test_prefill_rejects_bad_arguments(lib):
     assert pre(d=32) == UNSUPPORTED         # decode head dims only
     assert pre(ws=None) == WORKSPACE
     assert pre(wsb=100) == WORKSPACE
+
+
+def test_header_is_c99_and_links(lib, tmp_path):
+    """The header is a C header: a C99 translation unit that takes the address of every
+    declared entry point compiles warning-free and links against the library."""
+    import subprocess
+
+    import softmax_attention_block_b200 as P
+
+    names = declared_functions()
+    src = tmp_path / "use_header.c"
+    src.write_text(
+        '#include "path_attn.h"\n#include <stdio.h>\n'
+        "typedef void (*any_fn)(void);\n"
+        "int main(void) {\n    any_fn fns[] = {\n"
+        + "".join(f"        (any_fn)&{n},\n" for n in names)
+        + "    };\n    size_t n = sizeof fns / sizeof fns[0];\n"
+        '    printf("%zu %s\\n", n, path_status_string(PATH_OK));\n    return 0;\n}\n')
+    exe = tmp_path / "use_header"
+    libdir = os.path.dirname(P.LIB_PATH)
+    cmd = ["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+           "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+           "-L", libdir, "-l:libpath_attn.so", "-Wl,--allow-shlib-undefined",
+           f"-Wl,-rpath,{libdir}"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr

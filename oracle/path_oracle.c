@@ -362,8 +362,10 @@ double path_oracle_round_bf16(double x)
 }
 
 /*
- * One decode step of one head. K / V [capacity,d] hold n valid rows; g (NULL
- * without the gate) holds their gate biases and logf_t is log f_t.
+ * One decode step of one head (Paper-Notes "训练策略", inference paragraph;
+ * gist.science section 3 "Inferentie"). K / V [capacity,d] hold n valid rows;
+ * g (NULL without the gate) holds their gate biases c_t - c_j (Paper-Notes
+ * "PaTH-FoX 扩展" logit term) and logf_t is log f_t.
  */
 static void decode_head(const double *q_t, const double *k_new, const double *v_new,
                         const double *w_t, double beta_t, const double *logf_t, double scale,
@@ -450,7 +452,7 @@ int path_oracle_decode_step_gated(const double *q, const double *k_new,
 
 /*
  * The cache after a prefill of positions 0..L-1, by replaying the in-place
- * update position by position: before position t is appended, each key
+ * update of the inference paragraph (Paper-Notes "训练策略") position by position: before position t is appended, each key
  * already held is multiplied by H_t and each gate bias grows by log f_t.
  * k, v, w [B,H,L,d]; beta, log_f [B,H,L] (log_f may be NULL; g_cache is then
  * untouched). Writes rows 0..L-1 of k_cache, v_cache [B,H,capacity,d] and

@@ -14,7 +14,14 @@ Entry points (same names as the C ABI):
   log_f=None, g_cache=None) -> out`` (with ``log_f``: ``path_decode_step_gated``)
 - ``path_attn_prefill(q, k, v, w, beta, capacity, log_f=None, scale=None)
   -> (out, lse, k_cache, v_cache, g_cache)``
+- ``path_decode_step_gated(q, k_new, v_new, w, beta, log_f, k_cache, v_cache, g_cache,
+  n_cached, scale=None) -> out``
+- ``path_decode_step_noalloc(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=None)
+  -> out``
+- ``path_attn_wait_status(workspace) -> int`` (0 = no bounded wait gave up)
 - ``path_attn_workspace_bytes``, ``path_decode_workspace_bytes``, ``path_status_string``
+- diagnostics: ``path_kernel_launch_count()``, ``path_profile_enable(on)``,
+  ``path_profile_read() -> {stage: (total_ms, count)}``
 """
 from __future__ import annotations
 
@@ -40,6 +47,12 @@ def _mode(in_dtype, out_dtype):
         return PATH_BF16_F32OUT
     raise ValueError(f"unsupported dtypes: inputs {in_dtype}, outputs {out_dtype}")
 _lib = None
+
+
+class _StageTime(ctypes.Structure):
+    """path_stage_time of the C header."""
+    _fields_ = [("name", ctypes.c_char * 32), ("total_ms", ctypes.c_double),
+                ("count", ctypes.c_int)]
 
 
 class PathError(RuntimeError):
@@ -73,10 +86,17 @@ def lib() -> ctypes.CDLL:
                                              vp, fp, vp, vp, sz, vp]
         L.path_attn_prefill.argtypes = [vp, vp, vp, vp, fp, fp, f, i, i, i, i, i, vp, fp, vp, vp,
                                         fp, i, vp, sz, vp]
+        L.path_decode_step_noalloc.argtypes = [vp, vp, vp, vp, fp, f, i, i, i, i, i, i, vp, vp,
+                                               vp, vp]
         L.path_attn_wait_status.argtypes = [vp, vp]
         L.path_kernel_launch_count.restype = ctypes.c_ulonglong
+        L.path_profile_enable.argtypes = [i]
+        L.path_profile_enable.restype = i
+        L.path_profile_read.argtypes = [ctypes.POINTER(_StageTime), i]
+        L.path_profile_read.restype = i
         for fn in (L.path_attn_fwd, L.path_attn_bwd, L.path_decode_step,
-                   L.path_decode_step_gated, L.path_attn_prefill, L.path_attn_wait_status):
+                   L.path_decode_step_gated, L.path_decode_step_noalloc, L.path_attn_prefill,
+                   L.path_attn_wait_status):
             fn.restype = i
         _lib = L
     return _lib
@@ -221,19 +241,10 @@ def path_attn_bwd(q, k, v, w, beta, out, lse, dout, log_f=None, scale=None, grad
     return grads
 
 
-def path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=None, out=None,
-                     workspace=None, log_f=None, g_cache=None):
-    """One decode step; updates k_cache / v_cache ([B,H,cap,d]) in place. Returns out [B,H,d].
-
-    With the forget gate, log_f [B,H] fp32 is log f of the new position and g_cache
-    [B,H,cap] fp32 the cached keys' gate biases, also updated in place
-    (path_decode_step_gated)."""
+def _check_decode(q, k_new, v_new, w, beta, k_cache, v_cache, out, log_f, g_cache):
     if k_cache.dim() != 4 or k_cache.dtype not in _DT:
         raise ValueError("k_cache must be [B,H,capacity,d], float32 or bfloat16")
     B, H, cap, d = k_cache.shape
-    dt = _DT[k_cache.dtype]
-    if out is None:
-        out = torch.empty_like(q)
     if (log_f is None) != (g_cache is None):
         raise ValueError("log_f and g_cache go together")
     _expect("v_cache", v_cache, k_cache.shape, k_cache.dtype)
@@ -242,6 +253,20 @@ def path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale
     _expect("beta", beta, (B, H), torch.float32)
     _expect("log_f", log_f, (B, H), torch.float32)
     _expect("g_cache", g_cache, (B, H, cap), torch.float32)
+    return B, H, cap, d
+
+
+def path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=None, out=None,
+                     workspace=None, log_f=None, g_cache=None):
+    """One decode step; updates k_cache / v_cache ([B,H,cap,d]) in place. Returns out [B,H,d].
+
+    With the forget gate, log_f [B,H] fp32 is log f of the new position and g_cache
+    [B,H,cap] fp32 the cached keys' gate biases, also updated in place
+    (path_decode_step_gated)."""
+    if out is None:
+        out = torch.empty_like(q)
+    B, H, cap, d = _check_decode(q, k_new, v_new, w, beta, k_cache, v_cache, out, log_f, g_cache)
+    dt = _DT[k_cache.dtype]
     _check_dev(q, k_new, v_new, w, beta, k_cache, v_cache, out, log_f, g_cache, workspace)
     nbytes = path_decode_workspace_bytes(B, H, cap, d, k_cache.dtype)
     ws = _workspace(nbytes, q.device, workspace)
@@ -260,6 +285,57 @@ def path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale
     if st:
         raise PathError(st, where)
     return out
+
+
+def path_decode_step_gated(q, k_new, v_new, w, beta, log_f, k_cache, v_cache, g_cache, n_cached,
+                           scale=None, out=None, workspace=None):
+    """PaTH-FoX decode step: path_decode_step with the forget gate (log_f [B,H] fp32 of the
+    new position; g_cache [B,H,cap] fp32, the cached keys' gate biases, updated in place)."""
+    if log_f is None or g_cache is None:
+        raise ValueError("path_decode_step_gated needs log_f and g_cache")
+    return path_decode_step(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=scale,
+                            out=out, workspace=workspace, log_f=log_f, g_cache=g_cache)
+
+
+def path_decode_step_noalloc(q, k_new, v_new, w, beta, k_cache, v_cache, n_cached, scale=None,
+                             out=None):
+    """path_decode_step without a workspace (the library's fixed 4 MiB device scratch; see
+    the C header for its limit and its sharing between calls on one device)."""
+    if out is None:
+        out = torch.empty_like(q)
+    B, H, cap, d = _check_decode(q, k_new, v_new, w, beta, k_cache, v_cache, out, None, None)
+    _check_dev(q, k_new, v_new, w, beta, k_cache, v_cache, out)
+    st = lib().path_decode_step_noalloc(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(w), _ptr(beta),
+                                        _scale(scale, d), B, H, d, int(n_cached), cap,
+                                        _DT[k_cache.dtype], _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(out), _stream())
+    if st:
+        raise PathError(st, "path_decode_step_noalloc")
+    return out
+
+
+def path_attn_wait_status(workspace) -> int:
+    """Waits for the current stream, then returns 0, or PATH_ERR_TIMEOUT (5) if the last
+    path_attn_fwd / path_attn_bwd that used `workspace` had a bounded wait give up."""
+    _check_dev(workspace)
+    return int(lib().path_attn_wait_status(_ptr(workspace), _stream()))
+
+
+def path_kernel_launch_count() -> int:
+    """Kernels this library has launched in this process so far."""
+    return int(lib().path_kernel_launch_count())
+
+
+def path_profile_enable(on: bool) -> bool:
+    """Per-stage event timing on or off; returns the previous setting."""
+    return bool(lib().path_profile_enable(int(bool(on))))
+
+
+def path_profile_read(max_entries: int = 64) -> dict:
+    """Stage name -> (total ms, launches) of the stages timed since the last read."""
+    buf = (_StageTime * max_entries)()
+    n = lib().path_profile_read(buf, max_entries)
+    return {buf[i].name.decode(): (buf[i].total_ms, buf[i].count) for i in range(n)}
 
 
 def path_attn_prefill(q, k, v, w, beta, capacity, log_f=None, scale=None, out=None, lse=None,

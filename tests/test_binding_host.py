@@ -104,3 +104,27 @@ def test_prefill_checks_caches():
         P.path_attn_prefill(*args, g_cache=torch.zeros(B, H, 65))
     with pytest.raises(ValueError, match="CUDA tensors"):
         P.path_attn_prefill(*args)
+
+
+def test_wrappers_of_the_remaining_entry_points():
+    cap = 50
+    kc = torch.zeros(B, H, cap, D, dtype=torch.bfloat16)
+    vc = torch.zeros_like(kc)
+    s = [torch.zeros(B, H, D, dtype=torch.bfloat16) for _ in range(4)]
+    beta = torch.zeros(B, H)
+    with pytest.raises(ValueError, match="needs log_f and g_cache"):
+        P.path_decode_step_gated(*s, beta, None, kc, vc, None, 10)
+    with pytest.raises(ValueError, match="g_cache: dtype"):
+        P.path_decode_step_gated(*s, beta, torch.zeros(B, H), kc, vc,
+                                 torch.zeros(B, H, cap, dtype=torch.float64), 10)
+    with pytest.raises(ValueError, match="w: shape"):
+        P.path_decode_step_noalloc(*s[:3], torch.zeros(B, H, 2 * D, dtype=torch.bfloat16), beta,
+                                   kc, vc, 10)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        P.path_decode_step_noalloc(*s, beta, kc, vc, 10)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        P.path_attn_wait_status(torch.zeros(64, dtype=torch.uint8))
+    assert P.path_kernel_launch_count() >= 0
+    prev = P.path_profile_enable(True)
+    assert P.path_profile_enable(prev) is True
+    assert P.path_profile_read() == {}

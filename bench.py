@@ -24,7 +24,6 @@ tokens/s = B * L / step time, and the FlashAttention-equivalent 7 L^2 d count.
 from __future__ import annotations
 
 import argparse
-import ctypes
 import json
 import os
 import statistics
@@ -183,23 +182,10 @@ class ClockSampler:
                 "samples": len(rows), "samples_under_load": len(busy)}
 
 
-def lib_call(name, *args):
-    import softmax_attention_block_b200 as P
-    return getattr(P.lib(), name)(*args)
-
-
-class StageTime(ctypes.Structure):
-    _fields_ = [("name", ctypes.c_char * 32), ("total_ms", ctypes.c_double),
-                ("count", ctypes.c_int)]
-
-
 def read_profile():
+    """Stage name -> (total ms, launches) timed since the last read."""
     import softmax_attention_block_b200 as P
-    L = P.lib()
-    L.path_profile_read.argtypes = [ctypes.POINTER(StageTime), ctypes.c_int]
-    buf = (StageTime * 64)()
-    n = L.path_profile_read(buf, 64)
-    return {buf[i].name.decode(): (buf[i].total_ms, buf[i].count) for i in range(n)}
+    return P.path_profile_read(64)
 
 
 # ---------------------------------------------------------------- reference arm

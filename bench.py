@@ -8,7 +8,9 @@ H=24 L=4096 d=64 bf16, inputs resident in HBM. The decode step (B=32 H=32 d=128,
 64 steps) is timed after it and reported under "decode" (with the forget gate's per-key
 bias under "decode.gated"), and a prefill of the same sequences (forward plus the decode
 cache it leaves) under "prefill", and fwd+bwd at head dim 128 (B=8 H=12, the same model
-width) under "d128".
+width) under "d128". The other timed workloads: the forward latency at B=2 H=4 L=1024
+("fwd_latency"), PaTH-FoX fwd+bwd at B=1 H=24 L=16384 ("fox"), and the headline step with
+fp32 outputs and gradients ("f32out").
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -430,8 +432,17 @@ def run_ours(args):
 
     prefill = None if args.no_prefill else bench_prefill(P, x, w, ws, peaks, world,
                                                            max_over_ranks, barrier, args.steps)
-    del x, out, lse, grads, ws
+    del out, lse, grads, ws
     torch.cuda.empty_cache()
+    f32out = None if args.no_f32out else bench_f32out(P, x, w, world, max_over_ranks, barrier,
+                                                      args.steps)
+    del x
+    torch.cuda.empty_cache()
+    fwd_latency = None if args.no_fwd_latency else bench_fwd_latency(P, dev, peaks, world,
+                                                                     max_over_ranks, barrier)
+    fox = None if args.no_fox else bench_fox(
+        P, dev, peaks, world, max_over_ranks, barrier, 3,
+        cpu_sample=(rank == 0 and world == 1 and not args.no_cpu_baseline))
     decode = None if args.no_decode else bench_decode(P, dev, peaks, world, max_over_ranks,
                                                        barrier)
     d128 = None if args.no_d128 else bench_d128(P, dev, peaks, world, max_over_ranks, barrier,
@@ -456,7 +467,7 @@ def run_ours(args):
             "pct_bf16_peak": value / world / peaks["bf16_tflops_sustained"],
             "stages": stage_rows, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk, "decode": decode, "prefill": prefill,
-            "d128": d128}
+            "d128": d128, "f32out": f32out, "fwd_latency": fwd_latency, "fox": fox}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -510,6 +521,173 @@ def bench_prefill(P, x, w, ws, peaks, world, max_over_ranks, barrier, steps):
                          "frac": ach / peaks["hbm_gbs"] if ach else None, "traffic": traffic,
                          "traffic_unit": "bytes per launch", "algorithmic_bytes": bytes_launch,
                          "peak_source": f"{peaks['source']} HBM copy"}}
+
+
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2: written between timed calls of small workloads
+
+
+def timed_calls(call, n, flush, stream):
+    """Device time of n calls, each preceded by an untimed write of `flush` (evicts L2):
+    per-call CUDA events on the launching stream; returns ms per call."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / n
+
+
+def stage_roofline(stages, B, H, L, d, peaks):
+    """Dominant stage of a timed region -> roofline object against the sustained bf16 peak."""
+    if not stages:
+        return None
+    dom = max(stages, key=lambda n: stages[n][0])
+    per_launch_ms = stages[dom][0] / stages[dom][1]
+    f, bound = stage_model(dom, B, H, L, d)
+    ach = f / (per_launch_ms * 1e-3) / 1e12 if f else None
+    peak = peaks["bf16_tflops_sustained"]
+    return {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+            "frac": (ach / peak) if ach else None, "traffic": None,
+            "peak_source": f"{peaks['source']} bf16 dense (sustained)"}
+
+
+FWD_LATENCY = "fwd_bf16_l1024"
+FOX = "fox_fwdbwd_l16384"
+
+
+def bench_fwd_latency(P, dev, peaks, world, max_over_ranks, barrier, calls=20):
+    """Forward latency of the B=2 H=4 L=1024 bf16 workload (out + lse): one call is
+    launch-bound, so each timed call follows an L2 flush and is timed on its own."""
+    w = si.WORKLOADS[FWD_LATENCY]
+    xc = si.workload_inputs(FWD_LATENCY, seed=0)
+    x = {k: (v.to(dev) if v is not None else None) for k, v in xc.items()}
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    ws = torch.empty(P.path_attn_workspace_bytes(w.B, w.H, w.L, w.d, w.dtype, False),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def call():
+        P.path_attn_fwd(x["q"], x["k"], x["v"], x["w"], x["beta"], None, out=out, lse=lse,
+                        workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    barrier()
+    stream = torch.cuda.current_stream()
+    P.lib().path_profile_enable(1)
+    ms = max_over_ranks(timed_calls(call, calls, flush, stream))
+    P.lib().path_profile_enable(0)
+    stages = read_profile()
+    fl = 3.0 * w.L * w.L * w.d * w.B * w.H
+    del x, out, lse, ws, flush
+    return {"workload": f"{FWD_LATENCY}: bf16 forward B={w.B} H={w.H} L={w.L} d={w.d}, out + lse",
+            "ms_per_call": ms, "value": whole_job_rate(world, fl, ms) / 1e12, "unit": UNIT,
+            "flop_convention": "3 L^2 d per head (QK^T, PV, block transport)",
+            "l2": "flushed (256 MB written) before every timed call",
+            "stages_ms": {n: t / c for n, (t, c) in stages.items()}}
+
+
+def bench_fox(P, dev, peaks, world, max_over_ranks, barrier, steps, cpu_sample):
+    """PaTH-FoX fwd+bwd at B=1 H=24 L=16384 (the long-context workload): TFLOP/s by
+    11 L^2 d per head, tokens/s, the dominant stage's roofline, and the oracle on a
+    bounded sample (the first 4096 positions of one head)."""
+    w = si.WORKLOADS[FOX]
+    xc = si.workload_inputs(FOX, seed=0)
+    x = {k: (v.to(dev) if v is not None else None) for k, v in xc.items()}
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    grads = {n: torch.empty_like(x["q"]) for n in ("dq", "dk", "dv", "dw")}
+    grads["dbeta"] = torch.empty_like(x["beta"])
+    grads["dlog_f"] = torch.empty_like(x["log_f"])
+    ws = torch.empty(P.path_attn_workspace_bytes(w.B, w.H, w.L, w.d, w.dtype, True),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        P.path_attn_fwd(x["q"], x["k"], x["v"], x["w"], x["beta"], x["log_f"], out=out, lse=lse,
+                        workspace=ws)
+        P.path_attn_bwd(x["q"], x["k"], x["v"], x["w"], x["beta"], out, lse, x["dout"],
+                        x["log_f"], grads=grads, workspace=ws, reuse_fwd_workspace=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    stream = torch.cuda.current_stream()
+    P.lib().path_profile_enable(1)
+    ms = max_over_ranks(timed_calls(step, steps, flush, stream))
+    P.lib().path_profile_enable(0)
+    stages = read_profile()
+    fl = algorithmic_flops(w.B, w.H, w.L, w.d)
+    del x, out, lse, grads, ws, flush
+    torch.cuda.empty_cache()
+    res = {"workload": f"{FOX}: bf16 PaTH-FoX fwd+bwd B={w.B} H={w.H} L={w.L} d={w.d}",
+           "ms_per_step": ms, "value": whole_job_rate(world, fl, ms) / 1e12, "unit": UNIT,
+           "tokens_per_s": whole_job_rate(world, w.B * w.L, ms),
+           "pct_bf16_peak": fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+           "l2": "flushed (256 MB written) before every timed step",
+           "stages": {n: {"ms_per_launch": t / c, "launches": c} for n, (t, c) in stages.items()},
+           "roofline": stage_roofline(stages, w.B, w.H, w.L, w.d, peaks)}
+    if cpu_sample:
+        import oracle
+
+        xs = si.workload_inputs(FOX, heads=[0])
+        Ls = 4096
+        xs = {k: (v[:, :, :Ls].contiguous() if v is not None else None) for k, v in xs.items()}
+        t0 = time.perf_counter()
+        orc = oracle.default()
+        orc.fwd(xs["q"], xs["k"], xs["v"], xs["w"], xs["beta"], xs["log_f"])
+        orc.bwd(xs["q"], xs["k"], xs["v"], xs["w"], xs["beta"], xs["dout"], xs["log_f"])
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {
+            "value": algorithmic_flops(1, 1, Ls, w.d) / dt / 1e12, "unit": UNIT,
+            "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)), "kind": "oracle",
+            "sample": f"positions 0..{Ls - 1} of head 0 of {FOX} (a causal prefix), fwd+bwd in "
+                      f"fp64 ({dt:.1f} s); TFLOP/s on that prefix's 11*L^2*d FLOP"}
+    return res
+
+
+def bench_f32out(P, x, w, world, max_over_ranks, barrier, steps):
+    """The headline step with fp32 out, dout and gradients (PATH_BF16_F32OUT): the mode
+    whose outputs meet max-abs 2e-2 without the bf16 storage allowance."""
+    dev = x["q"].device
+    out = torch.empty(x["q"].shape, dtype=torch.float32, device=dev)
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    dout = x["dout"].float()
+    grads = {n: torch.empty(x["q"].shape, dtype=torch.float32, device=dev)
+             for n in ("dq", "dk", "dv", "dw")}
+    grads["dbeta"] = torch.empty_like(x["beta"])
+    ws = torch.empty(P.path_attn_workspace_bytes(w.B, w.H, w.L, w.d, w.dtype, True,
+                                                 torch.float32), dtype=torch.uint8, device=dev)
+
+    def step():
+        P.path_attn_fwd(x["q"], x["k"], x["v"], x["w"], x["beta"], None, out=out, lse=lse,
+                        workspace=ws)
+        P.path_attn_bwd(x["q"], x["k"], x["v"], x["w"], x["beta"], out, lse, dout, None,
+                        grads=grads, workspace=ws, reuse_fwd_workspace=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / steps
+    fl = algorithmic_flops(w.B, w.H, w.L, w.d)
+    del out, lse, dout, grads, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"{WORKLOAD} with fp32 out, dout and gradients (PATH_BF16_F32OUT)",
+            "ms_per_step": ms, "value": whole_job_rate(world, fl, ms) / 1e12, "unit": UNIT}
 
 
 D128 = (8, 12, 4096, 128)  # B, H, L, d: the headline model width (24 x 64) as 12 x 128
@@ -712,6 +890,9 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-d128", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-f32out", action="store_true")
+    ap.add_argument("--no-fwd-latency", action="store_true")
+    ap.add_argument("--no-fox", action="store_true")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES) + sorted(DECODE_PROFILE_CASES)
                     + sorted(PREFILL_PROFILE_CASES),
                     help="run one untimed fwd+bwd on a small shape (for profiler captures)")

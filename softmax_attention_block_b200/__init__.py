@@ -130,6 +130,9 @@ def _expect(name, t, shape, dtype):
 
 
 def _check_dev(*ts):
+    """All tensors contiguous, on one CUDA device, and that device the current one: the
+    library launches on the current device's stream and resolves its own per-device
+    state (the allocation-free decode's scratch array) through the current device."""
     ts = [t for t in ts if t is not None]
     for t in ts:
         if not t.is_cuda:
@@ -138,6 +141,10 @@ def _check_dev(*ts):
             raise ValueError("all tensors must be contiguous")
         if t.device != ts[0].device:
             raise ValueError("all tensors must be on one device")
+    if ts and ts[0].device.index != torch.cuda.current_device():
+        raise ValueError(f"tensors are on {ts[0].device} but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()}: call under "
+                         f"torch.cuda.device({ts[0].device})")
 
 
 def _check_attn_inputs(q, k, v, w, beta, log_f):

@@ -59,8 +59,12 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
     w.Vh = c.take<char>(nh * (size_t)y.L * d * 2);
     w.Sd = c.take<float>(nh * nb * BT * BT);
     PrepDims D{y.nh, y.L, y.d, y.nblk, types_of(dt).in, types_of(dt).out};
-    carve_prep_scratch(c, D, bwd, w.prep);
+    // the buffers above are the forward's, at the same offsets in a forward- and a
+    // backward-sized workspace (a backward may reuse the forward's); the rest only
+    // the backward path that reads it gets
+    const bool split_tf32 = y.d == 64 && D.dt == F32;  // fp32, head dim 64: split-TF32 UT kernels
     if (bwd) {
+        if (y.d != 64) carve_prep_scratch(c, D, true, w.prep);
         w.delta = c.take<float>(nh * Lp);
         w.dQt = c.take<float>(nh * Lp * d);
         w.dKt = c.take<float>(nh * Lp * d);
@@ -69,9 +73,11 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
         w.rowsum = c.take<float>(nh * Lp);
         w.colsum = c.take<float>(nh * Lp);
         w.lse_p = c.take<float>(nh * Lp);
-        w.dP64 = c.take<float>(nh * 2 * nb * d * d);
-        w.halves = c.take<float>(prep_forward_tc_supported(D) ? nh * nb * 4 * 64 * 64 : 0);
+        w.dP64 = split_tf32 ? c.take<float>(nh * 2 * nb * d * d) : nullptr;
+        w.halves = split_tf32 ? c.take<float>(nh * nb * 4 * 64 * 64) : nullptr;
         w.dout16 = c.take<char>(nh * (size_t)y.L * d * 2);
+    } else {
+        w.dP64 = w.halves = nullptr;
     }
     return c.bytes();
 }
@@ -84,6 +90,16 @@ bool fwd_dims_ok(int B, int H, int L, int d)
 }
 
 bool head_dim_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+// bf16 inputs at head dim 64 go through the tcgen05 UT kernels, which load q, k
+// and w by TMA: their base addresses must be 16-byte aligned.
+bool tma_inputs_ok(int d, path_dtype dt, const void *q, const void *k, const void *w)
+{
+    if (d != 64 || types_of(dt).in != BF16) return true;
+    const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                         reinterpret_cast<uintptr_t>(w);
+    return (al & 15u) == 0;
+}
 
 // Heads and 128-row blocks index launch grid dimensions limited to 65535.
 bool grid_ok(int B, int H, int L)
@@ -136,7 +152,9 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
     PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, t.mid, ws.halves};
     {
         Stage s("ut_prep", st);
-        if (prep_forward_tc_supported(D))
+        if (prep_forward_ut_supported(D, in))
+            TRY(prep_forward_ut(D, in, out, ws.err, st));  // no 64-half buffers: its adjoint recomputes
+        else if (prep_forward_tc_supported(D))
             TRY(prep_forward_tc(D, in, out, st));
         else
             TRY(prep_forward_rec(D, in, out, st));
@@ -216,6 +234,7 @@ path_status path_attn_fwd(const void *q, const void *k, const void *v, const voi
     if (!q || !k || !v || !w || !beta || !out || !lse) return PATH_ERR_INVALID_ARG;
     if (!fwd_dims_ok(B, H, L, d) || !isfinite(scale)) return PATH_ERR_INVALID_ARG;
     if (!head_dim_supported(d) || !dtype_ok(dt) || !grid_ok(B, H, L)) return PATH_ERR_UNSUPPORTED;
+    if (!tma_inputs_ok(d, dt, q, k, w)) return PATH_ERR_INVALID_ARG;
     AttnWs ws;
     return run_forward(q, k, v, w, beta, log_f, scale, make_layout(B, H, L, d, dt), dt, out, lse,
                        workspace, workspace_bytes, ws, reinterpret_cast<cudaStream_t>(stream));
@@ -236,6 +255,7 @@ path_status path_attn_prefill(const void *q, const void *k, const void *v, const
     const uintptr_t al = reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(k_cache) |
                          reinterpret_cast<uintptr_t>(v_cache);
     if (al & 15u) return PATH_ERR_INVALID_ARG;
+    if (!tma_inputs_ok(d, dt, q, k, w)) return PATH_ERR_INVALID_ARG;
     const Layout y = make_layout(B, H, L, d, dt);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     AttnWs ws;
@@ -261,6 +281,7 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
     if ((log_f == nullptr) != (dlog_f == nullptr)) return PATH_ERR_INVALID_ARG;
     if (!fwd_dims_ok(B, H, L, d) || !isfinite(scale)) return PATH_ERR_INVALID_ARG;
     if (!head_dim_supported(d) || !dtype_ok(dt) || !grid_ok(B, H, L)) return PATH_ERR_UNSUPPORTED;
+    if (!tma_inputs_ok(d, dt, q, k, w)) return PATH_ERR_INVALID_ARG;
     const Layout y = make_layout(B, H, L, d, dt);
     AttnWs ws;
     const size_t need = carve_attn(nullptr, y, dt, true, ws);
@@ -297,7 +318,10 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
     PrepDims D{y.nh, y.L, y.d, y.nblk, types_of(dt).in, types_of(dt).out};
     PrepInputs in{q, k, w, beta};
     PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta, ws.halves};
-    if (prep_backward_fused_supported(D)) {
+    if (prep_backward_ut_supported(D, in)) {
+        Stage s("ut_adj", st);
+        TRY(prep_backward_ut(D, in, gr, ws.err, st));
+    } else if (prep_backward_fused_supported(D)) {
         TRY(prep_backward_fused(D, in, gr, ws.dP64, st));  // times its two kernels itself
     } else {
         Stage s("ut_prep_bwd", st);

@@ -52,6 +52,17 @@ cudaError_t prep_forward_rec(const PrepDims &D, const PrepInputs &in, const Prep
 bool prep_forward_tc_supported(const PrepDims &D);
 cudaError_t prep_forward_tc(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
                             cudaStream_t st);
+// The same outputs for head dim 64 and bf16 inputs on tcgen05 (tensor memory),
+// with (I + A)^{-1} as a product of block-diagonal and nilpotent factors
+// (prep_fwd_ut.cu). q, k, w 16-byte aligned. err: device error word.
+bool prep_forward_ut_supported(const PrepDims &D, const PrepInputs &in);
+cudaError_t prep_forward_ut(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
+                            int *err, cudaStream_t st);
+// Adjoint of prep_forward_ut (one tcgen05 kernel per block: recomputes the halves'
+// transforms, composition adjoint, per-half UT adjoint). dQt and dKt are overwritten.
+bool prep_backward_ut_supported(const PrepDims &D, const PrepInputs &in);
+cudaError_t prep_backward_ut(const PrepDims &D, const PrepInputs &in, const PrepGrads &g, int *err,
+                             cudaStream_t st);
 cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
                           const PrepGrads &gr, cudaStream_t st);
 // Fused adjoint for head dim 64 (two 64-position halves per block). dQt and

@@ -1,0 +1,340 @@
+// Forward UT prep of one 128-position block on 5th-generation tensor cores
+// (tcgen05, accumulators in tensor memory), head dim 64, bf16 inputs.
+//
+// Per 64-position half (positions s..e, H_t = I - beta_t w_t w_t^T), the UT
+// transform in closed form (Paper-Notes "训练策略": T^{-1} = (I + strictLower(D W W^T))^{-1} D,
+// and the full-matrix form of the block's logits):
+//   A = strictLower(D W W^T), N = strictLower(W K^T), M = lower(Q W^T),
+//   [What | U] = (I + A)^{-1} D [W | N]
+//   Qtil = Q - M What, Ktil = K - U^T W, P = I - W^T What, Sd = lower(Q K^T - M U)
+// and the 128-block from its halves a (first) and b:
+//   Qtil[a] = Qtil_a, Qtil[b] = Qtil_b P_a, Ktil[a] = Ktil_a P_b^T, Ktil[b] = Ktil_b,
+//   P = P_b P_a, Sd = [[Sd_aa, 0], [Qtil_b Ktil_a^T, Sd_bb]].
+//
+// The inverse (I + A)^{-1} is not reached by substitution. With E the block
+// diagonal of I + A in 16 x 16 blocks (inverted on the CUDA cores) and
+// N' = E^{-1} A_off (A_off: A outside those blocks), N' is strictly lower in
+// 16-row blocks, so N'^4 = 0 and
+//   (I + A)^{-1} = (I + N')^{-1} E^{-1} = (I + N'^2)(I - N') E^{-1}.
+// Applied to D [W | N] that is three dependent products:
+//   Z = E^{-1} D [W | N],  Z1 = Z - N' Z (with N'^2 = N' N'),  [What | U] = Z1 + N'^2 Z1.
+// Every product is an M = 64 MMA on fp16 operands with fp32 accumulation (the
+// bf16 inputs are exact in fp16); both halves run side by side (ut_tc.cuh).
+#include "prep.cuh"
+#include "runtime.cuh"
+#include "ut_tc.cuh"
+
+namespace path {
+
+namespace {
+
+using namespace tc;
+using namespace uttc;
+
+constexpr int NT = 256;
+
+// shared-memory tiles (8 KB each)
+enum {
+    T_WA = 0, T_KA = 1, T_WB = 2, T_KB = 3,  // W_h, K_h adjacent: [W_h; K_h] is one 128-row B
+    T_QA = 4, T_QB = 5,
+    T_DA = 6, T_DB = 7,    // E^{-1}, then N'^2
+    T_F1 = 8,              // per half (b at +3): A_off, D W, D N (B of the first product)
+    T_MA = 14, T_MB = 15,  // -M
+    T_NA = 16, T_NB = 17,  // -N'
+    T_Z = 18,              // per half (b at +2): [Zw, Zn] = Z, then Z1, then [What, U]
+    NTILES = 22,
+    // composition operands (over the T_F1 tiles, free by then)
+    T_KTA = 8, T_QTB = 9, T_PA = 10, T_PB = 11,
+};
+constexpr int SA16_OFF = NTILES * TILE;              // [2][4][16][16] fp32 diagonal blocks of A
+constexpr int BETA_OFF = SA16_OFF + 2 * 4 * 256 * 4;  // [128] beta
+constexpr int BAR_OFF = BETA_OFF + 128 * 4;
+constexpr int SMEM = BAR_OFF + 64 + 1024;             // + 1024-byte alignment slack
+
+// tensor-memory columns
+constexpr int C_G = 0, C_N = 64, C_M = 128, C_S = 192;  // W W^T, W K^T, Q W^T, Q K^T (then Sd)
+constexpr int C_Z = 256;                               // N' | Zw | Zn (then Z1, [What | U])
+constexpr int C_N2 = 0;                                // N'^2
+constexpr int C_QT = 64, C_KT = 128, C_P = 0;          // -M What, U^T W, W^T What
+constexpr int C_C1 = 256, C_C2 = 320;                  // composition
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p)
+{
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__global__ void __launch_bounds__(NT, 1)
+    prep_fwd_ut_kernel(const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mQ,
+                       const __grid_constant__ CUtensorMap mK, const float *beta, int L, int nblk,
+                       f16 *Qt, f16 *Kt, f16 *Pm, float *Sd, float *halves, int *err)
+{
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = align1024(smraw);
+    auto tile = [&](int i) { return sm + i * TILE; };
+    const uint32_t s0 = smem_u32(sm);
+    auto ta = [&](int i) { return s0 + (uint32_t)i * TILE; };
+    float *sA16 = reinterpret_cast<float *>(sm + SA16_OFF);
+    float *sB = reinterpret_cast<float *>(sm + BETA_OFF);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + BAR_OFF);  // [0] loads, [1] MMA
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 2);
+    const int J = blockIdx.x, hd = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int Lp = nblk * BT;
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(tslot, 512);
+    // the E^{-1} tiles: only their diagonal blocks are written below
+    for (int i = tid; i < 2 * (int)TILE / 16; i += NT)
+        reinterpret_cast<uint4 *>(tile(T_DA))[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (tid < BT) {
+        const int p = J * BT + tid;
+        sB[tid] = p < L ? beta[(long long)hd * L + p] : 0.f;
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tslot;
+    if (tid == 0) {
+        // rows past L read as zero (w = 0, beta = 0: H = I there)
+        mbar_expect_tx(&bars[0], 6 * TILE);
+        for (int h = 0; h < 2; ++h) {
+            const int y = J * BT + h * HB;
+            tma_load_3d(tile(h ? T_WB : T_WA), &mW, 0, y, hd, &bars[0]);
+            tma_load_3d(tile(h ? T_KB : T_KA), &mK, 0, y, hd, &bars[0]);
+            tma_load_3d(tile(h ? T_QB : T_QA), &mQ, 0, y, hd, &bars[0]);
+        }
+    }
+    bool ok = mbar_wait(&bars[0], 0, WAIT_POLLS);
+    ok = __syncthreads_and(ok);
+
+    const Me me;
+    const int h = me.h, r = me.r, c0 = 32 * me.cg;
+    const float br = sB[h * HB + r];
+    uint32_t phase = 0;
+    // one level: operands written and fenced, barrier; one thread issues the
+    // products and commits; everyone waits for them
+    auto sync_operands = [&]() {
+        fence_async_smem();
+        fence_before_sync();
+        ok = __syncthreads_and(ok);
+    };
+    auto wait_mma = [&]() {
+        if (ok && !mbar_wait(&bars[1], phase, WAIT_POLLS)) ok = false;
+        phase ^= 1;
+        fence_after_sync();
+    };
+#define ISSUE(...)                                \
+    do {                                          \
+        if (ok && warp == 0) {                    \
+            fence_after_sync();                   \
+            if (lane == 0) {                      \
+                __VA_ARGS__;                      \
+                commit(&bars[1]);                 \
+            }                                     \
+            __syncwarp();                         \
+        }                                         \
+    } while (0)
+
+    float v[32], x[32];
+
+    // ---- level 0: [W; Q] [W; K]^T per half (bf16 operands)
+    ISSUE(for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t wk = ta(hh ? T_WB : T_WA);
+        mma64(dst(tbase, hh, C_G), wk, A_N, wk, B_T, 2, TILE, false, AB_BF16);
+        mma64(dst(tbase, hh, C_M), ta(hh ? T_QB : T_QA), A_N, wk, B_T, 2, TILE, false, AB_BF16);
+    });
+    wait_mma();
+    if (ok) {
+        // A = strictLower(D W W^T): diagonal 16-blocks to sA16 (fp32), the rest to A_off
+        me.ld(tbase, C_G, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int col = c0 + j;
+            const float a = col < r ? br * v[j] : 0.f;
+            if ((col >> 4) == (r >> 4)) {
+                sA16[((h * 4 + (r >> 4)) * 16 + (r & 15)) * 16 + (col & 15)] = a;
+                x[j] = 0.f;
+            } else {
+                x[j] = a;
+            }
+        }
+        st_tile_f16(tile(T_F1 + 3 * h), r, c0, x);
+        me.ld(tbase, C_N, v);  // D N, N = strictLower(W K^T)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = c0 + j < r ? br * v[j] : 0.f;
+        st_tile_f16(tile(T_F1 + 3 * h + 2), r, c0, v);
+        me.ld(tbase, C_M, v);  // -M, M = lower(Q W^T)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = c0 + j <= r ? -v[j] : 0.f;
+        st_tile_f16(tile(h ? T_MB : T_MA), r, c0, v);
+        // W to fp16 in place (an operand beside fp16 intermediates from here on), and D W
+        uint8_t *tw = tile(h ? T_WB : T_WA);
+        ld_tile_bf16(tw, r, c0, v);
+        st_tile_f16(tw, r, c0, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= br;
+        st_tile_f16(tile(T_F1 + 3 * h + 1), r, c0, v);
+    }
+    sync_operands();
+    if (ok) {
+        uint8_t *const dinv[2] = {tile(T_DA), tile(T_DB)};
+        diag_block_inverses(sA16, dinv);
+    }
+    sync_operands();
+
+    // ---- level 1: [N' | Zw | Zn] = E^{-1} [A_off | D W | D N]
+    ISSUE(for (int hh = 0; hh < 2; ++hh)
+              mma64(dst(tbase, hh, C_Z), ta(T_DA + hh), A_N, ta(T_F1 + 3 * hh), B_N, 3, TILE, false));
+    wait_mma();
+    if (ok) {
+        me.ld(tbase, C_Z, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = -v[j];
+        st_tile_f16(tile(T_NA + h), r, c0, v);
+        me.ld(tbase, C_Z + 64, v);
+        st_tile_f16(tile(T_Z + 2 * h), r, c0, v);
+        me.ld(tbase, C_Z + 128, v);
+        st_tile_f16(tile(T_Z + 2 * h + 1), r, c0, v);
+    }
+    sync_operands();
+
+    // ---- level 2: Z1 = Z + (-N') Z (in place in tensor memory), N'^2 = (-N')(-N')
+    ISSUE(for (int hh = 0; hh < 2; ++hh) {
+        mma64(dst(tbase, hh, C_Z + 64), ta(T_NA + hh), A_N, ta(T_Z + 2 * hh), B_N, 2, TILE, true);
+        mma64(dst(tbase, hh, C_N2), ta(T_NA + hh), A_N, ta(T_NA + hh), B_N, 1, TILE, false);
+    });
+    wait_mma();
+    if (ok) {
+        me.ld(tbase, C_Z + 64, v);
+        st_tile_f16(tile(T_Z + 2 * h), r, c0, v);
+        me.ld(tbase, C_Z + 128, v);
+        st_tile_f16(tile(T_Z + 2 * h + 1), r, c0, v);
+        me.ld(tbase, C_N2, v);
+        st_tile_f16(tile(T_DA + h), r, c0, v);
+    }
+    sync_operands();
+
+    // ---- level 3: [What | U] = Z1 + N'^2 Z1
+    ISSUE(for (int hh = 0; hh < 2; ++hh)
+              mma64(dst(tbase, hh, C_Z + 64), ta(T_DA + hh), A_N, ta(T_Z + 2 * hh), B_N, 2, TILE, true));
+    wait_mma();
+    if (ok) {
+        me.ld(tbase, C_Z + 64, v);
+        st_tile_f16(tile(T_Z + 2 * h), r, c0, v);
+        me.ld(tbase, C_Z + 128, v);
+        st_tile_f16(tile(T_Z + 2 * h + 1), r, c0, v);
+    }
+    sync_operands();
+
+    // ---- level 4: -M What, Q K^T - M U, U^T W, W^T What
+    ISSUE(for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t wh = ta(T_Z + 2 * hh), u = ta(T_Z + 2 * hh + 1), w = ta(hh ? T_WB : T_WA);
+        mma64(dst(tbase, hh, C_QT), ta(T_MA + hh), A_N, wh, B_N, 1, TILE, false);
+        mma64(dst(tbase, hh, C_S), ta(T_MA + hh), A_N, u, B_N, 1, TILE, true);
+        mma64(dst(tbase, hh, C_KT), u, A_T, w, B_N, 1, TILE, false);
+        mma64(dst(tbase, hh, C_P), w, A_T, wh, B_N, 1, TILE, false);
+    });
+    wait_mma();
+    const long long brow = (long long)hd * Lp + (long long)J * BT;  // block's first row in [nh, Lp]
+    float *sdb = Sd + ((long long)hd * nblk + J) * BT * BT;
+    float *hv = halves ? halves + ((long long)hd * nblk + J) * 4 * HB * HB : nullptr;
+    if (ok) {
+        // Qtil_h = Q - M What
+        me.ld(tbase, C_QT, v);
+        ld_tile_bf16(tile(h ? T_QB : T_QA), r, c0, x);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += x[j];
+        if (h == 0)
+            st_global(Qt + (brow + r) * HB + c0, v);
+        else
+            st_tile_f16(tile(T_QTB), r, c0, v);
+        if (hv && h == 1) st_global(hv + 1 * HB * HB + r * HB + c0, v);
+        // Ktil_h = K - U^T W
+        me.ld(tbase, C_KT, v);
+        ld_tile_bf16(tile(h ? T_KB : T_KA), r, c0, x);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = x[j] - v[j];
+        if (h == 1)
+            st_global(Kt + (brow + HB + r) * HB + c0, v);
+        else
+            st_tile_f16(tile(T_KTA), r, c0, v);
+        if (hv && h == 0) st_global(hv + 0 * HB * HB + r * HB + c0, v);
+        // P_h = I - W^T What
+        me.ld(tbase, C_P, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = (c0 + j == r ? 1.f : 0.f) - v[j];
+        st_tile_f16(tile(h ? T_PB : T_PA), r, c0, v);
+        if (hv) st_global(hv + (2 + h) * HB * HB + r * HB + c0, v);
+        // Sd_hh = lower(Q K^T - M U); the block above the diagonal blocks is zero
+        me.ld(tbase, C_S, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (c0 + j > r) v[j] = 0.f;
+        float *sdrow = sdb + (long long)(h * HB + r) * BT;
+        st_global(sdrow + h * HB + c0, v);
+        if (h == 0) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = 0.f;
+            st_global(sdrow + HB + c0, x);
+        }
+    }
+    sync_operands();
+
+    // ---- level 5: the 128-block from its halves
+    ISSUE({
+        mma64(dst(tbase, 0, C_C1), ta(T_KTA), A_N, ta(T_PB), B_T, 1, TILE, false);  // Ktil_a P_b^T
+        mma64(dst(tbase, 0, C_C2), ta(T_PB), A_N, ta(T_PA), B_N, 1, TILE, false);   // P_b P_a
+        mma64(dst(tbase, 1, C_C1), ta(T_QTB), A_N, ta(T_PA), B_N, 1, TILE, false);  // Qtil_b P_a
+        mma64(dst(tbase, 1, C_C2), ta(T_QTB), A_N, ta(T_KTA), B_T, 1, TILE, false); // Qtil_b Ktil_a^T
+    });
+    wait_mma();
+    if (ok) {
+        me.ld(tbase, C_C1, v);
+        if (h == 0)
+            st_global(Kt + (brow + r) * HB + c0, v);
+        else
+            st_global(Qt + (brow + HB + r) * HB + c0, v);
+        me.ld(tbase, C_C2, v);
+        if (h == 0)
+            st_global(Pm + (((long long)hd * nblk + J) * HB + r) * HB + c0, v);
+        else
+            st_global(sdb + (long long)(HB + r) * BT + c0, v);
+    }
+#undef ISSUE
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (!ok && tid == 0 && err) atomicCAS(err, 0, 21);
+    if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+}  // namespace
+
+bool prep_forward_ut_supported(const PrepDims &Dm, const PrepInputs &in)
+{
+    const uintptr_t al = reinterpret_cast<uintptr_t>(in.q) | reinterpret_cast<uintptr_t>(in.k) |
+                         reinterpret_cast<uintptr_t>(in.w);
+    return Dm.d == HB && Dm.dt == BF16 && (al & 15u) == 0 && (long long)Dm.L <= (1LL << 31) - 1;
+}
+
+cudaError_t prep_forward_ut(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out,
+                            int *err, cudaStream_t st)
+{
+    CUtensorMap mW, mQ, mK;
+    if (!make_map_3d(&mW, in.w, BF16, HB, Dm.L, Dm.nh, HB) ||
+        !make_map_3d(&mQ, in.q, BF16, HB, Dm.L, Dm.nh, HB) ||
+        !make_map_3d(&mK, in.k, BF16, HB, Dm.L, Dm.nh, HB))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(prep_fwd_ut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e != cudaSuccess) return e;
+    prep_fwd_ut_kernel<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(
+        mW, mQ, mK, in.beta, Dm.L, Dm.nblk, static_cast<f16 *>(out.Qt), static_cast<f16 *>(out.Kt),
+        static_cast<f16 *>(out.Pm), out.Sd, out.halves, err);
+    count_launches();
+    return cudaGetLastError();
+}
+
+}  // namespace path

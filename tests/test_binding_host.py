@@ -128,3 +128,24 @@ def test_wrappers_of_the_remaining_entry_points():
     prev = P.path_profile_enable(True)
     assert P.path_profile_enable(prev) is True
     assert P.path_profile_read() == {}
+
+
+class _OnDevice:
+    """Stands in for a contiguous CUDA tensor on device `index` (no GPU needed)."""
+    is_cuda = True
+
+    def __init__(self, index):
+        self.device = torch.device("cuda", index)
+
+    def is_contiguous(self):
+        return True
+
+
+def test_tensors_must_be_on_the_current_device(monkeypatch):
+    """The library launches on the current device: tensors elsewhere are refused."""
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+    with pytest.raises(ValueError, match="current CUDA device"):
+        P._check_dev(_OnDevice(0), _OnDevice(0))
+    with pytest.raises(ValueError, match="one device"):
+        P._check_dev(_OnDevice(1), _OnDevice(0))
+    P._check_dev(_OnDevice(1), None, _OnDevice(1))

@@ -51,22 +51,43 @@ def ulp_bf16(x):
     return np.exp2(np.floor(np.log2(a)) - 7)
 
 
+def nans(shape, dtype):
+    return torch.full(shape, float("nan"), dtype=dtype, device="cuda")
+
+
+def assert_all_finite(ts, where):
+    """Every element of every tensor was written: they all start as NaN."""
+    for n, t in ts.items():
+        bad = int((~torch.isfinite(t)).sum())
+        assert bad == 0, f"{where}: {n} has {bad} elements never written (NaN sentinel left)"
+
+
 def run_ours(P, x, backward, out_dtype=None, reuse=False):
+    """The library on x. Outputs, gradients and the workspace start filled with NaN
+    (the workspace as 0xFF bytes, a NaN in fp32 and fp16), so an element that no kernel
+    writes, or a workspace value read before any kernel wrote it, cannot pass."""
     d = to_dev(x)
     B, H, L, D = d["q"].shape
     od = out_dtype or d["q"].dtype
     nb = max(P.path_attn_workspace_bytes(B, H, L, D, d["q"].dtype, bwd, od)
              for bwd in (False, backward))
-    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    ws = torch.full((nb,), 0xFF, dtype=torch.uint8, device="cuda")
     out, lse = P.path_attn_fwd(d["q"], d["k"], d["v"], d["w"], d["beta"], d["log_f"],
-                               out_dtype=out_dtype, workspace=ws)
+                               out=nans(d["q"].shape, od), lse=nans((B, H, L), torch.float32),
+                               workspace=ws)
     assert P.lib().path_attn_wait_status(ws.data_ptr(), None) == 0, "forward wait timed out"
+    assert_all_finite({"out": out, "lse": lse}, "forward")
     g = None
     if backward:
+        grads = {n: nans(d["q"].shape, od) for n in ("dq", "dk", "dv", "dw")}
+        grads["dbeta"] = nans((B, H, L), torch.float32)
+        if d["log_f"] is not None:
+            grads["dlog_f"] = nans((B, H, L), torch.float32)
         g = P.path_attn_bwd(d["q"], d["k"], d["v"], d["w"], d["beta"], out, lse,
-                            d["dout"].to(out.dtype), d["log_f"], workspace=ws,
+                            d["dout"].to(out.dtype), d["log_f"], grads=grads, workspace=ws,
                             reuse_fwd_workspace=reuse)
         assert P.lib().path_attn_wait_status(ws.data_ptr(), None) == 0, "backward wait timed out"
+        assert_all_finite(g, "backward")
     torch.cuda.synchronize()
     return out, lse, g
 
@@ -203,6 +224,10 @@ def test_full_size_fox_l16384_sampled_heads(P):
 def _decode_check(P, B, H, d, n0, cap, steps, dtype, heads, tol):
     kc, vc, seq = si.make_decode_inputs(B, H, d, n0, cap, steps, dtype, seed=3)
     kd, vd = kc.cuda(), vc.cuda()
+    # cache rows past the cached ones start as NaN: each step must write its row
+    # before any read of it, and rows past the last step stay untouched
+    kd[..., n0:, :] = float("nan")
+    vd[..., n0:, :] = float("nan")
     sel = lambda t: t.reshape(B * H, *t.shape[2:])[heads].unsqueeze(0)
     ok = sel(kc).double().numpy().copy()
     ov = sel(vc).double().numpy().copy()
@@ -211,7 +236,8 @@ def _decode_check(P, B, H, d, n0, cap, steps, dtype, heads, tol):
     for t, s in enumerate(seq):
         sd = {k: v.cuda() for k, v in s.items()}
         out = P.path_decode_step(sd["q"], sd["k_new"], sd["v_new"], sd["w"], sd["beta"], kd, vd,
-                                 n0 + t)
+                                 n0 + t, out=nans(sd["q"].shape, dtype))
+        assert_all_finite({"out": out}, f"decode step {t}")
         ref = oracle.decode_step(sel(s["q"]), sel(s["k_new"]), sel(s["v_new"]), sel(s["w"]),
                                  sel(s["beta"]), ok, ov, n0 + t,
                                  round_bf16=(dtype == torch.bfloat16))
@@ -255,6 +281,9 @@ def _decode_check(P, B, H, d, n0, cap, steps, dtype, heads, tol):
           f"cache entries beyond tolerance {cache_bad}, entries differing "
           f"{int(np.sum(kg != kref))} of {kg.size}")
     np.testing.assert_array_equal(np64(sel(vd.cpu())[..., :n, :]), ov[..., :n, :])
+    assert_all_finite({"k_cache": kd[..., :n, :], "v_cache": vd[..., :n, :]}, "decode cache")
+    assert bool(torch.isnan(kd[..., n:, :]).all()) and bool(torch.isnan(vd[..., n:, :]).all()), \
+        "decode wrote cache rows past the last step"
     assert worst <= tol
     assert cache_bad == 0
 
@@ -303,10 +332,19 @@ def _cache_bar(got, ref, dtype):
 def _prefill_check(P, x, cap, heads=None):
     dd = to_dev(x)
     dtype = dd["q"].dtype
-    out, lse, kc, vc, gc = P.path_attn_prefill(dd["q"], dd["k"], dd["v"], dd["w"], dd["beta"],
-                                               cap, dd["log_f"])
-    torch.cuda.synchronize()
     B, H, L, d = dd["q"].shape
+    # outputs and caches start as NaN: rows 0..L-1 must be written, the rest left alone
+    fox = dd["log_f"] is not None
+    out, lse, kc, vc, gc = P.path_attn_prefill(
+        dd["q"], dd["k"], dd["v"], dd["w"], dd["beta"], cap, dd["log_f"],
+        out=nans(dd["q"].shape, dtype), lse=nans((B, H, L), torch.float32),
+        k_cache=nans((B, H, cap, d), dtype), v_cache=nans((B, H, cap, d), dtype),
+        g_cache=nans((B, H, cap), torch.float32) if fox else None)
+    torch.cuda.synchronize()
+    assert_all_finite({"out": out, "lse": lse, "k_cache": kc[..., :L, :], "v_cache": vc[..., :L, :]},
+                      "prefill")
+    if fox:
+        assert_all_finite({"g_cache": gc[..., :L]}, "prefill")
     pick = (lambda t: t) if heads is None else (
         lambda t: t.reshape(B * H, *t.shape[2:])[heads].unsqueeze(0))
     xs = x if heads is None else {k: (None if v is None else pick(v)) for k, v in x.items()}
@@ -327,10 +365,10 @@ def _prefill_check(P, x, cap, heads=None):
         # fp32 roundings of |c| and one of the difference, so |err| <= 3 2^-24 max|c|
         cmax = float(np.abs(np.cumsum(np64(xs["log_f"]), axis=-1)).max())
         assert eg <= 4 * 2.0 ** -24 * cmax + 1e-12, (eg, cmax)
-    # rows past L are left as the caller had them (zero here)
-    assert not kc[..., L:, :].any() and not vc[..., L:, :].any()
+    # rows past L are left as the caller had them (NaN here)
+    assert bool(torch.isnan(kc[..., L:, :]).all()) and bool(torch.isnan(vc[..., L:, :]).all())
     if gc is not None:
-        assert not gc[..., L:].any()
+        assert bool(torch.isnan(gc[..., L:]).all())
 
 
 @pytest.mark.parametrize("dtype,d,L,fox", [(torch.float32, 64, 300, False),

@@ -376,7 +376,6 @@ __global__ void __launch_bounds__(NT, 1)
                     // chain adjoint: operand for the next pair, or dKtil_J after pair (J+1, J)
                     float v[32];
                     tmem_ld32(tbase + C::T_AB + c0 + lane_off, v);
-                    tmem_wait_ld();
                     if (I > J + 1) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
@@ -398,7 +397,6 @@ __global__ void __launch_bounds__(NT, 1)
                     // dQtil rows of tile I (lane = query row)
                     float v[32];
                     tmem_ld32(tbase + C::T_DQ + c0 + lane_off, v);
-                    tmem_wait_ld();
                     uint8_t *box = stq + (c0 >> 5) * 16384 + j * 128;
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
@@ -411,7 +409,6 @@ __global__ void __launch_bounds__(NT, 1)
                     for (int c0 = 0; c0 < D; c0 += 32) {
                         float v[32];
                         tmem_ld32(tbase + C::T_DPI + c0 + lane_off, v);
-                        tmem_wait_ld();
                         if (j < D) {
                             uint8_t *box = stp + (c0 >> 5) * 8192 + j * 128;
 #pragma unroll
@@ -454,7 +451,6 @@ __global__ void __launch_bounds__(NT, 1)
             for (int c0 = 0; c0 < D; c0 += 32) {
                 float v[32];
                 tmem_ld32(tbase + C::T_DV + c0 + lane_off, v);  // warp-wide; rows past L drop
-                tmem_wait_ld();
                 if (gj < a.L) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) dst[c0 + e] = from_f<TO>(v[e]);

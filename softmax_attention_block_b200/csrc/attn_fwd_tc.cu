@@ -105,9 +105,13 @@ __global__ void __launch_bounds__(NT, 1)
     uint64_t *kv_full = bars + 1;
     uint64_t *kv_empty = bars + 1 + NS;
     uint64_t *s_full = bars + 1 + 2 * NS;
-    uint64_t *p_full = bars + 3 + 2 * NS;
-    uint64_t *o_full = bars + 4 + 2 * NS;  // [PB]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 + 2 * NS + C::PB);
+    // P of tile it is complete when p_full[it & 1] completes. One barrier per
+    // parity: a warp pair may finish tile it + 1 (its S and the P.V it folds are
+    // ready) before another pair has finished tile it, and its arrival must not
+    // count toward tile it's phase.
+    uint64_t *p_full = bars + 3 + 2 * NS;  // [2]
+    uint64_t *o_full = bars + 5 + 2 * NS;  // [PB]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 5 + 2 * NS + C::PB);
     uint8_t *sQ = sm + C::Q_OFF;
     uint8_t *sP = sm + C::P_OFF;
     auto sK = [&](int s) { return sm + C::ST_OFF + s * C::ST_BYTES; };
@@ -130,7 +134,8 @@ __global__ void __launch_bounds__(NT, 1)
         }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(p_full, NSOFT);
+        mbar_init(&p_full[0], NSOFT);
+        mbar_init(&p_full[1], NSOFT);
         for (int b = 0; b < C::PB; ++b) mbar_init(&o_full[b], 1);
         mbar_fence_init();
     }
@@ -210,7 +215,7 @@ __global__ void __launch_bounds__(NT, 1)
                 // after tile it's softmax, and its keys were loaded a tile earlier
                 for (int n = 1; ok && n <= 2 && n < niter; ++n) ok = issue_s(n);
                 for (int it = 0; ok && it < niter; ++it) {
-                    if (!mbar_wait(p_full, it & 1, WAIT_POLLS)) {
+                    if (!mbar_wait(&p_full[it & 1], (it >> 1) & 1, WAIT_POLLS)) {
                         ok = false;
                         break;
                     }
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(NT, 1)
                         ok = false;
                         break;
                     }
-                    if (!mbar_wait(p_full, it & 1, WAIT_POLLS)) {
+                    if (!mbar_wait(&p_full[it & 1], (it >> 1) & 1, WAIT_POLLS)) {
                         ok = false;
                         break;
                     }
@@ -281,7 +286,6 @@ __global__ void __launch_bounds__(NT, 1)
                     float *z0 = z, *z1 = z + 32;
                     tmem_ld32(tbase + b * 128 + c0s + lane_off, *reinterpret_cast<float(*)[32]>(z0));
                     tmem_ld32(tbase + b * 128 + c0s + 32 + lane_off, *reinterpret_cast<float(*)[32]>(z1));
-                    tmem_wait_ld();
                 }
                 if (it == 0) {  // the diagonal tile: causal mask
 #pragma unroll
@@ -317,7 +321,6 @@ __global__ void __launch_bounds__(NT, 1)
                     for (int c0 = 0; c0 < DH; c0 += 32) {
                         float v[32];
                         tmem_ld32(tbase + 256 + pb * D + c0o + c0 + lane_off, v);
-                        tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
                     }
@@ -351,7 +354,7 @@ __global__ void __launch_bounds__(NT, 1)
             }
             fence_async_smem();
             fence_before_sync();
-            mbar_arrive(p_full);
+            mbar_arrive(&p_full[it & 1]);
         }
         // the last PB tiles' P.V
         for (int t = niter - C::PB > 0 ? niter - C::PB : 0; t < niter; ++t) {
@@ -366,7 +369,6 @@ __global__ void __launch_bounds__(NT, 1)
                 for (int c0 = 0; c0 < DH; c0 += 32) {
                     float v[32];
                     tmem_ld32(tbase + 256 + pb * D + c0o + c0 + lane_off, v);
-                    tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(acc[c0 + j], corr, v[j]);
                 }

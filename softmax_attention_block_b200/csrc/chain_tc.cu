@@ -120,7 +120,6 @@ __global__ void __launch_bounds__(128)
         for (int c0 = 0; c0 < D; c0 += 32) {
             float v[32];
             tmem_ld32(tbase + c0 + lane_off, v);
-            tmem_wait_ld();
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
                 uint4 u;

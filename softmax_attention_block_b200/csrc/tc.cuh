@@ -138,13 +138,17 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 
 // 32 consecutive fp32 columns of this thread's lane (warp w reads lanes
 // 32*(w%4) .. 32*(w%4)+31; taddr must carry that lane offset in bits 31:16).
+// The load and its wait are one asm statement: the destination registers are
+// written asynchronously until tcgen05.wait::ld, and a separate wait statement
+// would not stop the compiler from scheduling their uses before it.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32])
 {
     uint32_t *u = reinterpret_cast<uint32_t *>(r);
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
           "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
           "=r"(u[13]), "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]),
@@ -156,7 +160,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32])
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 16 consecutive fp32 columns of this thread's lane (same addressing as tmem_ld32).
+// 16 consecutive fp32 columns of this thread's lane (same addressing as
+// tmem_ld32), without the wait: follow with tmem_wait_ld_tied on the registers.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16])
 {
     uint32_t *u = reinterpret_cast<uint32_t *>(r);

@@ -69,7 +69,6 @@ struct Me {
     __device__ __forceinline__ void ld(uint32_t tbase, int col, float (&v)[32]) const
     {
         tc::tmem_ld32(tbase + lane_off + (uint32_t)(col + 32 * cg), v);
-        tc::tmem_wait_ld();
     }
 };
 

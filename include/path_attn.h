@@ -264,6 +264,21 @@ unsigned long long path_kernel_launch_count(void);
 int path_profile_enable(int on);
 int path_profile_read(path_stage_time *out, int max_entries);
 
+/*
+ * Test hook for the bounded waits (process-wide, off by default; the pages have
+ * no counterpart). While on (on = 1), every tensor-core path_attn_fwd (bf16
+ * inputs, d = 64 or 128) makes the load producer of its last query tile skip
+ * the copy of that tile's first off-diagonal key / value block (it neither
+ * issues it nor announces its bytes), and every wait of that kernel gives up
+ * after 2 ms instead of 0.5 s. The tile that waits for the block then gives
+ * up: its rows of out and lse are written as NaN and path_attn_wait_status
+ * reports PATH_ERR_TIMEOUT; the other tiles complete normally and the CUDA
+ * context stays usable. The producer still waits for every copy it did issue
+ * before its block exits. Needs L > 128 (at least two query tiles). Returns
+ * PATH_OK, or PATH_ERR_INVALID_ARG if `on` is not 0 or 1.
+ */
+path_status path_test_withhold_kv_load(int on);
+
 #ifdef __cplusplus
 }
 #endif

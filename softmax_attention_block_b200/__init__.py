@@ -22,6 +22,7 @@ Entry points (same names as the C ABI):
 - ``path_attn_workspace_bytes``, ``path_decode_workspace_bytes``, ``path_status_string``
 - diagnostics: ``path_kernel_launch_count()``, ``path_profile_enable(on)``,
   ``path_profile_read() -> {stage: (total_ms, count)}``
+- test hook: ``path_test_withhold_kv_load(on)`` (makes the forward's bounded waits give up)
 """
 from __future__ import annotations
 
@@ -89,6 +90,8 @@ def lib() -> ctypes.CDLL:
         L.path_decode_step_noalloc.argtypes = [vp, vp, vp, vp, fp, f, i, i, i, i, i, i, vp, vp,
                                                vp, vp]
         L.path_attn_wait_status.argtypes = [vp, vp]
+        L.path_test_withhold_kv_load.argtypes = [i]
+        L.path_test_withhold_kv_load.restype = i
         L.path_kernel_launch_count.restype = ctypes.c_ulonglong
         L.path_profile_enable.argtypes = [i]
         L.path_profile_enable.restype = i
@@ -385,3 +388,11 @@ def path_attn_prefill(q, k, v, w, beta, capacity, log_f=None, scale=None, out=No
     if st:
         raise PathError(st, "path_attn_prefill")
     return out, lse, k_cache, v_cache, g_cache
+
+
+def path_test_withhold_kv_load(on: bool) -> None:
+    """Test hook of the bounded waits (include/path_attn.h): while on, the tensor-core
+    forward's last query tile never receives one key/value block and reports a timeout."""
+    st = lib().path_test_withhold_kv_load(1 if on else 0)
+    if st:
+        raise PathError(st, "path_test_withhold_kv_load")

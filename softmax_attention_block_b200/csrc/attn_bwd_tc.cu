@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(NT, 1)
             int issued = 0;
             for (int it = 0; it < niter; ++it) {
                 const int s = it & 1;
-                if (it >= 2 && !mbar_wait(&ld_empty[s], ((it >> 1) - 1) & 1, WAIT_POLLS)) {
+                if (it >= 2 && !mbar_wait(&ld_empty[s], ((it >> 1) - 1) & 1, WAIT_LIMIT_NS)) {
                     if (a.err) atomicCAS(a.err, 0, 11);
                     break;
                 }
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(NT, 1)
                 issued = it + 1;
             }
             for (int it = issued - 2 > 0 ? issued - 2 : 0; it < issued; ++it)
-                mbar_wait(&ld_full[it & 1], (it >> 1) & 1, WAIT_POLLS);
+                mbar_wait(&ld_full[it & 1], (it >> 1) & 1, WAIT_LIMIT_NS);
         }
     } else if (warp == W_MMA) {
         // the whole warp runs the issue loop (uniform descriptors); lane 0 issues
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(NT, 1)
             // MMA 1 of pair it: S^T = Khat Qtil^T (not on the diagonal), dP^T = V dO^T
             auto mma1 = [&](int it) -> bool {
                 const int s = it & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_POLLS)))
+                if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_LIMIT_NS)))
                     return false;
                 fence_after_sync();
                 const uint32_t kh0 = smem_u32(stage(s) + C::S_KH), q0 = smem_u32(stage(s) + C::S_Q),
@@ -181,14 +181,14 @@ __global__ void __launch_bounds__(NT, 1)
                 commit_if(lead, s_full);
                 return true;
             };
-            bool ok = __all_sync(0xffffffffu, mbar_wait(v_full, 0, WAIT_POLLS)) && mma1(0);
+            bool ok = __all_sync(0xffffffffu, mbar_wait(v_full, 0, WAIT_LIMIT_NS)) && mma1(0);
             for (int it = 0; ok && it < niter; ++it) {
                 const int s = it & 1, I = tile_of(it);
                 const bool diag = it == niter - 1;
                 // MMA 2 needs this pair's P / dS in shared memory, and overwrites the
                 // previous pair's results: drained by then?
-                const bool ready = mbar_wait(p_full, it & 1, WAIT_POLLS) &&
-                                   (it == 0 || mbar_wait(e_done, (it - 1) & 1, WAIT_POLLS));
+                const bool ready = mbar_wait(p_full, it & 1, WAIT_LIMIT_NS) &&
+                                   (it == 0 || mbar_wait(e_done, (it - 1) & 1, WAIT_LIMIT_NS));
                 if (!__all_sync(0xffffffffu, ready)) {  // the warp stays converged
                     ok = false;
                     break;
@@ -252,8 +252,8 @@ __global__ void __launch_bounds__(NT, 1)
             const int s = it & 1, I = tile_of(it);
             const bool diag = it == niter - 1;
             // s_full also orders this pair's P / dS writes after the previous MMA 2
-            if (ok && (!mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_POLLS) ||
-                       !mbar_wait(s_full, it & 1, WAIT_POLLS)))
+            if (ok && (!mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_LIMIT_NS) ||
+                       !mbar_wait(s_full, it & 1, WAIT_LIMIT_NS)))
                 ok = false;
             ok = __all_sync(0xffffffffu, ok);  // shuffles and TMEM loads below are warp-wide
             fence_after_sync();
@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(NT, 1)
         for (int it = 0; it < niter; ++it) {
             const int s = it & 1, I = tile_of(it);
             const bool diag = it == niter - 1;
-            if (ok && !mbar_wait(m2_full, it & 1, WAIT_POLLS)) ok = false;
+            if (ok && !mbar_wait(m2_full, it & 1, WAIT_LIMIT_NS)) ok = false;
             ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-wide
             fence_after_sync();
             uint8_t *stq = stage(s), *stp = stage(s) + 2 * 16384;  // dQtil: 2 x 16 KB, dP_I: 2 x 8 KB

@@ -111,7 +111,8 @@ __global__ void __launch_bounds__(NT, 1)
     // count toward tile it's phase.
     uint64_t *p_full = bars + 3 + 2 * NS;  // [2]
     uint64_t *o_full = bars + 5 + 2 * NS;  // [PB]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 5 + 2 * NS + C::PB);
+    uint64_t *mma_done = bars + 5 + 2 * NS + C::PB;  // every MMA of the CTA completed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6 + 2 * NS + C::PB);
     uint8_t *sQ = sm + C::Q_OFF;
     uint8_t *sP = sm + C::P_OFF;
     auto sK = [&](int s) { return sm + C::ST_OFF + s * C::ST_BYTES; };
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_init(&p_full[0], NSOFT);
         mbar_init(&p_full[1], NSOFT);
         for (int b = 0; b < C::PB; ++b) mbar_init(&o_full[b], 1);
+        mbar_init(mma_done, 1);
         mbar_fence_init();
     }
     if (warp == W_MMA) tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -147,15 +149,19 @@ __global__ void __launch_bounds__(NT, 1)
 
     if (warp == W_PROD) {
         if (lane == 0) {
-            int issued = 0;
+            int issued = 0, withheld = -1;
             mbar_expect_tx(q_full, C::TILE);
             for (int p = 0; p < C::PANELS; ++p)
                 tma_load_2d(sQ + p * 16384, &mQ, 64 * p, h * Lp + I * BT, q_full);
             for (int it = 0; it < niter; ++it) {
                 const int s = it % NS;
-                if (it >= NS && !mbar_wait(&kv_empty[s], ((it / NS) - 1) & 1, WAIT_POLLS)) {
+                if (it >= NS && !mbar_wait(&kv_empty[s], ((it / NS) - 1) & 1, a.limit_ns)) {
                     flag_error(a.err, 1);
                     break;
+                }
+                if (a.withhold && I == a.nblk - 1 && it == 1) {
+                    withheld = it;  // test hook: this stage's copies are never issued
+                    continue;
                 }
                 const int J = it == 0 ? I : I - it;
                 const uint32_t bytes = C::TILE + (it > 0 ? C::TILE : 0) + (FOX ? 512 : 0);
@@ -170,22 +176,24 @@ __global__ void __launch_bounds__(NT, 1)
                 if (FOX) bulk_load(sC(s), a.c + (long long)h * Lp + J * BT, 512, &kv_full[s]);
                 issued = it + 1;
             }
-            // never leave while copies into this CTA's shared memory are in flight
+            // never leave while copies into this CTA's shared memory are in flight:
+            // wait for every stage whose copies were issued (the copies complete on
+            // their own; the bound is the rule for every wait, set far above them)
             for (int it = issued - NS > 0 ? issued - NS : 0; it < issued; ++it)
-                mbar_wait(&kv_full[it % NS], (it / NS) & 1, WAIT_POLLS);
+                if (it != withheld) mbar_wait(&kv_full[it % NS], (it / NS) & 1, 8 * a.limit_ns);
         }
     } else if (warp == W_MMA) {
         if (lane == 0) {
             const uint32_t idS = idesc_f16(128, 128, AB_F16, 0, 0);
             const uint32_t idO = idesc_f16(128, D, AB_F16, 0, 1);
             const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
-            bool ok = mbar_wait(q_full, 0, WAIT_POLLS) && mbar_wait(&kv_full[0], 0, WAIT_POLLS);
+            bool ok = mbar_wait(q_full, 0, a.limit_ns) && mbar_wait(&kv_full[0], 0, a.limit_ns);
             fence_after_sync();
             // S = Qtil Khat^T of tile n into S buffer n & 1 (tile 0, the diagonal,
             // takes its logits from the UT prep)
             auto issue_s = [&](int n) -> bool {
                 const int s = n % NS, b = n & 1;
-                if (!mbar_wait(&kv_full[s], (n / NS) & 1, WAIT_POLLS)) return false;
+                if (!mbar_wait(&kv_full[s], (n / NS) & 1, a.limit_ns)) return false;
                 fence_after_sync();
                 const uint32_t k_addr = smem_u32(sK(s));
 #pragma unroll
@@ -215,7 +223,7 @@ __global__ void __launch_bounds__(NT, 1)
                 // after tile it's softmax, and its keys were loaded a tile earlier
                 for (int n = 1; ok && n <= 2 && n < niter; ++n) ok = issue_s(n);
                 for (int it = 0; ok && it < niter; ++it) {
-                    if (!mbar_wait(&p_full[it & 1], (it >> 1) & 1, WAIT_POLLS)) {
+                    if (!mbar_wait(&p_full[it & 1], (it >> 1) & 1, a.limit_ns)) {
                         ok = false;
                         break;
                     }
@@ -230,7 +238,7 @@ __global__ void __launch_bounds__(NT, 1)
                         ok = false;
                         break;
                     }
-                    if (!mbar_wait(&p_full[it & 1], (it >> 1) & 1, WAIT_POLLS)) {
+                    if (!mbar_wait(&p_full[it & 1], (it >> 1) & 1, a.limit_ns)) {
                         ok = false;
                         break;
                     }
@@ -239,6 +247,10 @@ __global__ void __launch_bounds__(NT, 1)
                 }
             }
             if (!ok) flag_error(a.err, 2);
+            // the tensor memory is freed after this warp leaves: no MMA it issued
+            // may still be running then (on the normal path they all completed)
+            commit(mma_done);
+            mbar_wait(mma_done, 0, 8 * a.limit_ns);
         }
     } else {
         // softmax: row r = TMEM lane; this warp owns S columns [c0s, c0s+64) and
@@ -265,11 +277,11 @@ __global__ void __launch_bounds__(NT, 1)
         // failed wait the work is skipped, never the barriers.
         for (int it = 0; it < niter; ++it) {
             const int s = it % NS, b = it & 1;
-            if (ok && FOX && !mbar_wait(&kv_full[s], (it / NS) & 1, WAIT_POLLS)) ok = false;
+            if (ok && FOX && !mbar_wait(&kv_full[s], (it / NS) & 1, a.limit_ns)) ok = false;
             const float *cj = sC(s) + c0s;
             float z[64];
             float pmax = -INFINITY;
-            if (ok && it > 0 && !mbar_wait(&s_full[b], ((it - 1) >> 1) & 1, WAIT_POLLS)) ok = false;
+            if (ok && it > 0 && !mbar_wait(&s_full[b], ((it - 1) >> 1) & 1, a.limit_ns)) ok = false;
             ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-wide
             if (ok) {
                 if (it == 0) {
@@ -311,7 +323,7 @@ __global__ void __launch_bounds__(NT, 1)
             // accumulator; its P buffer is then free for this tile's probabilities
             if (it >= C::PB) {
                 const int t = it - C::PB, pb = t % C::PB;
-                if (ok && !mbar_wait(&o_full[pb], (t / C::PB) & 1, WAIT_POLLS)) ok = false;
+                if (ok && !mbar_wait(&o_full[pb], (t / C::PB) & 1, a.limit_ns)) ok = false;
                 ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-wide
                 if (ok) {
                     fence_after_sync();
@@ -359,7 +371,7 @@ __global__ void __launch_bounds__(NT, 1)
         // the last PB tiles' P.V
         for (int t = niter - C::PB > 0 ? niter - C::PB : 0; t < niter; ++t) {
             const int pb = t % C::PB;
-            if (ok && !mbar_wait(&o_full[pb], (t / C::PB) & 1, WAIT_POLLS)) ok = false;
+            if (ok && !mbar_wait(&o_full[pb], (t / C::PB) & 1, a.limit_ns)) ok = false;
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 fence_after_sync();
@@ -448,7 +460,9 @@ cudaError_t attn_fwd_tc(const FwdArgs &f, Types t, int d, int *err, cudaStream_t
         mK = mQ;  // no off-diagonal tiles: never read
     }
     if (!make_map_3d(&mV, f.vh, F16, d, f.L, f.nh, 128)) return cudaErrorInvalidValue;
-    FwdTcArgs a{f.Sd, f.c, f.scale * 1.4426950408889634f, f.L, f.nblk, f.nh, npairs, f.out, f.lse, err};
+    const int withhold = withhold_kv_load() && f.nblk > 1;
+    FwdTcArgs a{f.Sd, f.c, f.scale * 1.4426950408889634f, f.L, f.nblk, f.nh, npairs, f.out, f.lse, err,
+                withhold ? 2000000ull : WAIT_LIMIT_NS, withhold};
     const bool fox = f.c != nullptr;
     const bool f32 = t.out == F32;
 #define L_(D_, FOX_, TO_) return launch<D_, FOX_, TO_>(mQ, mK, mV, a, st)

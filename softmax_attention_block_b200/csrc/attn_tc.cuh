@@ -13,6 +13,8 @@ struct FwdTcArgs {
     void *out;
     float *lse;
     int *err;          // device error word (first wait that gave up)
+    uint64_t limit_ns; // bound on every wait of the kernel
+    int withhold;      // test hook: the last query tile's producer skips one key/value load
 };
 
 struct BwdTcArgs {

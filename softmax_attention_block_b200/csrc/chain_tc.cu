@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(128)
             for (int p = 0; p < D / 64; ++p)
                 tma_load_2d(Pb[0] + p * (D * 128), &mP, 64 * p, (h * nblk + J + 1) * D, &p_full[0]);
         }
-        ok = mbar_wait(x_full, 0, WAIT_POLLS);
+        ok = mbar_wait(x_full, 0, WAIT_LIMIT_NS);
         if (ok) {
             for (int p = 0; p < D / 64; ++p) tma_store_2d(&mKh, 64 * p, pair_row(J + 1), X[0] + p * 16384);
             bulk_commit();
@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(128)
         const int t = I - J - 1;
         uint8_t *cur = X[t & 1], *nxt = X[(t + 1) & 1];
         if (tid == 0 && ok) {
-            ok = mbar_wait(&p_full[t & 1], (t >> 1) & 1, WAIT_POLLS);
+            ok = mbar_wait(&p_full[t & 1], (t >> 1) & 1, WAIT_LIMIT_NS);
             if (ok && I + 1 < last) {  // prefetch P_{I+1}; its buffer's last reader has completed
                 mbar_expect_tx(&p_full[(t + 1) & 1], C::PB);
                 for (int p = 0; p < D / 64; ++p)
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(128)
         }
         ok = __syncthreads_and(ok);
         if (!ok) break;
-        if (!mbar_wait(mma_done, t & 1, WAIT_POLLS)) ok = false;
+        if (!mbar_wait(mma_done, t & 1, WAIT_LIMIT_NS)) ok = false;
         ok = __syncthreads_and(ok);
         if (!ok) break;
         fence_after_sync();

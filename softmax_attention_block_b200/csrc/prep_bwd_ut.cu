@@ -139,6 +139,12 @@ __global__ void __launch_bounds__(NT, 1)
     const float *dsdb = dSd + ((long long)hd * nblk + J) * BT * BT;
 
     if (tid == 0) {
+        // every fp32 adjoint this block reads, on its way to L2 while the
+        // halves' transforms are recomputed
+        prefetch_l2(dQt + brow * HB, BT * HB * 4);
+        prefetch_l2(dKt + brow * HB, BT * HB * 4);
+        prefetch_l2(dPm + ((long long)hd * nblk + J) * HB * HB, HB * HB * 4);
+        prefetch_l2(dsdb, BT * BT * 4);
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
         mbar_fence_init();
@@ -172,10 +178,7 @@ __global__ void __launch_bounds__(NT, 1)
             tma_load_3d(tile(T_Q + h), &mQ, 0, y, hd, &bars[0]);
         }
     }
-    // the adjoints the halves take from the attention backward as they are
-    tile_from_f32(tile(T_DQ), dQt + brow * HB, HB);                  // dQ_a = dQtil[a]
-    tile_from_f32(tile(T_DK + 1), dKt + (brow + HB) * HB, HB);       // dK_b = dKtil[b]
-    bool ok = mbar_wait(&bars[0], 0, WAIT_POLLS);
+    bool ok = mbar_wait(&bars[0], 0, WAIT_LIMIT_NS);
     ok = __syncthreads_and(ok);
 
     const Me me;
@@ -188,7 +191,7 @@ __global__ void __launch_bounds__(NT, 1)
         ok = __syncthreads_and(ok);
     };
     auto wait_mma = [&]() {
-        if (ok && !mbar_wait(&bars[1], phase, WAIT_POLLS)) ok = false;
+        if (ok && !mbar_wait(&bars[1], phase, WAIT_LIMIT_NS)) ok = false;
         phase ^= 1;
         fence_after_sync();
     };
@@ -212,6 +215,9 @@ __global__ void __launch_bounds__(NT, 1)
         mma64(dst(tbase, hh, C_GN), wk, A_N, wk, B_T, 2, TILE, false, AB_BF16);
         mma64(dst(tbase, hh, C_M), ta(T_Q + hh), A_N, wk, B_T, 1, TILE, false, AB_BF16);
     });
+    // meanwhile: the adjoints the halves take from the attention backward as they are
+    tile_from_f32(tile(T_DQ), dQt + brow * HB, HB);             // dQ_a = dQtil[a]
+    tile_from_f32(tile(T_DK + 1), dKt + (brow + HB) * HB, HB);  // dK_b = dKtil[b]
     wait_mma();
     if (ok) {
         me.ld(tbase, C_GN, v);  // A = strictLower(D G): diagonal blocks fp32, the rest A_off

@@ -63,10 +63,24 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// Row r of a 64-row fp32 TMA box of 32 columns (128-byte rows, 128-byte swizzle).
+__device__ __forceinline__ void st_box_f32(uint8_t *box, int r, const float (&v)[32])
+{
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        *reinterpret_cast<float4 *>(box + r * 128 + ((k ^ (r & 7)) << 4)) =
+            make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+}
+
+// Outputs leave through shared-memory staging and TMA tensor stores: Qt, Kt
+// ([nh Lp, 64] fp16), Pm ([nh nblk 64, 64] fp16) in 64 x 64 tiles, Sd
+// ([nh nblk 128, 128] fp32) in 64-row boxes of 32 columns.
 __global__ void __launch_bounds__(NT, 1)
     prep_fwd_ut_kernel(const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mQ,
-                       const __grid_constant__ CUtensorMap mK, const float *beta, int L, int nblk,
-                       f16 *Qt, f16 *Kt, f16 *Pm, float *Sd, float *halves, int *err)
+                       const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mQt,
+                       const __grid_constant__ CUtensorMap mKt, const __grid_constant__ CUtensorMap mPm,
+                       const __grid_constant__ CUtensorMap mSd, const float *beta, int L, int nblk,
+                       int *err)
 {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
@@ -107,7 +121,7 @@ __global__ void __launch_bounds__(NT, 1)
             tma_load_3d(tile(h ? T_QB : T_QA), &mQ, 0, y, hd, &bars[0]);
         }
     }
-    bool ok = mbar_wait(&bars[0], 0, WAIT_POLLS);
+    bool ok = mbar_wait(&bars[0], 0, WAIT_LIMIT_NS);
     ok = __syncthreads_and(ok);
 
     const Me me;
@@ -122,7 +136,7 @@ __global__ void __launch_bounds__(NT, 1)
         ok = __syncthreads_and(ok);
     };
     auto wait_mma = [&]() {
-        if (ok && !mbar_wait(&bars[1], phase, WAIT_POLLS)) ok = false;
+        if (ok && !mbar_wait(&bars[1], phase, WAIT_LIMIT_NS)) ok = false;
         phase ^= 1;
         fence_after_sync();
     };
@@ -238,71 +252,75 @@ __global__ void __launch_bounds__(NT, 1)
         mma64(dst(tbase, hh, C_P), w, A_T, wh, B_N, 1, TILE, false);
     });
     wait_mma();
-    const long long brow = (long long)hd * Lp + (long long)J * BT;  // block's first row in [nh, Lp]
-    float *sdb = Sd + ((long long)hd * nblk + J) * BT * BT;
-    float *hv = halves ? halves + ((long long)hd * nblk + J) * 4 * HB * HB : nullptr;
+    // staging: tiles free by now (F4's and the composition's, kept apart so the
+    // first stores can still be reading theirs while the second are written)
+    enum { S_QA = 12, S_KB = 13, S_SDA = 6, S_SDB = 14, S_KA = 0, S_QB = 1, S_PM = 2, S_SDBA = 3 };
+    const int brow = hd * Lp + J * BT;            // block's first row in [nh Lp] (fits int32)
+    const int sdrow = (hd * nblk + J) * BT;       // and in [nh nblk 128]
     if (ok) {
         // Qtil_h = Q - M What
         me.ld(tbase, C_QT, v);
         ld_tile_bf16(tile(h ? T_QB : T_QA), r, c0, x);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] += x[j];
-        if (h == 0)
-            st_global(Qt + (brow + r) * HB + c0, v);
-        else
-            st_tile_f16(tile(T_QTB), r, c0, v);
-        if (hv && h == 1) st_global(hv + 1 * HB * HB + r * HB + c0, v);
+        st_tile_f16(tile(h ? T_QTB : S_QA), r, c0, v);
         // Ktil_h = K - U^T W
         me.ld(tbase, C_KT, v);
         ld_tile_bf16(tile(h ? T_KB : T_KA), r, c0, x);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = x[j] - v[j];
-        if (h == 1)
-            st_global(Kt + (brow + HB + r) * HB + c0, v);
-        else
-            st_tile_f16(tile(T_KTA), r, c0, v);
-        if (hv && h == 0) st_global(hv + 0 * HB * HB + r * HB + c0, v);
+        st_tile_f16(tile(h ? S_KB : T_KTA), r, c0, v);
         // P_h = I - W^T What
         me.ld(tbase, C_P, v);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = (c0 + j == r ? 1.f : 0.f) - v[j];
         st_tile_f16(tile(h ? T_PB : T_PA), r, c0, v);
-        if (hv) st_global(hv + (2 + h) * HB * HB + r * HB + c0, v);
-        // Sd_hh = lower(Q K^T - M U); the block above the diagonal blocks is zero
+        // Sd_hh = lower(Q K^T - M U) (the block above the diagonal blocks is never
+        // read: the attention kernels mask it)
         me.ld(tbase, C_S, v);
 #pragma unroll
         for (int j = 0; j < 32; ++j)
             if (c0 + j > r) v[j] = 0.f;
-        float *sdrow = sdb + (long long)(h * HB + r) * BT;
-        st_global(sdrow + h * HB + c0, v);
-        if (h == 0) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = 0.f;
-            st_global(sdrow + HB + c0, x);
-        }
+        st_box_f32(tile((h ? S_SDB : S_SDA) + me.cg), r, v);
     }
     sync_operands();
 
-    // ---- level 5: the 128-block from its halves
+    // ---- level 5: the 128-block from its halves; meanwhile Qtil[a], Ktil[b], Sd_aa, Sd_bb go out
     ISSUE({
         mma64(dst(tbase, 0, C_C1), ta(T_KTA), A_N, ta(T_PB), B_T, 1, TILE, false);  // Ktil_a P_b^T
         mma64(dst(tbase, 0, C_C2), ta(T_PB), A_N, ta(T_PA), B_N, 1, TILE, false);   // P_b P_a
         mma64(dst(tbase, 1, C_C1), ta(T_QTB), A_N, ta(T_PA), B_N, 1, TILE, false);  // Qtil_b P_a
         mma64(dst(tbase, 1, C_C2), ta(T_QTB), A_N, ta(T_KTA), B_T, 1, TILE, false); // Qtil_b Ktil_a^T
     });
+    const bool storer = tid == 32;  // issues every TMA store (and waits for its own groups)
+    if (ok && storer) {
+        tma_store_2d(&mQt, 0, brow, tile(S_QA));
+        tma_store_2d(&mKt, 0, brow + HB, tile(S_KB));
+        for (int b = 0; b < 2; ++b) {
+            tma_store_2d(&mSd, 32 * b, sdrow, tile(S_SDA + b));
+            tma_store_2d(&mSd, HB + 32 * b, sdrow + HB, tile(S_SDB + b));
+        }
+        bulk_commit();
+    }
     wait_mma();
     if (ok) {
         me.ld(tbase, C_C1, v);
-        if (h == 0)
-            st_global(Kt + (brow + r) * HB + c0, v);
-        else
-            st_global(Qt + (brow + HB + r) * HB + c0, v);
+        st_tile_f16(tile(h ? S_QB : S_KA), r, c0, v);  // Ktil[a] = Ktil_a P_b^T, Qtil[b] = Qtil_b P_a
         me.ld(tbase, C_C2, v);
         if (h == 0)
-            st_global(Pm + (((long long)hd * nblk + J) * HB + r) * HB + c0, v);
+            st_tile_f16(tile(S_PM), r, c0, v);         // P = P_b P_a
         else
-            st_global(sdb + (long long)(HB + r) * BT + c0, v);
+            st_box_f32(tile(S_SDBA + me.cg), r, v);    // Sd[b, a] = Qtil_b Ktil_a^T
     }
+    sync_operands();
+    if (ok && storer) {
+        tma_store_2d(&mKt, 0, brow, tile(S_KA));
+        tma_store_2d(&mQt, 0, brow + HB, tile(S_QB));
+        tma_store_2d(&mPm, 0, (hd * nblk + J) * HB, tile(S_PM));
+        for (int b = 0; b < 2; ++b) tma_store_2d(&mSd, 32 * b, sdrow + HB, tile(S_SDBA + b));
+        bulk_commit();
+    }
+    if (storer) bulk_wait_all();  // the staging is read (and written out) before the CTA exits
 #undef ISSUE
     fence_before_sync();
     __syncthreads();
@@ -317,22 +335,27 @@ bool prep_forward_ut_supported(const PrepDims &Dm, const PrepInputs &in)
 {
     const uintptr_t al = reinterpret_cast<uintptr_t>(in.q) | reinterpret_cast<uintptr_t>(in.k) |
                          reinterpret_cast<uintptr_t>(in.w);
-    return Dm.d == HB && Dm.dt == BF16 && (al & 15u) == 0 && (long long)Dm.L <= (1LL << 31) - 1;
+    // tile row coordinates of the output tensor maps are int32
+    return Dm.d == HB && Dm.dt == BF16 && (al & 15u) == 0 &&
+           (long long)Dm.nh * Dm.nblk * BT < (1LL << 31);
 }
 
 cudaError_t prep_forward_ut(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out,
                             int *err, cudaStream_t st)
 {
-    CUtensorMap mW, mQ, mK;
+    CUtensorMap mW, mQ, mK, mQt, mKt, mPm, mSd;
+    const uint64_t rows = (uint64_t)Dm.nh * Dm.nblk * BT;
     if (!make_map_3d(&mW, in.w, BF16, HB, Dm.L, Dm.nh, HB) ||
         !make_map_3d(&mQ, in.q, BF16, HB, Dm.L, Dm.nh, HB) ||
-        !make_map_3d(&mK, in.k, BF16, HB, Dm.L, Dm.nh, HB))
+        !make_map_3d(&mK, in.k, BF16, HB, Dm.L, Dm.nh, HB) ||
+        !make_map_2d(&mQt, out.Qt, F16, HB, rows, HB) || !make_map_2d(&mKt, out.Kt, F16, HB, rows, HB) ||
+        !make_map_2d(&mPm, out.Pm, F16, HB, (uint64_t)Dm.nh * Dm.nblk * HB, HB) ||
+        !make_map_f32_2d(&mSd, out.Sd, BT, rows, HB))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(prep_fwd_ut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
-    prep_fwd_ut_kernel<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(
-        mW, mQ, mK, in.beta, Dm.L, Dm.nblk, static_cast<f16 *>(out.Qt), static_cast<f16 *>(out.Kt),
-        static_cast<f16 *>(out.Pm), out.Sd, out.halves, err);
+    prep_fwd_ut_kernel<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(mW, mQ, mK, mQt, mKt, mPm, mSd, in.beta,
+                                                               Dm.L, Dm.nblk, err);
     count_launches();
     return cudaGetLastError();
 }

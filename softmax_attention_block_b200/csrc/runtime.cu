@@ -12,6 +12,7 @@ namespace path {
 namespace {
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<int> g_profile{0};
+std::atomic<int> g_withhold{0};
 struct Rec {
     const char *name;
     cudaEvent_t e0, e1;
@@ -21,6 +22,8 @@ std::vector<Rec> g_recs;
 }  // namespace
 
 void count_launches(int n) { g_launches.fetch_add((unsigned long long)n); }
+
+int withhold_kv_load() { return g_withhold.load(); }
 
 Stage::Stage(const char *name, cudaStream_t st) : name_(name), st_(st)
 {
@@ -87,3 +90,10 @@ int path_profile_read(path_stage_time *out, int max_entries)
 }
 
 }  // extern "C"
+
+extern "C" path_status path_test_withhold_kv_load(int on)
+{
+    if (on != 0 && on != 1) return PATH_ERR_INVALID_ARG;
+    path::g_withhold.store(on);
+    return PATH_OK;
+}

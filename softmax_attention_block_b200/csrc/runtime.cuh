@@ -8,6 +8,9 @@ namespace path {
 
 void count_launches(int n = 1);
 
+// path_test_withhold_kv_load's setting (0 or 1).
+int withhold_kv_load();
+
 // Brackets one stage of an entry point with events when profiling is on.
 class Stage {
   public:

@@ -242,7 +242,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     }
 }
 
-constexpr uint64_t WAIT_POLLS = 500000000ull;  // bound on every in-kernel wait: 0.5 s
+constexpr uint64_t WAIT_LIMIT_NS = 500000000ull;  // bound on every in-kernel wait: 0.5 s of wall-clock time
 
 }  // namespace tc
 }  // namespace path
@@ -317,6 +317,14 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, int x,
         :
         : "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(src))
         : "memory");
+}
+
+// Asynchronous prefetch of a contiguous range into L2 (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+                 "r"(bytes)
+                 : "memory");
 }
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }

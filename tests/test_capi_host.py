@@ -81,6 +81,20 @@ def test_fwd_rejects_bad_arguments(lib):
     assert fwd(lib, wsb=100) == WORKSPACE
 
 
+def test_fwd_rejects_unaligned_tma_inputs(lib):
+    # bf16 at head dim 64 loads q, k, w by TMA: 16-byte aligned bases only
+    assert fwd(lib, q=FAKE + 2) == INVALID
+    assert fwd(lib, w=FAKE + 8) == INVALID
+    # other head dims have no such rule: validation goes on to the (missing) workspace
+    assert fwd(lib, k=FAKE + 2, d=32, ws=None) == WORKSPACE
+
+
+def test_withhold_hook_arguments(lib):
+    assert lib.path_test_withhold_kv_load(2) == INVALID
+    assert lib.path_test_withhold_kv_load(-1) == INVALID
+    assert lib.path_test_withhold_kv_load(0) == 0
+
+
 def test_grid_limits_unsupported(lib):
     # heads and 128-row blocks index launch grid dimensions (at most 65535)
     assert fwd(lib, B=256, H=256) == UNSUPPORTED

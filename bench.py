@@ -10,7 +10,8 @@ bias under "decode.gated"), and a prefill of the same sequences (forward plus th
 cache it leaves) under "prefill", and fwd+bwd at head dim 128 (B=8 H=12, the same model
 width) under "d128". The other timed workloads: the forward latency at B=2 H=4 L=1024
 ("fwd_latency"), PaTH-FoX fwd+bwd at B=1 H=24 L=16384 ("fox"), and the headline step with
-fp32 outputs and gradients ("f32out").
+fp32 outputs and gradients ("f32out"), and the w / beta prologue at the headline layer
+("wbeta").
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -440,6 +441,8 @@ def run_ours(args):
     torch.cuda.empty_cache()
     fwd_latency = None if args.no_fwd_latency else bench_fwd_latency(P, dev, peaks, world,
                                                                      max_over_ranks, barrier)
+    wbeta = None if args.no_wbeta else bench_wbeta(P, dev, peaks, world, max_over_ranks, barrier,
+                                                   args.steps)
     fox = None if args.no_fox else bench_fox(
         P, dev, peaks, world, max_over_ranks, barrier, 3,
         cpu_sample=(rank == 0 and world == 1 and not args.no_cpu_baseline))
@@ -467,7 +470,8 @@ def run_ours(args):
             "pct_bf16_peak": value / world / peaks["bf16_tflops_sustained"],
             "stages": stage_rows, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk, "decode": decode, "prefill": prefill,
-            "d128": d128, "f32out": f32out, "fwd_latency": fwd_latency, "fox": fox}
+            "d128": d128, "f32out": f32out, "fwd_latency": fwd_latency, "fox": fox,
+            "wbeta": wbeta}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -690,6 +694,67 @@ def bench_f32out(P, x, w, world, max_over_ranks, barrier, steps):
             "ms_per_step": ms, "value": whole_job_rate(world, fl, ms) / 1e12, "unit": UNIT}
 
 
+# the w / beta prologue at the headline layer: B, L, D (= H d), rank, H, d, beta clip
+WBETA = (8, 4096, 1536, 64, 24, 64, 1.99)
+
+
+def bench_wbeta(P, dev, peaks, world, max_over_ranks, barrier, steps):
+    """The w / beta prologue (low-rank layer, short convolution, L2 norm, beta) forward and
+    backward at the headline layer width, bf16 inputs and outputs. Algorithmic bytes: what
+    the step must move at least (x read by both passes, w and beta written, dw and dbeta
+    read, dx written), against the HBM copy peak."""
+    B, L, D, r, H, d, bmax = WBETA
+    g = torch.Generator().manual_seed(0)
+    rn = lambda *s: torch.randn(*s, generator=g)
+    x = rn(B, L, D).to(torch.bfloat16).to(dev)
+    A = (rn(D, r) / D ** 0.5).to(torch.bfloat16).to(dev)
+    Bw = (rn(r, H * d) / r ** 0.5).to(torch.bfloat16).to(dev)
+    f = (rn(H * d, 3) * 0.5 + torch.tensor([1.0, 0.0, 0.0])).to(dev)
+    U = (rn(D, H) * (2.0 / D ** 0.5)).to(torch.bfloat16).to(dev)
+    b = rn(H).to(dev)
+    dw = rn(B, H, L, d).to(torch.bfloat16).to(dev)
+    dbeta = rn(B, H, L).to(dev)
+    ws = torch.empty(P.path_wbeta_workspace_bytes(B, L, D, r, H, d, torch.bfloat16, True),
+                     dtype=torch.uint8, device=dev)
+    w = torch.empty((B, H, L, d), dtype=torch.bfloat16, device=dev)
+    beta = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    grads = dict(dx=torch.empty_like(x), dA=torch.empty((D, r), device=dev),
+                 dBw=torch.empty((r, H * d), device=dev), df=torch.empty((H * d, 3), device=dev),
+                 dU=torch.empty((D, H), device=dev), db=torch.empty((H,), device=dev))
+
+    def step():
+        P.path_wbeta_fwd(x, A, Bw, f, U, b, H, bmax, w=w, beta=beta, workspace=ws)
+        P.path_wbeta_bwd(x, A, Bw, f, U, b, H, dw, dbeta, bmax, grads=grads, workspace=ws,
+                         reuse_fwd_workspace=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    P.lib().path_profile_enable(1)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    P.lib().path_profile_enable(0)
+    stages = read_profile()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / steps
+    nbytes = 2 * x.numel() * 2 + w.numel() * 2 * 2 + beta.numel() * 4 * 2 + x.numel() * 2
+    del x, A, Bw, f, U, b, dw, dbeta, ws, w, beta, grads
+    torch.cuda.empty_cache()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": f"w/beta prologue fwd+bwd bf16 B={B} L={L} D={D} rank={r} H={H} d={d}",
+            "ms_per_step": ms, "value": whole_job_rate(world, B * L, ms), "unit": "tokens/s",
+            "algorithmic_bytes": nbytes,
+            "roofline": {"kernel": "whole step", "bound": "hbm", "achieved": gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "traffic": None, "peak_source": f"{peaks['source']} HBM copy"},
+            "stages_ms": {n: t / c for n, (t, c) in stages.items()}}
+
+
 D128 = (8, 12, 4096, 128)  # B, H, L, d: the headline model width (24 x 64) as 12 x 128
 
 
@@ -893,6 +958,7 @@ def main():
     ap.add_argument("--no-f32out", action="store_true")
     ap.add_argument("--no-fwd-latency", action="store_true")
     ap.add_argument("--no-fox", action="store_true")
+    ap.add_argument("--no-wbeta", action="store_true")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES) + sorted(DECODE_PROFILE_CASES)
                     + sorted(PREFILL_PROFILE_CASES),
                     help="run one untimed fwd+bwd on a small shape (for profiler captures)")

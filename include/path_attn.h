@@ -240,6 +240,44 @@ path_status path_attn_prefill(const void *q, const void *k, const void *v, const
                               size_t workspace_bytes, path_stream_t stream);
 
 /*
+ * The w / beta prologue: the model-layer step that makes the attention's w and
+ * beta from token features x (Paper-Notes "关键设计": w_t from a low-rank linear
+ * layer, a short convolution with filter size 3 and L2 normalisation;
+ * beta_t = 2 sigmoid(u^T x_t + b); gist.science section 2). Per sequence, position t,
+ * head h, channel c of the H d channels:
+ *   wt_t = (x_t A) Bw;   z_t[c] = f[c,0] wt_t[c] + f[c,1] wt_{t-1}[c] + f[c,2] wt_{t-2}[c]
+ *   (wt = 0 before the sequence start);   w_t^h = z_t^h / max(|z_t^h|, 1e-6);
+ *   beta_t^h = min(2 sigmoid(x_t . U[:, h] + b[h]), beta_max)
+ * Layouts (row-major, contiguous): x [B,L,D]; A [D,r]; Bw [r,H*d]; U [D,H] (in the
+ * input type of dt); f [H*d,3], b [H] fp32. Outputs w [B,H,L,d] (the output type of
+ * dt) and beta [B,H,L] fp32: the inputs path_attn_fwd takes. beta_max in (0, 2]
+ * (2: no clip; bf16 training clips, e.g. 1.99). d in {16, 32, 64, 128}.
+ * The low-rank products and their adjoints run as cuBLASLt GEMMs in fp32 (TF32
+ * tensor cores for bf16 inputs, which TF32 holds exactly); its scratch is part of
+ * `workspace` (path_wbeta_workspace_bytes). Errors as for path_attn_fwd.
+ */
+size_t path_wbeta_workspace_bytes(int B, int L, int D, int r, int H, int d, path_dtype dt,
+                                  int for_bwd);
+path_status path_wbeta_fwd(const void *x, const void *A, const void *Bw, const float *f,
+                           const void *U, const float *b, float beta_max, int B, int L, int D,
+                           int r, int H, int d, path_dtype dt, void *w, float *beta,
+                           void *workspace, size_t workspace_bytes, path_stream_t stream);
+/*
+ * Backward of sum(w * dw) + sum(beta * dbeta): dx [B,L,D] (output type of dt) and
+ * the parameter gradients dA [D,r], dBw [r,H*d], df [H*d,3], dU [D,H], db [H] (fp32,
+ * overwritten, summed over all B*L positions in a fixed order). dw [B,H,L,d] in the
+ * output type, dbeta [B,H,L] fp32 (e.g. path_attn_bwd's dw and dbeta). beta gets no
+ * gradient where the clip holds. flags: PATH_BWD_REUSE_FWD_WORKSPACE when
+ * `workspace` (sized for the backward) holds the matching path_wbeta_fwd's state.
+ */
+path_status path_wbeta_bwd(const void *x, const void *A, const void *Bw, const float *f,
+                           const void *U, const float *b, float beta_max, int B, int L, int D,
+                           int r, int H, int d, path_dtype dt, const void *dw, const float *dbeta,
+                           void *dx, float *dA, float *dBw, float *df, float *dU, float *db,
+                           unsigned flags, void *workspace, size_t workspace_bytes,
+                           path_stream_t stream);
+
+/*
  * Diagnostics (host-side, process-wide; not needed for normal use).
  *
  * path_kernel_launch_count: number of CUDA kernels this library has launched

@@ -22,6 +22,9 @@ Entry points (same names as the C ABI):
 - ``path_attn_workspace_bytes``, ``path_decode_workspace_bytes``, ``path_status_string``
 - diagnostics: ``path_kernel_launch_count()``, ``path_profile_enable(on)``,
   ``path_profile_read() -> {stage: (total_ms, count)}``
+- the w / beta prologue: ``path_wbeta_fwd(x, A, Bw, f, U, b, H, beta_max=2.0) -> (w, beta)``,
+  ``path_wbeta_bwd(x, A, Bw, f, U, b, H, dw, dbeta, beta_max=2.0) -> dict``,
+  ``path_wbeta_workspace_bytes``
 - test hook: ``path_test_withhold_kv_load(on)`` (makes the forward's bounded waits give up)
 """
 from __future__ import annotations
@@ -90,6 +93,14 @@ def lib() -> ctypes.CDLL:
         L.path_decode_step_noalloc.argtypes = [vp, vp, vp, vp, fp, f, i, i, i, i, i, i, vp, vp,
                                                vp, vp]
         L.path_attn_wait_status.argtypes = [vp, vp]
+        L.path_wbeta_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+        L.path_wbeta_workspace_bytes.restype = sz
+        L.path_wbeta_fwd.argtypes = [vp, vp, vp, fp, vp, fp, f, i, i, i, i, i, i, i, vp, fp, vp, sz,
+                                     vp]
+        L.path_wbeta_bwd.argtypes = [vp, vp, vp, fp, vp, fp, f, i, i, i, i, i, i, i, vp, fp, vp, fp,
+                                     fp, fp, fp, fp, ctypes.c_uint, vp, sz, vp]
+        L.path_wbeta_fwd.restype = i
+        L.path_wbeta_bwd.restype = i
         L.path_test_withhold_kv_load.argtypes = [i]
         L.path_test_withhold_kv_load.restype = i
         L.path_kernel_launch_count.restype = ctypes.c_ulonglong
@@ -396,3 +407,89 @@ def path_test_withhold_kv_load(on: bool) -> None:
     st = lib().path_test_withhold_kv_load(1 if on else 0)
     if st:
         raise PathError(st, "path_test_withhold_kv_load")
+
+
+# ---------------------------------------------------------------- the w / beta prologue
+def path_wbeta_workspace_bytes(B, L, D, r, H, d, dtype, for_bwd=False, out_dtype=None) -> int:
+    mode = _mode(dtype, out_dtype or dtype)
+    return int(lib().path_wbeta_workspace_bytes(B, L, D, r, H, d, mode, int(bool(for_bwd))))
+
+
+def _check_wbeta(x, A, Bw, f, U, b, H):
+    if x.dim() != 3 or x.dtype not in _DT:
+        raise ValueError("x must be [B,L,D], float32 or bfloat16")
+    B, L, D = x.shape
+    if A.dim() != 2 or A.shape[0] != D:
+        raise ValueError(f"A: shape {tuple(A.shape)}, expected ({D}, r)")
+    r = A.shape[1]
+    if Bw.dim() != 2 or Bw.shape[0] != r or Bw.shape[1] % H:
+        raise ValueError(f"Bw: shape {tuple(Bw.shape)}, expected ({r}, H*d) with H={H}")
+    d = Bw.shape[1] // H
+    _expect("A", A, (D, r), x.dtype)
+    _expect("Bw", Bw, (r, H * d), x.dtype)
+    _expect("U", U, (D, H), x.dtype)
+    _expect("f", f, (H * d, 3), torch.float32)
+    _expect("b", b, (H,), torch.float32)
+    return B, L, D, r, d
+
+
+def path_wbeta_fwd(x, A, Bw, f, U, b, H, beta_max=2.0, w=None, beta=None, workspace=None,
+                   out_dtype=None):
+    """w [B,H,L,d] (out_dtype, default x's dtype) and beta [B,H,L] fp32 from x [B,L,D]:
+    w = per-head L2 normalisation of the 3-tap causal convolution (filter f [H*d,3]) of
+    (x A) Bw; beta = min(2 sigmoid(x U + b), beta_max)."""
+    B, L, D, r, d = _check_wbeta(x, A, Bw, f, U, b, H)
+    od = out_dtype or x.dtype
+    if w is None:
+        w = torch.empty((B, H, L, d), dtype=od, device=x.device)
+    if beta is None:
+        beta = torch.empty((B, H, L), dtype=torch.float32, device=x.device)
+    _expect("w", w, (B, H, L, d), od)
+    _expect("beta", beta, (B, H, L), torch.float32)
+    mode = _mode(x.dtype, od)
+    _check_dev(x, A, Bw, f, U, b, w, beta, workspace)
+    nbytes = path_wbeta_workspace_bytes(B, L, D, r, H, d, x.dtype, False, od)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = lib().path_wbeta_fwd(_ptr(x), _ptr(A), _ptr(Bw), _ptr(f), _ptr(U), _ptr(b), float(beta_max),
+                              B, L, D, r, H, d, mode, _ptr(w), _ptr(beta), _ptr(ws), nbytes,
+                              _stream())
+    if st:
+        raise PathError(st, "path_wbeta_fwd")
+    return w, beta
+
+
+def path_wbeta_bwd(x, A, Bw, f, U, b, H, dw, dbeta, beta_max=2.0, grads=None, workspace=None,
+                   reuse_fwd_workspace=False):
+    """Gradients of sum(w * dw) + sum(beta * dbeta): dict dx (dw's dtype), dA, dBw, df, dU,
+    db (fp32)."""
+    if reuse_fwd_workspace and workspace is None:
+        raise ValueError("reuse_fwd_workspace needs the forward's workspace")
+    B, L, D, r, d = _check_wbeta(x, A, Bw, f, U, b, H)
+    od = dw.dtype
+    _expect("dw", dw, (B, H, L, d), od)
+    _expect("dbeta", dbeta, (B, H, L), torch.float32)
+    if grads is None:
+        dev = x.device
+        grads = dict(dx=torch.empty((B, L, D), dtype=od, device=dev),
+                     dA=torch.empty((D, r), dtype=torch.float32, device=dev),
+                     dBw=torch.empty((r, H * d), dtype=torch.float32, device=dev),
+                     df=torch.empty((H * d, 3), dtype=torch.float32, device=dev),
+                     dU=torch.empty((D, H), dtype=torch.float32, device=dev),
+                     db=torch.empty((H,), dtype=torch.float32, device=dev))
+    _expect("dx", grads["dx"], (B, L, D), od)
+    for n, shp in (("dA", (D, r)), ("dBw", (r, H * d)), ("df", (H * d, 3)), ("dU", (D, H)),
+                   ("db", (H,))):
+        _expect(n, grads[n], shp, torch.float32)
+    mode = _mode(x.dtype, od)
+    _check_dev(x, A, Bw, f, U, b, dw, dbeta, workspace, *grads.values())
+    nbytes = path_wbeta_workspace_bytes(B, L, D, r, H, d, x.dtype, True, od)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = lib().path_wbeta_bwd(_ptr(x), _ptr(A), _ptr(Bw), _ptr(f), _ptr(U), _ptr(b), float(beta_max),
+                              B, L, D, r, H, d, mode, _ptr(dw), _ptr(dbeta), _ptr(grads["dx"]),
+                              _ptr(grads["dA"]), _ptr(grads["dBw"]), _ptr(grads["df"]),
+                              _ptr(grads["dU"]), _ptr(grads["db"]),
+                              PATH_BWD_REUSE_FWD_WORKSPACE if reuse_fwd_workspace else 0, _ptr(ws),
+                              nbytes, _stream())
+    if st:
+        raise PathError(st, "path_wbeta_bwd")
+    return grads

@@ -55,7 +55,7 @@ def build(verbose: bool = False, extra_flags=()) -> str:
     if jobs or not os.path.exists(LIB):
         tmp = LIB + f".tmp{os.getpid()}"
         run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", tmp,
-             "-lcudart"])
+             "-lcudart", "-lcublasLt"])
         os.replace(tmp, LIB)
     return LIB
 

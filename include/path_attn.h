@@ -86,6 +86,20 @@ const char *path_status_string(path_status s);
  * The workspace is scratch (its contents on entry are ignored), except that
  * path_attn_bwd with PATH_BWD_REUSE_FWD_WORKSPACE reads what the forward left
  * in it. Alignment: 256 bytes.
+ * Size: with nh = B*H, nblk = ceil(L/128) and the transported-key count
+ * npairs = nblk (nblk - 1) / 2, the leading term is the stored key tiles
+ * (every key block J carried to every later query block I, fp16 at bf16 inputs,
+ * fp32 at fp32 inputs): nh * npairs * 128 * d * s bytes (s = 2 or 4), about
+ * nh * L^2 * d * s / 256 (51.5 GB at nh = 24, L = 65536, d = 64, bf16; one
+ * B200 has 180 GB). The rest grows linearly: at bf16 inputs
+ * nh * (Lp * (516 + 4 d) + L * 2 d) bytes for the forward and
+ * nh * (Lp * (1044 + 12 d) + L * 4 d) for the backward (block logits and their
+ * adjoints, boundary-adjusted queries / keys, per-position terms, 16-bit copies
+ * of v and dout; Lp = 128 nblk), plus nh * nblk * d^2 * 2 (forward) or * 6
+ * (backward) for the block products and their adjoints, each buffer rounded up
+ * to 256 bytes; a backward at a head dim other than 64 also holds the per-block
+ * scratch of its closed-form adjoint, nh * nblk * (14 * 128^2 + 3 * 128 d) * 4
+ * bytes. At nh = 24, L = 65536, d = 64, bf16 the forward needs 53.0 GB.
  */
 size_t path_attn_workspace_bytes(int B, int H, int L, int d, path_dtype dt, int for_bwd);
 
@@ -181,7 +195,11 @@ path_status path_decode_step(const void *q, const void *k_new, const void *v_new
  *   returns PATH_ERR_WORKSPACE and launches nothing. Within it, the rows per
  *   chunk grow (256, 1024, 4096 or 16384) until the partials fit.
  * - The first call on each device looks up the array's device address (with
- *   that device current); make that first call before any stream capture.
+ *   that device current); make that first call before any stream capture. The
+ *   address is kept for the life of the process: after cudaDeviceReset (or
+ *   anything else that tears down and re-creates the device's primary context)
+ *   it no longer names the array, so do not call this entry point again in a
+ *   process that has reset the device.
  * - Every call on a device shares that device's array and leaves its last
  *   contents there. Nothing in it needs clearing between calls, but calls on
  *   one device whose work overlaps on the GPU (e.g. on unordered streams)

@@ -387,27 +387,54 @@ __global__ void delta_kernel(const T *out, const T *dout, float *delta, int L, i
 }
 
 // c_t = sum_{s<=t} log f_s (fp64 running sum), padded rows repeat the last value
-__global__ void gate_prefix_kernel(const float *logf, float *c, int L, int Lp, int nh)
+// Block-wide inclusive scan of one double per thread (blockDim.x = GATE_NT).
+constexpr int GATE_NT = 1024;
+
+__device__ double block_inclusive_scan(double v)
 {
-    const int h = blockIdx.x * blockDim.x + threadIdx.x;
-    if (h >= nh) return;
-    double acc = 0.0;
-    for (int t = 0; t < Lp; ++t) {
-        if (t < L) acc += logf[(long long)h * L + t];
-        c[(long long)h * Lp + t] = (float)acc;
+    __shared__ double sh[GATE_NT];
+    sh[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = 1; o < GATE_NT; o <<= 1) {
+        const double add = threadIdx.x >= (unsigned)o ? sh[threadIdx.x - o] : 0.0;
+        __syncthreads();
+        sh[threadIdx.x] += add;
+        __syncthreads();
+    }
+    return sh[threadIdx.x];
+}
+
+// c_t = sum_{s<=t} log f_s (0 past L), accumulated in fp64: one block per head, each
+// thread a contiguous chunk of positions (chunk sums, a block scan of them, the chunk).
+__global__ void __launch_bounds__(GATE_NT) gate_prefix_kernel(const float *logf, float *c, int L, int Lp)
+{
+    const long long h = blockIdx.x;
+    const int n = (Lp + GATE_NT - 1) / GATE_NT, t0 = threadIdx.x * n, t1 = min(t0 + n, Lp);
+    const float *lf = logf + h * L;
+    double s = 0.0;
+    for (int t = t0; t < t1 && t < L; ++t) s += lf[t];
+    double acc = block_inclusive_scan(s) - s;
+    for (int t = t0; t < t1; ++t) {
+        if (t < L) acc += lf[t];
+        c[h * Lp + t] = (float)acc;
     }
 }
 
-// dlogf_s = sum_{t>=s} (rowsum_t - colsum_t)
-__global__ void gate_grad_kernel(const float *rowsum, const float *colsum, float *dlogf, int L,
-                                 int Lp, int nh)
+// dlogf_s = sum_{t>=s} (rowsum_t - colsum_t), in fp64: one block per head, thread k the
+// k-th chunk from the end.
+__global__ void __launch_bounds__(GATE_NT) gate_grad_kernel(const float *rowsum, const float *colsum,
+                                                           float *dlogf, int L, int Lp)
 {
-    const int h = blockIdx.x * blockDim.x + threadIdx.x;
-    if (h >= nh) return;
-    double acc = 0.0;
-    for (int t = L - 1; t >= 0; --t) {
-        acc += (double)rowsum[(long long)h * Lp + t] - (double)colsum[(long long)h * Lp + t];
-        dlogf[(long long)h * L + t] = (float)acc;
+    const long long h = blockIdx.x;
+    const int n = (L + GATE_NT - 1) / GATE_NT;
+    const int t1 = L - threadIdx.x * n, t0 = max(t1 - n, 0);  // chunk [t0, t1), counted from the end
+    const float *rs = rowsum + h * Lp, *cs = colsum + h * Lp;
+    double s = 0.0;
+    for (int t = t0; t < t1; ++t) s += (double)rs[t] - (double)cs[t];
+    double acc = block_inclusive_scan(s) - s;
+    for (int t = t1 - 1; t >= t0; --t) {
+        acc += (double)rs[t] - (double)cs[t];
+        dlogf[h * L + t] = (float)acc;
     }
 }
 
@@ -529,7 +556,7 @@ cudaError_t compute_delta(const BwdArgs &a, Types t, int d, cudaStream_t st)
 
 cudaError_t gate_prefix(const float *logf, float *c, int L, int Lp, int nh, cudaStream_t st)
 {
-    gate_prefix_kernel<<<ceil_div(nh, 64), 64, 0, st>>>(logf, c, L, Lp, nh);
+    gate_prefix_kernel<<<nh, GATE_NT, 0, st>>>(logf, c, L, Lp);
     count_launches();
     return cudaGetLastError();
 }
@@ -537,7 +564,7 @@ cudaError_t gate_prefix(const float *logf, float *c, int L, int Lp, int nh, cuda
 cudaError_t gate_grad(const float *rowsum, const float *colsum, float *dlogf, int L, int Lp, int nh,
                       cudaStream_t st)
 {
-    gate_grad_kernel<<<ceil_div(nh, 64), 64, 0, st>>>(rowsum, colsum, dlogf, L, Lp, nh);
+    gate_grad_kernel<<<nh, GATE_NT, 0, st>>>(rowsum, colsum, dlogf, L, Lp);
     count_launches();
     return cudaGetLastError();
 }

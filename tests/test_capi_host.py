@@ -69,6 +69,28 @@ def fwd(lib, **kw):
                              a["wsb"], None)
 
 
+def _ws_formula(nh, L, d, bwd):
+    """path_attn_workspace_bytes at bf16, restated from the header's size formula."""
+    nblk = -(-L // 128)
+    Lp, npairs = 128 * nblk, nblk * (nblk - 1) // 2
+    khat = nh * npairs * 128 * d * 2
+    lin = nh * (Lp * (1044 + 12 * d) + L * 4 * d) if bwd else nh * (Lp * (516 + 4 * d) + L * 2 * d)
+    prods = nh * nblk * d * d * (6 if bwd else 2)
+    scratch = nh * nblk * (14 * 128 * 128 + 3 * 128 * d) * 4 if bwd and d != 64 else 0
+    return khat + lin + prods + scratch
+
+
+@pytest.mark.parametrize("nh,L,d", [(24, 4096, 64), (3, 300, 64), (24, 65536, 64), (12, 4096, 128)])
+def test_workspace_follows_the_stated_formula(lib, nh, L, d):
+    for bwd in (0, 1):
+        got = lib.path_attn_workspace_bytes(1, nh, L, d, BF16, bwd)
+        ref = _ws_formula(nh, L, d, bwd)
+        # within the 256-byte rounding of each of the (at most 24) buffers
+        assert ref <= got <= ref + 24 * 256, (nh, L, d, bwd, got, ref)
+    if (nh, L) == (24, 65536):
+        assert 52.9e9 < lib.path_attn_workspace_bytes(1, 24, 65536, 64, BF16, 0) < 53.1e9
+
+
 def test_fwd_rejects_bad_arguments(lib):
     assert fwd(lib, q=None) == INVALID
     assert fwd(lib, lse=None) == INVALID

@@ -503,7 +503,7 @@ cudaError_t launch(const CUtensorMap *m, const BwdTcArgs &a, cudaStream_t st)
 
 bool attn_bwd_tc_supported(Types t, int d) { return t.in == BF16 && t.mid == F16 && d == 64; }
 
-cudaError_t attn_bwd_tc_prepare(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16,
+cudaError_t attn_bwd_tc_prepare(const BwdArgs &b, Types t, int d, float *lse_p, void *dout_bf16,
                                 cudaStream_t st)
 {
     const int Lp = b.nblk * BT;
@@ -511,7 +511,7 @@ cudaError_t attn_bwd_tc_prepare(const BwdArgs &b, Types t, float *lse_p, void *d
     row_terms_kernel<<<592, 256, 0, st>>>(b.lse, b.c, lse_p, b.delta, b.scale, b.L, Lp, b.nh);
     count_launches();
     if (t.out == F32) {
-        const long long n = (long long)b.nh * b.L * D;
+        const long long n = (long long)b.nh * b.L * d;
         f32_to_bf16_kernel<<<1184, 256, 0, st>>>(static_cast<const float *>(b.dout),
                                                  static_cast<bf16 *>(dout_bf16), n);
         count_launches();

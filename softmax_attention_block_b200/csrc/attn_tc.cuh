@@ -31,10 +31,14 @@ struct BwdTcArgs {
 bool attn_bwd_tc_supported(Types t, int d);
 // lse_p: [nh, Lp] scratch; dout_bf16: [nh, L, d] scratch (used when dout is fp32).
 // attn_bwd_tc_prepare (per-query terms, bf16 dout) runs first on the same stream.
-cudaError_t attn_bwd_tc_prepare(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16,
+cudaError_t attn_bwd_tc_prepare(const BwdArgs &b, Types t, int d, float *lse_p, void *dout_bf16,
                                 cudaStream_t st);
 cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16, int *err,
                         cudaStream_t st);
+// Head dim 128 (attn_bwd128_tc.cu): the same contract, 64-query sub-tiles.
+bool attn_bwd128_tc_supported(Types t, int d);
+cudaError_t attn_bwd128_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16, int *err,
+                           cudaStream_t st);
 
 bool attn_fwd_tc_supported(Types t, int d);
 // Key-side transport chain (fp16 tensors, d in {64, 128}).

@@ -300,18 +300,21 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
               lse,       ws.delta, ws.dQt,   ws.dKt, ws.dPm, ws.dSd,
               dv,        ws.rowsum, ws.colsum};
     const Types t = types_of(dt);
-    const bool tc = attn_bwd_tc_supported(t, d) && tc_rows_fit(y) &&
+    const bool tc = (attn_bwd_tc_supported(t, d) || attn_bwd128_tc_supported(t, d)) && tc_rows_fit(y) &&
                     !((reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(dout)) & 15u);
     if (tc) {
         {
             Stage s_d("delta", st);
             TRY(compute_delta(a, t, d, st));
-            TRY(attn_bwd_tc_prepare(a, t, ws.lse_p, ws.dout16, st));
+            TRY(attn_bwd_tc_prepare(a, t, d, ws.lse_p, ws.dout16, st));
         }
         TRY(cudaMemsetAsync(ws.dQt, 0, sizeof(float) * (size_t)y.nh * y.Lp * d, st));
         TRY(cudaMemsetAsync(ws.rowsum, 0, sizeof(float) * (size_t)y.nh * y.Lp, st));
         Stage s_b("attn_bwd", st);
-        TRY(attn_bwd_tc(a, t, ws.lse_p, ws.dout16, ws.err, st));
+        if (d == 128)
+            TRY(attn_bwd128_tc(a, t, ws.lse_p, ws.dout16, ws.err, st));
+        else
+            TRY(attn_bwd_tc(a, t, ws.lse_p, ws.dout16, ws.err, st));
     } else {
         TRY(attn_bwd_simt(a, t, d, st));
     }

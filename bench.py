@@ -58,16 +58,15 @@ def fa_equiv_flops(B, H, L, d):
 
 # fp32 FMA peak from unit counts and clocks: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz
 ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-# dense TF32 / BF16 nominal ratio (1.1 / 2.25 PFLOP/s), to derive a TF32 peak
-TF32_PER_BF16 = 1.1 / 2.25
 
 
 def stage_model(name, B, H, L, d, BT=128):
     """(algorithmic FLOP of one launch, bound) of a stage; causal, leading order.
 
     Tensor-core stages count the products of the blockwise algorithm; the UT
-    prep stages count the fp32 arithmetic of the per-block recurrences and
-    64x64 products they are made of ("tf32": products on TF32 tensor cores)."""
+    stages at head dim 64 count the 64x64x64 products their tcgen05 kernels
+    issue (fp16 operands), at other head dims the fp32 arithmetic of the
+    per-block recurrences and closed-form adjoint ("alu")."""
     nh, nblk, HB = B * H, -(-L // BT), 64
     per = {
         "attn_fwd": (2.0 * L * L * d, "tensor"),                      # QK^T + PV
@@ -77,17 +76,15 @@ def stage_model(name, B, H, L, d, BT=128):
         "attn_bwd_q": (3.0 * L * L * d, "tensor"),                    # S, dP, dQ (SIMT path)
         "attn_bwd_k": (4.0 * L * L * d + 2.0 * L * L * d * d / BT, "tensor"),
         "chain": (1.0 * L * L * d * d / BT, "tensor"),               # key-side block transport
-        # head dim 64 (tensor-core prep): per 64-half 8 products 64x64xd and a
-        # 64x128 triangular solve, then 4 products composing the 128-block;
-        # other head dims: rank-one recurrences (keys with in-block logits,
-        # queries, block product)
-        "ut_prep": ((2 * (8 * 2.0 * HB * HB * d + HB * HB * 128.0) + 4 * 2.0 * HB * HB * d, "tf32")
+        # head dim 64: per 128-block 36 products of 64x64 by 64x64 (both halves'
+        # UT in the closed form, boundary terms, the block's composition); other
+        # head dims: rank-one recurrences (keys with in-block logits, queries,
+        # block product)
+        "ut_prep": ((36 * 2.0 * HB ** 3, "tensor")
                     if d == 64 else (BT * BT / 2 * 10.0 * d + BT * 4.0 * d * d, "alu")),
-        # per 128-block: 8 products of 64x64 by 64xd (the halves' quantities come
-        # from the forward's UT prep)
-        "ut_adj_compose": (nblk * 8 * 2.0 * HB * HB * d, "tf32"),
-        # per 64-half: 22 products and two 64x128 triangular solves
-        "ut_adj64": (2 * nblk * (22 * 2.0 * HB * HB * d + 2 * HB * HB * 128.0), "tf32"),
+        # head dim 64: per 128-block 84 such products (the halves' UT recomputed,
+        # the composition's adjoint, both halves' UT adjoints)
+        "ut_adj": (nblk * 84 * 2.0 * HB ** 3, "tensor"),
         "ut_prep_bwd": (nblk * (8 * 2.0 * HB * HB * d + 4 * HB * HB * 4.0 * d
                                 + 2 * 24 * 2.0 * HB * HB * d), "alu"),
     }
@@ -101,7 +98,10 @@ def stage_model(name, B, H, L, d, BT=128):
 # B=1 H=24 L=4096 d=64 case (profiles/ summaries), scaled to the benchmark's
 # B=8 by the heads processed; None where the kernel changed since the capture.
 DRAM_BYTES_B1H24 = {
-    "attn_bwd": 325.6e6 + 95.3e6,
+    "attn_bwd": 325.6e6 + 96.1e6,
+    "attn_fwd": 274.1e6 + 9.8e6,
+    "ut_prep": 38.2e6 + 18.2e6,
+    "ut_adj": 151.6e6 + 34.0e6,
 }
 DRAM_BYTES_PREFILL_CACHE_B4H24 = 157.2e6
 
@@ -345,10 +345,6 @@ def run_ours(args):
         ach = f / (per_launch_ms * 1e-3) / 1e12 if f else None
         if bound == "alu":
             peak, src = ALU_F32_TFLOPS, "fp32 FMA from unit counts and max clock"
-        elif bound == "tf32":
-            peak = peaks["bf16_tflops_sustained"] * TF32_PER_BF16
-            src = f"{peaks['source']} bf16 dense (sustained) x nominal tf32/bf16 ratio"
-            bound = "tensor"
         else:
             peak = peaks["bf16_tflops_sustained"]
             src = f"{peaks['source']} bf16 dense (sustained)"
@@ -889,6 +885,7 @@ PROFILE_CASES = {
     # name: (B, H, L, d, log_f) -- one untimed fwd + bwd, for profiler captures
     "b1h24l4096": (1, 24, 4096, 64, False),
     "b1h6l16384fox": (1, 6, 16384, 64, True),
+    "b1h12l4096d128": (1, 12, 4096, 128, False),
 }
 # name: (B, H, d, cached rows) -- two untimed decode steps on a 16K-row cache
 DECODE_PROFILE_CASES = {

@@ -97,9 +97,10 @@ const char *path_status_string(path_status s);
  * adjoints, boundary-adjusted queries / keys, per-position terms, 16-bit copies
  * of v and dout; Lp = 128 nblk), plus nh * nblk * d^2 * 2 (forward) or * 6
  * (backward) for the block products and their adjoints, each buffer rounded up
- * to 256 bytes; a backward at a head dim other than 64 also holds the per-block
- * scratch of its closed-form adjoint, nh * nblk * (14 * 128^2 + 3 * 128 d) * 4
- * bytes. At nh = 24, L = 65536, d = 64, bf16 the forward needs 53.0 GB.
+ * to 256 bytes; a backward that is not bf16 at head dim 64 (fp32 inputs, or
+ * another head dim) also holds the per-block scratch of its closed-form adjoint,
+ * nh * nblk * (14 * 128^2 + 3 * 128 d) * 4 bytes. At nh = 24, L = 65536, d = 64,
+ * bf16 the forward needs 53.0 GB.
  */
 size_t path_attn_workspace_bytes(int B, int H, int L, int d, path_dtype dt, int for_bwd);
 

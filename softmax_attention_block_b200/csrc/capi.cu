@@ -40,10 +40,17 @@ struct AttnWs {
     // backward only
     float *delta, *dQt, *dKt, *dPm, *dSd, *rowsum, *colsum;
     float *lse_p;     // lse padded to Lp (tensor-core backward)
-    float *dP64;      // per-half block-product adjoints (fused prep adjoint)
-    float *halves = nullptr;  // 64-half quantities of the tensor-core prep (head dim 64)
     void *dout16;     // bf16 copy of an fp32 dout (tensor-core backward)
 };
+
+// bf16 inputs at head dim 64 take the tcgen05 UT kernels (prep_fwd_ut.cu,
+// prep_bwd_ut.cu), whose adjoint needs no scratch; every other case takes the
+// fp32 recurrences and the closed-form adjoint on CUDA cores (prep_fwd_rec.cu,
+// prep.cu), which hold fp32 accuracy for fp32 inputs.
+bool ut_tc_path(const Layout &y, path_dtype dt)
+{
+    return y.d == 64 && types_of(dt).in == BF16 && (long long)y.nh * y.nblk * BT < (1LL << 31);
+}
 
 // The single description of the workspace: used both to size and to carve it.
 size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &w)
@@ -62,9 +69,8 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
     // the buffers above are the forward's, at the same offsets in a forward- and a
     // backward-sized workspace (a backward may reuse the forward's); the rest only
     // the backward path that reads it gets
-    const bool split_tf32 = y.d == 64 && D.dt == F32;  // fp32, head dim 64: split-TF32 UT kernels
     if (bwd) {
-        if (y.d != 64) carve_prep_scratch(c, D, true, w.prep);
+        if (!ut_tc_path(y, dt)) carve_prep_scratch(c, D, true, w.prep);
         w.delta = c.take<float>(nh * Lp);
         w.dQt = c.take<float>(nh * Lp * d);
         w.dKt = c.take<float>(nh * Lp * d);
@@ -73,11 +79,7 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
         w.rowsum = c.take<float>(nh * Lp);
         w.colsum = c.take<float>(nh * Lp);
         w.lse_p = c.take<float>(nh * Lp);
-        w.dP64 = split_tf32 ? c.take<float>(nh * 2 * nb * d * d) : nullptr;
-        w.halves = split_tf32 ? c.take<float>(nh * nb * 4 * 64 * 64) : nullptr;
         w.dout16 = c.take<char>(nh * (size_t)y.L * d * 2);
-    } else {
-        w.dP64 = w.halves = nullptr;
     }
     return c.bytes();
 }
@@ -149,13 +151,11 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
     const Types t = types_of(dt);
     PrepDims D{y.nh, y.L, y.d, y.nblk, t.in, t.out};
     PrepInputs in{q, k, w, beta};
-    PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, t.mid, ws.halves};
+    PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, t.mid};
     {
         Stage s("ut_prep", st);
-        if (prep_forward_ut_supported(D, in))
-            TRY(prep_forward_ut(D, in, out, ws.err, st));  // no 64-half buffers: its adjoint recomputes
-        else if (prep_forward_tc_supported(D))
-            TRY(prep_forward_tc(D, in, out, st));
+        if (ut_tc_path(y, dt))
+            TRY(prep_forward_ut(D, in, out, ws.err, st));
         else
             TRY(prep_forward_rec(D, in, out, st));
     }
@@ -183,7 +183,6 @@ path_status run_forward(const void *q, const void *k, const void *v, const void 
     // reuses it needs beyond the forward's own buffers
     const bool for_bwd = workspace_bytes >= carve_attn(nullptr, y, dt, true, ws);
     carve_attn(workspace, y, dt, for_bwd, ws);
-    if (!for_bwd) ws.halves = nullptr;
     TRY(cudaMemsetAsync(ws.err, 0, sizeof(int), st));
     path_status s = run_prep_and_chain(q, k, w, beta, log_f, y, dt, ws, st);
     if (s != PATH_OK) return s;
@@ -320,12 +319,10 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
     }
     PrepDims D{y.nh, y.L, y.d, y.nblk, types_of(dt).in, types_of(dt).out};
     PrepInputs in{q, k, w, beta};
-    PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta, ws.halves};
-    if (prep_backward_ut_supported(D, in)) {
+    PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta};
+    if (ut_tc_path(y, dt)) {
         Stage s("ut_adj", st);
         TRY(prep_backward_ut(D, in, gr, ws.err, st));
-    } else if (prep_backward_fused_supported(D)) {
-        TRY(prep_backward_fused(D, in, gr, ws.dP64, st));  // times its two kernels itself
     } else {
         Stage s("ut_prep_bwd", st);
         TRY(prep_backward(D, in, ws.prep, gr, st));

@@ -1,5 +1,7 @@
-// Per-block UT transform / boundary adjustment: forward by recurrences
-// (prep_fwd_rec.cu), adjoint through the closed form (prep.cu).
+// Per-block UT transform / boundary adjustment. bf16 inputs at head dim 64: the
+// tcgen05 kernels (prep_fwd_ut.cu, prep_bwd_ut.cu). Otherwise (fp32 inputs, other
+// head dims): forward by recurrences in fp32 (prep_fwd_rec.cu), adjoint through
+// the closed form on CUDA cores (prep.cu).
 #pragma once
 #include "common.cuh"
 
@@ -21,9 +23,6 @@ struct PrepOutputs {
     void *Pm;       // [nh, nblk, d, d] block products (type tdt)
     float *Sd;      // [nh, nblk, BT, BT] diagonal-block bilinear logits (lower part)
     int tdt;
-    // optional (head dim 64, tensor-core prep): per block the 64-half quantities
-    // Ktil_a, Qtil_b, P_a, P_b ([nh, nblk, 4, 64, 64] fp32) for the backward
-    float *halves = nullptr;
 };
 
 struct PrepGrads {
@@ -32,7 +31,6 @@ struct PrepGrads {
     const float *dSd;        // [nh, nblk, BT, BT], zero above the diagonal
     void *dq, *dk, *dw;      // [nh, L, d] (type dt)
     float *dbeta;            // [nh, L]
-    const float *halves = nullptr;  // PrepOutputs::halves of the forward (fused adjoint)
 };
 
 struct PrepScratch {
@@ -47,11 +45,6 @@ size_t prep_scratch_bytes(const PrepDims &D, bool backward);
 // Qtil, Ktil, P, Sd of every 128-block, computed by per-row recurrences in fp32.
 cudaError_t prep_forward_rec(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
                              cudaStream_t st);
-// The same outputs for head dim 64, by the UT transform of each 64-position half on
-// the tensor cores (split TF32) and a 128-level composition.
-bool prep_forward_tc_supported(const PrepDims &D);
-cudaError_t prep_forward_tc(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
-                            cudaStream_t st);
 // The same outputs for head dim 64 and bf16 inputs on tcgen05 (tensor memory),
 // with (I + A)^{-1} as a product of block-diagonal and nilpotent factors
 // (prep_fwd_ut.cu). q, k, w 16-byte aligned. err: device error word.
@@ -65,11 +58,6 @@ cudaError_t prep_backward_ut(const PrepDims &D, const PrepInputs &in, const Prep
                              cudaStream_t st);
 cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
                           const PrepGrads &gr, cudaStream_t st);
-// Fused adjoint for head dim 64 (two 64-position halves per block). dQt and
-// dKt are overwritten; dP64: [nh, 2 nblk, 64, 64] scratch.
-bool prep_backward_fused_supported(const PrepDims &D);
-cudaError_t prep_backward_fused(const PrepDims &D, const PrepInputs &in, const PrepGrads &g,
-                                float *dP64, cudaStream_t st);
 cudaError_t scale_rows(const float *in, float *out, const float *beta, int L, int nblk, int batch,
                        cudaStream_t st);
 

@@ -513,6 +513,7 @@ bool prep_backward_ut_supported(const PrepDims &Dm, const PrepInputs &in)
 cudaError_t prep_backward_ut(const PrepDims &Dm, const PrepInputs &in, const PrepGrads &g, int *err,
                              cudaStream_t st)
 {
+    if (!prep_backward_ut_supported(Dm, in)) return cudaErrorInvalidValue;
     CUtensorMap m[3];
     if (!make_map_3d(&m[0], in.w, BF16, HB, Dm.L, Dm.nh, HB) ||
         !make_map_3d(&m[1], in.q, BF16, HB, Dm.L, Dm.nh, HB) ||

@@ -343,6 +343,7 @@ bool prep_forward_ut_supported(const PrepDims &Dm, const PrepInputs &in)
 cudaError_t prep_forward_ut(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out,
                             int *err, cudaStream_t st)
 {
+    if (!prep_forward_ut_supported(Dm, in)) return cudaErrorInvalidValue;
     CUtensorMap mW, mQ, mK, mQt, mKt, mPm, mSd;
     const uint64_t rows = (uint64_t)Dm.nh * Dm.nblk * BT;
     if (!make_map_3d(&mW, in.w, BF16, HB, Dm.L, Dm.nh, HB) ||

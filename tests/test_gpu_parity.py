@@ -100,10 +100,8 @@ def oracle_results(x, backward):
     return r
 
 
-def compare(ours, ref, mode, report, f32_scaled=False):
-    """ours/ref: dicts name -> array. mode: 'f32', 'bf16in_f32out' or 'bf16'.
-    f32_scaled: the fp32 bar becomes 1e-4 max(1, max|ref|), for cases built to keep
-    magnitudes large, where 1e-4 absolute asks more than fp32 arithmetic holds."""
+def compare(ours, ref, mode, report):
+    """ours/ref: dicts name -> array. mode: 'f32', 'bf16in_f32out' or 'bf16'."""
     errs, bad = {}, {}
     for n, r in ref.items():
         got = np64(ours[n])
@@ -111,8 +109,7 @@ def compare(ours, ref, mode, report, f32_scaled=False):
         errs[n] = float(diff.max()) if diff.size else 0.0
         errs[n + "/max|ref|"] = errs[n] / max(float(np.abs(r).max()), 1e-30)
         if mode == "f32":
-            scale = max(1.0, float(np.abs(r).max())) if f32_scaled and diff.size else 1.0
-            ok = errs[n] <= 1e-4 * scale
+            ok = errs[n] <= 1e-4
         elif mode == "bf16in_f32out" or n in ("lse", "dbeta"):
             ok = errs[n] <= 2e-2
         elif n in STORED_BF16:
@@ -510,14 +507,13 @@ def test_beta_zero_is_causal_softmax_attention(P, dtype, d, L):
 def test_reflections_beta_two_fp32(P):
     """beta = 2 with unit w: every H is a reflection (orthogonal), so the transported keys
     keep their norms over the whole sequence and nothing decays: dw reaches |15| here. The
-    fp32 path's products keep about 21 significant bits (split TF32), so the bar is 1e-4 of
-    the largest reference magnitude; the absolute 1e-4 of the other fp32 cases is for
-    values of order one."""
+    bar is the absolute 1e-4 of every fp32 case (plain fp32 arithmetic of the key-cache
+    recurrence stays near 8e-6 on this input)."""
     x = si.make_inputs(1, 2, 257, 64, torch.float32, seed=9, clip_beta=False)
     x["beta"] = torch.full_like(x["beta"], 2.0)
     ref = oracle_results(x, True)
     out, lse, g = run_ours(P, x, True)
-    compare(ours_dict(out, lse, g), ref, "f32", "beta=2 reflections", f32_scaled=True)
+    compare(ours_dict(out, lse, g), ref, "f32", "beta=2 reflections")
 
 
 @pytest.mark.parametrize("dtype,mode", [(torch.float32, "f32"),

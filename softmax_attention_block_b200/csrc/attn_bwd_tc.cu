@@ -5,25 +5,29 @@
 // for S^T, dP^T, dV and the chain adjoint Abar. Per tile pair:
 //   MMA 1:  S^T  = Khat_{J,I} Qtil_I^T          (fp16)
 //           dP^T = V_J dO_I^T                    (bf16)
-//           issued right after the previous pair's MMA 2, whose launch waits for
-//           the softmax to have consumed that pair's S^T / dP^T
 //   threads: P = exp(scale S + c_i - c_j - lse_i), dZ = P (dP - delta_i),
-//            dS = scale dZ; P^T (bf16) and dS^T (fp16) to shared memory;
+//            dS = scale dZ; P^T (bf16) into tensor memory over the S^T columns
+//            already read, dS^T (fp16) to shared memory (two buffers);
 //            [gate] row sums of dS by warp reduce-scatter, column sums per thread
-//   MMA 2:  dV   += P^T dO_I                              (bf16)
-//           dP_I += Abar_{I+1}^T Khat_{J,I}                (fp16; operand
-//                   [Abar | Khat] so the M=128 form applies, top half kept)
+//   MMA 2:  dV   += P^T dO_I                   (bf16, A = P^T from tensor memory)
+//           dP_I += Abar_{I+1}^T Khat_{J,I}     (fp16; operand [Abar | Khat] so
+//                   the M=128 form applies, top half kept)
 //           Abar  = Abar_{I+1} P_I + dS^T Qtil_I           (fp16, fp32 in TMEM)
 //           dQtil_I += dS Khat_{J,I}                       (fp16)
 // Khat_{J,I+1} = Khat_{J,I} P_I^T, so Abar is the adjoint carried back along
-// the key-side transport chain; after the pair (J+1, J) it is dKtil_J. dQtil
-// and dP are staged in shared memory by the drain warps and accumulate across
-// CTAs by TMA tensor reduce-add; the gate's row sums by fp32 atomics.
-// The diagonal tile takes its logits from the UT prep and writes dS to the
-// prep's adjoint instead (dSd), which carries it to dQ, dK, dW, dbeta.
+// the key-side transport chain; after the pair (J+1, J) it is dKtil_J. dQtil is
+// staged in the pair's spent dS^T buffer by the drain warps and accumulates
+// across CTAs by TMA tensor reduce-add; dP_I by fp32 vector atomics; the gate's
+// row sums by fp32 atomics. The diagonal tile takes its logits from the UT prep
+// and writes dS to the prep's adjoint instead (dSd), which carries it to dQ,
+// dK, dW, dbeta.
 //
-// Every accumulator has its own TMEM columns, so MMA 1 of the next pair and
-// the softmax on its results run while the drain empties this pair's MMA 2.
+// Issue order of the MMA warp per pair: dV (reads this pair's P^T), the next
+// pair's MMA 1 (overwrites S^T / P^T and dP^T: the tensor pipe runs one
+// thread's MMAs in issue order), then the rest of MMA 2. So the softmax of the
+// next pair runs while the rest of this pair's MMA 2 executes, and the drain of
+// this pair's results runs under the softmax after it. The operand stage goes
+// back to the producer when the MMAs that read it complete.
 #include <type_traits>
 
 #include "attn.cuh"
@@ -50,18 +54,22 @@ struct BCfg {
     static constexpr int TILE = 128 * D * 2;     // 16 KB
     static constexpr int AB_OFF = 0;             // Abar operand (fp16), before the stages
     static constexpr int V_OFF = AB_OFF + TILE;
-    static constexpr int PT_OFF = V_OFF + TILE;  // P^T  [keys x queries] bf16, 2 panels
-    static constexpr int DS_OFF = PT_OFF + 2 * 16384;  // dS^T [keys x queries] fp16
-    static constexpr int ST_OFF = DS_OFF + 2 * 16384;
+    // dS^T [keys x queries] fp16, 2 panels of 64 queries; two buffers (pairs it % 2),
+    // each the fp32 staging of that pair's dQtil once MMA 2 has read it
+    static constexpr int DS_BYTES = 2 * 16384;
+    static constexpr int DS_OFF = V_OFF + TILE;
+    static constexpr int ST_OFF = DS_OFF + 2 * DS_BYTES;
     // stage: Khat, Qtil, dO, P_I (8 KB), rows (lse, delta, c: 3 x 512 B)
     static constexpr int S_KH = 0, S_Q = TILE, S_DO = 2 * TILE, S_P = 3 * TILE, S_ROW = 3 * TILE + 8192;
     static constexpr int ST_BYTES = 3 * TILE + 8192 + 2048;
     static constexpr int CS_OFF = ST_OFF + 2 * ST_BYTES;  // [128] column-sum exchange
     static constexpr int BAR_OFF = CS_OFF + 512;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
-    // TMEM columns: no two accumulators share columns
+    // TMEM columns: no two accumulators share columns; P^T (packed bf16) sits in
+    // the S^T columns, query block q (16 queries) at column 64 (q / 4) + 8 (q % 4)
     static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_AB = 320, T_DQ = 384, T_DPI = 448;
 };
+static_assert(BCfg::SMEM <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ void named_barrier(int id, int nthreads)
 {
@@ -78,18 +86,19 @@ __global__ void __launch_bounds__(NT, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                   const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mDO,
                   const __grid_constant__ CUtensorMap mP, const __grid_constant__ CUtensorMap mDQ,
-                  const __grid_constant__ CUtensorMap mDPI, BwdTcArgs a)
+                  BwdTcArgs a)
 {
     using C = BCfg;
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
-    uint8_t *sAb = sm + C::AB_OFF, *sV = sm + C::V_OFF, *sPt = sm + C::PT_OFF, *sDs = sm + C::DS_OFF;
+    uint8_t *sAb = sm + C::AB_OFF, *sV = sm + C::V_OFF, *sDs = sm + C::DS_OFF;
     float *sCs = reinterpret_cast<float *>(sm + C::CS_OFF);
     auto stage = [&](int s) { return sm + C::ST_OFF + s * C::ST_BYTES; };
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::BAR_OFF);
     uint64_t *v_full = bars, *ld_full = bars + 1, *ld_empty = bars + 3, *s_full = bars + 5,
-             *p_full = bars + 7, *m2_full = bars + 8, *e_done = bars + 9;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
+             *p_full = bars + 7, *m2_full = bars + 8, *e_done = bars + 9, *ds_free = bars + 10,
+             *mma_done = bars + 12;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
 
     // key tiles along x: the CTAs of one head run together and share its Q, dO
     // tiles in L2 (heads along x, longest tiles first, measured slower)
@@ -109,6 +118,9 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_init(p_full, NEW);
         mbar_init(m2_full, 1);
         mbar_init(e_done, NDR);
+        mbar_init(&ds_free[0], 1);
+        mbar_init(&ds_free[1], 1);
+        mbar_init(mma_done, 1);
         mbar_fence_init();
     }
     if (warp == W_MMA) tmem_alloc(tmem_slot, 512);
@@ -122,8 +134,20 @@ __global__ void __launch_bounds__(NT, 1)
             mbar_expect_tx(v_full, C::TILE);
             tma_load_3d(sV, &mV, 0, J * BT, h, v_full);
             int issued = 0;
+            // the tiles of pair it into L2 (its loads are issued two pairs later, when
+            // its stage comes back, and then read L2 instead of HBM)
+            auto prefetch = [&](int it) {
+                const int I = tile_of(it);
+                if (it != niter - 1) {
+                    tma_prefetch_2d(&mK, 0, (int)((h * a.npairs + (long long)I * (I - 1) / 2 + J) * BT));
+                    tma_prefetch_2d(&mQ, 0, h * Lp + I * BT);
+                    if (I < last) tma_prefetch_2d(&mP, 0, (h * nblk + I) * D);
+                }
+                tma_prefetch_3d(&mDO, 0, I * BT, h);
+            };
             for (int it = 0; it < niter; ++it) {
                 const int s = it & 1;
+                if (it + 2 < niter) prefetch(it + 2);
                 if (it >= 2 && !mbar_wait(&ld_empty[s], ((it >> 1) - 1) & 1, WAIT_LIMIT_NS)) {
                     if (a.err) atomicCAS(a.err, 0, 11);
                     break;
@@ -158,8 +182,7 @@ __global__ void __launch_bounds__(NT, 1)
             const uint32_t idDV = idesc_f16(128, D, AB_BF16, 0, 1);
             const uint32_t idAbP = idesc_f16(128, D, AB_F16, 0, 1);
             const uint32_t idMN = idesc_f16(128, D, AB_F16, 1, 1);
-            const uint32_t ab0 = smem_u32(sAb), v0 = smem_u32(sV), pt0 = smem_u32(sPt),
-                           ds0 = smem_u32(sDs);
+            const uint32_t ab0 = smem_u32(sAb), v0 = smem_u32(sV);
             // MMA 1 of pair it: S^T = Khat Qtil^T (not on the diagonal), dP^T = V dO^T
             auto mma1 = [&](int it) -> bool {
                 const int s = it & 1;
@@ -185,23 +208,32 @@ __global__ void __launch_bounds__(NT, 1)
             for (int it = 0; ok && it < niter; ++it) {
                 const int s = it & 1, I = tile_of(it);
                 const bool diag = it == niter - 1;
-                // MMA 2 needs this pair's P / dS in shared memory, and overwrites the
-                // previous pair's results: drained by then?
-                const bool ready = mbar_wait(p_full, it & 1, WAIT_LIMIT_NS) &&
-                                   (it == 0 || mbar_wait(e_done, (it - 1) & 1, WAIT_LIMIT_NS));
-                if (!__all_sync(0xffffffffu, ready)) {  // the warp stays converged
+                // this pair's P^T (tensor memory) and dS^T (shared memory) are written
+                if (!__all_sync(0xffffffffu, mbar_wait(p_full, it & 1, WAIT_LIMIT_NS))) {
                     ok = false;
                     break;
                 }
                 fence_after_sync();
                 const uint32_t kh0 = smem_u32(stage(s) + C::S_KH), q0 = smem_u32(stage(s) + C::S_Q),
-                               do0 = smem_u32(stage(s) + C::S_DO), p0 = smem_u32(stage(s) + C::S_P);
-                // dV += P^T dO   (K = 128 queries)
+                               do0 = smem_u32(stage(s) + C::S_DO), p0 = smem_u32(stage(s) + C::S_P),
+                               ds0 = smem_u32(sDs + s * C::DS_BYTES);
+                // dV += P^T dO   (K = 128 queries, A from tensor memory)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss_if(lead, tbase + C::T_DV, desc_sw128(pt0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                           desc_sw128(do0 + kk * 2048, 16384, 1024), idDV, (it > 0 || kk > 0));
+                    mma_ts_if(lead, tbase + C::T_DV, tbase + C::T_S + 64 * (kk >> 2) + 8 * (kk & 3),
+                              desc_sw128(do0 + kk * 2048, 16384, 1024), idDV, (it > 0 || kk > 0));
+                // the next pair's MMA 1 overwrites the P^T just read (in issue order)
+                if (it + 1 < niter && !mma1(it + 1)) {
+                    ok = false;
+                    break;
+                }
                 if (!diag) {
+                    // the drain has taken the previous pair's Abar, dQtil, dP_I out
+                    if (!__all_sync(0xffffffffu, it == 0 || mbar_wait(e_done, (it - 1) & 1, WAIT_LIMIT_NS))) {
+                        ok = false;
+                        break;
+                    }
+                    fence_after_sync();
                     if (I < last) {
                         // dP_I (+)= [Abar | Khat]^T Khat  (rows 0..63 = Abar^T Khat)
                         const uint32_t lbo = kh0 - ab0;
@@ -226,16 +258,14 @@ __global__ void __launch_bounds__(NT, 1)
                         mma_ss_if(lead, tbase + C::T_DQ, desc_sw128(ds0 + kk * 2048, 16384, 1024),
                                desc_sw128(kh0 + kk * 2048, 16384, 1024), idMN, kk > 0);
                 }
-                commit_if(lead, m2_full);  // the drain frees the stage after using it
-                // the next pair's MMA 1 (S^T / dP^T were consumed before this MMA 2);
-                // its completion also orders the next softmax's P / dS writes after
-                // this MMA 2's reads
-                if (it + 1 < niter && !mma1(it + 1)) {
-                    ok = false;
-                    break;
-                }
+                commit_if(lead, m2_full);
+                commit_if(lead, &ld_empty[s]);  // the stage's operands are read once these complete
             }
             if (!ok && lead && a.err) atomicCAS(a.err, 0, 12);
+            // every MMA this warp issued completes before the CTA frees tensor memory
+            commit_if(lead, mma_done);
+            if (!__all_sync(0xffffffffu, mbar_wait(mma_done, 0, WAIT_LIMIT_NS)) && lead && a.err)
+                atomicCAS(a.err, 0, 15);
         }
     } else if (warp < W_DRAIN0) {
         // softmax warpgroups: warpgroup g takes query columns [64g, 64g + 64);
@@ -247,33 +277,24 @@ __global__ void __launch_bounds__(NT, 1)
         const float k1 = a.scale * LOG2E;
         const float cj2 = FOX ? a.c[(long long)h * Lp + gj] * LOG2E : 0.f;
         float colsum = 0.f;
-        bool ok = true;
+        bool ok = true, ds_late = false;
         for (int it = 0; it < niter; ++it) {
             const int s = it & 1, I = tile_of(it);
             const bool diag = it == niter - 1;
-            // s_full also orders this pair's P / dS writes after the previous MMA 2
+            // s_full: this pair's S^T / dP^T are in tensor memory, and the previous pair's
+            // dV products, which read P^T from the columns written below, have completed
             if (ok && (!mbar_wait(&ld_full[s], (it >> 1) & 1, WAIT_LIMIT_NS) ||
                        !mbar_wait(s_full, it & 1, WAIT_LIMIT_NS)))
                 ok = false;
-            ok = __all_sync(0xffffffffu, ok);  // shuffles and TMEM loads below are warp-wide
+            ok = __all_sync(0xffffffffu, ok);  // shuffles and TMEM accesses below are warp-wide
             fence_after_sync();
             const float *rows = reinterpret_cast<const float *>(stage(s) + C::S_ROW);
             const float *sd = a.Sd + ((long long)h * nblk + J) * BT * BT;
             float *dsd = a.dSd + ((long long)h * nblk + J) * BT * BT;
-            // one 16-column chunk; the diagonal tile (logits from the UT prep, causal
-            // mask, dS also to the prep's adjoint) is its own instantiation
-            auto chunk = [&](auto dg, int c) {
+            uint8_t *sDsb = sDs + s * C::DS_BYTES;
+            // one 16-column chunk: sv / dp hold S and dP on entry, P and dS on exit
+            auto chunk = [&](auto dg, int c, float (&sv)[16], float (&dp)[16]) {
                 constexpr bool DG = decltype(dg)::value;
-                float sv[16], dp[16];
-                if (DG) {
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) sv[u] = sd[(c + u) * BT + j];
-                } else {
-                    tmem_ld16(tbase + C::T_S + c + lane_off, sv);
-                }
-                tmem_ld16(tbase + C::T_DP + c + lane_off, dp);
-                tmem_wait_ld_tied(sv, dp);
-                float pv[16], dsv[16];
                 const float4 *nb4 = reinterpret_cast<const float4 *>(rows + c);
                 const float4 *sd4 = reinterpret_cast<const float4 *>(rows + 128 + c);
 #pragma unroll
@@ -287,30 +308,36 @@ __global__ void __launch_bounds__(NT, 1)
                         float p = ex2(x);
                         if (DG && i < j) p = 0.f;
                         const float ds = p * fmaf(dp[u], a.scale, -sdv[e]);
-                        pv[u] = p;
-                        dsv[u] = ds;
+                        sv[u] = p;
+                        dp[u] = ds;
                         if (DG) dsd[(long long)i * BT + j] = ds;
                     }
                 }
                 uint32_t pb[8], db[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const __nv_bfloat162 bb = __floats2bfloat162_rn(pv[2 * k], pv[2 * k + 1]);
+                    const __nv_bfloat162 bb = __floats2bfloat162_rn(sv[2 * k], sv[2 * k + 1]);
                     pb[k] = *reinterpret_cast<const uint32_t *>(&bb);
-                    const __half2 hh = __floats2half2_rn(dsv[2 * k], dsv[2 * k + 1]);
+                    const __half2 hh = __floats2half2_rn(dp[2 * k], dp[2 * k + 1]);
                     db[k] = *reinterpret_cast<const uint32_t *>(&hh);
                 }
+                // P^T of these 16 queries: 8 packed columns, inside the S^T columns this
+                // warpgroup has already read
+                tmem_st8(tbase + C::T_S + 64 * g + ((c & 63) >> 1) + lane_off, pb);
+                // before the first dS^T store: the drain's staging of pair it - 2 has
+                // left this buffer (a wait that gives up flags the error; the stores go on)
+                if ((c & 63) == 0 && it >= 2 && !mbar_wait(&ds_free[s], ((it >> 1) - 1) & 1, WAIT_LIMIT_NS))
+                    ds_late = true;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const uint32_t off = (c >> 6) * 16384 + sw128_offset(j, (c & 63) + 8 * hf);
-                    *reinterpret_cast<uint4 *>(sPt + off) =
-                        make_uint4(pb[4 * hf], pb[4 * hf + 1], pb[4 * hf + 2], pb[4 * hf + 3]);
-                    *reinterpret_cast<uint4 *>(sDs + off) =
+                    *reinterpret_cast<uint4 *>(sDsb + off) =
                         make_uint4(db[4 * hf], db[4 * hf + 1], db[4 * hf + 2], db[4 * hf + 3]);
                 }
                 if (FOX) {
                     // gate: row and column sums of the same fp16-rounded dS that the
                     // MMAs read, so the crossing sums in the gate gradient cancel
+                    float *dsv = dp;
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const float2 f2 = __half22float2(*reinterpret_cast<const __half2 *>(&db[k]));
@@ -334,13 +361,38 @@ __global__ void __launch_bounds__(NT, 1)
                         atomicAdd(a.rowsum + (long long)h * Lp + I * BT + c + (lane >> 1), dsv[0] / a.scale);
                 }
             };
-#pragma unroll 1
-            for (int c = 64 * g; ok && c < 64 * g + 64; c += 16) {
+            // the four chunks of this warpgroup, the next chunk's loads in flight while
+            // one is computed; the diagonal tile (logits from the UT prep, causal mask,
+            // dS also to the prep's adjoint) is its own instantiation
+            auto pass = [&](auto dg) {
+                constexpr bool DG = decltype(dg)::value;
+                float sv[2][16], dp[2][16];
+                auto load = [&](int b, int c) {
+                    if (DG) {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) sv[b][u] = sd[(c + u) * BT + j];
+                    } else {
+                        tmem_ld16(tbase + C::T_S + c + lane_off, sv[b]);
+                    }
+                    tmem_ld16(tbase + C::T_DP + c + lane_off, dp[b]);
+                };
+                load(0, 64 * g);
+                tmem_wait_ld_tied(sv[0], dp[0]);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int b = q4 & 1, c = 64 * g + 16 * q4;
+                    if (q4 < 3) load(b ^ 1, c + 16);
+                    chunk(dg, c, sv[b], dp[b]);
+                    if (q4 < 3) tmem_wait_ld_tied(sv[b ^ 1], dp[b ^ 1]);
+                }
+            };
+            if (ok) {
                 if (diag)
-                    chunk(std::true_type{}, c);
+                    pass(std::true_type{});
                 else
-                    chunk(std::false_type{}, c);
+                    pass(std::false_type{});
             }
+            tmem_wait_st();
             fence_async_smem();
             fence_before_sync();
             mbar_arrive(p_full);
@@ -348,19 +400,20 @@ __global__ void __launch_bounds__(NT, 1)
         // column sums: warpgroup 1 hands its half to warpgroup 0
         if (g == 1) sCs[j] = colsum;
         named_barrier(1, NEW);
-        if (!ok && a.err) atomicCAS(a.err, 0, 13);
+        if ((!ok || ds_late) && a.err) atomicCAS(a.err, 0, 13);
         if (ok && g == 0 && a.colsum && gj < a.L) a.colsum[(long long)h * Lp + gj] = (colsum + sCs[j]) / a.scale;
     } else if (warp < W_PROD) {
         // drain warpgroup: thread j = lane j of TMEM (key row for Abar and dV, query
         // row for dQtil, row f < 64 of dP_I); all 64 columns of each result.
-        // dQtil and dP_I leave through fp32 staging (128B-swizzled boxes of 32
-        // columns) in this pair's operand stage, free once MMA 2 has completed,
-        // and bulk tensor reduce-add; the stage goes back to the producer after the
-        // reductions have read it.
+        // dQtil leaves through fp32 staging (128B-swizzled boxes of 32 columns) in
+        // this pair's dS^T buffer, spent once MMA 2 has completed, and bulk tensor
+        // reduce-add; the buffer goes back to the softmax after the reduction has
+        // read it. dP_I leaves by fp32 vector atomics.
         const int j = tid - 32 * W_DRAIN0;
         const int gj = J * BT + j;
         const bool leader = j == 0;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        float dpv[2][32];  // this thread's row of dP_I
         bool ok = true;
         for (int it = 0; it < niter; ++it) {
             const int s = it & 1, I = tile_of(it);
@@ -368,8 +421,28 @@ __global__ void __launch_bounds__(NT, 1)
             if (ok && !mbar_wait(m2_full, it & 1, WAIT_LIMIT_NS)) ok = false;
             ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-wide
             fence_after_sync();
-            uint8_t *stq = stage(s), *stp = stage(s) + 2 * 16384;  // dQtil: 2 x 16 KB, dP_I: 2 x 8 KB
+            uint8_t *stq = sDs + s * C::DS_BYTES;  // dQtil: 2 x 16 KB
             const bool drain = ok && !diag;
+            if (drain) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    // dQtil rows of tile I (lane = query row)
+                    float v[32];
+                    tmem_ld32(tbase + C::T_DQ + c0 + lane_off, v);
+                    uint8_t *box = stq + (c0 >> 5) * 16384 + j * 128;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        *reinterpret_cast<float4 *>(box + ((k ^ (j & 7)) << 4)) =
+                            make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                }
+                fence_async_smem();
+            }
+            named_barrier(2, NDR);  // every staging row written: the reduction starts first
+            if (leader && drain) {
+                tma_reduce_add_2d(&mDQ, 0, h * Lp + I * BT, stq);
+                tma_reduce_add_2d(&mDQ, 32, h * Lp + I * BT, stq + 16384);
+                bulk_commit();
+            }
             if (drain) {
 #pragma unroll 1
                 for (int c0 = 0; c0 < D; c0 += 32) {
@@ -392,50 +465,27 @@ __global__ void __launch_bounds__(NT, 1)
                             *reinterpret_cast<float4 *>(dk + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
                     }
                 }
-#pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    // dQtil rows of tile I (lane = query row)
-                    float v[32];
-                    tmem_ld32(tbase + C::T_DQ + c0 + lane_off, v);
-                    uint8_t *box = stq + (c0 >> 5) * 16384 + j * 128;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        *reinterpret_cast<float4 *>(box + ((k ^ (j & 7)) << 4)) =
-                            make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-                }
                 if (I < last) {
-                    // dP_I rows f = 0..63 live in lanes 0..63 (the first two warps)
-#pragma unroll 1
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        float v[32];
-                        tmem_ld32(tbase + C::T_DPI + c0 + lane_off, v);
-                        if (j < D) {
-                            uint8_t *box = stp + (c0 >> 5) * 8192 + j * 128;
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                *reinterpret_cast<float4 *>(box + ((k ^ (j & 7)) << 4)) =
-                                    make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-                        }
-                    }
+                    // dP_I rows f = 0..63 live in lanes 0..63 (the first two warps);
+                    // they leave by atomics once the tensor memory is released
+                    tmem_ld32(tbase + C::T_DPI + lane_off, dpv[0]);
+                    tmem_ld32(tbase + C::T_DPI + 32 + lane_off, dpv[1]);
                 }
                 fence_async_smem();
             }
             // TMEM results read and Abar written: MMA 2 of the next pair may go
             fence_before_sync();
             mbar_arrive(e_done);
-            named_barrier(2, NDR);  // every staging row written
+            if (drain && I < last && j < D) {
+                float4 *dpi = reinterpret_cast<float4 *>(a.dPm + (((long long)h * nblk + I) * D + j) * D);
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    atomicAdd(dpi + k, make_float4(dpv[k >> 3][4 * (k & 7)], dpv[k >> 3][4 * (k & 7) + 1],
+                                                   dpv[k >> 3][4 * (k & 7) + 2], dpv[k >> 3][4 * (k & 7) + 3]));
+            }
             if (leader) {
-                if (drain) {
-                    tma_reduce_add_2d(&mDQ, 0, h * Lp + I * BT, stq);
-                    tma_reduce_add_2d(&mDQ, 32, h * Lp + I * BT, stq + 16384);
-                    if (I < last) {
-                        tma_reduce_add_2d(&mDPI, 0, (h * nblk + I) * D, stp);
-                        tma_reduce_add_2d(&mDPI, 32, (h * nblk + I) * D, stp + 8192);
-                    }
-                    bulk_commit();
-                    bulk_wait_read<0>();
-                }
-                mbar_arrive(&ld_empty[s]);  // the producer may refill this stage
+                if (drain) bulk_wait_read<0>();
+                mbar_arrive(&ds_free[s]);  // the softmax may write this dS^T buffer again
             }
         }
         if (leader) bulk_wait_all();
@@ -494,7 +544,7 @@ cudaError_t launch(const CUtensorMap *m, const BwdTcArgs &a, cudaStream_t st)
     auto k = bwd_tc_kernel<FOX, TO>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BCfg::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<dim3(a.nblk, a.nh), NT, BCfg::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], a);
+    k<<<dim3(a.nblk, a.nh), NT, BCfg::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], a);
     count_launches();
     return cudaGetLastError();
 }
@@ -525,7 +575,7 @@ cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16
     const int Lp = b.nblk * BT;
     const long long npairs = (long long)b.nblk * (b.nblk - 1) / 2;
     const void *dob = t.out == F32 ? dout_bf16 : b.dout;
-    CUtensorMap m[7];
+    CUtensorMap m[6];
     if (!make_map_2d(&m[0], b.Qt, F16, D, (uint64_t)b.nh * Lp, 128)) return cudaErrorInvalidValue;
     if (npairs > 0) {
         if (!make_map_2d(&m[1], b.Khat, F16, D, (uint64_t)b.nh * npairs * BT, 128)) return cudaErrorInvalidValue;
@@ -535,8 +585,7 @@ cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16
     if (!make_map_3d(&m[2], b.v, BF16, D, b.L, b.nh, 128) ||
         !make_map_3d(&m[3], dob, BF16, D, b.L, b.nh, 128) ||
         !make_map_2d(&m[4], b.Pm, F16, D, (uint64_t)b.nh * b.nblk * D, D) ||
-        !make_map_f32_2d(&m[5], b.dQt, D, (uint64_t)b.nh * Lp, 128) ||
-        !make_map_f32_2d(&m[6], b.dPm, D, (uint64_t)b.nh * b.nblk * D, 64))
+        !make_map_f32_2d(&m[5], b.dQt, D, (uint64_t)b.nh * Lp, 128))
         return cudaErrorInvalidValue;
     BwdTcArgs a{b.Sd, b.c, lse_p, b.delta, b.scale, b.L, b.nblk, b.nh, npairs,
                 b.dQt, b.dKt, b.dPm, b.dSd, b.dv, b.rowsum, b.colsum, err};

@@ -82,6 +82,21 @@ __device__ __forceinline__ void mma_ss_if(uint32_t issue, uint32_t tmem_d, uint6
         : "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(issue));
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, A (M x K, K-major) read from tensor memory:
+// row m in lane m, 16-bit elements k, k+1 packed low / high in column k / 2.
+// Issued like mma_ss_if.
+__device__ __forceinline__ void mma_ts_if(uint32_t issue, uint32_t tmem_d, uint32_t tmem_a,
+                                          uint64_t bdesc, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %5, 0;\n\t"
+        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+        :
+        : "r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(issue));
+}
+
 // commit() by the threads with `issue` != 0 only (the lane that issued the MMAs).
 __device__ __forceinline__ void commit_if(uint32_t issue, uint64_t *bar)
 {
@@ -173,6 +188,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16])
           "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
         : "r"(taddr));
 }
+
+// 8 consecutive 32-bit columns of this thread's lane (addressing as tmem_ld32);
+// complete once tmem_wait_st() returns.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+        :
+        : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Waits for this thread's TMEM loads; the registers of `a` and `b` are tied to
 // the wait, so no use of them can be scheduled before it (needed when loads
@@ -324,6 +353,22 @@ __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
 {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
                  "r"(bytes)
+                 : "memory");
+}
+
+// L2 prefetch of the tile a tma_load_2d / tma_load_3d with the same map and
+// coordinates would copy (no shared memory, no completion signal).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, int y)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, int y, int z)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z)
                  : "memory");
 }
 

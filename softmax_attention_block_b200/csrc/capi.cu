@@ -44,9 +44,11 @@ struct AttnWs {
 };
 
 // bf16 inputs at head dim 64 take the tcgen05 UT kernels (prep_fwd_ut.cu,
-// prep_bwd_ut.cu), whose adjoint needs no scratch; every other case takes the
-// fp32 recurrences and the closed-form adjoint on CUDA cores (prep_fwd_rec.cu,
-// prep.cu), which hold fp32 accuracy for fp32 inputs.
+// prep_bwd_ut.cu), whose adjoint needs no scratch. Other bf16 cases take the
+// closed form by batched products on the tensor cores in TF32 (prep.cu,
+// gemm_tc.cu), forward and adjoint; fp32 inputs take the fp32 recurrences
+// forward and the closed-form adjoint on CUDA cores (prep_fwd_rec.cu, prep.cu,
+// gemm_batched.cu), which hold fp32 accuracy.
 bool ut_tc_path(const Layout &y, path_dtype dt)
 {
     return y.d == 64 && types_of(dt).in == BF16 && (long long)y.nh * y.nblk * BT < (1LL << 31);
@@ -69,8 +71,10 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
     // the buffers above are the forward's, at the same offsets in a forward- and a
     // backward-sized workspace (a backward may reuse the forward's); the rest only
     // the backward path that reads it gets
+    // closed-form scratch: the backward's adjoint, and the forward of bf16 inputs
+    // (fp32 inputs take the recurrences forward)
+    if (!ut_tc_path(y, dt) && (bwd || D.dt != F32)) carve_prep_scratch(c, D, bwd, w.prep);
     if (bwd) {
-        if (!ut_tc_path(y, dt)) carve_prep_scratch(c, D, true, w.prep);
         w.delta = c.take<float>(nh * Lp);
         w.dQt = c.take<float>(nh * Lp * d);
         w.dKt = c.take<float>(nh * Lp * d);
@@ -154,10 +158,14 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
     PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, t.mid};
     {
         Stage s("ut_prep", st);
-        if (ut_tc_path(y, dt))
+        if (ut_tc_path(y, dt)) {
             TRY(prep_forward_ut(D, in, out, ws.err, st));
-        else
+        } else if (D.dt != F32) {
+            ws.prep.err = ws.err;
+            TRY(prep_forward_gemm(D, in, out, ws.prep, st));
+        } else {
             TRY(prep_forward_rec(D, in, out, st));
+        }
     }
     ChainArgs ca{ws.Kt, ws.Pm, ws.Khat, y.nblk, y.nh};
     {
@@ -325,6 +333,7 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
         TRY(prep_backward_ut(D, in, gr, ws.err, st));
     } else {
         Stage s("ut_prep_bwd", st);
+        ws.prep.err = ws.err;
         TRY(prep_backward(D, in, ws.prep, gr, st));
     }
     if (log_f) {

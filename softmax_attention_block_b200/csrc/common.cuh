@@ -131,9 +131,14 @@ struct GemmArgs {
     int c_seq = -1;          // if >= 0: output rows with blk*BT + r >= c_seq are not written
     int nblk = 1;
     int batch = 1;           // number of batch items (heads * nblk)
+    int *err = nullptr;      // device error word (tensor-core version: a wait that gave up)
 };
 
-// Launches the batched GEMM on `stream`. Returns cudaGetLastError().
+// Launches the batched GEMM on `stream` (fp32 on CUDA cores). Returns cudaGetLastError().
 cudaError_t gemm_batched(const GemmArgs &g, cudaStream_t stream);
+// The same product on the tensor cores in TF32 (gemm_tc.cu), for M, N, K <= 128,
+// multiples of 4, operands addressable four elements at a time.
+bool gemm_tc_supported(const GemmArgs &g);
+cudaError_t gemm_batched_tc(const GemmArgs &g, cudaStream_t stream);
 
 }  // namespace path

@@ -22,10 +22,10 @@ __device__ __forceinline__ float op_elem(const Operand &o, long long base, int r
     return load_as_f(o.p, o.dt, base + (long long)sr * o.ld + sc);
 }
 
-__global__ void __launch_bounds__(256) gemm_batched_kernel(GemmArgs g)
+__global__ void __launch_bounds__(256, 4) gemm_batched_kernel(GemmArgs g)
 {
-    __shared__ float As[TK][TM + 4];
-    __shared__ float Bs[TK][TN + 4];
+    __shared__ float As[TK][TM + 1];
+    __shared__ float Bs[TK][TN + 1];
     const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
     for (int z = blockIdx.z; z < g.batch; z += gridDim.z) {
@@ -38,13 +38,32 @@ __global__ void __launch_bounds__(256) gemm_batched_kernel(GemmArgs g)
         const long long bbase = (long long)h * T.b.sh + (long long)blk * T.b.sb;
         float part[4][4] = {};
         for (int k0 = 0; k0 < g.K; k0 += TK) {
-            for (int e = threadIdx.x; e < TK * TM; e += 256) {
-                const int kk = e / TM, mm = e % TM;
-                As[kk][mm] = op_elem(T.a, abase, m0 + mm, k0 + kk, blk, g.M, g.K);
+            // consecutive threads take consecutive stored elements (coalesced)
+            if (T.a.trans) {  // stored [k][m]
+#pragma unroll 1
+                for (int e = threadIdx.x; e < TK * TM; e += 256) {
+                    const int kk = e / TM, mm = e % TM;
+                    As[kk][mm] = op_elem(T.a, abase, m0 + mm, k0 + kk, blk, g.M, g.K);
+                }
+            } else {          // stored [m][k]
+#pragma unroll 1
+                for (int e = threadIdx.x; e < TK * TM; e += 256) {
+                    const int kk = e % TK, mm = e / TK;
+                    As[kk][mm] = op_elem(T.a, abase, m0 + mm, k0 + kk, blk, g.M, g.K);
+                }
             }
-            for (int e = threadIdx.x; e < TK * TN; e += 256) {
-                const int kk = e / TN, nn = e % TN;
-                Bs[kk][nn] = op_elem(T.b, bbase, k0 + kk, n0 + nn, blk, g.K, g.N);
+            if (T.b.trans) {  // stored [n][k]
+#pragma unroll 1
+                for (int e = threadIdx.x; e < TK * TN; e += 256) {
+                    const int kk = e % TK, nn = e / TK;
+                    Bs[kk][nn] = op_elem(T.b, bbase, k0 + kk, n0 + nn, blk, g.K, g.N);
+                }
+            } else {          // stored [k][n]
+#pragma unroll 1
+                for (int e = threadIdx.x; e < TK * TN; e += 256) {
+                    const int kk = e / TN, nn = e % TN;
+                    Bs[kk][nn] = op_elem(T.b, bbase, k0 + kk, n0 + nn, blk, g.K, g.N);
+                }
             }
             __syncthreads();
 #pragma unroll

@@ -19,8 +19,13 @@ namespace path {
 
 namespace {
 
-// Tinv = (I + A)^{-1} for strictly lower A (forward substitution, one block
-// per CTA), and X = Tinv diag(beta).
+// Tinv = (I + A)^{-1} for strictly lower A, and X = Tinv diag(beta), one block
+// per CTA, by forward substitution in 16 x 16 blocks: the eight diagonal blocks
+// first (their own 16-step substitutions, side by side), then block row I,
+// I = 1..7: S_IJ = sum_{K=J}^{I-1} A_IK Tinv_KJ for every J < I, and
+// Tinv_IJ = -Tinv_II S_IJ. Every output of a step is an independent dot
+// product, so a step is one pass of the CTA.
+constexpr int TB = 16, NTB = BT / TB;
 __global__ void __launch_bounds__(256) tri_inverse_kernel(const float *A, float *Tinv, float *X,
                                                           const float *beta, int L, int nblk,
                                                           int batch)
@@ -28,29 +33,53 @@ __global__ void __launch_bounds__(256) tri_inverse_kernel(const float *A, float 
     extern __shared__ float sm[];
     float *sA = sm;              // [BT][BT]
     float *sT = sm + BT * BT;    // [BT][BT]
-    __shared__ float part[2][BT];
+    float *sS = sT + BT * BT;    // [NTB - 1][TB][TB] block sums of one block row
     for (int z = blockIdx.x; z < batch; z += gridDim.x) {
         const int h = z / nblk, blk = z % nblk;
         const long long base = (long long)z * BT * BT;
-        for (int e = threadIdx.x; e < BT * BT; e += blockDim.x) {
-            sA[e] = A[base + e];
-            sT[e] = 0.f;
+        for (int e = threadIdx.x; e < BT * BT / 4; e += blockDim.x) {
+            reinterpret_cast<float4 *>(sA)[e] = reinterpret_cast<const float4 *>(A + base)[e];
+            reinterpret_cast<float4 *>(sT)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         __syncthreads();
-        const int c = threadIdx.x % BT, half = threadIdx.x / BT;
-        if (half == 0) sT[c * BT + c] = 1.f;
-        __syncthreads();
-        for (int i = 1; i < BT; ++i) {
-            // row i, column c < i: -sum_{k=c}^{i-1} A[i][k] Tinv[k][c]; k split in two halves
-            float s = 0.f;
-            if (c < i) {
-                const int mid = (c + i) / 2;
-                const int k0 = half == 0 ? c : mid, k1 = half == 0 ? mid : i;
-                for (int k = k0; k < k1; ++k) s = fmaf(sA[i * BT + k], sT[k * BT + c], s);
+        // diagonal blocks: thread (block I, column c) runs the 16-step substitution
+        if (threadIdx.x < BT) {
+            const int I = threadIdx.x / TB, c = threadIdx.x % TB, o = I * TB;
+            float t[TB];
+#pragma unroll
+            for (int r = 0; r < TB; ++r) {
+                float s = r == c ? 1.f : 0.f;
+#pragma unroll
+                for (int k = 0; k < r; ++k) s = fmaf(-sA[(o + r) * BT + o + k], t[k], s);
+                t[r] = r < c ? 0.f : s;
             }
-            part[half][c] = s;
+#pragma unroll
+            for (int r = 0; r < TB; ++r) sT[(o + r) * BT + o + c] = t[r];
+        }
+        __syncthreads();
+        for (int I = 1; I < NTB; ++I) {
+            // S_IJ[r][c] = sum_{K=J}^{I-1} sum_m A_IK[r][m] Tinv_KJ[m][c]; Tinv_KJ = 0 for K < J
+            for (int e = threadIdx.x; e < I * TB * TB; e += blockDim.x) {
+                const int J = e / (TB * TB), r = (e / TB) % TB, c = e % TB;
+                const float *arow = sA + (I * TB + r) * BT;
+                float s0 = 0.f, s1 = 0.f;
+                for (int k = J * TB; k < I * TB; k += 2) {
+                    s0 = fmaf(arow[k], sT[k * BT + J * TB + c], s0);
+                    s1 = fmaf(arow[k + 1], sT[(k + 1) * BT + J * TB + c], s1);
+                }
+                sS[e] = s0 + s1;
+            }
             __syncthreads();
-            if (half == 0 && c < i) sT[i * BT + c] = -(part[0][c] + part[1][c]);
+            // Tinv_IJ = -Tinv_II S_IJ
+            for (int e = threadIdx.x; e < I * TB * TB; e += blockDim.x) {
+                const int J = e / (TB * TB), r = (e / TB) % TB, c = e % TB;
+                const float *trow = sT + (I * TB + r) * BT + I * TB;
+                const float *scol = sS + J * TB * TB + c;
+                float s = 0.f;
+#pragma unroll
+                for (int m = 0; m < TB; ++m) s = fmaf(trow[m], scol[m * TB], s);
+                sT[(I * TB + r) * BT + J * TB + c] = -s;
+            }
             __syncthreads();
         }
         for (int e = threadIdx.x; e < BT * BT; e += blockDim.x) {
@@ -195,6 +224,15 @@ static void out_blk(GemmArgs &g, const PrepDims &D, float *p, int rows, int cols
         if (e_ != cudaSuccess) return e_;     \
     } while (0)
 
+// bf16 / fp16 inputs: the products on the tensor cores in TF32; fp32 inputs: fp32
+// on CUDA cores (the fp32 mode's precision)
+static cudaError_t gemm(const PrepDims &D, GemmArgs g, const PrepScratch &s, cudaStream_t st)
+{
+    g.err = s.err;
+    if (D.dt != F32 && gemm_tc_supported(g)) return gemm_batched_tc(g, st);
+    return gemm_batched(g, st);
+}
+
 size_t prep_scratch_bytes(const PrepDims &D, bool backward)
 {
     Carver c(nullptr);
@@ -239,17 +277,17 @@ static cudaError_t prep_core(const PrepDims &D, const PrepInputs &in, const Prep
         GemmArgs g = base_args(D, BT, BT, d);
         term(g, W, T_(W), 1.f);
         out_blk(g, D, s.G, BT, BT);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
         g.rowscale = in.beta;
         g.rs_sh = L;
         g.rs_sb = BT;
         g.rs_seq = L;
         out_blk(g, D, s.A, BT, BT, MASK_STRICT_LOWER);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
     }
     {
         const int batch = D.nh * nb;
-        const size_t smem = 2 * BT * BT * sizeof(float);
+        const size_t smem = (2 * BT * BT + (NTB - 1) * TB * TB) * sizeof(float);
         CK(cudaFuncSetAttribute(tri_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem));
         tri_inverse_kernel<<<grid_for(batch), 256, smem, st>>>(s.A, s.Tinv, s.X, in.beta, L, nb,
@@ -262,25 +300,72 @@ static cudaError_t prep_core(const PrepDims &D, const PrepInputs &in, const Prep
         GemmArgs g = base_args(D, BT, d, BT);
         term(g, X, W, 1.f);
         out_blk(g, D, s.What, BT, d);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
     }
     {   // N = strictLower(W K^T)
         GemmArgs g = base_args(D, BT, BT, d);
         term(g, W, T_(K), 1.f);
         out_blk(g, D, s.N, BT, BT, MASK_STRICT_LOWER);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
     }
     {   // U = X N
         GemmArgs g = base_args(D, BT, BT, BT);
         term(g, X, blk_mat(s.N, F32, nb, BT, BT), 1.f);
         out_blk(g, D, s.U, BT, BT);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
     }
     {   // M = lower(Q W^T)
         GemmArgs g = base_args(D, BT, BT, d);
         term(g, Q, T_(W), 1.f);
         out_blk(g, D, s.M, BT, BT, MASK_LOWER);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
+    }
+    return cudaSuccess;
+}
+
+cudaError_t prep_forward_gemm(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
+                              const PrepScratch &s, cudaStream_t st)
+{
+    CK(prep_core(D, in, s, st));
+    const int L = D.L, d = D.d, nb = D.nblk, Lp = nb * BT;
+    const Operand W = user_rows(in.w, D.dt, L, d), K = user_rows(in.k, D.dt, L, d),
+                  Q = user_rows(in.q, D.dt, L, d);
+    const Operand U = blk_mat(s.U, F32, nb, BT, BT), M = blk_mat(s.M, F32, nb, BT, BT),
+                  What = blk_mat(s.What, F32, nb, BT, d);
+    {   // P = I - W^T What
+        GemmArgs g = base_args(D, d, d, BT);
+        term(g, T_(W), What, -1.f);
+        g.add_identity = 1;
+        set_out(g, out.Pm, out.tdt, (long long)nb * d * d, (long long)d * d, d, -1);
+        CK(gemm(D, g, s, st));
+    }
+    {   // Qtil = Q - M What (rows past L: zero)
+        GemmArgs g = base_args(D, BT, d, BT);
+        term(g, M, What, -1.f);
+        g.addend = Q;
+        g.gamma = 1.f;
+        set_out(g, out.Qt, out.tdt, (long long)Lp * d, (long long)BT * d, d, -1);
+        CK(gemm(D, g, s, st));
+    }
+    {   // Ktil = K - U^T W
+        GemmArgs g = base_args(D, BT, d, BT);
+        term(g, T_(U), W, -1.f);
+        g.addend = K;
+        g.gamma = 1.f;
+        set_out(g, out.Kt, out.tdt, (long long)Lp * d, (long long)BT * d, d, -1);
+        CK(gemm(D, g, s, st));
+    }
+    {   // Sd = lower(Q K^T - M U)
+        GemmArgs g = base_args(D, BT, BT, d);
+        term(g, Q, T_(K), 1.f);
+        out_blk(g, D, out.Sd, BT, BT);
+        CK(gemm(D, g, s, st));
+        GemmArgs g2 = base_args(D, BT, BT, BT);
+        term(g2, M, U, -1.f);
+        g2.addend = blk_mat(out.Sd, F32, nb, BT, BT);
+        g2.gamma = 1.f;
+        out_blk(g2, D, out.Sd, BT, BT, MASK_LOWER);
+        CK(gemm(D, g2, s, st));
     }
     return cudaSuccess;
 }
@@ -309,13 +394,13 @@ cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScr
         GemmArgs g = base_args(D, BT, BT, BT);
         term(g, dSl, T_(U), -1.f);
         out_blk(g, D, s.dM, BT, BT, MASK_LOWER);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
         GemmArgs g2 = base_args(D, BT, BT, d);
         term(g2, dQt, T_(What), -1.f);
         g2.addend = dM;
         g2.gamma = 1.f;
         out_blk(g2, D, s.dM, BT, BT, MASK_LOWER);
-        CK(gemm_batched(g2, st));
+        CK(gemm(D, g2, s, st));
     }
     {   // dq = dQt + dSl K + dM W
         GemmArgs g = base_args(D, BT, d, BT);
@@ -324,25 +409,25 @@ cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScr
         g.addend = dQt;
         g.gamma = 1.f;
         set_out(g, gr.dq, D.odt, ush, usb, d, L);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
     }
     {   // dU = -M^T dSl - W dKt^T
         GemmArgs g = base_args(D, BT, BT, BT);
         term(g, T_(M), dSl, -1.f);
         out_blk(g, D, s.dU, BT, BT);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
         GemmArgs g2 = base_args(D, BT, BT, d);
         term(g2, W, T_(dKt), -1.f);
         g2.addend = dU;
         g2.gamma = 1.f;
         out_blk(g2, D, s.dU, BT, BT);
-        CK(gemm_batched(g2, st));
+        CK(gemm(D, g2, s, st));
     }
     {   // dN = strictLower(X^T dU)
         GemmArgs g = base_args(D, BT, BT, BT);
         term(g, T_(X), dU, 1.f);
         out_blk(g, D, s.dN, BT, BT, MASK_STRICT_LOWER);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
     }
     {   // dk = dKt + dSl^T Q + dN^T W
         GemmArgs g = base_args(D, BT, d, BT);
@@ -351,41 +436,41 @@ cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScr
         g.addend = dKt;
         g.gamma = 1.f;
         set_out(g, gr.dk, D.odt, ush, usb, d, L);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
     }
     {   // dWhat = -M^T dQt - W dP
         GemmArgs g = base_args(D, BT, d, BT);
         term(g, T_(M), dQt, -1.f);
         out_blk(g, D, s.dWhat, BT, d);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
         GemmArgs g2 = base_args(D, BT, d, d);
         term(g2, W, dP, -1.f);
         g2.addend = dWhat;
         g2.gamma = 1.f;
         out_blk(g2, D, s.dWhat, BT, d);
-        CK(gemm_batched(g2, st));
+        CK(gemm(D, g2, s, st));
     }
     {   // dX = dU N^T + dWhat W^T
         GemmArgs g = base_args(D, BT, BT, BT);
         term(g, dU, T_(Nm), 1.f);
         out_blk(g, D, s.dX, BT, BT);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
         GemmArgs g2 = base_args(D, BT, BT, d);
         term(g2, dWhat, T_(W), 1.f);
         g2.addend = dX;
         g2.gamma = 1.f;
         out_blk(g2, D, s.dX, BT, BT);
-        CK(gemm_batched(g2, st));
+        CK(gemm(D, g2, s, st));
     }
     {   // dA = strictLower(-(Tinv^T dX) X^T)   (adjoint of Tinv = (I + A)^{-1}, X = Tinv D)
         GemmArgs g = base_args(D, BT, BT, BT);
         term(g, T_(Tinv), dX, 1.f);
         out_blk(g, D, s.tmp, BT, BT);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
         GemmArgs g2 = base_args(D, BT, BT, BT);
         term(g2, tmp, T_(X), -1.f);
         out_blk(g2, D, s.dA, BT, BT, MASK_STRICT_LOWER);
-        CK(gemm_batched(g2, st));
+        CK(gemm(D, g2, s, st));
     }
     // dG = strictLower(D dA): dA is strictly lower already, scale its rows by beta
     CK(scale_rows(s.dA, s.dG, in.beta, L, nb, D.nh * nb, st));
@@ -402,13 +487,13 @@ cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScr
         term(g, dN, K, 1.f);
         term(g, T_(dM), Q, 1.f);
         out_blk(g, D, s.dWacc, BT, d);
-        CK(gemm_batched(g, st));
+        CK(gemm(D, g, s, st));
         GemmArgs g2 = base_args(D, BT, d, d);
         term(g2, What, T_(dP), -1.f);
         g2.addend = dWacc;
         g2.gamma = 1.f;
         out_blk(g2, D, s.dWacc, BT, d);
-        CK(gemm_batched(g2, st));
+        CK(gemm(D, g2, s, st));
         GemmArgs g3 = base_args(D, BT, d, BT);
         term(g3, T_(X), dWhat, 1.f);
         term(g3, dGm, W, 1.f);
@@ -416,7 +501,7 @@ cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScr
         g3.addend = dWacc;
         g3.gamma = 1.f;
         set_out(g3, gr.dw, D.odt, ush, usb, d, L);
-        CK(gemm_batched(g3, st));
+        CK(gemm(D, g3, s, st));
     }
     return cudaSuccess;
 }

@@ -38,6 +38,7 @@ struct PrepScratch {
           *M = nullptr, *What = nullptr;
     float *dM = nullptr, *dU = nullptr, *dN = nullptr, *dX = nullptr, *tmp = nullptr,
           *dA = nullptr, *dG = nullptr, *dWhat = nullptr, *dWacc = nullptr;
+    int *err = nullptr;  // device error word of the call
 };
 
 void carve_prep_scratch(Carver &c, const PrepDims &D, bool backward, PrepScratch &s);
@@ -56,6 +57,10 @@ cudaError_t prep_forward_ut(const PrepDims &D, const PrepInputs &in, const PrepO
 bool prep_backward_ut_supported(const PrepDims &D, const PrepInputs &in);
 cudaError_t prep_backward_ut(const PrepDims &D, const PrepInputs &in, const PrepGrads &g, int *err,
                              cudaStream_t st);
+// The same outputs from the closed form by batched products (bf16 inputs at head
+// dims other than 64; TF32 tensor cores), through the forward part of `s`.
+cudaError_t prep_forward_gemm(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
+                              const PrepScratch &s, cudaStream_t st);
 cudaError_t prep_backward(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
                           const PrepGrads &gr, cudaStream_t st);
 cudaError_t scale_rows(const float *in, float *out, const float *beta, int L, int nblk, int batch,

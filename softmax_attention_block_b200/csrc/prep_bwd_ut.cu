@@ -139,15 +139,22 @@ __global__ void __launch_bounds__(NT, 1)
     const float *dsdb = dSd + ((long long)hd * nblk + J) * BT * BT;
 
     if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_fence_init();
+        mbar_expect_tx(&bars[0], 6 * TILE);
+        for (int h = 0; h < 2; ++h) {
+            const int y = J * BT + h * HB;
+            tma_load_3d(tile(T_W + 2 * h), &mW, 0, y, hd, &bars[0]);
+            tma_load_3d(tile(T_K + 2 * h), &mK, 0, y, hd, &bars[0]);
+            tma_load_3d(tile(T_Q + h), &mQ, 0, y, hd, &bars[0]);
+        }
         // every fp32 adjoint this block reads, on its way to L2 while the
         // halves' transforms are recomputed
         prefetch_l2(dQt + brow * HB, BT * HB * 4);
         prefetch_l2(dKt + brow * HB, BT * HB * 4);
         prefetch_l2(dPm + ((long long)hd * nblk + J) * HB * HB, HB * HB * 4);
         prefetch_l2(dsdb, BT * BT * 4);
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        mbar_fence_init();
     }
     if (warp == 0) tmem_alloc(tslot, 512);
     // E^{-1} tiles (only their diagonal blocks are written below) and the identity
@@ -169,15 +176,6 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = *tslot;
-    if (tid == 0) {
-        mbar_expect_tx(&bars[0], 6 * TILE);
-        for (int h = 0; h < 2; ++h) {
-            const int y = J * BT + h * HB;
-            tma_load_3d(tile(T_W + 2 * h), &mW, 0, y, hd, &bars[0]);
-            tma_load_3d(tile(T_K + 2 * h), &mK, 0, y, hd, &bars[0]);
-            tma_load_3d(tile(T_Q + h), &mQ, 0, y, hd, &bars[0]);
-        }
-    }
     bool ok = mbar_wait(&bars[0], 0, WAIT_LIMIT_NS);
     ok = __syncthreads_and(ok);
 
@@ -398,6 +396,7 @@ __global__ void __launch_bounds__(NT, 1)
         mma64(dst(tbase, hh, C_DQ), ta(T_DS + hh), A_N, ta(T_K + 2 * hh), B_N, 1, TILE, false);
         mma64(dst(tbase, hh, C_DQ), ta(T_M + hh), A_N, ta(T_W + 2 * hh), B_N, 1, TILE, true);
     });
+    ld_global(dQt + (brow + h * HB + r) * HB + c0, x);  // in flight during the MMAs
     wait_mma();
     const long long grow = (long long)hd * L + (long long)J * BT + h * HB + r;  // row in [nh, L]
     const bool valid = J * BT + h * HB + r < L;
@@ -411,7 +410,6 @@ __global__ void __launch_bounds__(NT, 1)
         st_tile_f16(tile(T_P + h), r, c0, v);    // dN = strictLower(D dR_n)
         // dq = dQ + dS K + dM W
         me.ld(tbase, C_DQ, v);
-        ld_global(dQt + (brow + h * HB + r) * HB + c0, x);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] += x[j];
         if (valid) st_global(dq + grow * HB + c0, v);
@@ -427,6 +425,8 @@ __global__ void __launch_bounds__(NT, 1)
         mma64(dst(tbase, hh, C_DKK), ta(T_P + hh), A_T, w, B_N, 1, TILE, true);
         mma64(dst(tbase, hh, C_GN2), w, A_N, w, B_T, 2, TILE, false);
     });
+    float xk[32];
+    ld_global(dKt + (brow + h * HB + r) * HB + c0, xk);  // in flight during the MMAs
     wait_mma();
     if (ok) {
         // dbeta_r = dR_w[r].W[r] + dR_n[r].N[r] + sum_c dA[r][c] G[r][c]
@@ -451,9 +451,8 @@ __global__ void __launch_bounds__(NT, 1)
         sPart[me.cg * BT + h * HB + r] = s;
         // dk = dK + dS^T Q + dN^T W
         me.ld(tbase, C_DKK, v);
-        ld_global(dKt + (brow + h * HB + r) * HB + c0, x);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] += x[j];
+        for (int j = 0; j < 32; ++j) v[j] += xk[j];
         if (valid) st_global(dk + grow * HB + c0, v);
     }
     sync_operands();

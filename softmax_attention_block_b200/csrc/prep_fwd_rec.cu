@@ -14,6 +14,8 @@
 // Sd_tj = q_t . k_j after every step (the in-place key update of the
 // inference paragraph, applied inside the block); thread i carries q_i
 // through H_i, ..., H_s; thread c carries column c of I through H_s, ..., H_e.
+// The three roles are separate CTAs of 128 threads, so that a thread's vector
+// of up to 128 fp32 values stays in registers.
 // Positions past the sequence end have beta = 0 and w = 0 (H = I).
 #include "prep.cuh"
 #include "runtime.cuh"
@@ -24,8 +26,9 @@ namespace {
 
 template <int D>
 struct RecCfg {
-    static constexpr int NT = 2 * BT + (D < 32 ? 32 : D);  // keys, queries, P columns
-    static constexpr int MIN_CTAS = D <= 32 ? 2 : 1;
+    // one role per CTA (grid z: 0 keys, 1 queries, 2 columns of P), one vector
+    // of D fp32 values per thread, kept in registers
+    static constexpr int NT = BT;
     static constexpr int LDS = D + 4;  // shared row stride: 16-byte rows for vector reads
 };
 
@@ -64,17 +67,17 @@ __device__ __forceinline__ void apply_h(float (&x)[D], const float *sW, const fl
 }
 
 template <typename T, typename TM, int D>
-__global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
+__global__ void __launch_bounds__(RecCfg<D>::NT)
     prep_fwd_rec_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ w,
                         const float *__restrict__ beta, int L, int nblk, TM *Qt, TM *Kt, TM *Pm,
-                        float *Sd)
+                        float *Sd, int role0)
 {
     constexpr int LDS = RecCfg<D>::LDS;
     extern __shared__ __align__(16) float sm[];
     float *sW = sm;              // [BT][D+4]
-    float *sQ = sW + BT * LDS;   // [BT][D+4]
-    float *sB = sQ + BT * LDS;   // [BT]
-    const int J = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    float *sB = sW + BT * LDS;   // [BT]
+    float *sQ = sB + BT;         // [BT][D+4], keys role only
+    const int J = blockIdx.x, h = blockIdx.y, role = role0 + blockIdx.z, tid = threadIdx.x;
     const int Lp = nblk * BT;
     const long long row0 = (long long)h * L + (long long)J * BT;  // first row of the block in [nh, L]
     const int nvalid = min(BT, L - J * BT);
@@ -82,12 +85,12 @@ __global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
         const int r = e / D, c = e % D;
         const bool ok = r < nvalid;
         sW[r * LDS + c] = ok ? to_f(w[(row0 + r) * D + c]) : 0.f;
-        sQ[r * LDS + c] = ok ? to_f(q[(row0 + r) * D + c]) : 0.f;
+        if (role == 0) sQ[r * LDS + c] = ok ? to_f(q[(row0 + r) * D + c]) : 0.f;
     }
     for (int r = tid; r < BT; r += blockDim.x) sB[r] = r < nvalid ? beta[row0 + r] : 0.f;
     __syncthreads();
 
-    if (tid < BT) {
+    if (role == 0) {
         // keys: Ktil and the diagonal-block logits
         const int j = tid;
         float x[D];
@@ -109,12 +112,12 @@ __global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
         TM *dst = Kt + ((long long)h * Lp + (long long)J * BT + j) * D;
 #pragma unroll
         for (int c = 0; c < D; ++c) dst[c] = from_f<TM>(x[c]);
-    } else if (tid < 2 * BT) {
+    } else if (role == 1) {
         // queries: Qtil_i = H_s ... H_i q_i (apply H_i first)
-        const int i = tid - BT;
+        const int i = tid;
         float x[D];
 #pragma unroll
-        for (int c = 0; c < D; ++c) x[c] = sQ[i * LDS + c];
+        for (int c = 0; c < D; ++c) x[c] = i < nvalid ? to_f(q[(row0 + i) * D + c]) : 0.f;
         for (int t = (i | 31); t >= 0; --t)
             if (t <= i) apply_h<D>(x, sW, sB, t);
         TM *dst = Qt + ((long long)h * Lp + (long long)J * BT + i) * D;
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
         for (int c = 0; c < D; ++c) dst[c] = from_f<TM>(x[c]);
     } else {
         // block product P = H_e ... H_s, one column per thread
-        const int col = tid - 2 * BT;
+        const int col = tid;
         if (col < D) {
             float x[D];
 #pragma unroll
@@ -138,16 +141,22 @@ __global__ void __launch_bounds__(RecCfg<D>::NT, RecCfg<D>::MIN_CTAS)
 template <typename T, typename TM, int D>
 cudaError_t run(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out, cudaStream_t st)
 {
-    const size_t smem = (2 * BT * RecCfg<D>::LDS + BT) * sizeof(float);
+    // keys (W, beta and Q in shared memory), then queries and P columns (W, beta)
+    const size_t smem_w = (BT * RecCfg<D>::LDS + BT) * sizeof(float);
+    const size_t smem_k = smem_w + BT * RecCfg<D>::LDS * sizeof(float);
     auto kern = prep_fwd_rec_kernel<T, TM, D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(Dm.nblk, Dm.nh), RecCfg<D>::NT, smem, st>>>(
-        static_cast<const T *>(in.q), static_cast<const T *>(in.k), static_cast<const T *>(in.w),
-        in.beta, Dm.L, Dm.nblk, static_cast<TM *>(out.Qt), static_cast<TM *>(out.Kt),
-        static_cast<TM *>(out.Pm), out.Sd);
-    count_launches();
-    return cudaGetLastError();
+    for (int role0 = 0; role0 < 2; ++role0) {
+        kern<<<dim3(Dm.nblk, Dm.nh, role0 == 0 ? 1 : 2), RecCfg<D>::NT, role0 == 0 ? smem_k : smem_w, st>>>(
+            static_cast<const T *>(in.q), static_cast<const T *>(in.k), static_cast<const T *>(in.w),
+            in.beta, Dm.L, Dm.nblk, static_cast<TM *>(out.Qt), static_cast<TM *>(out.Kt),
+            static_cast<TM *>(out.Pm), out.Sd, role0);
+        count_launches();
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 template <int D>

@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(NT, 1)
                        const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mQt,
                        const __grid_constant__ CUtensorMap mKt, const __grid_constant__ CUtensorMap mPm,
                        const __grid_constant__ CUtensorMap mSd, const float *beta, int L, int nblk,
-                       int *err)
+                       int nsm, int *err)
 {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
@@ -98,6 +98,25 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
         mbar_fence_init();
+        // rows past L read as zero (w = 0, beta = 0: H = I there)
+        mbar_expect_tx(&bars[0], 6 * TILE);
+        for (int h = 0; h < 2; ++h) {
+            const int y = J * BT + h * HB;
+            tma_load_3d(tile(h ? T_WB : T_WA), &mW, 0, y, hd, &bars[0]);
+            tma_load_3d(tile(h ? T_KB : T_KA), &mK, 0, y, hd, &bars[0]);
+            tma_load_3d(tile(h ? T_QB : T_QA), &mQ, 0, y, hd, &bars[0]);
+        }
+        // one CTA per SM, started in grid order: the block nsm places further on
+        // starts on an SM this wave frees; its inputs go to L2 meanwhile
+        const long long n2 = (long long)hd * nblk + J + nsm;
+        if (n2 < (long long)nblk * gridDim.y) {
+            const int J2 = (int)(n2 % nblk), h2 = (int)(n2 / nblk);
+            for (int h = 0; h < 2; ++h) {
+                tma_prefetch_3d(&mW, 0, J2 * BT + h * HB, h2);
+                tma_prefetch_3d(&mK, 0, J2 * BT + h * HB, h2);
+                tma_prefetch_3d(&mQ, 0, J2 * BT + h * HB, h2);
+            }
+        }
     }
     if (warp == 0) tmem_alloc(tslot, 512);
     // the E^{-1} tiles: only their diagonal blocks are written below
@@ -111,16 +130,6 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = *tslot;
-    if (tid == 0) {
-        // rows past L read as zero (w = 0, beta = 0: H = I there)
-        mbar_expect_tx(&bars[0], 6 * TILE);
-        for (int h = 0; h < 2; ++h) {
-            const int y = J * BT + h * HB;
-            tma_load_3d(tile(h ? T_WB : T_WA), &mW, 0, y, hd, &bars[0]);
-            tma_load_3d(tile(h ? T_KB : T_KA), &mK, 0, y, hd, &bars[0]);
-            tma_load_3d(tile(h ? T_QB : T_QA), &mQ, 0, y, hd, &bars[0]);
-        }
-    }
     bool ok = mbar_wait(&bars[0], 0, WAIT_LIMIT_NS);
     ok = __syncthreads_and(ok);
 
@@ -356,7 +365,7 @@ cudaError_t prep_forward_ut(const PrepDims &Dm, const PrepInputs &in, const Prep
     cudaError_t e = cudaFuncSetAttribute(prep_fwd_ut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
     prep_fwd_ut_kernel<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(mW, mQ, mK, mQt, mKt, mPm, mSd, in.beta,
-                                                               Dm.L, Dm.nblk, err);
+                                                               Dm.L, Dm.nblk, sm_count(), err);
     count_launches();
     return cudaGetLastError();
 }

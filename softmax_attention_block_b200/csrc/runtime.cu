@@ -25,6 +25,20 @@ void count_launches(int n) { g_launches.fetch_add((unsigned long long)n); }
 
 int withhold_kv_load() { return g_withhold.load(); }
 
+int sm_count()
+{
+    static std::atomic<int> cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int n = cache[dev].load();
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            return 148;
+        cache[dev].store(n);
+    }
+    return n;
+}
+
 Stage::Stage(const char *name, cudaStream_t st) : name_(name), st_(st)
 {
     if (!g_profile.load()) return;

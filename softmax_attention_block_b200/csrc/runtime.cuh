@@ -11,6 +11,10 @@ void count_launches(int n = 1);
 // path_test_withhold_kv_load's setting (0 or 1).
 int withhold_kv_load();
 
+// Streaming multiprocessors of the current device (cached per device; 148 if
+// the query fails).
+int sm_count();
+
 // Brackets one stage of an entry point with events when profiling is on.
 class Stage {
   public:

@@ -76,7 +76,9 @@ def _ws_formula(nh, L, d, bwd):
     khat = nh * npairs * 128 * d * 2
     lin = nh * (Lp * (1044 + 12 * d) + L * 4 * d) if bwd else nh * (Lp * (516 + 4 * d) + L * 2 * d)
     prods = nh * nblk * d * d * (6 if bwd else 2)
-    scratch = nh * nblk * (14 * 128 * 128 + 3 * 128 * d) * 4 if bwd and d != 64 else 0
+    scratch = 0
+    if d != 64:
+        scratch = nh * nblk * ((14 * 128 * 128 + 3 * 128 * d) if bwd else (7 * 128 * 128 + 128 * d)) * 4
     return khat + lin + prods + scratch
 
 

@@ -7,8 +7,8 @@
 // at head dim 128 (the fp32-output gradient error of dw tripled). fp32 inputs
 // keep the CUDA-core gemm_batched.
 //
-// One CTA of 512 threads per batch item (head, block): C [M x N] with M, N, K
-// <= 128. Per term and 64-wide half of K the operands are staged in shared
+// One CTA of 256 threads per batch item (head, block), three CTAs per SM: C
+// [M x N] with M, N, K <= 128. Per term and 32-wide quarter of K the operands are staged in shared
 // memory as fp32 K-major 128-byte-swizzled panels of 32 K-values (A: M rows
 // padded to 128, B: N rows), masks, the sequence limit and alpha applied while
 // staging; one thread issues the MMAs into a tensor-memory accumulator shared
@@ -24,11 +24,11 @@ namespace {
 
 using namespace tc;
 
-constexpr int NT = 512;
+constexpr int NT = 256;
 constexpr int RP = 128;                    // rows of a staged operand (padded)
 constexpr int PANEL = RP * 128;            // bytes of one 32-wide K panel
-constexpr int KH = 64;                     // K staged per round
-constexpr int OPB = 2 * PANEL;             // bytes of one staged operand part (64 K values)
+constexpr int KH = 32;                     // K staged per round
+constexpr int OPB = PANEL;                 // bytes of one staged operand part (32 K values)
 constexpr int SMEM = 4 * OPB + 1024 + 64;  // A hi / lo, B hi / lo, alignment slack, barrier + TMEM slot
 
 // Instruction descriptor of tcgen05.mma kind::tf32 (fp32 accumulation, both
@@ -122,7 +122,9 @@ __device__ __forceinline__ float ld1(const void *p, long long i)
 // 4 kg columns is written as zero. Every thread writes whole 16-byte chunks (4
 // consecutive k of one row r); each warp covers the 8 swizzle positions of its
 // rows evenly; each thread's loads are all in flight before its stores.
-template <bool KMAJ, int DT>
+// EXACT: 16-bit values times alpha = +-1 are TF32 values: no lo part is staged
+// (the products that would read it are not issued)
+template <bool KMAJ, int DT, bool EXACT>
 __device__ void stage1(const Operand &o, long long base, int R, float alpha, uint8_t *hi, uint8_t *lo,
                        int blk, int K, int kb, int kglog)
 {
@@ -177,11 +179,14 @@ __device__ void stage1(const Operand &o, long long base, int R, float alpha, uin
                 // masks act on stored (row, column)
                 const int sr = KMAJ ? r : k0 + u, sc = KMAJ ? k0 + u : r;
                 const bool z = (mask == MASK_LOWER && sc > sr) || (mask == MASK_STRICT_LOWER && sc >= sr);
-                split_tf32(z ? 0.f : alpha * v[b][u], h4[u], l4[u]);
+                if (EXACT)
+                    h4[u] = z ? 0.f : alpha * v[b][u], l4[u] = 0.f;
+                else
+                    split_tf32(z ? 0.f : alpha * v[b][u], h4[u], l4[u]);
             }
             const uint32_t off = kmaj_offset(r, 4 * g);
             *reinterpret_cast<float4 *>(hi + off) = make_float4(h4[0], h4[1], h4[2], h4[3]);
-            *reinterpret_cast<float4 *>(lo + off) = make_float4(l4[0], l4[1], l4[2], l4[3]);
+            if (!EXACT) *reinterpret_cast<float4 *>(lo + off) = make_float4(l4[0], l4[1], l4[2], l4[3]);
         }
     }
 }
@@ -198,21 +203,27 @@ __device__ void stage(const Operand &o, long long base, int R, bool kmaj, float 
         }
         return;
     }
-#define STAGE_CASE(DT)                                                                     \
+#define STAGE_CASE(DT, EX)                                                                 \
     if (o.dt == DT) {                                                                      \
         if (kmaj)                                                                          \
-            stage1<true, DT>(o, base, R, alpha, hi, lo, blk, K, kb, kglog);                \
+            stage1<true, DT, EX>(o, base, R, alpha, hi, lo, blk, K, kb, kglog);            \
         else                                                                               \
-            stage1<false, DT>(o, base, R, alpha, hi, lo, blk, K, kb, kglog);               \
+            stage1<false, DT, EX>(o, base, R, alpha, hi, lo, blk, K, kb, kglog);           \
         return;                                                                            \
     }
-    STAGE_CASE(F32)
-    STAGE_CASE(BF16)
-    STAGE_CASE(F16)
+    const bool unit = alpha == 1.f || alpha == -1.f;
+    STAGE_CASE(F32, false)
+    if (unit) {
+        STAGE_CASE(BF16, true)
+        STAGE_CASE(F16, true)
+    } else {
+        STAGE_CASE(BF16, false)
+        STAGE_CASE(F16, false)
+    }
 #undef STAGE_CASE
 }
 
-__global__ void __launch_bounds__(NT, 1) gemm_tc_kernel(GemmArgs g)
+__global__ void __launch_bounds__(NT, 3) gemm_tc_kernel(GemmArgs g)
 {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -243,7 +254,7 @@ __global__ void __launch_bounds__(NT, 1) gemm_tc_kernel(GemmArgs g)
             const long long bbase = (long long)h * T.b.sh + (long long)blk * T.b.sb;
             for (int kb = 0; kb < g.K; kb += KH) {
                 const int kspan = g.K - kb < KH ? g.K - kb : KH;
-                const int kglog = kspan == 64 ? 4 : kspan == 32 ? 3 : 2;
+                const int kglog = kspan == 32 ? 3 : 2;
                 // A: logical [M x K], stored [M x K] (K-major) unless transposed
                 stage(T.a, abase, g.M, !T.a.trans, T.alpha, sAh, sAl, blk, g.K, kb, kglog);
                 // B: logical [K x N] staged as [N x K], stored [N x K] when transposed
@@ -256,13 +267,24 @@ __global__ void __launch_bounds__(NT, 1) gemm_tc_kernel(GemmArgs g)
                     if (lane == 0) {
                         const uint32_t ah = smem_u32(sAh), al = smem_u32(sAl), bh = smem_u32(sBh),
                                        bl = smem_u32(sBl);
+                        // operands exact in TF32 have no lo part: their lo product is not issued
+                        const bool a_lo = !(T.a.dt != F32 && (T.alpha == 1.f || T.alpha == -1.f));
+                        const bool b_lo = T.b.dt == F32;
                         for (int kk = 0; kk < kspan / 8; ++kk) {
                             const uint32_t off = (uint32_t)(kk >> 2) * PANEL + (uint32_t)(kk & 3) * 32;
                             // small terms first
-                            mma_tf32(tbase, desc_sw128(al + off, 16, 1024), desc_sw128(bh + off, 16, 1024), id,
+                            if (a_lo) {
+                                mma_tf32(tbase, desc_sw128(al + off, 16, 1024), desc_sw128(bh + off, 16, 1024), id,
+                                         first ? 0u : 1u);
+                                first = false;
+                            }
+                            if (b_lo) {
+                                mma_tf32(tbase, desc_sw128(ah + off, 16, 1024), desc_sw128(bl + off, 16, 1024), id,
+                                         first ? 0u : 1u);
+                                first = false;
+                            }
+                            mma_tf32(tbase, desc_sw128(ah + off, 16, 1024), desc_sw128(bh + off, 16, 1024), id,
                                      first ? 0u : 1u);
-                            mma_tf32(tbase, desc_sw128(ah + off, 16, 1024), desc_sw128(bl + off, 16, 1024), id, 1u);
-                            mma_tf32(tbase, desc_sw128(ah + off, 16, 1024), desc_sw128(bh + off, 16, 1024), id, 1u);
                             first = false;
                         }
                         commit(bar);
@@ -276,7 +298,7 @@ __global__ void __launch_bounds__(NT, 1) gemm_tc_kernel(GemmArgs g)
                 fence_after_sync();
             }
         }
-        // epilogue: thread = row r (lane quarter warp % 4), 32-column chunk warp / 4
+        // epilogue: thread = row r (lane quarter warp % 4), 32-column chunks of half warp / 4
         const int r = (warp & 3) * 32 + lane, chalf = warp >> 2;
         const long long cbase = (long long)h * g.csh + (long long)blk * g.csb;
         const long long ebase = (long long)h * g.addend.sh + (long long)blk * g.addend.sb;
@@ -287,8 +309,8 @@ __global__ void __launch_bounds__(NT, 1) gemm_tc_kernel(GemmArgs g)
                      ? 0.f
                      : g.rowscale[(long long)h * g.rs_sh + (long long)blk * g.rs_sb + r];
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const int nchunk = (Np + 31) / 32;  // 32-column chunks, one per warp group
-        for (int q = chalf; q < nchunk; q += 4) {
+        const int nchunk = (Np + 31) / 32;  // 32-column chunks, split between the warp groups
+        for (int q = chalf; q < nchunk; q += 2) {
             const int c0 = 32 * q;
             float v[32];
             tmem_ld32(tbase + lane_off + (uint32_t)c0, v);  // columns past Np are in the allocation
@@ -345,7 +367,7 @@ bool aligned_operand(const Operand &o)
 bool gemm_tc_supported(const GemmArgs &g)
 {
     if (g.M < 1 || g.M > 128 || g.N < 1 || g.N > 128 || g.K < 1 || g.K > 128) return false;
-    // K in 64-wide rounds of 16, 32 or 64 (4-wide K groups: a power of two >= 4)
+    // K in 32-wide rounds of 16 or 32 (4-wide K groups: a power of two >= 4)
     if (g.M % 4 != 0 || g.N % 4 != 0 || (g.K != 16 && g.K != 32 && g.K != 64 && g.K != 128)) return false;
     for (int t = 0; t < g.nterms; ++t)
         if (!aligned_operand(g.t[t].a) || !aligned_operand(g.t[t].b)) return false;

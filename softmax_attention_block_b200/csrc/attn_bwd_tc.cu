@@ -134,20 +134,8 @@ __global__ void __launch_bounds__(NT, 1)
             mbar_expect_tx(v_full, C::TILE);
             tma_load_3d(sV, &mV, 0, J * BT, h, v_full);
             int issued = 0;
-            // the tiles of pair it into L2 (its loads are issued two pairs later, when
-            // its stage comes back, and then read L2 instead of HBM)
-            auto prefetch = [&](int it) {
-                const int I = tile_of(it);
-                if (it != niter - 1) {
-                    tma_prefetch_2d(&mK, 0, (int)((h * a.npairs + (long long)I * (I - 1) / 2 + J) * BT));
-                    tma_prefetch_2d(&mQ, 0, h * Lp + I * BT);
-                    if (I < last) tma_prefetch_2d(&mP, 0, (h * nblk + I) * D);
-                }
-                tma_prefetch_3d(&mDO, 0, I * BT, h);
-            };
             for (int it = 0; it < niter; ++it) {
                 const int s = it & 1;
-                if (it + 2 < niter) prefetch(it + 2);
                 if (it >= 2 && !mbar_wait(&ld_empty[s], ((it >> 1) - 1) & 1, WAIT_LIMIT_NS)) {
                     if (a.err) atomicCAS(a.err, 0, 11);
                     break;

@@ -99,8 +99,8 @@ const char *path_status_string(path_status s);
  * (backward) for the block products and their adjoints, each buffer rounded up
  * to 256 bytes; a backward that is not bf16 at head dim 64 (fp32 inputs, or
  * another head dim) also holds the per-block scratch of its closed-form adjoint,
- * nh * nblk * (14 * 128^2 + 3 * 128 d) * 4 bytes, and a bf16 forward at a head
- * dim other than 64 the forward part of it, nh * nblk * (7 * 128^2 + 128 d) * 4
+ * nh * nblk * (14 * 128^2 + 3 * 128 d) * 4 bytes, and a bf16 forward at head
+ * dim 16 or 32 the forward part of it, nh * nblk * (7 * 128^2 + 128 d) * 4
  * bytes. At nh = 24, L = 65536, d = 64, bf16 the forward needs 53.0 GB.
  */
 size_t path_attn_workspace_bytes(int B, int H, int L, int d, path_dtype dt, int for_bwd);

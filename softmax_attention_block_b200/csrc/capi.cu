@@ -44,14 +44,21 @@ struct AttnWs {
 };
 
 // bf16 inputs at head dim 64 take the tcgen05 UT kernels (prep_fwd_ut.cu,
-// prep_bwd_ut.cu), whose adjoint needs no scratch. Other bf16 cases take the
-// closed form by batched products on the tensor cores in TF32 (prep.cu,
-// gemm_tc.cu), forward and adjoint; fp32 inputs take the fp32 recurrences
+// prep_bwd_ut.cu), whose adjoint needs no scratch; at head dim 128 the forward
+// takes prep_fwd_ut128.cu. Other bf16 cases take the closed form by batched
+// products on the tensor cores in TF32 (prep.cu, gemm_tc.cu), forward and adjoint; fp32 inputs take the fp32 recurrences
 // forward and the closed-form adjoint on CUDA cores (prep_fwd_rec.cu, prep.cu,
 // gemm_batched.cu), which hold fp32 accuracy.
 bool ut_tc_path(const Layout &y, path_dtype dt)
 {
     return y.d == 64 && types_of(dt).in == BF16 && (long long)y.nh * y.nblk * BT < (1LL << 31);
+}
+
+// bf16 inputs at head dim 128: the forward UT prep on tcgen05 (prep_fwd_ut128.cu);
+// the adjoint keeps the closed form by batched products.
+bool ut128_fwd_path(const Layout &y, path_dtype dt)
+{
+    return y.d == 128 && types_of(dt).in == BF16 && (long long)y.nh * y.nblk * BT < (1LL << 31);
 }
 
 // The single description of the workspace: used both to size and to carve it.
@@ -72,8 +79,9 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
     // backward-sized workspace (a backward may reuse the forward's); the rest only
     // the backward path that reads it gets
     // closed-form scratch: the backward's adjoint, and the forward of bf16 inputs
-    // (fp32 inputs take the recurrences forward)
-    if (!ut_tc_path(y, dt) && (bwd || D.dt != F32)) carve_prep_scratch(c, D, bwd, w.prep);
+    // at head dims 16 and 32 (fp32 inputs take the recurrences forward)
+    if (!ut_tc_path(y, dt) && (bwd || (D.dt != F32 && !ut128_fwd_path(y, dt))))
+        carve_prep_scratch(c, D, bwd, w.prep);
     if (bwd) {
         w.delta = c.take<float>(nh * Lp);
         w.dQt = c.take<float>(nh * Lp * d);
@@ -97,11 +105,11 @@ bool fwd_dims_ok(int B, int H, int L, int d)
 
 bool head_dim_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
-// bf16 inputs at head dim 64 go through the tcgen05 UT kernels, which load q, k
-// and w by TMA: their base addresses must be 16-byte aligned.
+// bf16 inputs at head dims 64 and 128 go through the tcgen05 UT kernels, which
+// load q, k and w by TMA: their base addresses must be 16-byte aligned.
 bool tma_inputs_ok(int d, path_dtype dt, const void *q, const void *k, const void *w)
 {
-    if (d != 64 || types_of(dt).in != BF16) return true;
+    if ((d != 64 && d != 128) || types_of(dt).in != BF16) return true;
     const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                          reinterpret_cast<uintptr_t>(w);
     return (al & 15u) == 0;
@@ -160,6 +168,8 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
         Stage s("ut_prep", st);
         if (ut_tc_path(y, dt)) {
             TRY(prep_forward_ut(D, in, out, ws.err, st));
+        } else if (ut128_fwd_path(y, dt)) {
+            TRY(prep_forward_ut128(D, in, out, ws.err, st));
         } else if (D.dt != F32) {
             ws.prep.err = ws.err;
             TRY(prep_forward_gemm(D, in, out, ws.prep, st));

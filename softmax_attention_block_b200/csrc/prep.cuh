@@ -1,7 +1,8 @@
 // Per-block UT transform / boundary adjustment. bf16 inputs at head dim 64: the
-// tcgen05 kernels (prep_fwd_ut.cu, prep_bwd_ut.cu). Otherwise (fp32 inputs, other
-// head dims): forward by recurrences in fp32 (prep_fwd_rec.cu), adjoint through
-// the closed form on CUDA cores (prep.cu).
+// tcgen05 kernels (prep_fwd_ut.cu, prep_bwd_ut.cu); at head dim 128 the forward
+// on tcgen05 (prep_fwd_ut128.cu). Otherwise: the closed form by batched products
+// (prep.cu; on the tensor cores for bf16 inputs), or for fp32 inputs the forward
+// by recurrences in fp32 (prep_fwd_rec.cu).
 #pragma once
 #include "common.cuh"
 
@@ -52,6 +53,10 @@ cudaError_t prep_forward_rec(const PrepDims &D, const PrepInputs &in, const Prep
 bool prep_forward_ut_supported(const PrepDims &D, const PrepInputs &in);
 cudaError_t prep_forward_ut(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
                             int *err, cudaStream_t st);
+// The same at head dim 128 (prep_fwd_ut128.cu; outputs fp16). q, k, w 16-byte aligned.
+bool prep_forward_ut128_supported(const PrepDims &D, const PrepInputs &in);
+cudaError_t prep_forward_ut128(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
+                               int *err, cudaStream_t st);
 // Adjoint of prep_forward_ut (one tcgen05 kernel per block: recomputes the halves'
 // transforms, composition adjoint, per-half UT adjoint). dQt and dKt are overwritten.
 bool prep_backward_ut_supported(const PrepDims &D, const PrepInputs &in);

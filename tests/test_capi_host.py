@@ -77,12 +77,13 @@ def _ws_formula(nh, L, d, bwd):
     lin = nh * (Lp * (1044 + 12 * d) + L * 4 * d) if bwd else nh * (Lp * (516 + 4 * d) + L * 2 * d)
     prods = nh * nblk * d * d * (6 if bwd else 2)
     scratch = 0
-    if d != 64:
+    if d != 64 and (bwd or d != 128):
         scratch = nh * nblk * ((14 * 128 * 128 + 3 * 128 * d) if bwd else (7 * 128 * 128 + 128 * d)) * 4
     return khat + lin + prods + scratch
 
 
-@pytest.mark.parametrize("nh,L,d", [(24, 4096, 64), (3, 300, 64), (24, 65536, 64), (12, 4096, 128)])
+@pytest.mark.parametrize("nh,L,d", [(24, 4096, 64), (3, 300, 64), (24, 65536, 64), (12, 4096, 128),
+                                    (5, 700, 32)])
 def test_workspace_follows_the_stated_formula(lib, nh, L, d):
     for bwd in (0, 1):
         got = lib.path_attn_workspace_bytes(1, nh, L, d, BF16, bwd)
@@ -106,9 +107,10 @@ def test_fwd_rejects_bad_arguments(lib):
 
 
 def test_fwd_rejects_unaligned_tma_inputs(lib):
-    # bf16 at head dim 64 loads q, k, w by TMA: 16-byte aligned bases only
+    # bf16 at head dims 64 and 128 loads q, k, w by TMA: 16-byte aligned bases only
     assert fwd(lib, q=FAKE + 2) == INVALID
     assert fwd(lib, w=FAKE + 8) == INVALID
+    assert fwd(lib, k=FAKE + 4, d=128) == INVALID
     # other head dims have no such rule: validation goes on to the (missing) workspace
     assert fwd(lib, k=FAKE + 2, d=32, ws=None) == WORKSPACE
 

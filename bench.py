@@ -751,7 +751,7 @@ def bench_wbeta(P, dev, peaks, world, max_over_ranks, barrier, steps):
             "stages_ms": {n: t / c for n, (t, c) in stages.items()}}
 
 
-D128 = (8, 12, 4096, 128)  # B, H, L, d: the headline model width (24 x 64) as 12 x 128
+D128 = "fwdbwd_bf16_l4096_d128"  # the headline model width (24 x 64) as 12 heads of 128
 
 
 def d128_flops(B, H, L, d):
@@ -763,8 +763,9 @@ def d128_flops(B, H, L, d):
 
 def bench_d128(P, dev, peaks, world, max_over_ranks, barrier, steps):
     """fwd+bwd at head dim 128 (same model width as the headline), per stage."""
-    B, H, L, d = D128
-    xc = si.make_inputs(B, H, L, d, torch.bfloat16, seed=0)
+    w = si.WORKLOADS[D128]
+    B, H, L, d = w.B, w.H, w.L, w.d
+    xc = si.workload_inputs(D128)
     x = {k: (v.to(dev) if v is not None else None) for k, v in xc.items()}
     del xc
     out = torch.empty_like(x["q"])

@@ -97,10 +97,12 @@ const char *path_status_string(path_status s);
  * adjoints, boundary-adjusted queries / keys, per-position terms, 16-bit copies
  * of v and dout; Lp = 128 nblk), plus nh * nblk * d^2 * 2 (forward) or * 6
  * (backward) for the block products and their adjoints, each buffer rounded up
- * to 256 bytes; a backward that is not bf16 at head dim 64 (fp32 inputs, or
- * another head dim) also holds the per-block scratch of its closed-form adjoint,
- * nh * nblk * (14 * 128^2 + 3 * 128 d) * 4 bytes, and a bf16 forward at head
- * dim 16 or 32 the forward part of it, nh * nblk * (7 * 128^2 + 128 d) * 4
+ * to 256 bytes; a bf16 backward at head dim 128 also holds per-block quantities
+ * of the UT transform that a forward into the same workspace leaves for the
+ * adjoint, nh * nblk * 245760 bytes; a backward that is neither (fp32 inputs, or
+ * bf16 at head dim 16 or 32) holds the per-block scratch of its closed-form
+ * adjoint, nh * nblk * (14 * 128^2 + 3 * 128 d) * 4 bytes, and a bf16 forward at
+ * head dim 16 or 32 the forward part of it, nh * nblk * (7 * 128^2 + 128 d) * 4
  * bytes. At nh = 24, L = 65536, d = 64, bf16 the forward needs 53.0 GB.
  */
 size_t path_attn_workspace_bytes(int B, int H, int L, int d, path_dtype dt, int for_bwd);
@@ -137,10 +139,14 @@ path_status path_attn_fwd(const void *q, const void *k, const void *v, const voi
  * through the same blockwise algorithm as the forward.
  * flags: 0, or PATH_BWD_REUSE_FWD_WORKSPACE when `workspace` is the buffer
  * the matching path_attn_fwd call used (sized with for_bwd != 0 at that
- * call), holding what that call left there, with q, k, w, beta and log_f
- * unchanged since: the backward then reuses the forward's block transforms
- * and transported keys instead of recomputing them. Unknown flag bits are
- * PATH_ERR_INVALID_ARG.
+ * call, and that size or more given as its workspace_bytes), holding what that
+ * call left there, with q, k, w, beta and log_f unchanged since: the backward
+ * then reuses the forward's block transforms and transported keys instead of
+ * recomputing them. At bf16, head dim 128, the forward leaves per-block
+ * quantities of the UT transform for the backward only when its workspace_bytes
+ * covers the backward size; a reusing backward after a forward that was given
+ * less writes no dq, dk, dw, dbeta and path_attn_wait_status reports
+ * PATH_ERR_WORKSPACE. Unknown flag bits are PATH_ERR_INVALID_ARG.
  */
 path_status path_attn_bwd(const void *q, const void *k, const void *v, const void *w,
                           const float *beta, const float *log_f, float scale, int B, int H,
@@ -155,8 +161,10 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
  * bytes of the workspace, writes NaN to the rows it could not finish, frees
  * its tensor memory and returns instead of hanging. This call waits for
  * `stream`, then returns PATH_ERR_TIMEOUT if the last path_attn_fwd /
- * path_attn_bwd that used `workspace` recorded such an event, else PATH_OK
- * (PATH_ERR_CUDA if the read-back itself fails). It synchronises the host.
+ * path_attn_bwd that used `workspace` recorded such an event, PATH_ERR_WORKSPACE
+ * if a reusing backward found the forward's saved quantities missing (see
+ * path_attn_bwd), else PATH_OK (PATH_ERR_CUDA if the read-back itself fails).
+ * It synchronises the host.
  */
 path_status path_attn_wait_status(const void *workspace, path_stream_t stream);
 

@@ -206,9 +206,11 @@ def path_attn_fwd(q, k, v, w, beta, log_f=None, scale=None, out=None, lse=None, 
     _check_dev(q, k, v, w, beta, log_f, out, lse, workspace)
     nbytes = path_attn_workspace_bytes(B, H, L, d, q.dtype, False, out.dtype)
     ws = _workspace(nbytes, q.device, workspace)
+    # the buffer's whole size: a backward-sized workspace also receives what a
+    # backward that reuses it reads
     st = lib().path_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(beta), _ptr(log_f),
                              _scale(scale, d), B, H, L, d, dt, _ptr(out), _ptr(lse), _ptr(ws),
-                             nbytes, _stream())
+                             ws.numel() * ws.element_size(), _stream())
     if st:
         raise PathError(st, "path_attn_fwd")
     return out, lse

@@ -53,10 +53,31 @@ cudaError_t prep_forward_rec(const PrepDims &D, const PrepInputs &in, const Prep
 bool prep_forward_ut_supported(const PrepDims &D, const PrepInputs &in);
 cudaError_t prep_forward_ut(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
                             int *err, cudaStream_t st);
+// Per-block quantities of the head-dim-128 UT kernels that the forward leaves for the
+// adjoint (fp16, row-major; blk = head * nblk + block, h = half):
+//   What [blk][h][64][128], U, X, M [blk][h][64][64], Kta, Qtb [blk][64][128]
+//   (Ktil_a, Qtil_b), Pa, Pb [blk][128][128] (P_a, P_b); and the adjoint's own
+//   dP [blk][h][128][128] (the halves' dP).
+struct Ut128Save {
+    f16 *What = nullptr, *U = nullptr, *X = nullptr, *M = nullptr, *Kta = nullptr,
+        *Qtb = nullptr, *Pa = nullptr, *Pb = nullptr, *dP = nullptr;
+};
+void carve_ut128_save(Carver &c, const PrepDims &D, Ut128Save &s);
 // The same at head dim 128 (prep_fwd_ut128.cu; outputs fp16). q, k, w 16-byte aligned.
+// save: NULL, or the area the adjoint reads (prep_backward_ut128).
 bool prep_forward_ut128_supported(const PrepDims &D, const PrepInputs &in);
 cudaError_t prep_forward_ut128(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
-                               int *err, cudaStream_t st);
+                               const Ut128Save *save, int *err, cudaStream_t st);
+// Adjoint of prep_forward_ut128 from what it saved: the composition adjoint (one
+// kernel per block) and the per-half UT adjoint (one kernel per half block).
+// dQt and dKt are overwritten. `saved`: a device word the caller sets to bytes
+// UT128_SAVED_BYTE when the save area holds the forward's values; otherwise the
+// kernels record ERR_UT128_NOT_SAVED in *err and write no gradient.
+constexpr int UT128_SAVED_WORD = 1;       // index in the workspace's error words
+constexpr int UT128_SAVED_BYTE = 0x5A;    // memset byte of a valid save
+constexpr int ERR_UT128_NOT_SAVED = 30;
+cudaError_t prep_backward_ut128(const PrepDims &D, const PrepInputs &in, const PrepGrads &g,
+                                const Ut128Save &save, const int *saved, int *err, cudaStream_t st);
 // Adjoint of prep_forward_ut (one tcgen05 kernel per block: recomputes the halves'
 // transforms, composition adjoint, per-half UT adjoint). dQt and dKt are overwritten.
 bool prep_backward_ut_supported(const PrepDims &D, const PrepInputs &in);

@@ -20,6 +20,12 @@
 // four results of the halves' last level (M What, U^T W, W^T What in two row
 // blocks, and M U added to Q K^T) exceed the 512 tensor-memory columns by one
 // row block of P_h: that one is issued after the others have been read.
+//
+// With a save area (a workspace sized for the backward) the kernel also writes
+// what the adjoint (prep_bwd_ut128.cu) reads instead of recomputing it: per
+// half What, U, M and X = (I + A)^{-1} (the same three factors applied to the
+// identity: Z1x = (I - N') E^{-1}, X = (I + N'^2) Z1x), and the composition's
+// inputs Ktil_a, Qtil_b, P_a, P_b, all fp16 as the products read them.
 #include "prep.cuh"
 #include "runtime.cuh"
 #include "ut_tc.cuh"
@@ -53,7 +59,7 @@ static_assert(SMEM <= 227 * 1024, "shared memory of one CTA");
 // tensor-memory columns (both halves share them: lane offsets 0 / 16)
 constexpr int C_G = 0, C_N = 64, C_M = 128, C_S = 192;  // W W^T, W K^T, Q W^T, Q K^T (then Sd)
 constexpr int C_Z = 256;                                // N' | Zw (2) | Zn, then Z1, [What | U]
-constexpr int C_N2 = 0;                                 // N'^2
+constexpr int C_N2 = 0, C_ZX = 64;                      // N'^2; saving: the X products
 constexpr int C_QT = 0, C_KT = 256, C_P0 = 384;         // -M What, U^T W, rows 0..63 of W^T What
 constexpr int C_P1 = 0;                                 // rows 64..127 of W^T What
 constexpr int C_C1 = 0, C_C2 = 128, C_C3 = 256;         // composition
@@ -75,12 +81,13 @@ __device__ __forceinline__ void st_box_f32(uint8_t *box, int r, const float (&v)
 // Outputs leave through shared-memory staging and TMA tensor stores: Qt, Kt
 // ([nh Lp, 128] fp16) and Pm ([nh nblk 128, 128] fp16) in 64 x 64 tiles, Sd
 // ([nh nblk 128, 128] fp32) in 64-row boxes of 32 columns.
+template <bool SAVE>
 __global__ void __launch_bounds__(NT, 1)
     prep_fwd_ut128_kernel(const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mQ,
                           const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mQt,
                           const __grid_constant__ CUtensorMap mKt, const __grid_constant__ CUtensorMap mPm,
                           const __grid_constant__ CUtensorMap mSd, const float *beta, int L, int nblk,
-                          int nsm, int *err)
+                          int nsm, Ut128Save sv, int *err)
 {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
@@ -140,6 +147,8 @@ __global__ void __launch_bounds__(NT, 1)
     const int h = me.h, r = me.r, c0 = 32 * me.cg;
     const float br = sB[h * HB + r];
     const int F = T_F + 4 * h;  // this half's F / Z tiles
+    const long long blk = (long long)hd * nblk + J;
+    const long long hrow = (blk * 2 + h) * HB + r;  // this thread's row in the per-half save arrays
     uint32_t phase = 0;
     // one level: operands written and fenced, barrier; one thread issues the
     // products and commits; everyone waits for them
@@ -197,7 +206,10 @@ __global__ void __launch_bounds__(NT, 1)
         st_tile_f16(tile(F + 3), r, c0, v);
         me.ld(tbase, C_M, v);  // -M, M = lower(Q W^T)
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = c0 + j <= r ? -v[j] : 0.f;
+        for (int j = 0; j < 32; ++j) v[j] = c0 + j <= r ? v[j] : 0.f;
+        if (SAVE) st_global(sv.M + hrow * HB + c0, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = -v[j];
         st_tile_f16(tile(T_M + h), r, c0, v);
         // W to fp16 in place (an operand beside fp16 intermediates from here on), and D W
 #pragma unroll 1
@@ -235,10 +247,12 @@ __global__ void __launch_bounds__(NT, 1)
     }
     sync_operands();
 
-    // ---- level 2: Z1 = Z + (-N') Z (in place in tensor memory), N'^2 = (-N')(-N')
+    // ---- level 2: Z1 = Z + (-N') Z (in place in tensor memory), N'^2 = (-N')(-N');
+    // saving: (-N') E^{-1}, so that Z1x = E^{-1} + (-N') E^{-1}
     ISSUE(for (int hh = 0; hh < 2; ++hh) {
         mma64(dst(tbase, hh, C_Z + 64), ta(T_NN + hh), A_N, ta(T_F + 4 * hh), B_N, 3, TILE, true);
         mma64(dst(tbase, hh, C_N2), ta(T_NN + hh), A_N, ta(T_NN + hh), B_N, 1, TILE, false);
+        if (SAVE) mma64(dst(tbase, hh, C_ZX), ta(T_NN + hh), A_N, ta(T_E + hh), B_N, 1, TILE, false);
     });
     wait_mma();
     if (ok) {
@@ -247,20 +261,42 @@ __global__ void __launch_bounds__(NT, 1)
             me.ld(tbase, C_Z + 64 + 64 * m, v);
             st_tile_f16(tile(F + m), r, c0, v);
         }
+        if (SAVE) {  // Z1x over the D N tile (read by level 1); E^{-1} read before N'^2 replaces it
+            me.ld(tbase, C_ZX, v);
+            ld_tile_f16(tile(T_E + h), r, c0, x);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += x[j];
+            st_tile_f16(tile(F + 3), r, c0, v);
+        }
         me.ld(tbase, C_N2, v);
         st_tile_f16(tile(T_E + h), r, c0, v);
     }
     sync_operands();
 
-    // ---- level 3: [What | U] = Z1 + N'^2 Z1
-    ISSUE(for (int hh = 0; hh < 2; ++hh)
-              mma64(dst(tbase, hh, C_Z + 64), ta(T_E + hh), A_N, ta(T_F + 4 * hh), B_N, 3, TILE, true));
+    // ---- level 3: [What | U] = Z1 + N'^2 Z1; saving: N'^2 Z1x (X = Z1x + N'^2 Z1x)
+    ISSUE(for (int hh = 0; hh < 2; ++hh) {
+        mma64(dst(tbase, hh, C_Z + 64), ta(T_E + hh), A_N, ta(T_F + 4 * hh), B_N, 3, TILE, true);
+        if (SAVE) mma64(dst(tbase, hh, C_ZX), ta(T_E + hh), A_N, ta(T_F + 4 * hh + 3), B_N, 1, TILE, false);
+    });
     wait_mma();
     if (ok) {
 #pragma unroll 1
         for (int m = 0; m < 3; ++m) {
             me.ld(tbase, C_Z + 64 + 64 * m, v);
             st_tile_f16(tile(F + m), r, c0, v);
+            if (SAVE) {
+                if (m < 2)
+                    st_global(sv.What + hrow * DH + 64 * m + c0, v);
+                else
+                    st_global(sv.U + hrow * HB + c0, v);
+            }
+        }
+        if (SAVE) {
+            me.ld(tbase, C_ZX, v);
+            ld_tile_f16(tile(F + 3), r, c0, x);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += x[j];
+            st_global(sv.X + hrow * HB + c0, v);
         }
     }
     sync_operands();
@@ -286,6 +322,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] += x[j];
             st_tile_f16(tile(T_Q(h, c)), r, c0, v);
+            if (SAVE && h == 1) st_global(sv.Qtb + (blk * HB + r) * DH + 64 * c + c0, v);
         }
         // Ktil_h = K - U^T W, over K_h in place (fp16)
 #pragma unroll 1
@@ -295,6 +332,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = x[j] - v[j];
             st_tile_f16(tile(T_K(h, c)), r, c0, v);
+            if (SAVE && h == 0) st_global(sv.Kta + (blk * HB + r) * DH + 64 * c + c0, v);
         }
         // Sd_hh = lower(Q K^T - M U) (the block above the diagonal blocks is never
         // read: the attention kernels mask it), over the -M and -N' tiles
@@ -333,6 +371,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = (64 * rb + r == 64 * ck + c0 + j ? 1.f : 0.f) - v[j];
                 st_tile_f16(tile(h ? T_F + 4 + 2 * ck + rb : T_F + 2 * rb + ck), r, c0, v);
+                if (SAVE) st_global((h ? sv.Pb : sv.Pa) + (blk * DH + 64 * rb + r) * DH + 64 * ck + c0, v);
             }
     }
     sync_operands();
@@ -402,7 +441,7 @@ bool prep_forward_ut128_supported(const PrepDims &Dm, const PrepInputs &in)
 }
 
 cudaError_t prep_forward_ut128(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out,
-                               int *err, cudaStream_t st)
+                               const Ut128Save *save, int *err, cudaStream_t st)
 {
     if (!prep_forward_ut128_supported(Dm, in) || out.tdt != F16) return cudaErrorInvalidValue;
     CUtensorMap mW, mQ, mK, mQt, mKt, mPm, mSd;
@@ -414,11 +453,11 @@ cudaError_t prep_forward_ut128(const PrepDims &Dm, const PrepInputs &in, const P
         !make_map_2d(&mPm, out.Pm, F16, DH, (uint64_t)Dm.nh * Dm.nblk * DH, HB) ||
         !make_map_f32_2d(&mSd, out.Sd, BT, rows, HB))
         return cudaErrorInvalidValue;
-    cudaError_t e =
-        cudaFuncSetAttribute(prep_fwd_ut128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    auto k = save ? prep_fwd_ut128_kernel<true> : prep_fwd_ut128_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
-    prep_fwd_ut128_kernel<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(mW, mQ, mK, mQt, mKt, mPm, mSd, in.beta,
-                                                                  Dm.L, Dm.nblk, sm_count(), err);
+    k<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(mW, mQ, mK, mQt, mKt, mPm, mSd, in.beta, Dm.L, Dm.nblk,
+                                              sm_count(), save ? *save : Ut128Save{}, err);
     count_launches();
     return cudaGetLastError();
 }

@@ -17,6 +17,8 @@ headline shapes):
 - ``fwd_bf16_l1024``     bf16 forward, B=2 H=4 L=1024 d=64
 - ``fwdbwd_bf16_l4096``  bf16 forward+backward, B=8 H=24 L=4096 d=64
 - ``fox_fwdbwd_l16384``  bf16 PaTH-FoX forward+backward, B=1 H=24 L=16384 d=64
+- ``fwdbwd_bf16_l4096_d128``  bf16 forward+backward at head dim 128, B=8 H=12 L=4096
+  (the headline's model width as 12 heads of 128)
 - ``decode_bf16_c16k``   bf16 decode, B=32 H=32 d=128, cache 16384 -> 16448, 64 steps
 """
 from __future__ import annotations
@@ -50,6 +52,7 @@ WORKLOADS = {
         Workload("fwdbwd_bf16_l4096", 8, 24, 4096, 64, torch.bfloat16, backward=True),
         Workload("fox_fwdbwd_l16384", 1, 24, 16384, 64, torch.bfloat16, fox=True,
                  backward=True),
+        Workload("fwdbwd_bf16_l4096_d128", 8, 12, 4096, 128, torch.bfloat16, backward=True),
         Workload("decode_bf16_c16k", 32, 32, 0, 128, torch.bfloat16, n0=16384, steps=64),
     )
 }

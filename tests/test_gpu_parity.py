@@ -214,6 +214,12 @@ def test_full_size_l4096_sampled_heads(P):
     _sampled_full_size(P, "fwdbwd_bf16_l4096", [0, 77, 191], ["bf16", "bf16in_f32out"])
 
 
+def test_full_size_d128_sampled_heads(P):
+    """Head dim 128 at the benchmark's shape (32 blocks per head, 96 heads), oracle on
+    the first and last head."""
+    _sampled_full_size(P, "fwdbwd_bf16_l4096_d128", [0, 95], ["bf16", "bf16in_f32out"])
+
+
 def test_forward_is_deterministic_at_full_size(P):
     """The forward has no atomics: repeated calls on the headline workload give the same
     bits (each call starts from a NaN-filled workspace). A softmax warp pair running a

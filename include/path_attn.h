@@ -97,11 +97,11 @@ const char *path_status_string(path_status s);
  * adjoints, boundary-adjusted queries / keys, per-position terms, 16-bit copies
  * of v and dout; Lp = 128 nblk), plus nh * nblk * d^2 * 2 (forward) or * 6
  * (backward) for the block products and their adjoints, each buffer rounded up
- * to 256 bytes; a bf16 backward at head dim 128 also holds per-block quantities
- * of the UT transform that a forward into the same workspace leaves for the
- * adjoint, nh * nblk * 245760 bytes; a backward that is neither (fp32 inputs, or
- * bf16 at head dim 16 or 32) holds the per-block scratch of its closed-form
- * adjoint, nh * nblk * (14 * 128^2 + 3 * 128 d) * 4 bytes, and a bf16 forward at
+ * to 256 bytes; a bf16 backward at head dim 64 or 128 also holds per-block
+ * quantities of the UT transform that a forward into the same workspace leaves
+ * for the adjoint, nh * nblk * 98304 bytes at d = 64 and nh * nblk * 245760 at
+ * d = 128; a backward that is neither (fp32 inputs, or bf16 at head dim 16 or
+ * 32) holds the per-block scratch of its closed-form adjoint, nh * nblk * (14 * 128^2 + 3 * 128 d) * 4 bytes, and a bf16 forward at
  * head dim 16 or 32 the forward part of it, nh * nblk * (7 * 128^2 + 128 d) * 4
  * bytes. At nh = 24, L = 65536, d = 64, bf16 the forward needs 53.0 GB.
  */
@@ -142,7 +142,7 @@ path_status path_attn_fwd(const void *q, const void *k, const void *v, const voi
  * call, and that size or more given as its workspace_bytes), holding what that
  * call left there, with q, k, w, beta and log_f unchanged since: the backward
  * then reuses the forward's block transforms and transported keys instead of
- * recomputing them. At bf16, head dim 128, the forward leaves per-block
+ * recomputing them. At bf16, head dims 64 and 128, the forward leaves per-block
  * quantities of the UT transform for the backward only when its workspace_bytes
  * covers the backward size; a reusing backward after a forward that was given
  * less writes no dq, dk, dw, dbeta and path_attn_wait_status reports

@@ -37,7 +37,7 @@ struct AttnWs {
     void *Vh;  // fp16 copy of v for the tensor-core forward
     float *Sd;
     PrepScratch prep;
-    Ut128Save save;   // head dim 128, bf16, backward-sized workspace
+    UtSave save;   // head dim 128, bf16, backward-sized workspace
     // backward only
     float *delta, *dQt, *dKt, *dPm, *dSd, *rowsum, *colsum;
     float *lse_p;     // lse padded to Lp (tensor-core backward)
@@ -45,9 +45,11 @@ struct AttnWs {
 };
 
 // bf16 inputs at head dim 64 take the tcgen05 UT kernels (prep_fwd_ut.cu,
-// prep_bwd_ut.cu), whose adjoint needs no scratch; at head dim 128 those of
-// prep_fwd_ut128.cu and prep_bwd_ut128.cu. Other bf16 cases take the closed form
-// by batched products on the tensor cores in TF32 (prep.cu, gemm_tc.cu), forward and adjoint; fp32 inputs take the fp32 recurrences
+// prep_bwd_ut.cu), at head dim 128 those of prep_fwd_ut128.cu and
+// prep_bwd_ut128.cu; a forward into a backward-sized workspace leaves per-block
+// quantities there that their adjoint reads (UtSave). Other bf16 cases take the
+// closed form by batched products on the tensor cores in TF32 (prep.cu,
+// gemm_tc.cu), forward and adjoint; fp32 inputs take the fp32 recurrences
 // forward and the closed-form adjoint on CUDA cores (prep_fwd_rec.cu, prep.cu,
 // gemm_batched.cu), which hold fp32 accuracy.
 bool ut_tc_path(const Layout &y, path_dtype dt)
@@ -55,9 +57,6 @@ bool ut_tc_path(const Layout &y, path_dtype dt)
     return y.d == 64 && types_of(dt).in == BF16 && (long long)y.nh * y.nblk * BT < (1LL << 31);
 }
 
-// bf16 inputs at head dim 128: the UT prep and its adjoint on tcgen05
-// (prep_fwd_ut128.cu, prep_bwd_ut128.cu); a forward into a backward-sized
-// workspace leaves per-block quantities there that the adjoint reads.
 bool ut128_path(const Layout &y, path_dtype dt)
 {
     return y.d == 128 && types_of(dt).in == BF16 && (long long)y.nh * y.nblk * 2 * 128 < (1LL << 31);
@@ -82,9 +81,9 @@ size_t carve_attn(void *base, const Layout &y, path_dtype dt, bool bwd, AttnWs &
     // the backward path that reads it gets
     // closed-form scratch: the backward's adjoint, and the forward of bf16 inputs
     // at head dims 16 and 32 (fp32 inputs take the recurrences forward)
-    if (ut128_path(y, dt)) {
-        if (bwd) carve_ut128_save(c, D, w.save);
-    } else if (!ut_tc_path(y, dt) && (bwd || D.dt != F32)) {
+    if (ut_tc_path(y, dt) || ut128_path(y, dt)) {
+        if (bwd) carve_ut_save(c, D, w.save);
+    } else if (bwd || D.dt != F32) {
         carve_prep_scratch(c, D, bwd, w.prep);
     }
     if (bwd) {
@@ -171,14 +170,15 @@ path_status run_prep_and_chain(const void *q, const void *k, const void *w, cons
     PrepOutputs out{ws.Qt, ws.Kt, ws.Pm, ws.Sd, t.mid};
     {
         Stage s("ut_prep", st);
-        if (ut_tc_path(y, dt)) {
-            TRY(prep_forward_ut(D, in, out, ws.err, st));
-        } else if (ut128_path(y, dt)) {
-            // the save flag tells a backward that reuses this workspace whether the
+        if (ut_tc_path(y, dt) || ut128_path(y, dt)) {
+            // the save word tells a backward that reuses this workspace whether the
             // per-block quantities it reads were written by this call
             const bool save = ws.save.What != nullptr;
-            TRY(cudaMemsetAsync(ws.err + UT128_SAVED_WORD, save ? UT128_SAVED_BYTE : 0, sizeof(int), st));
-            TRY(prep_forward_ut128(D, in, out, save ? &ws.save : nullptr, ws.err, st));
+            TRY(cudaMemsetAsync(ws.err + UT_SAVED_WORD, save ? UT_SAVED_BYTE : 0, sizeof(int), st));
+            if (y.d == 64)
+                TRY(prep_forward_ut(D, in, out, save ? &ws.save : nullptr, ws.err, st));
+            else
+                TRY(prep_forward_ut128(D, in, out, save ? &ws.save : nullptr, ws.err, st));
         } else if (D.dt != F32) {
             ws.prep.err = ws.err;
             TRY(prep_forward_gemm(D, in, out, ws.prep, st));
@@ -349,10 +349,10 @@ path_status path_attn_bwd(const void *q, const void *k, const void *v, const voi
     PrepGrads gr{ws.dQt, ws.dKt, ws.dPm, ws.dSd, dq, dk, dw, dbeta};
     if (ut_tc_path(y, dt)) {
         Stage s("ut_adj", st);
-        TRY(prep_backward_ut(D, in, gr, ws.err, st));
+        TRY(prep_backward_ut(D, in, gr, ws.save, ws.err + UT_SAVED_WORD, ws.err, st));
     } else if (ut128_path(y, dt)) {
         Stage s("ut_adj", st);
-        TRY(prep_backward_ut128(D, in, gr, ws.save, ws.err + UT128_SAVED_WORD, ws.err, st));
+        TRY(prep_backward_ut128(D, in, gr, ws.save, ws.err + UT_SAVED_WORD, ws.err, st));
     } else {
         Stage s("ut_prep_bwd", st);
         ws.prep.err = ws.err;
@@ -373,7 +373,7 @@ path_status path_attn_wait_status(const void *workspace, path_stream_t stream)
     if (cudaMemcpyAsync(&code, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
         return PATH_ERR_CUDA;
-    if (code == ERR_UT128_NOT_SAVED) return PATH_ERR_WORKSPACE;
+    if (code == ERR_UT_NOT_SAVED) return PATH_ERR_WORKSPACE;
     return code ? PATH_ERR_TIMEOUT : PATH_OK;
 }
 

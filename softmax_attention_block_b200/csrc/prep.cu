@@ -266,6 +266,20 @@ void carve_prep_scratch(Carver &c, const PrepDims &D, bool backward, PrepScratch
     }
 }
 
+void carve_ut_save(Carver &c, const PrepDims &D, UtSave &s)
+{
+    const size_t nb = (size_t)D.nh * D.nblk, d = D.d, hb = BT / 2;
+    s.What = c.take<f16>(nb * 2 * hb * d);
+    s.U = c.take<f16>(nb * 2 * hb * hb);
+    s.X = c.take<f16>(nb * 2 * hb * hb);
+    s.M = c.take<f16>(nb * 2 * hb * hb);
+    s.Kta = c.take<f16>(nb * hb * d);
+    s.Qtb = c.take<f16>(nb * hb * d);
+    s.Pa = c.take<f16>(nb * d * d);
+    s.Pb = c.take<f16>(nb * d * d);
+    s.dP = d == 128 ? c.take<f16>(nb * 2 * d * d) : nullptr;
+}
+
 // Closed-form forward quantities the adjoint needs: A, G, Tinv, X, What, N, U, M.
 static cudaError_t prep_core(const PrepDims &D, const PrepInputs &in, const PrepScratch &s,
                              cudaStream_t st)

@@ -47,42 +47,46 @@ size_t prep_scratch_bytes(const PrepDims &D, bool backward);
 // Qtil, Ktil, P, Sd of every 128-block, computed by per-row recurrences in fp32.
 cudaError_t prep_forward_rec(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
                              cudaStream_t st);
-// The same outputs for head dim 64 and bf16 inputs on tcgen05 (tensor memory),
-// with (I + A)^{-1} as a product of block-diagonal and nilpotent factors
-// (prep_fwd_ut.cu). q, k, w 16-byte aligned. err: device error word.
-bool prep_forward_ut_supported(const PrepDims &D, const PrepInputs &in);
-cudaError_t prep_forward_ut(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
-                            int *err, cudaStream_t st);
-// Per-block quantities of the head-dim-128 UT kernels that the forward leaves for the
-// adjoint (fp16, row-major; blk = head * nblk + block, h = half):
-//   What [blk][h][64][128], U, X, M [blk][h][64][64], Kta, Qtb [blk][64][128]
-//   (Ktil_a, Qtil_b), Pa, Pb [blk][128][128] (P_a, P_b); and the adjoint's own
-//   dP [blk][h][128][128] (the halves' dP).
-struct Ut128Save {
+// Per-block quantities of the tcgen05 UT kernels (head dims 64 and 128) that the
+// forward leaves for the adjoint in a backward-sized workspace (fp16, row-major;
+// blk = head * nblk + block, h = half):
+//   What [blk][h][64][d], U, X, M [blk][h][64][64], Kta, Qtb [blk][64][d]
+//   (Ktil_a, Qtil_b), Pa, Pb [blk][d][d] (P_a, P_b); at d = 128 also the
+//   adjoint's own dP [blk][h][128][128] (the halves' dP).
+struct UtSave {
     f16 *What = nullptr, *U = nullptr, *X = nullptr, *M = nullptr, *Kta = nullptr,
         *Qtb = nullptr, *Pa = nullptr, *Pb = nullptr, *dP = nullptr;
 };
-void carve_ut128_save(Carver &c, const PrepDims &D, Ut128Save &s);
+void carve_ut_save(Carver &c, const PrepDims &D, UtSave &s);
+// A device word of the workspace tells the adjoint whether the save area holds the
+// forward's values (bytes UT_SAVED_BYTE); without them the adjoint kernels record
+// ERR_UT_NOT_SAVED in the error word and write no gradient.
+constexpr int UT_SAVED_WORD = 1;       // index in the workspace's error words
+constexpr int UT_SAVED_BYTE = 0x5A;    // memset byte of a valid save
+constexpr int ERR_UT_NOT_SAVED = 30;
+// The same outputs for head dim 64 and bf16 inputs on tcgen05 (tensor memory),
+// with (I + A)^{-1} as a product of block-diagonal and nilpotent factors
+// (prep_fwd_ut.cu). q, k, w 16-byte aligned. err: device error word. save: NULL,
+// or the area the adjoint reads (prep_backward_ut).
+bool prep_forward_ut_supported(const PrepDims &D, const PrepInputs &in);
+cudaError_t prep_forward_ut(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
+                            const UtSave *save, int *err, cudaStream_t st);
 // The same at head dim 128 (prep_fwd_ut128.cu; outputs fp16). q, k, w 16-byte aligned.
 // save: NULL, or the area the adjoint reads (prep_backward_ut128).
 bool prep_forward_ut128_supported(const PrepDims &D, const PrepInputs &in);
 cudaError_t prep_forward_ut128(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,
-                               const Ut128Save *save, int *err, cudaStream_t st);
+                               const UtSave *save, int *err, cudaStream_t st);
 // Adjoint of prep_forward_ut128 from what it saved: the composition adjoint (one
 // kernel per block) and the per-half UT adjoint (one kernel per half block).
-// dQt and dKt are overwritten. `saved`: a device word the caller sets to bytes
-// UT128_SAVED_BYTE when the save area holds the forward's values; otherwise the
-// kernels record ERR_UT128_NOT_SAVED in *err and write no gradient.
-constexpr int UT128_SAVED_WORD = 1;       // index in the workspace's error words
-constexpr int UT128_SAVED_BYTE = 0x5A;    // memset byte of a valid save
-constexpr int ERR_UT128_NOT_SAVED = 30;
+// dQt and dKt are overwritten. saved: the workspace's save word (UT_SAVED_WORD).
 cudaError_t prep_backward_ut128(const PrepDims &D, const PrepInputs &in, const PrepGrads &g,
-                                const Ut128Save &save, const int *saved, int *err, cudaStream_t st);
-// Adjoint of prep_forward_ut (one tcgen05 kernel per block: recomputes the halves'
-// transforms, composition adjoint, per-half UT adjoint). dQt and dKt are overwritten.
+                                const UtSave &save, const int *saved, int *err, cudaStream_t st);
+// Adjoint of prep_forward_ut from what it saved (one tcgen05 kernel per block:
+// composition adjoint, per-half UT adjoint). dQt and dKt are overwritten. saved:
+// the workspace's save word (UT_SAVED_WORD).
 bool prep_backward_ut_supported(const PrepDims &D, const PrepInputs &in);
-cudaError_t prep_backward_ut(const PrepDims &D, const PrepInputs &in, const PrepGrads &g, int *err,
-                             cudaStream_t st);
+cudaError_t prep_backward_ut(const PrepDims &D, const PrepInputs &in, const PrepGrads &g,
+                             const UtSave &save, const int *saved, int *err, cudaStream_t st);
 // The same outputs from the closed form by batched products (bf16 inputs at head
 // dims other than 64; TF32 tensor cores), through the forward part of `s`.
 cudaError_t prep_forward_gemm(const PrepDims &D, const PrepInputs &in, const PrepOutputs &out,

@@ -7,10 +7,10 @@
 // product (dP) and of the block's logits (dSd). This kernel carries them to
 // dq, dk, dw and dbeta:
 //
-// 1. It recomputes each half's UT transform (Paper-Notes "训练策略":
-//    T^{-1} = (I + strictLower(D W W^T))^{-1} D) as the forward prep does, with
-//    the inverse itself: X = (I + A)^{-1} = (I + N'^2)(I - N') E^{-1}, and
-//    [What | U | X] = X [D W | D N | I].
+// 1. It reads each half's UT transform (Paper-Notes "训练策略":
+//    T^{-1} = (I + strictLower(D W W^T))^{-1} D) from what the forward prep
+//    saved (prep_fwd_ut.cu): What, U, M, the inverse X = (I + A)^{-1} itself,
+//    and the composition's inputs Ktil_a, Qtil_b, P_a, P_b.
 // 2. The halves compose the block (Qtil[b] = Qtil_b P_a, Ktil[a] = Ktil_a P_b^T,
 //    P = P_b P_a, Sd[b,a] = Qtil_b Ktil_a^T), so the block's adjoints become
 //    per-half ones:
@@ -41,36 +41,31 @@ using namespace tc;
 using namespace uttc;
 
 constexpr int NT = 256;
+constexpr int SAVED_WORD = UT_SAVED_BYTE * 0x01010101;
 
 // shared-memory tiles (8 KB each); "_h" = half a at the index, half b at +1
 // unless noted
 enum {
     T_W = 0, T_K = 1,       // W_h at 2h, K_h at 2h + 1 ([W_h; K_h] is one 128-row operand)
     T_Q = 4,                // Q_h
-    T_E = 6,                // E^{-1}_h -> N'^2_h -> (Ktil_a, Qtil_b) -> dP_h
-    T_F1 = 8,               // per half (b at +3): A_off, D W, D N
-    T_NN = 8,               // -N'_h -> (dQtil[b], dKtil[a]) -> dWhat_h -> dR_n_h -> dG_h
-    T_Z = 10,               // per half (b at +3): Zw, Zn, Zx -> What, U, X
-    T_I = 16,               // identity -> dP (the block's)
+    T_E = 6,                // (Ktil_a, Qtil_b) -> dP_h
+    T_NN = 8,               // (dQtil[b], dKtil[a]) -> dWhat_h -> dR_n_h -> dG_h
+    T_Z = 10,               // per half (b at +3): What, U, X
+    T_DPB = 16,             // dP (the block's)
     T_M = 17,               // M_h -> dM_h
     T_P = 19,               // (P_a, P_b) -> dU_h -> dN_h
     T_DSBA = 21,            // dSd[b, a]
     T_DQ = 22,              // dQ_h -> dR_w_h
     T_DK = 24,              // dK_h
-    T_DS = 26,              // dS_h (tile 27 first holds the fp32 diagonal blocks of A)
+    T_DS = 26,              // dS_h
     NTILES = 28,
 };
-constexpr int SA16_OFF = 27 * TILE;   // [2][4][16][16] fp32, over tile 27 until dS is loaded
 constexpr int BETA_OFF = NTILES * TILE;
 constexpr int PART_OFF = BETA_OFF + 128 * 4;  // [2][128] dbeta partial sums
 constexpr int BAR_OFF = PART_OFF + 256 * 4;
 constexpr int SMEM = BAR_OFF + 64 + 1024;
 
 // tensor-memory columns
-constexpr int C_GN = 0, C_M = 128;                    // W [W; K]^T, Q W^T
-constexpr int C_Z = 256;                              // N' | Zw | Zn | Zx -> (., What, U, X)
-constexpr int C_N2 = 0;                               // N'^2
-constexpr int C_F4 = 0;                               // U_a^T W_a | M_b What_b, then W^T What at +64
 constexpr int C_CA = 128;                             // dKtil_a | dQtil_b, then dP_a | dP_b at +64
 constexpr int C_B1 = 0;                               // dWhat', dU', dM' at +0, +64, +128
 constexpr int C_DR = 256;                             // dR_w | dR_n (held to the end)
@@ -108,6 +103,45 @@ __device__ __forceinline__ void tile_from_f32(uint8_t *tile, const float *src, l
     }
 }
 
+// N 64 x 64 fp32 blocks (row stride ld floats, 16-byte aligned) into fp16
+// tiles, every load in flight before the first store; the whole CTA, no barrier.
+template <int N>
+__device__ __forceinline__ void tiles_from_f32(uint8_t *const (&tiles)[N], const float *const (&src)[N],
+                                               const int (&ld)[N])
+{
+    const int t = threadIdx.x, row = t >> 2, c = (t & 3) * 16;
+    float4 q[N][4];
+#pragma unroll
+    for (int n = 0; n < N; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            q[n][i] = reinterpret_cast<const float4 *>(src[n] + (long long)row * ld[n] + c)[i];
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+        const float *f = reinterpret_cast<const float *>(q[n]);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            uint4 u;
+            __half2 *hh = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hh[i] = __floats2half2_rn(f[8 * j + 2 * i], f[8 * j + 2 * i + 1]);
+            *reinterpret_cast<uint4 *>(tiles[n] + sw128_offset(row, c + 8 * j)) = u;
+        }
+    }
+}
+
+// Row r, columns [c0, c0 + 32) of an fp16 tile negated in place.
+__device__ __forceinline__ void negate_in_place(uint8_t *tile, int r, int c0)
+{
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint4 *p = reinterpret_cast<uint4 *>(tile + sw128_offset(r, c0 + 8 * j));
+        uint4 u = *p;
+        u.x ^= 0x80008000u, u.y ^= 0x80008000u, u.z ^= 0x80008000u, u.w ^= 0x80008000u;
+        *p = u;
+    }
+}
+
 // Row r, columns [c0, c0 + 32) of a bf16 tile converted to fp16 in place.
 __device__ __forceinline__ void to_f16_in_place(uint8_t *tile, int r, int c0)
 {
@@ -119,16 +153,20 @@ __device__ __forceinline__ void to_f16_in_place(uint8_t *tile, int r, int c0)
 template <typename TO>
 __global__ void __launch_bounds__(NT, 1)
     prep_bwd_ut_kernel(const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mQ,
-                       const __grid_constant__ CUtensorMap mK, const float *beta, int L, int nblk,
+                       const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mH,
+                       const __grid_constant__ CUtensorMap mB, const float *beta, int L, int nblk,
                        float *dQt, float *dKt, const float *dPm, const float *dSd, TO *dq, TO *dk,
-                       TO *dw, float *dbeta, int *err)
+                       TO *dw, float *dbeta, int nsm, const int *saved, int *err)
 {
+    if (*saved != SAVED_WORD) {  // nothing to read: record it, write nothing
+        if (threadIdx.x == 0 && err) atomicCAS(err, 0, ERR_UT_NOT_SAVED);
+        return;
+    }
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
     auto tile = [&](int i) { return sm + i * TILE; };
     const uint32_t s0 = smem_u32(sm);
     auto ta = [&](int i) { return s0 + (uint32_t)i * TILE; };
-    float *sA16 = reinterpret_cast<float *>(sm + SA16_OFF);
     float *sB = reinterpret_cast<float *>(sm + BETA_OFF);
     float *sPart = reinterpret_cast<float *>(sm + PART_OFF);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + BAR_OFF);  // [0] loads, [1] MMA
@@ -136,48 +174,66 @@ __global__ void __launch_bounds__(NT, 1)
     const int J = blockIdx.x, hd = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Lp = nblk * BT;
     const long long brow = (long long)hd * Lp + (long long)J * BT;  // block's first row in [nh, Lp]
-    const float *dsdb = dSd + ((long long)hd * nblk + J) * BT * BT;
+    const long long blk = (long long)hd * nblk + J;
+    const float *dsdb = dSd + blk * BT * BT;
+    // the save area's tensor maps: mH over the per-half arrays What, U, X, M
+    // ([nblk_all 2 64, 64] each, stacked in that order at stride hstride rows),
+    // mB over the per-block ones Kta, Qtb, Pa, Pb ([nblk_all 64, 64], bstride rows)
+    const long long nb_all = (long long)nblk * gridDim.y;
+    const int hstride = (int)(nb_all * 2 * HB), bstride = (int)(nb_all * HB);
 
     if (tid == 0) {
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
         mbar_fence_init();
-        mbar_expect_tx(&bars[0], 6 * TILE);
+        mbar_expect_tx(&bars[0], 18 * TILE);
         for (int h = 0; h < 2; ++h) {
-            const int y = J * BT + h * HB;
+            const int y = J * BT + h * HB, yh = (int)(blk * 2 + h) * HB;
             tma_load_3d(tile(T_W + 2 * h), &mW, 0, y, hd, &bars[0]);
             tma_load_3d(tile(T_K + 2 * h), &mK, 0, y, hd, &bars[0]);
             tma_load_3d(tile(T_Q + h), &mQ, 0, y, hd, &bars[0]);
+            for (int m = 0; m < 3; ++m)  // What, U, X
+                tma_load_2d(tile(T_Z + 3 * h + m), &mH, 0, m * hstride + yh, &bars[0]);
+            tma_load_2d(tile(T_M + h), &mH, 0, 3 * hstride + yh, &bars[0]);
+            tma_load_2d(tile(T_E + h), &mB, 0, h * bstride + (int)blk * HB, &bars[0]);  // Ktil_a, Qtil_b
+            tma_load_2d(tile(T_P + h), &mB, 0, (2 + h) * bstride + (int)blk * HB, &bars[0]);  // P_a, P_b
         }
-        // every fp32 adjoint this block reads, on its way to L2 while the
-        // halves' transforms are recomputed
-        prefetch_l2(dQt + brow * HB, BT * HB * 4);
-        prefetch_l2(dKt + brow * HB, BT * HB * 4);
-        prefetch_l2(dPm + ((long long)hd * nblk + J) * HB * HB, HB * HB * 4);
-        prefetch_l2(dsdb, BT * BT * 4);
+        // one CTA per SM, started in grid order: the block nsm places further on
+        // starts on an SM this wave frees; what it reads goes to L2 meanwhile
+        const long long n2 = blk + nsm;
+        if (n2 < nb_all) {
+            const int J2 = (int)(n2 % nblk), h2 = (int)(n2 / nblk);
+            for (int h = 0; h < 2; ++h) {
+                tma_prefetch_3d(&mW, 0, J2 * BT + h * HB, h2);
+                tma_prefetch_3d(&mK, 0, J2 * BT + h * HB, h2);
+                tma_prefetch_3d(&mQ, 0, J2 * BT + h * HB, h2);
+                for (int m = 0; m < 4; ++m) tma_prefetch_2d(&mH, 0, m * hstride + (int)(n2 * 2 + h) * HB);
+                for (int m = 0; m < 2; ++m) tma_prefetch_2d(&mB, 0, (2 * m + h) * bstride + (int)n2 * HB);
+            }
+            const long long brow2 = (long long)h2 * Lp + (long long)J2 * BT;
+            prefetch_l2(dQt + brow2 * HB, BT * HB * 4);
+            prefetch_l2(dKt + brow2 * HB, BT * HB * 4);
+            prefetch_l2(dPm + n2 * HB * HB, HB * HB * 4);
+            prefetch_l2(dSd + n2 * BT * BT, BT * BT * 4);
+        }
     }
     if (warp == 0) tmem_alloc(tslot, 512);
-    // E^{-1} tiles (only their diagonal blocks are written below) and the identity
-    for (int i = tid; i < 2 * (int)TILE / 16; i += NT)
-        reinterpret_cast<uint4 *>(tile(T_E))[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (tid < HB) {
-        float one[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) one[j] = 0.f;
-        st_tile_f16(tile(T_I), tid, 32, one);
-        st_tile_f16(tile(T_I), tid, 0, one);
-        *reinterpret_cast<__half *>(tile(T_I) + sw128_offset(tid, tid)) = __float2half_rn(1.f);
-    }
     if (tid < BT) {
         const int p = J * BT + tid;
         sB[tid] = p < L ? beta[(long long)hd * L + p] : 0.f;
+    }
+    {   // the fp32 adjoints the composition adjoint reads, as fp16 operands
+        uint8_t *const t[4] = {tile(T_NN), tile(T_NN + 1), tile(T_DPB), tile(T_DSBA)};
+        const float *const src[4] = {dQt + (brow + HB) * HB, dKt + brow * HB, dPm + blk * HB * HB,
+                                     dsdb + (long long)HB * BT};  // dQtil[b], dKtil[a], dP, dSd[b, a]
+        const int ld[4] = {HB, HB, HB, BT};
+        tiles_from_f32(t, src, ld);
     }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = *tslot;
     bool ok = mbar_wait(&bars[0], 0, WAIT_LIMIT_NS);
-    ok = __syncthreads_and(ok);
 
     const Me me;
     const int h = me.h, r = me.r, c0 = 32 * me.cg;
@@ -206,131 +262,11 @@ __global__ void __launch_bounds__(NT, 1)
     } while (0)
 
     float v[32], x[32];
-
-    // ---- F0: W [W; K]^T and Q W^T per half (bf16 operands)
-    ISSUE(for (int hh = 0; hh < 2; ++hh) {
-        const uint32_t wk = ta(T_W + 2 * hh);
-        mma64(dst(tbase, hh, C_GN), wk, A_N, wk, B_T, 2, TILE, false, AB_BF16);
-        mma64(dst(tbase, hh, C_M), ta(T_Q + hh), A_N, wk, B_T, 1, TILE, false, AB_BF16);
-    });
-    // meanwhile: the adjoints the halves take from the attention backward as they are
-    tile_from_f32(tile(T_DQ), dQt + brow * HB, HB);             // dQ_a = dQtil[a]
-    tile_from_f32(tile(T_DK + 1), dKt + (brow + HB) * HB, HB);  // dK_b = dKtil[b]
-    wait_mma();
-    if (ok) {
-        me.ld(tbase, C_GN, v);  // A = strictLower(D G): diagonal blocks fp32, the rest A_off
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int col = c0 + j;
-            const float a = col < r ? br * v[j] : 0.f;
-            if ((col >> 4) == (r >> 4)) {
-                sA16[((h * 4 + (r >> 4)) * 16 + (r & 15)) * 16 + (col & 15)] = a;
-                x[j] = 0.f;
-            } else {
-                x[j] = a;
-            }
-        }
-        st_tile_f16(tile(T_F1 + 3 * h), r, c0, x);
-        me.ld(tbase, C_GN + 64, v);  // D N
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = c0 + j < r ? br * v[j] : 0.f;
-        st_tile_f16(tile(T_F1 + 3 * h + 2), r, c0, v);
-        me.ld(tbase, C_M, v);  // M = lower(Q W^T)
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (c0 + j > r) v[j] = 0.f;
-        st_tile_f16(tile(T_M + h), r, c0, v);
-        // W, K, Q to fp16 in place; D W
-        ld_tile_bf16(tile(T_W + 2 * h), r, c0, v);
-        st_tile_f16(tile(T_W + 2 * h), r, c0, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] *= br;
-        st_tile_f16(tile(T_F1 + 3 * h + 1), r, c0, v);
+    if (ok) {  // W, K, Q (bf16 inputs, exact in fp16) beside the fp16 operands; M from the saved -M
+        to_f16_in_place(tile(T_W + 2 * h), r, c0);
         to_f16_in_place(tile(T_K + 2 * h), r, c0);
         to_f16_in_place(tile(T_Q + h), r, c0);
-    }
-    sync_operands();
-    if (ok) {
-        uint8_t *const dinv[2] = {tile(T_E), tile(T_E + 1)};
-        diag_block_inverses(sA16, dinv);
-    }
-    sync_operands();
-
-    // ---- F1: [N' | Zw | Zn] = E^{-1} [A_off | D W | D N], Zx = E^{-1} I
-    ISSUE(for (int hh = 0; hh < 2; ++hh) {
-        mma64(dst(tbase, hh, C_Z), ta(T_E + hh), A_N, ta(T_F1 + 3 * hh), B_N, 3, TILE, false);
-        mma64(dst(tbase, hh, C_Z + 192), ta(T_E + hh), A_N, ta(T_I), B_N, 1, TILE, false);
-    });
-    // meanwhile: the halves' own logit adjoints (tile 27 held A's diagonal blocks)
-    tile_from_f32(tile(T_DS), dsdb, BT);                               // dS_a = dSd[a, a]
-    tile_from_f32(tile(T_DS + 1), dsdb + (long long)HB * BT + HB, BT);  // dS_b = dSd[b, b]
-    wait_mma();
-    if (ok) {
-        me.ld(tbase, C_Z, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = -v[j];
-        st_tile_f16(tile(T_NN + h), r, c0, v);
-        me.ld(tbase, C_Z + 64, v);
-        st_tile_f16(tile(T_Z + 3 * h), r, c0, v);
-        me.ld(tbase, C_Z + 128, v);
-        st_tile_f16(tile(T_Z + 3 * h + 1), r, c0, v);
-    }
-    sync_operands();
-
-    // ---- F2: Z1 = Z + (-N') Z (Zx's fp16 copy is the E^{-1} tile), N'^2
-    ISSUE(for (int hh = 0; hh < 2; ++hh) {
-        mma64(dst(tbase, hh, C_Z + 64), ta(T_NN + hh), A_N, ta(T_Z + 3 * hh), B_N, 2, TILE, true);
-        mma64(dst(tbase, hh, C_Z + 192), ta(T_NN + hh), A_N, ta(T_E + hh), B_N, 1, TILE, true);
-        mma64(dst(tbase, hh, C_N2), ta(T_NN + hh), A_N, ta(T_NN + hh), B_N, 1, TILE, false);
-    });
-    wait_mma();
-    if (ok) {
-#pragma unroll 1
-        for (int m = 0; m < 3; ++m) {
-            me.ld(tbase, C_Z + 64 + 64 * m, v);
-            st_tile_f16(tile(T_Z + 3 * h + m), r, c0, v);
-        }
-        me.ld(tbase, C_N2, v);
-        st_tile_f16(tile(T_E + h), r, c0, v);
-    }
-    sync_operands();
-
-    // ---- F3: [What | U | X] = Z1 + N'^2 Z1
-    ISSUE(for (int hh = 0; hh < 2; ++hh)
-              mma64(dst(tbase, hh, C_Z + 64), ta(T_E + hh), A_N, ta(T_Z + 3 * hh), B_N, 3, TILE, true));
-    // meanwhile: the block's adjoints that the composition adjoint reads
-    tile_from_f32(tile(T_NN), dQt + (brow + HB) * HB, HB);                  // dQtil[b]
-    tile_from_f32(tile(T_NN + 1), dKt + brow * HB, HB);                     // dKtil[a]
-    tile_from_f32(tile(T_I), dPm + ((long long)hd * nblk + J) * HB * HB, HB);  // dP
-    tile_from_f32(tile(T_DSBA), dsdb + (long long)HB * BT, BT);              // dSd[b, a]
-    wait_mma();
-    if (ok) {
-#pragma unroll 1
-        for (int m = 0; m < 3; ++m) {
-            me.ld(tbase, C_Z + 64 + 64 * m, v);
-            st_tile_f16(tile(T_Z + 3 * h + m), r, c0, v);
-        }
-    }
-    sync_operands();
-
-    // ---- F4: the halves' quantities the composition uses: Ktil_a, Qtil_b, P_a, P_b
-    ISSUE({
-        mma64(dst(tbase, 0, C_F4), ta(T_Z + 1), A_T, ta(T_W), B_N, 1, TILE, false);      // U_a^T W_a
-        mma64(dst(tbase, 1, C_F4), ta(T_M + 1), A_N, ta(T_Z + 3), B_N, 1, TILE, false);  // M_b What_b
-        for (int hh = 0; hh < 2; ++hh)                                                  // W^T What
-            mma64(dst(tbase, hh, C_F4 + 64), ta(T_W + 2 * hh), A_T, ta(T_Z + 3 * hh), B_N, 1, TILE, false);
-    });
-    wait_mma();
-    if (ok) {
-        me.ld(tbase, C_F4, v);
-        ld_tile_f16(tile(h ? T_Q + 1 : T_K), r, c0, x);  // K_a or Q_b
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = x[j] - v[j];
-        st_tile_f16(tile(T_E + h), r, c0, v);  // Ktil_a (h = 0), Qtil_b (h = 1)
-        me.ld(tbase, C_F4 + 64, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = (c0 + j == r ? 1.f : 0.f) - v[j];
-        st_tile_f16(tile(T_P + h), r, c0, v);  // P_h
+        negate_in_place(tile(T_M + h), r, c0);
     }
     sync_operands();
 
@@ -340,13 +276,20 @@ __global__ void __launch_bounds__(NT, 1)
         mma64(dst(tbase, 0, C_CA), ta(T_NN + 1), A_N, ta(T_P + 1), B_N, 1, TILE, false);
         mma64(dst(tbase, 0, C_CA), ta(T_DSBA), A_T, ta(T_E + 1), B_N, 1, TILE, true);
         mma64(dst(tbase, 0, C_CA + 64), ta(T_E + 1), A_T, ta(T_NN), B_N, 1, TILE, false);
-        mma64(dst(tbase, 0, C_CA + 64), ta(T_P + 1), A_T, ta(T_I), B_N, 1, TILE, true);
+        mma64(dst(tbase, 0, C_CA + 64), ta(T_P + 1), A_T, ta(T_DPB), B_N, 1, TILE, true);
         // b: dQtil_b = dQtil[b] P_a^T + dSd[b,a] Ktil_a; dP_b = dKtil[a]^T Ktil_a + dP P_a^T
         mma64(dst(tbase, 1, C_CA), ta(T_NN), A_N, ta(T_P), B_T, 1, TILE, false);
         mma64(dst(tbase, 1, C_CA), ta(T_DSBA), A_N, ta(T_E), B_N, 1, TILE, true);
         mma64(dst(tbase, 1, C_CA + 64), ta(T_NN + 1), A_T, ta(T_E), B_N, 1, TILE, false);
-        mma64(dst(tbase, 1, C_CA + 64), ta(T_I), A_N, ta(T_P), B_T, 1, TILE, true);
+        mma64(dst(tbase, 1, C_CA + 64), ta(T_DPB), A_N, ta(T_P), B_T, 1, TILE, true);
     });
+    {   // meanwhile: the halves' own adjoints as fp16 operands
+        uint8_t *const t[4] = {tile(T_DQ), tile(T_DK + 1), tile(T_DS), tile(T_DS + 1)};
+        const float *const src[4] = {dQt + brow * HB, dKt + (brow + HB) * HB, dsdb,
+                                     dsdb + (long long)HB * BT + HB};  // dQ_a, dK_b, dS_a, dS_b
+        const int ld[4] = {HB, HB, BT, BT};
+        tiles_from_f32(t, src, ld);
+    }
     wait_mma();
     if (ok) {
         me.ld(tbase, C_CA, v);
@@ -489,15 +432,15 @@ __global__ void __launch_bounds__(NT, 1)
 
 template <typename TO>
 cudaError_t launch(const CUtensorMap *m, const PrepDims &Dm, const PrepInputs &in,
-                   const PrepGrads &g, int *err, cudaStream_t st)
+                   const PrepGrads &g, const int *saved, int *err, cudaStream_t st)
 {
     auto k = prep_bwd_ut_kernel<TO>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
     k<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(
-        m[0], m[1], m[2], in.beta, Dm.L, Dm.nblk, const_cast<float *>(g.dQt),
+        m[0], m[1], m[2], m[3], m[4], in.beta, Dm.L, Dm.nblk, const_cast<float *>(g.dQt),
         const_cast<float *>(g.dKt), g.dPm, g.dSd, static_cast<TO *>(g.dq), static_cast<TO *>(g.dk),
-        static_cast<TO *>(g.dw), g.dbeta, err);
+        static_cast<TO *>(g.dw), g.dbeta, sm_count(), saved, err);
     count_launches();
     return cudaGetLastError();
 }
@@ -506,20 +449,28 @@ cudaError_t launch(const CUtensorMap *m, const PrepDims &Dm, const PrepInputs &i
 
 bool prep_backward_ut_supported(const PrepDims &Dm, const PrepInputs &in)
 {
-    return prep_forward_ut_supported(Dm, in);
+    // the save area's stacked maps index up to 4 nh nblk 128 rows (int32)
+    return prep_forward_ut_supported(Dm, in) && (long long)Dm.nh * Dm.nblk * 4 * BT < (1LL << 31);
 }
 
-cudaError_t prep_backward_ut(const PrepDims &Dm, const PrepInputs &in, const PrepGrads &g, int *err,
-                             cudaStream_t st)
+cudaError_t prep_backward_ut(const PrepDims &Dm, const PrepInputs &in, const PrepGrads &g,
+                             const UtSave &sv, const int *saved, int *err, cudaStream_t st)
 {
     if (!prep_backward_ut_supported(Dm, in)) return cudaErrorInvalidValue;
-    CUtensorMap m[3];
+    // What, U, X, M and Kta, Qtb, Pa, Pb lie back to back (carve_ut_save): one map each
+    const uint64_t nb = (uint64_t)Dm.nh * Dm.nblk, hsz = nb * 2 * HB * HB, bsz = nb * HB * HB;
+    if (sv.U != sv.What + hsz || sv.X != sv.U + hsz || sv.M != sv.X + hsz || sv.Qtb != sv.Kta + bsz ||
+        sv.Pa != sv.Qtb + bsz || sv.Pb != sv.Pa + bsz)
+        return cudaErrorInvalidValue;
+    CUtensorMap m[5];
     if (!make_map_3d(&m[0], in.w, BF16, HB, Dm.L, Dm.nh, HB) ||
         !make_map_3d(&m[1], in.q, BF16, HB, Dm.L, Dm.nh, HB) ||
-        !make_map_3d(&m[2], in.k, BF16, HB, Dm.L, Dm.nh, HB))
+        !make_map_3d(&m[2], in.k, BF16, HB, Dm.L, Dm.nh, HB) ||
+        !make_map_2d(&m[3], sv.What, F16, HB, 4 * nb * 2 * HB, HB) ||
+        !make_map_2d(&m[4], sv.Kta, F16, HB, 4 * nb * HB, HB))
         return cudaErrorInvalidValue;
-    if (Dm.odt == F32) return launch<float>(m, Dm, in, g, err, st);
-    return launch<bf16>(m, Dm, in, g, err, st);
+    if (Dm.odt == F32) return launch<float>(m, Dm, in, g, saved, err, st);
+    return launch<bf16>(m, Dm, in, g, saved, err, st);
 }
 
 }  // namespace path

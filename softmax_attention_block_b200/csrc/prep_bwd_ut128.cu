@@ -1,5 +1,5 @@
 // Adjoint of the head-dim-128 UT prep (prep_fwd_ut128.cu) on tcgen05, bf16
-// inputs, from the per-half quantities that forward saved (Ut128Save).
+// inputs, from the per-half quantities that forward saved (UtSave).
 //
 // The attention backward hands over, per block, the adjoints of the
 // boundary-adjusted queries / keys (dQtil, dKtil: 128 rows), of the block
@@ -42,7 +42,7 @@ using namespace uttc;
 
 constexpr int NT = 256;
 constexpr int DH = 128;  // head dim
-constexpr int SAVED_WORD = UT128_SAVED_BYTE * 0x01010101;
+constexpr int SAVED_WORD = UT_SAVED_BYTE * 0x01010101;
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
 {
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(NT, 1)
                           const int *saved, int *err)
 {
     if (*saved != SAVED_WORD) {  // nothing to read: record it, write nothing
-        if (threadIdx.x == 0 && err) atomicCAS(err, 0, ERR_UT128_NOT_SAVED);
+        if (threadIdx.x == 0 && err) atomicCAS(err, 0, ERR_UT_NOT_SAVED);
         return;
     }
     extern __shared__ uint8_t smraw[];
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(NT, 1)
                      const float *dSd, TO *dq, TO *dk, TO *dw, float *dbeta, const int *saved, int *err)
 {
     if (*saved != SAVED_WORD) {
-        if (threadIdx.x == 0 && err) atomicCAS(err, 0, ERR_UT128_NOT_SAVED);
+        if (threadIdx.x == 0 && err) atomicCAS(err, 0, ERR_UT_NOT_SAVED);
         return;
     }
     extern __shared__ uint8_t smraw[];
@@ -511,22 +511,8 @@ cudaError_t launch_adj(const CUtensorMap *m, const PrepDims &Dm, const PrepInput
 
 }  // namespace
 
-void carve_ut128_save(Carver &c, const PrepDims &D, Ut128Save &s)
-{
-    const size_t nb = (size_t)D.nh * D.nblk;
-    s.What = c.take<f16>(nb * 2 * HB * DH);
-    s.U = c.take<f16>(nb * 2 * HB * HB);
-    s.X = c.take<f16>(nb * 2 * HB * HB);
-    s.M = c.take<f16>(nb * 2 * HB * HB);
-    s.Kta = c.take<f16>(nb * HB * DH);
-    s.Qtb = c.take<f16>(nb * HB * DH);
-    s.Pa = c.take<f16>(nb * DH * DH);
-    s.Pb = c.take<f16>(nb * DH * DH);
-    s.dP = c.take<f16>(nb * 2 * DH * DH);
-}
-
 cudaError_t prep_backward_ut128(const PrepDims &Dm, const PrepInputs &in, const PrepGrads &g,
-                                const Ut128Save &sv, const int *saved, int *err, cudaStream_t st)
+                                const UtSave &sv, const int *saved, int *err, cudaStream_t st)
 {
     if (!prep_forward_ut128_supported(Dm, in) || (long long)Dm.nh * Dm.nblk * 2 * DH >= (1LL << 31))
         return cudaErrorInvalidValue;

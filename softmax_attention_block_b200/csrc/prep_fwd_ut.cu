@@ -20,6 +20,13 @@
 //   Z = E^{-1} D [W | N],  Z1 = Z - N' Z (with N'^2 = N' N'),  [What | U] = Z1 + N'^2 Z1.
 // Every product is an M = 64 MMA on fp16 operands with fp32 accumulation (the
 // bf16 inputs are exact in fp16); both halves run side by side (ut_tc.cuh).
+//
+// With a save area (a workspace sized for the backward) the kernel also writes
+// what the adjoint (prep_bwd_ut.cu) reads instead of recomputing it: per half
+// What, U, -M and X = (I + A)^{-1} (the same factors applied to the identity:
+// Z1x = (I - N') E^{-1}, X = (I + N'^2) Z1x), and the composition's inputs
+// Ktil_a, Qtil_b, P_a, P_b, all fp16 as the products read them, by TMA stores
+// of the operand tiles.
 #include "prep.cuh"
 #include "runtime.cuh"
 #include "ut_tc.cuh"
@@ -54,7 +61,7 @@ constexpr int SMEM = BAR_OFF + 64 + 1024;             // + 1024-byte alignment s
 // tensor-memory columns
 constexpr int C_G = 0, C_N = 64, C_M = 128, C_S = 192;  // W W^T, W K^T, Q W^T, Q K^T (then Sd)
 constexpr int C_Z = 256;                               // N' | Zw | Zn (then Z1, [What | U])
-constexpr int C_N2 = 0;                                // N'^2
+constexpr int C_N2 = 0, C_ZX = 64;                     // N'^2; saving: the X products
 constexpr int C_QT = 64, C_KT = 128, C_P = 0;          // -M What, U^T W, W^T What
 constexpr int C_C1 = 256, C_C2 = 320;                  // composition
 
@@ -75,11 +82,13 @@ __device__ __forceinline__ void st_box_f32(uint8_t *box, int r, const float (&v)
 // Outputs leave through shared-memory staging and TMA tensor stores: Qt, Kt
 // ([nh Lp, 64] fp16), Pm ([nh nblk 64, 64] fp16) in 64 x 64 tiles, Sd
 // ([nh nblk 128, 128] fp32) in 64-row boxes of 32 columns.
+template <bool SAVE>
 __global__ void __launch_bounds__(NT, 1)
     prep_fwd_ut_kernel(const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mQ,
                        const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mQt,
                        const __grid_constant__ CUtensorMap mKt, const __grid_constant__ CUtensorMap mPm,
-                       const __grid_constant__ CUtensorMap mSd, const float *beta, int L, int nblk,
+                       const __grid_constant__ CUtensorMap mSd, const __grid_constant__ CUtensorMap mSvH,
+                       const __grid_constant__ CUtensorMap mSvB, const float *beta, int L, int nblk,
                        int nsm, int *err)
 {
     extern __shared__ uint8_t smraw[];
@@ -136,6 +145,12 @@ __global__ void __launch_bounds__(NT, 1)
     const Me me;
     const int h = me.h, r = me.r, c0 = 32 * me.cg;
     const float br = sB[h * HB + r];
+    const int blk = hd * nblk + J;
+    // the save maps: mSvH over What, U, X, -M ([nb 2 64, 64] each, stacked at
+    // hstride rows), mSvB over Kta, Qtb, Pa, Pb ([nb 64, 64] each, bstride rows)
+    const int hstride = nblk * gridDim.y * 2 * HB, bstride = nblk * gridDim.y * HB;
+    constexpr int T_ZX = 12;  // + h: Z1x (over F1 tiles, free from level 1 to 4)
+    const bool storer = tid == 32;  // issues every TMA store (and waits for its own groups)
     uint32_t phase = 0;
     // one level: operands written and fenced, barrier; one thread issues the
     // products and commits; everyone waits for them
@@ -202,6 +217,10 @@ __global__ void __launch_bounds__(NT, 1)
         st_tile_f16(tile(T_F1 + 3 * h + 1), r, c0, v);
     }
     sync_operands();
+    if (SAVE && ok && storer) {  // -M of both halves
+        for (int hh = 0; hh < 2; ++hh) tma_store_2d(&mSvH, 0, 3 * hstride + (blk * 2 + hh) * HB, tile(T_MA + hh));
+        bulk_commit();
+    }
     if (ok) {
         uint8_t *const dinv[2] = {tile(T_DA), tile(T_DB)};
         diag_block_inverses(sA16, dinv);
@@ -224,10 +243,12 @@ __global__ void __launch_bounds__(NT, 1)
     }
     sync_operands();
 
-    // ---- level 2: Z1 = Z + (-N') Z (in place in tensor memory), N'^2 = (-N')(-N')
+    // ---- level 2: Z1 = Z + (-N') Z (in place in tensor memory), N'^2 = (-N')(-N');
+    // saving: (-N') E^{-1}, so that Z1x = E^{-1} + (-N') E^{-1}
     ISSUE(for (int hh = 0; hh < 2; ++hh) {
         mma64(dst(tbase, hh, C_Z + 64), ta(T_NA + hh), A_N, ta(T_Z + 2 * hh), B_N, 2, TILE, true);
         mma64(dst(tbase, hh, C_N2), ta(T_NA + hh), A_N, ta(T_NA + hh), B_N, 1, TILE, false);
+        if (SAVE) mma64(dst(tbase, hh, C_ZX), ta(T_NA + hh), A_N, ta(T_DA + hh), B_N, 1, TILE, false);
     });
     wait_mma();
     if (ok) {
@@ -235,22 +256,49 @@ __global__ void __launch_bounds__(NT, 1)
         st_tile_f16(tile(T_Z + 2 * h), r, c0, v);
         me.ld(tbase, C_Z + 128, v);
         st_tile_f16(tile(T_Z + 2 * h + 1), r, c0, v);
+        if (SAVE) {  // E^{-1} read before N'^2 replaces it
+            me.ld(tbase, C_ZX, v);
+            ld_tile_f16(tile(T_DA + h), r, c0, x);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += x[j];
+            st_tile_f16(tile(T_ZX + h), r, c0, v);
+        }
         me.ld(tbase, C_N2, v);
         st_tile_f16(tile(T_DA + h), r, c0, v);
     }
     sync_operands();
 
-    // ---- level 3: [What | U] = Z1 + N'^2 Z1
-    ISSUE(for (int hh = 0; hh < 2; ++hh)
-              mma64(dst(tbase, hh, C_Z + 64), ta(T_DA + hh), A_N, ta(T_Z + 2 * hh), B_N, 2, TILE, true));
+    // ---- level 3: [What | U] = Z1 + N'^2 Z1; saving: N'^2 Z1x (X = Z1x + N'^2 Z1x)
+    ISSUE(for (int hh = 0; hh < 2; ++hh) {
+        mma64(dst(tbase, hh, C_Z + 64), ta(T_DA + hh), A_N, ta(T_Z + 2 * hh), B_N, 2, TILE, true);
+        if (SAVE) mma64(dst(tbase, hh, C_ZX), ta(T_DA + hh), A_N, ta(T_ZX + hh), B_N, 1, TILE, false);
+    });
     wait_mma();
     if (ok) {
         me.ld(tbase, C_Z + 64, v);
         st_tile_f16(tile(T_Z + 2 * h), r, c0, v);
         me.ld(tbase, C_Z + 128, v);
         st_tile_f16(tile(T_Z + 2 * h + 1), r, c0, v);
+        if (SAVE) {  // X over -N' (read by no product since level 2)
+            me.ld(tbase, C_ZX, v);
+            ld_tile_f16(tile(T_ZX + h), r, c0, x);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += x[j];
+            st_tile_f16(tile(T_NA + h), r, c0, v);
+        }
     }
+    // the -M tiles become staging in level 4's epilogue: their save is read by now
+    if (SAVE && storer) bulk_wait_read<0>();
     sync_operands();
+    if (SAVE && ok && storer) {
+        for (int hh = 0; hh < 2; ++hh) {
+            const int y = (blk * 2 + hh) * HB;
+            tma_store_2d(&mSvH, 0, y, tile(T_Z + 2 * hh));                 // What
+            tma_store_2d(&mSvH, 0, hstride + y, tile(T_Z + 2 * hh + 1));   // U
+            tma_store_2d(&mSvH, 0, 2 * hstride + y, tile(T_NA + hh));      // X
+        }
+        bulk_commit();
+    }
 
     // ---- level 4: -M What, Q K^T - M U, U^T W, W^T What
     ISSUE(for (int hh = 0; hh < 2; ++hh) {
@@ -301,8 +349,9 @@ __global__ void __launch_bounds__(NT, 1)
         mma64(dst(tbase, 1, C_C1), ta(T_QTB), A_N, ta(T_PA), B_N, 1, TILE, false);  // Qtil_b P_a
         mma64(dst(tbase, 1, C_C2), ta(T_QTB), A_N, ta(T_KTA), B_T, 1, TILE, false); // Qtil_b Ktil_a^T
     });
-    const bool storer = tid == 32;  // issues every TMA store (and waits for its own groups)
     if (ok && storer) {
+        if (SAVE)  // the composition's inputs: Ktil_a, Qtil_b, P_a, P_b
+            for (int i = 0; i < 4; ++i) tma_store_2d(&mSvB, 0, i * bstride + blk * HB, tile(T_KTA + i));
         tma_store_2d(&mQt, 0, brow, tile(S_QA));
         tma_store_2d(&mKt, 0, brow + HB, tile(S_KB));
         for (int b = 0; b < 2; ++b) {
@@ -350,7 +399,7 @@ bool prep_forward_ut_supported(const PrepDims &Dm, const PrepInputs &in)
 }
 
 cudaError_t prep_forward_ut(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out,
-                            int *err, cudaStream_t st)
+                            const UtSave *save, int *err, cudaStream_t st)
 {
     if (!prep_forward_ut_supported(Dm, in)) return cudaErrorInvalidValue;
     CUtensorMap mW, mQ, mK, mQt, mKt, mPm, mSd;
@@ -362,10 +411,23 @@ cudaError_t prep_forward_ut(const PrepDims &Dm, const PrepInputs &in, const Prep
         !make_map_2d(&mPm, out.Pm, F16, HB, (uint64_t)Dm.nh * Dm.nblk * HB, HB) ||
         !make_map_f32_2d(&mSd, out.Sd, BT, rows, HB))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(prep_fwd_ut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    CUtensorMap mSvH{}, mSvB{};  // unused without a save area
+    if (save) {
+        // What, U, X, M and Kta, Qtb, Pa, Pb lie back to back (carve_ut_save): one map each
+        const uint64_t nb = (uint64_t)Dm.nh * Dm.nblk, hsz = nb * 2 * HB * HB, bsz = nb * HB * HB;
+        if (save->U != save->What + hsz || save->X != save->U + hsz || save->M != save->X + hsz ||
+            save->Qtb != save->Kta + bsz || save->Pa != save->Qtb + bsz || save->Pb != save->Pa + bsz ||
+            nb * 4 * BT >= (1ull << 31))
+            return cudaErrorInvalidValue;
+        if (!make_map_2d(&mSvH, save->What, F16, HB, 4 * nb * 2 * HB, HB) ||
+            !make_map_2d(&mSvB, save->Kta, F16, HB, 4 * nb * HB, HB))
+            return cudaErrorInvalidValue;
+    }
+    auto k = save ? prep_fwd_ut_kernel<true> : prep_fwd_ut_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
-    prep_fwd_ut_kernel<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(mW, mQ, mK, mQt, mKt, mPm, mSd, in.beta,
-                                                               Dm.L, Dm.nblk, sm_count(), err);
+    k<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(mW, mQ, mK, mQt, mKt, mPm, mSd, mSvH, mSvB, in.beta, Dm.L,
+                                              Dm.nblk, sm_count(), err);
     count_launches();
     return cudaGetLastError();
 }

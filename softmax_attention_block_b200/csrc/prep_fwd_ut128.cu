@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(NT, 1)
                           const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mQt,
                           const __grid_constant__ CUtensorMap mKt, const __grid_constant__ CUtensorMap mPm,
                           const __grid_constant__ CUtensorMap mSd, const float *beta, int L, int nblk,
-                          int nsm, Ut128Save sv, int *err)
+                          int nsm, UtSave sv, int *err)
 {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
@@ -441,7 +441,7 @@ bool prep_forward_ut128_supported(const PrepDims &Dm, const PrepInputs &in)
 }
 
 cudaError_t prep_forward_ut128(const PrepDims &Dm, const PrepInputs &in, const PrepOutputs &out,
-                               const Ut128Save *save, int *err, cudaStream_t st)
+                               const UtSave *save, int *err, cudaStream_t st)
 {
     if (!prep_forward_ut128_supported(Dm, in) || out.tdt != F16) return cudaErrorInvalidValue;
     CUtensorMap mW, mQ, mK, mQt, mKt, mPm, mSd;
@@ -457,7 +457,7 @@ cudaError_t prep_forward_ut128(const PrepDims &Dm, const PrepInputs &in, const P
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
     k<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(mW, mQ, mK, mQt, mKt, mPm, mSd, in.beta, Dm.L, Dm.nblk,
-                                              sm_count(), save ? *save : Ut128Save{}, err);
+                                              sm_count(), save ? *save : UtSave{}, err);
     count_launches();
     return cudaGetLastError();
 }

@@ -77,9 +77,9 @@ def _ws_formula(nh, L, d, bwd):
     lin = nh * (Lp * (1044 + 12 * d) + L * 4 * d) if bwd else nh * (Lp * (516 + 4 * d) + L * 2 * d)
     prods = nh * nblk * d * d * (6 if bwd else 2)
     scratch = 0
-    if d == 128:  # the UT quantities the forward leaves for the adjoint
-        scratch = nh * nblk * 245760 if bwd else 0
-    elif d != 64:
+    if d in (64, 128):  # the UT quantities the forward leaves for the adjoint
+        scratch = nh * nblk * (98304 if d == 64 else 245760) if bwd else 0
+    else:
         scratch = nh * nblk * ((14 * 128 * 128 + 3 * 128 * d) if bwd else (7 * 128 * 128 + 128 * d)) * 4
     return khat + lin + prods + scratch
 

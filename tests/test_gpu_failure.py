@@ -60,13 +60,14 @@ def test_forward_wait_gives_up_reports_and_recovers(P, d):
 PATH_ERR_WORKSPACE = 3
 
 
-def test_reuse_after_a_forward_that_saved_nothing(P):
-    """At bf16, head dim 128, a reusing backward reads per-block quantities that the
+@pytest.mark.parametrize("d", [64, 128])
+def test_reuse_after_a_forward_that_saved_nothing(P, d):
+    """At bf16, head dims 64 and 128, a reusing backward reads per-block quantities that the
     forward leaves only when its workspace_bytes covers the backward size. A forward
     told less (C ABI, on the same backward-sized buffer) leaves none: the backward then
     writes no gradient and reports PATH_ERR_WORKSPACE, and the next forward given the
     whole buffer makes a reusing backward correct again."""
-    x = si.make_inputs(1, 2, 200, 128, torch.bfloat16, seed=12)
+    x = si.make_inputs(1, 2, 200, d, torch.bfloat16, seed=12)
     dd = to_dev(x)
     B, H, L, D = dd["q"].shape
     nb_bwd = P.path_attn_workspace_bytes(B, H, L, D, torch.bfloat16, True)

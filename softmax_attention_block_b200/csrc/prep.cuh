@@ -50,7 +50,7 @@ cudaError_t prep_forward_rec(const PrepDims &D, const PrepInputs &in, const Prep
 // Per-block quantities of the tcgen05 UT kernels (head dims 64 and 128) that the
 // forward leaves for the adjoint in a backward-sized workspace (fp16, row-major;
 // blk = head * nblk + block, h = half):
-//   What [blk][h][64][d], U, X, M [blk][h][64][64], Kta, Qtb [blk][64][d]
+//   What [blk][h][64][d], U, X, M [blk][h][64][64] (M holds -lower(Q W^T)), Kta, Qtb [blk][64][d]
 //   (Ktil_a, Qtil_b), Pa, Pb [blk][d][d] (P_a, P_b); at d = 128 also the
 //   adjoint's own dP [blk][h][128][128] (the halves' dP).
 struct UtSave {

@@ -78,70 +78,6 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// 64 x 64 fp32 rows (row stride ld floats, 16-byte aligned) into an fp16 tile;
-// the whole CTA, no barrier.
-__device__ __forceinline__ void tile_from_f32(uint8_t *tile, const float *src, long long ld)
-{
-    const int t = threadIdx.x, row = t >> 2, c = (t & 3) * 16;
-    const float4 *p = reinterpret_cast<const float4 *>(src + (long long)row * ld + c);
-    float f[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float4 q = p[i];
-        f[4 * i] = q.x;
-        f[4 * i + 1] = q.y;
-        f[4 * i + 2] = q.z;
-        f[4 * i + 3] = q.w;
-    }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        uint4 u;
-        __half2 *hh = reinterpret_cast<__half2 *>(&u);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) hh[i] = __floats2half2_rn(f[8 * j + 2 * i], f[8 * j + 2 * i + 1]);
-        *reinterpret_cast<uint4 *>(tile + sw128_offset(row, c + 8 * j)) = u;
-    }
-}
-
-// N 64 x 64 fp32 blocks (row stride ld floats, 16-byte aligned) into fp16
-// tiles, every load in flight before the first store; the whole CTA, no barrier.
-template <int N>
-__device__ __forceinline__ void tiles_from_f32(uint8_t *const (&tiles)[N], const float *const (&src)[N],
-                                               const int (&ld)[N])
-{
-    const int t = threadIdx.x, row = t >> 2, c = (t & 3) * 16;
-    float4 q[N][4];
-#pragma unroll
-    for (int n = 0; n < N; ++n)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            q[n][i] = reinterpret_cast<const float4 *>(src[n] + (long long)row * ld[n] + c)[i];
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-        const float *f = reinterpret_cast<const float *>(q[n]);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            uint4 u;
-            __half2 *hh = reinterpret_cast<__half2 *>(&u);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) hh[i] = __floats2half2_rn(f[8 * j + 2 * i], f[8 * j + 2 * i + 1]);
-            *reinterpret_cast<uint4 *>(tiles[n] + sw128_offset(row, c + 8 * j)) = u;
-        }
-    }
-}
-
-// Row r, columns [c0, c0 + 32) of an fp16 tile negated in place.
-__device__ __forceinline__ void negate_in_place(uint8_t *tile, int r, int c0)
-{
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        uint4 *p = reinterpret_cast<uint4 *>(tile + sw128_offset(r, c0 + 8 * j));
-        uint4 u = *p;
-        u.x ^= 0x80008000u, u.y ^= 0x80008000u, u.z ^= 0x80008000u, u.w ^= 0x80008000u;
-        *p = u;
-    }
-}
-
 // Row r, columns [c0, c0 + 32) of a bf16 tile converted to fp16 in place.
 __device__ __forceinline__ void to_f16_in_place(uint8_t *tile, int r, int c0)
 {

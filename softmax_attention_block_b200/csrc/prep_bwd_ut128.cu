@@ -49,31 +49,6 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// 64 x 64 fp32 rows (row stride ld floats, 16-byte aligned) into an fp16 tile;
-// the whole CTA, no barrier.
-__device__ __forceinline__ void tile_from_f32(uint8_t *tile, const float *src, long long ld)
-{
-    const int t = threadIdx.x, row = t >> 2, c = (t & 3) * 16;
-    const float4 *p = reinterpret_cast<const float4 *>(src + (long long)row * ld + c);
-    float f[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float4 q = p[i];
-        f[4 * i] = q.x;
-        f[4 * i + 1] = q.y;
-        f[4 * i + 2] = q.z;
-        f[4 * i + 3] = q.w;
-    }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        uint4 u;
-        __half2 *hh = reinterpret_cast<__half2 *>(&u);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) hh[i] = __floats2half2_rn(f[8 * j + 2 * i], f[8 * j + 2 * i + 1]);
-        *reinterpret_cast<uint4 *>(tile + sw128_offset(row, c + 8 * j)) = u;
-    }
-}
-
 // A 64 x 64 bf16 tile converted to fp16 in place (the products' operand type);
 // the whole CTA, no barrier.
 __device__ __forceinline__ void tile_bf16_to_f16(uint8_t *tile)
@@ -162,13 +137,19 @@ __global__ void __launch_bounds__(NT, 1)
     // the fp32 adjoints as fp16 operands
     const float *dsdb = dSd + blk * BT * BT;
     const float *dpb = dPm + blk * DH * DH;
-    for (int c = 0; c < 2; ++c) {
-        tile_from_f32(tile(CA_DKA + c), dKt + brow * DH + 64 * c, DH);         // dKtil[a]
-        tile_from_f32(tile(CA_DQB + c), dQt + (brow + HB) * DH + 64 * c, DH);  // dQtil[b]
-        for (int rb = 0; rb < 2; ++rb)
-            tile_from_f32(tile(CA_DP + 2 * rb + c), dpb + 64 * rb * DH + 64 * c, DH);
+    {   // dKtil[a], dQtil[b], dSd[b, a]
+        uint8_t *const t[5] = {tile(CA_DKA), tile(CA_DKA + 1), tile(CA_DQB), tile(CA_DQB + 1), tile(CA_DSBA)};
+        const float *const src[5] = {dKt + brow * DH, dKt + brow * DH + 64, dQt + (brow + HB) * DH,
+                                     dQt + (brow + HB) * DH + 64, dsdb + (long long)HB * BT};
+        const int ld[5] = {DH, DH, DH, DH, BT};
+        tiles_from_f32(t, src, ld);
     }
-    tile_from_f32(tile(CA_DSBA), dsdb + (long long)HB * BT, BT);  // dSd[b, a]
+    {   // dP
+        uint8_t *const t[4] = {tile(CA_DP), tile(CA_DP + 1), tile(CA_DP + 2), tile(CA_DP + 3)};
+        const float *const src[4] = {dpb, dpb + 64, dpb + 64 * DH, dpb + 64 * DH + 64};
+        const int ld[4] = {DH, DH, DH, DH};
+        tiles_from_f32(t, src, ld);
+    }
     fence_async_smem();
     fence_before_sync();
     __syncthreads();
@@ -308,11 +289,13 @@ __global__ void __launch_bounds__(NT, 1)
         tma_load_2d(tile(U_M), &mM, 0, srow, &bars[0]);
     }
     if (warp == 0) tmem_alloc(tslot, 512);
-    for (int c = 0; c < 2; ++c) {
-        tile_from_f32(tile(U_DQ + c), dQt + hrow * DH + 64 * c, DH);
-        tile_from_f32(tile(U_DK + c), dKt + hrow * DH + 64 * c, DH);
+    {   // dQ, dK and dS = dSd[h, h] as fp16 operands
+        uint8_t *const t[5] = {tile(U_DQ), tile(U_DQ + 1), tile(U_DK), tile(U_DK + 1), tile(U_DS)};
+        const float *const src[5] = {dQt + hrow * DH, dQt + hrow * DH + 64, dKt + hrow * DH, dKt + hrow * DH + 64,
+                                     dSd + blk * BT * BT + (long long)hf * HB * BT + hf * HB};
+        const int ld[5] = {DH, DH, DH, DH, BT};
+        tiles_from_f32(t, src, ld);
     }
-    tile_from_f32(tile(U_DS), dSd + blk * BT * BT + (long long)hf * HB * BT + hf * HB, BT);  // dSd[h, h]
     if (tid < HB) {
         const int p = prow0 + tid;
         sB[tid] = p < L ? beta[(long long)hd * L + p] : 0.f;
@@ -323,9 +306,10 @@ __global__ void __launch_bounds__(NT, 1)
     fence_after_sync();
     const uint32_t tbase = *tslot;
     bool ok = mbar_wait(&bars[0], 0, WAIT_LIMIT_NS);
-    if (ok) {  // W, K, Q (bf16 inputs, exact in fp16) beside the fp16 operands
+    if (ok) {  // W, K, Q (bf16 inputs, exact in fp16) beside the fp16 operands; M from the saved -M
         for (int i = 0; i < 4; ++i) tile_bf16_to_f16(tile(U_W + i));
         for (int c = 0; c < 2; ++c) tile_bf16_to_f16(tile(U_Q + c));
+        negate_tile(tile(U_M));
     }
     fence_async_smem();
     ok = __syncthreads_and(ok);

@@ -23,9 +23,10 @@
 //
 // With a save area (a workspace sized for the backward) the kernel also writes
 // what the adjoint (prep_bwd_ut128.cu) reads instead of recomputing it: per
-// half What, U, M and X = (I + A)^{-1} (the same three factors applied to the
+// half What, U, -M and X = (I + A)^{-1} (the same three factors applied to the
 // identity: Z1x = (I - N') E^{-1}, X = (I + N'^2) Z1x), and the composition's
-// inputs Ktil_a, Qtil_b, P_a, P_b, all fp16 as the products read them.
+// inputs Ktil_a, Qtil_b, P_a, P_b, all fp16 as the products read them (What, U,
+// X and -M by TMA stores of the operand tiles).
 #include "prep.cuh"
 #include "runtime.cuh"
 #include "ut_tc.cuh"
@@ -86,7 +87,8 @@ __global__ void __launch_bounds__(NT, 1)
     prep_fwd_ut128_kernel(const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mQ,
                           const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mQt,
                           const __grid_constant__ CUtensorMap mKt, const __grid_constant__ CUtensorMap mPm,
-                          const __grid_constant__ CUtensorMap mSd, const float *beta, int L, int nblk,
+                          const __grid_constant__ CUtensorMap mSd, const __grid_constant__ CUtensorMap mSvW,
+                          const __grid_constant__ CUtensorMap mSvH, const float *beta, int L, int nblk,
                           int nsm, UtSave sv, int *err)
 {
     extern __shared__ uint8_t smraw[];
@@ -148,7 +150,10 @@ __global__ void __launch_bounds__(NT, 1)
     const float br = sB[h * HB + r];
     const int F = T_F + 4 * h;  // this half's F / Z tiles
     const long long blk = (long long)hd * nblk + J;
-    const long long hrow = (blk * 2 + h) * HB + r;  // this thread's row in the per-half save arrays
+    // the save maps: mSvW over What ([nb 2 64, 128]), mSvH over U, X, -M ([nb 2 64, 64]
+    // each, stacked at hs rows); a half's rows start at hy
+    const int hs = nblk * gridDim.y * 2 * HB;
+    const bool storer = tid == 32;  // issues every TMA store (and waits for its own groups)
     uint32_t phase = 0;
     // one level: operands written and fenced, barrier; one thread issues the
     // products and commits; everyone waits for them
@@ -206,10 +211,7 @@ __global__ void __launch_bounds__(NT, 1)
         st_tile_f16(tile(F + 3), r, c0, v);
         me.ld(tbase, C_M, v);  // -M, M = lower(Q W^T)
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = c0 + j <= r ? v[j] : 0.f;
-        if (SAVE) st_global(sv.M + hrow * HB + c0, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = -v[j];
+        for (int j = 0; j < 32; ++j) v[j] = c0 + j <= r ? -v[j] : 0.f;
         st_tile_f16(tile(T_M + h), r, c0, v);
         // W to fp16 in place (an operand beside fp16 intermediates from here on), and D W
 #pragma unroll 1
@@ -223,6 +225,10 @@ __global__ void __launch_bounds__(NT, 1)
         }
     }
     sync_operands();
+    if (SAVE && ok && storer) {  // -M of both halves
+        for (int hh = 0; hh < 2; ++hh) tma_store_2d(&mSvH, 0, 2 * hs + (int)(blk * 2 + hh) * HB, tile(T_M + hh));
+        bulk_commit();
+    }
     if (ok) {
         uint8_t *const dinv[2] = {tile(T_E), tile(T_E + 1)};
         diag_block_inverses(sA16, dinv);
@@ -284,22 +290,28 @@ __global__ void __launch_bounds__(NT, 1)
         for (int m = 0; m < 3; ++m) {
             me.ld(tbase, C_Z + 64 + 64 * m, v);
             st_tile_f16(tile(F + m), r, c0, v);
-            if (SAVE) {
-                if (m < 2)
-                    st_global(sv.What + hrow * DH + 64 * m + c0, v);
-                else
-                    st_global(sv.U + hrow * HB + c0, v);
-            }
         }
-        if (SAVE) {
+        if (SAVE) {  // X over Z1x
             me.ld(tbase, C_ZX, v);
             ld_tile_f16(tile(F + 3), r, c0, x);
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] += x[j];
-            st_global(sv.X + hrow * HB + c0, v);
+            st_tile_f16(tile(F + 3), r, c0, v);
         }
     }
+    // the -M tiles become staging in level 4's epilogue: their save is read by now
+    if (SAVE && storer) bulk_wait_read<0>();
     sync_operands();
+    if (SAVE && ok && storer) {  // What, U, X of both halves
+        for (int hh = 0; hh < 2; ++hh) {
+            const int f = T_F + 4 * hh, hy = (int)(blk * 2 + hh) * HB;
+            tma_store_2d(&mSvW, 0, hy, tile(f));
+            tma_store_2d(&mSvW, 64, hy, tile(f + 1));
+            tma_store_2d(&mSvH, 0, hy, tile(f + 2));
+            tma_store_2d(&mSvH, 0, hs + hy, tile(f + 3));
+        }
+        bulk_commit();
+    }
 
     // ---- level 4: -M What, Q K^T - M U, U^T W, rows 0..63 of W^T What
     // (What_h: tiles F, F + 1; U_h: F + 2; W_h's two column tiles 2 TILE apart)
@@ -342,13 +354,14 @@ __global__ void __launch_bounds__(NT, 1)
             if (c0 + j > r) v[j] = 0.f;
         st_box_f32(tile(T_M + 2 * h + me.cg), r, v);
     }
+    // P_h goes over the What / U / X tiles in level 4b's epilogue: their save is read by now
+    if (SAVE && storer) bulk_wait_read<0>();
     sync_operands();
 
     // ---- level 4b: rows 64..127 of W^T What, over the (read) -M What columns;
     // meanwhile Qtil[a], Ktil[b], Sd_aa, Sd_bb go out
     ISSUE(for (int hh = 0; hh < 2; ++hh)
               mma64(dst(tbase, hh, C_P1), ta(T_W(hh, 1)), A_T, ta(T_F + 4 * hh), B_N, 2, TILE, false));
-    const bool storer = tid == 32;  // issues every TMA store (and waits for its own groups)
     if (ok && storer) {
         for (int c = 0; c < 2; ++c) {
             tma_store_2d(&mQt, 64 * c, brow, tile(T_Q(0, c)));
@@ -453,11 +466,21 @@ cudaError_t prep_forward_ut128(const PrepDims &Dm, const PrepInputs &in, const P
         !make_map_2d(&mPm, out.Pm, F16, DH, (uint64_t)Dm.nh * Dm.nblk * DH, HB) ||
         !make_map_f32_2d(&mSd, out.Sd, BT, rows, HB))
         return cudaErrorInvalidValue;
+    CUtensorMap mSvW{}, mSvH{};  // unused without a save area
+    if (save) {
+        // U, X, M lie back to back (carve_ut_save): one map
+        const uint64_t nb = (uint64_t)Dm.nh * Dm.nblk, hsz = nb * 2 * HB * HB;
+        if (save->X != save->U + hsz || save->M != save->X + hsz || nb * 3 * BT >= (1ull << 31))
+            return cudaErrorInvalidValue;
+        if (!make_map_2d(&mSvW, save->What, F16, DH, nb * 2 * HB, HB) ||
+            !make_map_2d(&mSvH, save->U, F16, HB, 3 * nb * 2 * HB, HB))
+            return cudaErrorInvalidValue;
+    }
     auto k = save ? prep_fwd_ut128_kernel<true> : prep_fwd_ut128_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
-    k<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(mW, mQ, mK, mQt, mKt, mPm, mSd, in.beta, Dm.L, Dm.nblk,
-                                              sm_count(), save ? *save : UtSave{}, err);
+    k<<<dim3(Dm.nblk, Dm.nh), NT, SMEM, st>>>(mW, mQ, mK, mQt, mKt, mPm, mSd, mSvW, mSvH, in.beta, Dm.L,
+                                              Dm.nblk, sm_count(), save ? *save : UtSave{}, err);
     count_launches();
     return cudaGetLastError();
 }

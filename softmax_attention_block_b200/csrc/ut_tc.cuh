@@ -149,6 +149,59 @@ __device__ __forceinline__ void st_global(float *dst, const float (&v)[32])
         reinterpret_cast<float4 *>(dst)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
 }
 
+// N 64 x 64 fp32 blocks (row stride ld floats, 16-byte aligned) into fp16
+// tiles, every load in flight before the first store; the whole CTA (256
+// threads, 16 values each per block), no barrier.
+template <int N>
+__device__ __forceinline__ void tiles_from_f32(uint8_t *const (&tiles)[N], const float *const (&src)[N],
+                                               const int (&ld)[N])
+{
+    const int t = threadIdx.x, row = t >> 2, c = (t & 3) * 16;
+    float4 q[N][4];
+#pragma unroll
+    for (int n = 0; n < N; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            q[n][i] = reinterpret_cast<const float4 *>(src[n] + (long long)row * ld[n] + c)[i];
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+        const float *f = reinterpret_cast<const float *>(q[n]);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            uint4 u;
+            __half2 *hh = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hh[i] = __floats2half2_rn(f[8 * j + 2 * i], f[8 * j + 2 * i + 1]);
+            *reinterpret_cast<uint4 *>(tiles[n] + tc::sw128_offset(row, c + 8 * j)) = u;
+        }
+    }
+}
+
+// Row r, columns [c0, c0 + 32) of an fp16 tile negated in place.
+__device__ __forceinline__ void negate_in_place(uint8_t *tile, int r, int c0)
+{
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint4 *p = reinterpret_cast<uint4 *>(tile + tc::sw128_offset(r, c0 + 8 * j));
+        uint4 u = *p;
+        u.x ^= 0x80008000u, u.y ^= 0x80008000u, u.z ^= 0x80008000u, u.w ^= 0x80008000u;
+        *p = u;
+    }
+}
+
+// A 64 x 64 fp16 tile negated in place; the whole CTA (256 threads), no barrier.
+__device__ __forceinline__ void negate_tile(uint8_t *tile)
+{
+    const int t = threadIdx.x, row = t >> 2, c = (t & 3) * 16;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        uint4 *p = reinterpret_cast<uint4 *>(tile + tc::sw128_offset(row, c + 8 * j));
+        uint4 u = *p;
+        u.x ^= 0x80008000u, u.y ^= 0x80008000u, u.z ^= 0x80008000u, u.w ^= 0x80008000u;
+        *p = u;
+    }
+}
+
 // 32 fp32 values from global memory (16-byte aligned source).
 __device__ __forceinline__ void ld_global(const float *src, float (&v)[32])
 {

@@ -64,10 +64,16 @@ def stage_model(name, B, H, L, d, BT=128):
     """(algorithmic FLOP of one launch, bound) of a stage; causal, leading order.
 
     Tensor-core stages count the products of the blockwise algorithm; the UT
-    stages at head dim 64 count the 64x64x64 products their tcgen05 kernels
-    issue (fp16 operands), at other head dims the fp32 arithmetic of the
+    stages at head dims 64 and 128 count the 64x64x64 products their tcgen05
+    kernels issue (fp16 operands), at other head dims the fp32 arithmetic of the
     per-block recurrences and closed-form adjoint ("alu")."""
     nh, nblk, HB = B * H, -(-L // BT), 64
+    # 64x64x64 products per 128-block of the tcgen05 UT kernels: the prep (both
+    # halves' closed-form UT, boundary terms, the block's composition; at d = 128
+    # every d-wide product is two) and the adjoint (composition adjoint and both
+    # halves' UT adjoints, the halves' transform read from the forward's save)
+    ut_prep_products = {64: 36, 128: 74}
+    ut_adj_products = {64: 52, 128: 124}
     per = {
         "attn_fwd": (2.0 * L * L * d, "tensor"),                      # QK^T + PV
         # S, dP, dV, dK, dQ recomputed / formed once per causal pair, plus the
@@ -76,21 +82,16 @@ def stage_model(name, B, H, L, d, BT=128):
         "attn_bwd_q": (3.0 * L * L * d, "tensor"),                    # S, dP, dQ (SIMT path)
         "attn_bwd_k": (4.0 * L * L * d + 2.0 * L * L * d * d / BT, "tensor"),
         "chain": (1.0 * L * L * d * d / BT, "tensor"),               # key-side block transport
-        # head dim 64: per 128-block 36 products of 64x64 by 64x64 (both halves'
-        # UT in the closed form, boundary terms, the block's composition); other
-        # head dims: rank-one recurrences (keys with in-block logits, queries,
+        # other head dims: rank-one recurrences (keys with in-block logits, queries,
         # block product)
-        "ut_prep": ((36 * 2.0 * HB ** 3, "tensor")
-                    if d == 64 else (BT * BT / 2 * 10.0 * d + BT * 4.0 * d * d, "alu")),
-        # head dim 64: per 128-block 84 such products (the halves' UT recomputed,
-        # the composition's adjoint, both halves' UT adjoints)
-        "ut_adj": (nblk * 84 * 2.0 * HB ** 3, "tensor"),
+        "ut_prep": ((nblk * ut_prep_products[d] * 2.0 * HB ** 3, "tensor") if d in ut_prep_products
+                    else (nblk * (BT * BT / 2 * 10.0 * d + BT * 4.0 * d * d), "alu")),
+        "ut_adj": ((nblk * ut_adj_products[d] * 2.0 * HB ** 3, "tensor") if d in ut_adj_products
+                   else (0.0, None)),
         "ut_prep_bwd": (nblk * (8 * 2.0 * HB * HB * d + 4 * HB * HB * 4.0 * d
                                 + 2 * 24 * 2.0 * HB * HB * d), "alu"),
     }
     f, bound = per.get(name, (0.0, None))
-    if name == "ut_prep":
-        f *= nblk
     return f * nh, bound
 
 
@@ -98,10 +99,10 @@ def stage_model(name, B, H, L, d, BT=128):
 # B=1 H=24 L=4096 d=64 case (profiles/ summaries), scaled to the benchmark's
 # B=8 by the heads processed; None where the kernel changed since the capture.
 DRAM_BYTES_B1H24 = {
-    "attn_bwd": 325.7e6 + 98.3e6,
+    "attn_bwd": None,
     "attn_fwd": 274.1e6 + 9.8e6,
-    "ut_prep": 38.2e6 + 16.7e6,
-    "ut_adj": 151.0e6 + 29.3e6,
+    "ut_prep": 38.2e6 + 85.7e6,
+    "ut_adj": 235.2e6 + 39.6e6,
 }
 DRAM_BYTES_PREFILL_CACHE_B4H24 = 157.2e6
 

@@ -63,6 +63,14 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ void flag_error(int *err, int code)
 {
     if (err) atomicCAS(err, 0, code);
@@ -266,6 +274,10 @@ __global__ void __launch_bounds__(NT, 1)
         float *redl = red + 512;                                  // [2][128]
         const float k1 = a.scale_log2;
         const float ci2 = FOX ? a.c[(long long)h * Lp + gi] * LOG2E : 0.f;
+        // without the gate and with a positive scale, the logits stay unscaled: the
+        // row max scales after the fact and the scale joins the exponent's FFMA
+        const bool fast = !FOX && k1 > 0.f;
+        const float kx = fast ? k1 : 1.f;
         float acc[DH];
 #pragma unroll
         for (int e = 0; e < DH; ++e) acc[e] = 0.f;
@@ -303,17 +315,19 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
                     for (int j = 0; j < 64; ++j) {
                         const float bias = FOX ? ci2 - cj[j] * LOG2E : 0.f;
-                        z[j] = c0s + j <= r ? fmaf(z[j], k1, bias) : -INFINITY;
-                        pmax = fmaxf(pmax, z[j]);
+                        const float t = fast ? z[j] : fmaf(z[j], k1, bias);
+                        z[j] = c0s + j <= r ? t : -INFINITY;
                     }
-                } else {
+                } else if (!fast) {
 #pragma unroll
                     for (int j = 0; j < 64; ++j) {
                         const float bias = FOX ? ci2 - cj[j] * LOG2E : 0.f;
                         z[j] = fmaf(z[j], k1, bias);
-                        pmax = fmaxf(pmax, z[j]);
                     }
                 }
+#pragma unroll
+                for (int j = 0; j < 64; j += 2) pmax = fmax3(pmax, z[j], z[j + 1]);
+                if (fast) pmax *= k1;
             }
             float *rb = red + (it & 1) * 256;
             rb[hf * 128 + r] = pmax;
@@ -350,8 +364,8 @@ __global__ void __launch_bounds__(NT, 1)
                     __half2 *hh = reinterpret_cast<__half2 *>(&u);
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2) {
-                        const float p0 = ex2(z[g * 8 + 2 * q2] - m_new);
-                        const float p1 = ex2(z[g * 8 + 2 * q2 + 1] - m_new);
+                        const float p0 = ex2(fmaf(z[g * 8 + 2 * q2], kx, -m_new));
+                        const float p1 = ex2(fmaf(z[g * 8 + 2 * q2 + 1], kx, -m_new));
                         rowsum += p0 + p1;
                         hh[q2] = __floats2half2_rn(p0, p1);
                     }

@@ -487,6 +487,22 @@ def test_hand_worked_example(P):
             np.testing.assert_allclose(np64(out.cpu())[0, 0, :, :2], ro, atol=1e-5)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("scale", [-0.125, 0.0])
+def test_forward_with_non_positive_scale(P, d, scale):
+    """Without the gate and with a positive scale the tensor-core softmax keeps the
+    logits unscaled and scales the row max instead; a zero or negative scale takes the
+    per-element path. Both against the oracle at the same scale."""
+    x = si.make_inputs(1, 2, 300, d, torch.bfloat16, seed=13)
+    dd = to_dev(x)
+    out, lse = P.path_attn_fwd(dd["q"], dd["k"], dd["v"], dd["w"], dd["beta"], None, scale=scale,
+                               out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ro, rl = oracle.fwd(x["q"], x["k"], x["v"], x["w"], x["beta"], None, scale=scale)
+    compare({"out": out, "lse": lse}, {"out": ro, "lse": rl}, "bf16in_f32out",
+            f"scale={scale} d={d}")
+
+
 # ---------------------------------------------------------------- degenerate cases
 @pytest.mark.parametrize("dtype,d,L", [(torch.float32, 64, 300), (torch.bfloat16, 64, 333),
                                        (torch.bfloat16, 128, 200)])

@@ -99,7 +99,7 @@ const char *path_status_string(path_status s);
  * (backward) for the block products and their adjoints, each buffer rounded up
  * to 256 bytes; a bf16 backward at head dim 64 or 128 also holds per-block
  * quantities of the UT transform that a forward into the same workspace leaves
- * for the adjoint, nh * nblk * 114688 bytes at d = 64 and nh * nblk * 245760 at
+ * for the adjoint, nh * nblk * 98304 bytes at d = 64 and nh * nblk * 245760 at
  * d = 128; a backward that is neither (fp32 inputs, or bf16 at head dim 16 or
  * 32) holds the per-block scratch of its closed-form adjoint, nh * nblk * (14 * 128^2 + 3 * 128 d) * 4 bytes, and a bf16 forward at
  * head dim 16 or 32 the forward part of it, nh * nblk * (7 * 128^2 + 128 d) * 4

@@ -277,7 +277,7 @@ void carve_ut_save(Carver &c, const PrepDims &D, UtSave &s)
     s.Qtb = c.take<f16>(nb * hb * d);
     s.Pa = c.take<f16>(nb * d * d);
     s.Pb = c.take<f16>(nb * d * d);
-    s.dP = c.take<f16>(nb * 2 * d * d);
+    s.dP = d == 128 ? c.take<f16>(nb * 2 * d * d) : nullptr;
 }
 
 // Closed-form forward quantities the adjoint needs: A, G, Tinv, X, What, N, U, M.

@@ -51,8 +51,8 @@ cudaError_t prep_forward_rec(const PrepDims &D, const PrepInputs &in, const Prep
 // forward leaves for the adjoint in a backward-sized workspace (fp16, row-major;
 // blk = head * nblk + block, h = half):
 //   What [blk][h][64][d], U, X, M [blk][h][64][64] (M holds -lower(Q W^T)), Kta, Qtb [blk][64][d]
-//   (Ktil_a, Qtil_b), Pa, Pb [blk][d][d] (P_a, P_b); and the adjoint's own
-//   dP [blk][h][d][d] (the halves' dP).
+//   (Ktil_a, Qtil_b), Pa, Pb [blk][d][d] (P_a, P_b); at d = 128 also the
+//   adjoint's own dP [blk][h][128][128] (the halves' dP).
 struct UtSave {
     f16 *What = nullptr, *U = nullptr, *X = nullptr, *M = nullptr, *Kta = nullptr,
         *Qtb = nullptr, *Pa = nullptr, *Pb = nullptr, *dP = nullptr;
@@ -81,9 +81,10 @@ cudaError_t prep_forward_ut128(const PrepDims &D, const PrepInputs &in, const Pr
 // dQt and dKt are overwritten. saved: the workspace's save word (UT_SAVED_WORD).
 cudaError_t prep_backward_ut128(const PrepDims &D, const PrepInputs &in, const PrepGrads &g,
                                 const UtSave &save, const int *saved, int *err, cudaStream_t st);
-// Adjoint of prep_forward_ut from what it saved: the composition adjoint (one
-// kernel per block) and the per-half UT adjoint (one kernel per half block).
-// dQt and dKt are overwritten. saved: the workspace's save word (UT_SAVED_WORD).
+// Adjoint of prep_forward_ut from what it saved: one kernel per half block forms
+// the half's adjoints from the block's (composition adjoint) and applies the UT
+// adjoint. dQt and dKt are read only. saved: the workspace's save word
+// (UT_SAVED_WORD).
 bool prep_backward_ut_supported(const PrepDims &D, const PrepInputs &in);
 cudaError_t prep_backward_ut(const PrepDims &D, const PrepInputs &in, const PrepGrads &g,
                              const UtSave &save, const int *saved, int *err, cudaStream_t st);

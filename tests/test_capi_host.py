@@ -78,7 +78,7 @@ def _ws_formula(nh, L, d, bwd):
     prods = nh * nblk * d * d * (6 if bwd else 2)
     scratch = 0
     if d in (64, 128):  # the UT quantities the forward leaves for the adjoint
-        scratch = nh * nblk * (114688 if d == 64 else 245760) if bwd else 0
+        scratch = nh * nblk * (98304 if d == 64 else 245760) if bwd else 0
     else:
         scratch = nh * nblk * ((14 * 128 * 128 + 3 * 128 * d) if bwd else (7 * 128 * 128 + 128 * d)) * 4
     return khat + lin + prods + scratch

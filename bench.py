@@ -102,7 +102,7 @@ DRAM_BYTES_B1H24 = {
     "attn_bwd": 325.96e6 + 97.03e6,
     "attn_fwd": 274.1e6 + 9.8e6,
     "ut_prep": 38.2e6 + 85.7e6,
-    "ut_adj": 75.5e6 + 4.8e6 + 176.7e6 + 24.3e6,
+    "ut_adj": 214.4e6 + 24.1e6,
 }
 DRAM_BYTES_PREFILL_CACHE_B4H24 = 157.2e6
 

@@ -17,7 +17,7 @@
 // Khat_{J,I+1} = Khat_{J,I} P_I^T, so Abar is the adjoint carried back along
 // the key-side transport chain; after the pair (J+1, J) it is dKtil_J. dQtil is
 // staged in the pair's spent dS^T buffer by the drain warps and accumulates
-// across CTAs by TMA tensor reduce-add; dP_I by fp32 vector atomics; the gate's
+// across CTAs by TMA tensor reduce-add, and so does dP_I (through an 8 KB box); the gate's
 // row sums by fp32 atomics. The diagonal tile takes its logits from the UT prep
 // and writes dS to the prep's adjoint instead (dSd), which carries it to dQ,
 // dK, dW, dbeta.
@@ -64,7 +64,9 @@ struct BCfg {
     static constexpr int ST_BYTES = 3 * TILE + 8192 + 2048;
     static constexpr int CS_OFF = ST_OFF + 2 * ST_BYTES;  // [128] column-sum exchange
     static constexpr int BAR_OFF = CS_OFF + 512;
-    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    // dP_I staging: one fp32 box of 64 rows x 32 columns (128-byte swizzle)
+    static constexpr int DPI_OFF = (BAR_OFF + 256 + 1023) / 1024 * 1024;
+    static constexpr int SMEM = DPI_OFF + 8192 + 1024;
     // TMEM columns: no two accumulators share columns; P^T (packed bf16) sits in
     // the S^T columns, query block q (16 queries) at column 64 (q / 4) + 8 (q % 4)
     static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_AB = 320, T_DQ = 384, T_DPI = 448;
@@ -86,13 +88,14 @@ __global__ void __launch_bounds__(NT, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                   const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mDO,
                   const __grid_constant__ CUtensorMap mP, const __grid_constant__ CUtensorMap mDQ,
-                  BwdTcArgs a)
+                  const __grid_constant__ CUtensorMap mDPI, BwdTcArgs a)
 {
     using C = BCfg;
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
     uint8_t *sAb = sm + C::AB_OFF, *sV = sm + C::V_OFF, *sDs = sm + C::DS_OFF;
     float *sCs = reinterpret_cast<float *>(sm + C::CS_OFF);
+    uint8_t *sDpi = sm + C::DPI_OFF;
     auto stage = [&](int s) { return sm + C::ST_OFF + s * C::ST_BYTES; };
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::BAR_OFF);
     uint64_t *v_full = bars, *ld_full = bars + 1, *ld_empty = bars + 3, *s_full = bars + 5,
@@ -396,7 +399,7 @@ __global__ void __launch_bounds__(NT, 1)
         // dQtil leaves through fp32 staging (128B-swizzled boxes of 32 columns) in
         // this pair's dS^T buffer, spent once MMA 2 has completed, and bulk tensor
         // reduce-add; the buffer goes back to the softmax after the reduction has
-        // read it. dP_I leaves by fp32 vector atomics.
+        // read it. dP_I leaves the same way through its own 8 KB staging box.
         const int j = tid - 32 * W_DRAIN0;
         const int gj = J * BT + j;
         const bool leader = j == 0;
@@ -464,12 +467,26 @@ __global__ void __launch_bounds__(NT, 1)
             // TMEM results read and Abar written: MMA 2 of the next pair may go
             fence_before_sync();
             mbar_arrive(e_done);
-            if (drain && I < last && j < D) {
-                float4 *dpi = reinterpret_cast<float4 *>(a.dPm + (((long long)h * nblk + I) * D + j) * D);
+            if (I < last && j < D) {
+                // dP_I (rows j < 64: the first two drain warps) leaves by bulk tensor
+                // reduce-add, 32 columns at a time through one 8 KB staging box
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    atomicAdd(dpi + k, make_float4(dpv[k >> 3][4 * (k & 7)], dpv[k >> 3][4 * (k & 7) + 1],
-                                                   dpv[k >> 3][4 * (k & 7) + 2], dpv[k >> 3][4 * (k & 7) + 3]));
+                for (int hb = 0; hb < 2; ++hb) {
+                    if (drain) {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            *reinterpret_cast<float4 *>(sDpi + j * 128 + ((k ^ (j & 7)) << 4)) =
+                                make_float4(dpv[hb][4 * k], dpv[hb][4 * k + 1], dpv[hb][4 * k + 2], dpv[hb][4 * k + 3]);
+                        fence_async_smem();
+                    }
+                    named_barrier(3, 64);  // the box is written
+                    if (leader && drain) {
+                        tma_reduce_add_2d(&mDPI, 32 * hb, (h * nblk + I) * D, sDpi);
+                        bulk_commit();
+                        bulk_wait_read<0>();
+                    }
+                    named_barrier(3, 64);  // and read: it may be written again
+                }
             }
             if (leader) {
                 if (drain) bulk_wait_read<0>();
@@ -532,7 +549,7 @@ cudaError_t launch(const CUtensorMap *m, const BwdTcArgs &a, cudaStream_t st)
     auto k = bwd_tc_kernel<FOX, TO>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BCfg::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<dim3(a.nblk, a.nh), NT, BCfg::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], a);
+    k<<<dim3(a.nblk, a.nh), NT, BCfg::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], a);
     count_launches();
     return cudaGetLastError();
 }
@@ -563,7 +580,7 @@ cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16
     const int Lp = b.nblk * BT;
     const long long npairs = (long long)b.nblk * (b.nblk - 1) / 2;
     const void *dob = t.out == F32 ? dout_bf16 : b.dout;
-    CUtensorMap m[6];
+    CUtensorMap m[7];
     if (!make_map_2d(&m[0], b.Qt, F16, D, (uint64_t)b.nh * Lp, 128)) return cudaErrorInvalidValue;
     if (npairs > 0) {
         if (!make_map_2d(&m[1], b.Khat, F16, D, (uint64_t)b.nh * npairs * BT, 128)) return cudaErrorInvalidValue;
@@ -573,7 +590,8 @@ cudaError_t attn_bwd_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_bf16
     if (!make_map_3d(&m[2], b.v, BF16, D, b.L, b.nh, 128) ||
         !make_map_3d(&m[3], dob, BF16, D, b.L, b.nh, 128) ||
         !make_map_2d(&m[4], b.Pm, F16, D, (uint64_t)b.nh * b.nblk * D, D) ||
-        !make_map_f32_2d(&m[5], b.dQt, D, (uint64_t)b.nh * Lp, 128))
+        !make_map_f32_2d(&m[5], b.dQt, D, (uint64_t)b.nh * Lp, 128) ||
+        !make_map_f32_2d(&m[6], b.dPm, D, (uint64_t)b.nh * b.nblk * D, D))
         return cudaErrorInvalidValue;
     BwdTcArgs a{b.Sd, b.c, lse_p, b.delta, b.scale, b.L, b.nblk, b.nh, npairs,
                 b.dQt, b.dKt, b.dPm, b.dSd, b.dv, b.rowsum, b.colsum, err};

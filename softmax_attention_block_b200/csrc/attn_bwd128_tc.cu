@@ -12,8 +12,10 @@
 //   MMA 2: dV += P^T dO_q;  Abar (+)= [Abar_{I+1} P_I] + dS^T Qtil_q;
 //          dQtil_q = dS Khat_{J,I} (64 x 128, over the spent S^T / dP^T columns);
 //          once per block: dP_I = Abar_{I+1}^T Khat_{J,I}
-//   drain: dQtil_q and dP_I to the global accumulators by vector atomics; after the
-//          block, Abar to the operand tile (fp16) or, after block J+1, to dKtil_J.
+//   drain: dQtil_q and dP_I to the global accumulators by bulk tensor reduce-add,
+//          staged as fp32 boxes in the spent P^T / dS^T buffers (32 KB: dQtil_q at
+//          once, dP_I in two rounds); after the block, Abar to the operand tile
+//          (fp16) or, after block J+1, to dKtil_J.
 // The diagonal block takes its logits from the UT prep and hands dS to its adjoint
 // (dSd), as at head dim 64. One thread issues the loads and the products; all
 // threads run the softmax and the drain in sequence; every wait is bounded.
@@ -74,7 +76,8 @@ template <bool FOX, typename TO>
 __global__ void __launch_bounds__(NT, 1)
     bwd128_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                      const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mDO,
-                     const __grid_constant__ CUtensorMap mP, BwdTcArgs a)
+                     const __grid_constant__ CUtensorMap mP, const __grid_constant__ CUtensorMap mDQ,
+                     const __grid_constant__ CUtensorMap mDPI, BwdTcArgs a)
 {
     using C = C128;
     extern __shared__ uint8_t smraw[];
@@ -307,33 +310,60 @@ __global__ void __launch_bounds__(NT, 1)
         if (ok && tid == 0 && s + 2 < nsub) load_sub(s + 2);
         // ---- drain
         if (ok && !diag) {
+            // staging: the spent P^T and dS^T buffers, 32 KB of fp32 boxes of 32
+            // columns (128-byte rows, 128-byte swizzle)
+            uint8_t *stg = sm + C::PT_OFF;
             // dQtil of the sub-tile (M = 64: rows 16 quarter + t in lanes 32 quarter + t, t < 16;
-            // the TMEM loads are warp-wide, the upper lanes' values are not used)
+            // the TMEM loads are warp-wide, the upper lanes' values are not used): four
+            // boxes of 64 rows
             {
                 const int qi = 16 * (warp & 3) + (lane & 15);
-                float *dst = a.dQt + ((long long)h * Lp + I * BT + q * QS + qi) * D + 64 * cg;
-#pragma unroll 1
+#pragma unroll
                 for (int c0 = 0; c0 < 64; c0 += 32) {
                     float v[32];
                     tmem_ld32(tbase + C::T_DQ + 64 * cg + c0 + lane_off, v);
                     if (lane < 16) {
+                        uint8_t *box = stg + (2 * cg + c0 / 32) * 8192 + qi * 128;
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            atomicAdd(reinterpret_cast<float4 *>(dst + c0 + e),
-                                      make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]));
+                        for (int k = 0; k < 8; ++k)
+                            *reinterpret_cast<float4 *>(box + ((k ^ (qi & 7)) << 4)) =
+                                make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
                     }
+                }
+                fence_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    for (int b = 0; b < 4; ++b)
+                        tma_reduce_add_2d(&mDQ, 32 * b, h * Lp + I * BT + q * QS, stg + b * 8192);
+                    bulk_commit();
                 }
             }
             if (q == 0 && hasP) {
-                // dP_I rows f = j (lane), columns [64 cg, 64 cg + 64)
-                float *dst = a.dPm + (((long long)h * nblk + I) * D + j) * D + 64 * cg;
+                // dP_I rows f = j (lane), columns [64 cg, 64 cg + 64): in two rounds (one
+                // per column half) of two boxes of 128 rows, once the staging is read
 #pragma unroll 1
-                for (int c0 = 0; c0 < 64; c0 += 32) {
-                    float v[32];
-                    tmem_ld32(tbase + C::T_DPI + 64 * cg + c0 + lane_off, v);
+                for (int half = 0; half < 2; ++half) {
+                    if (tid == 0) bulk_wait_read<0>();
+                    __syncthreads();
+                    if (cg == half) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        atomicAdd(reinterpret_cast<float4 *>(dst + c0 + e), make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]));
+                        for (int c0 = 0; c0 < 64; c0 += 32) {
+                            float v[32];
+                            tmem_ld32(tbase + C::T_DPI + 64 * cg + c0 + lane_off, v);
+                            uint8_t *box = stg + (c0 / 32) * 16384 + j * 128;
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                *reinterpret_cast<float4 *>(box + ((k ^ (j & 7)) << 4)) =
+                                    make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                        }
+                    }
+                    fence_async_smem();
+                    __syncthreads();
+                    if (tid == 0) {
+                        for (int b = 0; b < 2; ++b)
+                            tma_reduce_add_2d(&mDPI, 64 * half + 32 * b, (h * nblk + I) * D, stg + b * 16384);
+                        bulk_commit();
+                    }
                 }
             }
             if (q == 1) {
@@ -360,6 +390,8 @@ __global__ void __launch_bounds__(NT, 1)
                 }
             }
         }
+        // the next sub-tile's softmax writes P^T and dS^T: the staging's reads end first
+        if (tid == 0) bulk_wait_read<0>();
         fence_async_smem();
         fence_before_sync();
         ok = __syncthreads_and(ok);
@@ -399,6 +431,7 @@ __global__ void __launch_bounds__(NT, 1)
         for (int t = done_sub; t < issued_sub; ++t) mbar_wait(&sub_full[t & 1], (t >> 1) & 1, 8 * WAIT_LIMIT_NS);
         commit(mma_done);
         mbar_wait(mma_done, 0, 8 * WAIT_LIMIT_NS);
+        bulk_wait_all();  // and every reduction from the staging has completed
     }
     fence_before_sync();
     __syncthreads();
@@ -412,7 +445,7 @@ cudaError_t launch(const CUtensorMap *m, const BwdTcArgs &a, cudaStream_t st)
     auto k = bwd128_tc_kernel<FOX, TO>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C128::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<dim3(a.nblk, a.nh), NT, C128::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], a);
+    k<<<dim3(a.nblk, a.nh), NT, C128::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], a);
     count_launches();
     return cudaGetLastError();
 }
@@ -427,7 +460,7 @@ cudaError_t attn_bwd128_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_b
     const int Lp = b.nblk * BT;
     const long long npairs = (long long)b.nblk * (b.nblk - 1) / 2;
     const void *dob = t.out == F32 ? dout_bf16 : b.dout;
-    CUtensorMap m[5];
+    CUtensorMap m[7];
     if (!make_map_2d(&m[0], b.Qt, F16, D, (uint64_t)b.nh * Lp, QS)) return cudaErrorInvalidValue;
     if (npairs > 0) {
         if (!make_map_2d(&m[1], b.Khat, F16, D, (uint64_t)b.nh * npairs * BT, BT)) return cudaErrorInvalidValue;
@@ -436,7 +469,9 @@ cudaError_t attn_bwd128_tc(const BwdArgs &b, Types t, float *lse_p, void *dout_b
     }
     if (!make_map_3d(&m[2], b.v, BF16, D, b.L, b.nh, BT) ||
         !make_map_3d(&m[3], dob, BF16, D, b.L, b.nh, QS) ||
-        !make_map_2d(&m[4], b.Pm, F16, D, (uint64_t)b.nh * b.nblk * D, D))
+        !make_map_2d(&m[4], b.Pm, F16, D, (uint64_t)b.nh * b.nblk * D, D) ||
+        !make_map_f32_2d(&m[5], b.dQt, D, (uint64_t)b.nh * Lp, QS) ||
+        !make_map_f32_2d(&m[6], b.dPm, D, (uint64_t)b.nh * b.nblk * D, D))
         return cudaErrorInvalidValue;
     BwdTcArgs a{b.Sd, b.c, lse_p, b.delta, b.scale, b.L, b.nblk, b.nh, npairs,
                 b.dQt, b.dKt, b.dPm, b.dSd, b.dv, b.rowsum, b.colsum, err};

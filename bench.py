@@ -99,7 +99,7 @@ def stage_model(name, B, H, L, d, BT=128):
 # B=1 H=24 L=4096 d=64 case (profiles/ summaries), scaled to the benchmark's
 # B=8 by the heads processed; None where the kernel changed since the capture.
 DRAM_BYTES_B1H24 = {
-    "attn_bwd": 325.96e6 + 97.03e6,
+    "attn_bwd": 326.02e6 + 95.38e6,
     "attn_fwd": 274.1e6 + 9.8e6,
     "ut_prep": 38.2e6 + 85.7e6,
     "ut_adj": 214.4e6 + 24.1e6,

@@ -66,7 +66,9 @@ struct BCfg {
     static constexpr int BAR_OFF = CS_OFF + 512;
     // dP_I staging: one fp32 box of 64 rows x 32 columns (128-byte swizzle)
     static constexpr int DPI_OFF = (BAR_OFF + 256 + 1023) / 1024 * 1024;
-    static constexpr int SMEM = DPI_OFF + 8192 + 1024;
+    // gate: per-warp row-sum partials [2 pairs][2 warpgroups][4 warps][64 queries]
+    static constexpr int RS_OFF = DPI_OFF + 8192;
+    static constexpr int SMEM = RS_OFF + 4096 + 1024;
     // TMEM columns: no two accumulators share columns; P^T (packed bf16) sits in
     // the S^T columns, query block q (16 queries) at column 64 (q / 4) + 8 (q % 4)
     static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_AB = 320, T_DQ = 384, T_DPI = 448;
@@ -96,6 +98,7 @@ __global__ void __launch_bounds__(NT, 1)
     uint8_t *sAb = sm + C::AB_OFF, *sV = sm + C::V_OFF, *sDs = sm + C::DS_OFF;
     float *sCs = reinterpret_cast<float *>(sm + C::CS_OFF);
     uint8_t *sDpi = sm + C::DPI_OFF;
+    float *sRs = reinterpret_cast<float *>(sm + C::RS_OFF);
     auto stage = [&](int s) { return sm + C::ST_OFF + s * C::ST_BYTES; };
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::BAR_OFF);
     uint64_t *v_full = bars, *ld_full = bars + 1, *ld_empty = bars + 3, *s_full = bars + 5,
@@ -348,8 +351,9 @@ __global__ void __launch_bounds__(NT, 1)
                         }
                     }
                     dsv[0] += __shfl_xor_sync(0xffffffffu, dsv[0], 1);
-                    if (!(lane & 1))
-                        atomicAdd(a.rowsum + (long long)h * Lp + I * BT + c + (lane >> 1), dsv[0] / a.scale);
+                    // this warp's 32 keys' part of query c + m's row sum, combined with
+                    // the other three warps' after the pass
+                    if (!(lane & 1)) sRs[(((it & 1) * 2 + g) * 4 + (warp & 3)) * 64 + (c & 63) + (lane >> 1)] = dsv[0];
                 }
             };
             // the four chunks of this warpgroup, the next chunk's loads in flight while
@@ -382,6 +386,15 @@ __global__ void __launch_bounds__(NT, 1)
                     pass(std::true_type{});
                 else
                     pass(std::false_type{});
+            }
+            if (FOX) {
+                // the row sums of dS over the tile's 128 keys: one atomic per query
+                named_barrier(4 + g, 128);
+                if (ok && j < 64) {
+                    const float *rs = sRs + ((it & 1) * 2 + g) * 4 * 64 + j;
+                    atomicAdd(a.rowsum + (long long)h * Lp + I * BT + 64 * g + j,
+                              (rs[0] + rs[64] + rs[128] + rs[192]) / a.scale);
+                }
             }
             tmem_wait_st();
             fence_async_smem();

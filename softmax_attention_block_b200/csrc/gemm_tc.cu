@@ -1,11 +1,12 @@
 // Batched small GEMM of the closed-form UT transform on 5th-generation tensor
 // cores (tcgen05, kind::tf32): the same contract as gemm_batched (GemmArgs),
-// for the bf16-input paths. Products are split TF32: each operand is staged as
-// hi (rounded to TF32) and lo (the fp32 remainder), and every K step adds
-// hi.hi + hi.lo + lo.hi, so the products hold about 21 significant bits. One
-// TF32 pass was measured too coarse for the closed form of a 128-position block
-// at head dim 128 (the fp32-output gradient error of dw tripled). fp32 inputs
-// keep the CUDA-core gemm_batched.
+// for bf16 inputs at the head dims without per-half UT kernels (16, 32).
+// Products are split TF32: each operand is staged as hi (rounded to TF32) and
+// lo (the fp32 remainder), and every K step adds hi.hi + hi.lo + lo.hi, so the
+// products hold about 21 significant bits. One TF32 pass was measured too
+// coarse for the closed form of a 128-position block at head dim 128, when that
+// head dim still ran here (the fp32-output gradient error of dw tripled). fp32
+// inputs keep the CUDA-core gemm_batched.
 //
 // One CTA of 256 threads per batch item (head, block), three CTAs per SM: C
 // [M x N] with M, N, K <= 128. Per term and 32-wide quarter of K the operands are staged in shared

@@ -99,12 +99,17 @@ def stage_model(name, B, H, L, d, BT=128):
 # B=1 H=24 L=4096 d=64 case (profiles/ summaries), scaled to the benchmark's
 # B=8 by the heads processed; None where the kernel changed since the capture.
 DRAM_BYTES_B1H24 = {
-    "attn_bwd": 326.02e6 + 95.38e6,
+    "attn_bwd": 325.66e6 + 94.57e6,
     "attn_fwd": 274.1e6 + 9.8e6,
     "ut_prep": 38.2e6 + 85.7e6,
     "ut_adj": 214.4e6 + 24.1e6,
 }
 DRAM_BYTES_PREFILL_CACHE_B4H24 = 157.2e6
+# The same for the forget-gate workload's kernels, from a capture of B=1 H=6 L=16384
+# d=64, scaled by the heads processed.
+DRAM_BYTES_FOX_B1H6 = {
+    "attn_bwd": 933.63e6 + 103.36e6,
+}
 
 
 def load_peaks():
@@ -541,8 +546,9 @@ def timed_calls(call, n, flush, stream):
     return sum(a.elapsed_time(b) for a, b in evs) / n
 
 
-def stage_roofline(stages, B, H, L, d, peaks):
-    """Dominant stage of a timed region -> roofline object against the sustained bf16 peak."""
+def stage_roofline(stages, B, H, L, d, peaks, traffic_per_head=None):
+    """Dominant stage of a timed region -> roofline object against the sustained bf16 peak.
+    traffic_per_head: DRAM bytes per launch per head of the kernels captured, by stage."""
     if not stages:
         return None
     dom = max(stages, key=lambda n: stages[n][0])
@@ -550,8 +556,10 @@ def stage_roofline(stages, B, H, L, d, peaks):
     f, bound = stage_model(dom, B, H, L, d)
     ach = f / (per_launch_ms * 1e-3) / 1e12 if f else None
     peak = peaks["bf16_tflops_sustained"]
+    t = (traffic_per_head or {}).get(dom)
     return {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-            "frac": (ach / peak) if ach else None, "traffic": None,
+            "frac": (ach / peak) if ach else None,
+            "traffic": t * B * H if t is not None else None, "traffic_unit": "bytes per launch",
             "peak_source": f"{peaks['source']} bf16 dense (sustained)"}
 
 
@@ -633,7 +641,8 @@ def bench_fox(P, dev, peaks, world, max_over_ranks, barrier, steps, cpu_sample):
            "pct_bf16_peak": fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
            "l2": "flushed (256 MB written) before every timed step",
            "stages": {n: {"ms_per_launch": t / c, "launches": c} for n, (t, c) in stages.items()},
-           "roofline": stage_roofline(stages, w.B, w.H, w.L, w.d, peaks)}
+           "roofline": stage_roofline(stages, w.B, w.H, w.L, w.d, peaks,
+                                      {k: v / 6.0 for k, v in DRAM_BYTES_FOX_B1H6.items()})}
     if cpu_sample:
         import oracle
 
